@@ -1,0 +1,109 @@
+"""fp64 oracle of the Muon step -- TEST INFRASTRUCTURE ONLY (see package doc).
+
+Sources (page title, then section):
+
+* [MC] "MuonClip: speed, then stability" -- §02 "Momentum remembers.
+  Orthogonalization redistributes." (momentum, Nesterov, quintic NS step and
+  its coefficients, orientation), §03 "Making Muon scale" (0.2*sqrt(max(n,m))
+  scale, decoupled decay W <- W - eta*(O + lambda*W)), §07 "One complete
+  training step" (step order).
+* [MV] "Muon and MuonClip: orthogonalised updates for LLM training" --
+  §2 "Newton-Schulz: an odd polynomial on singular values" (X0 = G/||G||_F,
+  A = X X^T, X = aX + (bA + cA A)X, phi(x) = ax + bx^3 + cx^5, m <= n cost
+  rule), "The Muon optimizer" (M <- mu M + G; Moonlight form of the update).
+* [MS] "About Muon: Muon At Scale" -- "Why Not Bernstein's Multiplier?"
+  (update snippet: p *= 1 - lr*wd; p += -lr*scale*u, scale = 0.2*sqrt(max)).
+
+Readings where the pages are silent (each also listed in the design doc):
+
+* Nesterov lookahead: [MC] §02 only says one "may be applied".  Read as the
+  recurrence applied once more with the current gradient, U = G + mu*M_t, in
+  the pages' own sum convention M_t = mu*M_{t-1} + G_t.
+* Orientation: the NS input is transposed only when rows > cols, so that
+  A = X X^T is min(m,n) square; a square matrix is not transposed.
+* Normalisation: X0 = U / max(||U||_F, eps) with eps = 1e-7, so that a zero
+  matrix gives a zero update ([MV] prints U/||U||_F with no eps).
+* Scale: 0.2*sqrt(max(rows, cols)) ([MC] §03, [MV], [MS]); weight decay acts
+  on the pre-update W.
+"""
+from __future__ import annotations
+
+import numpy as np
+
+
+def phi(x, a: float, b: float, c: float):
+    """The scalar odd quintic phi(x) = a x + b x^3 + c x^5 that one NS step
+    applies to every singular value ([MV] §2, odd-polynomial identity)."""
+    x = np.asarray(x, dtype=np.float64)
+    return a * x + b * x ** 3 + c * x ** 5
+
+
+def phi_iter(x, steps: int, a: float, b: float, c: float):
+    """phi applied ``steps`` times."""
+    y = np.asarray(x, dtype=np.float64)
+    for _ in range(steps):
+        y = phi(y, a, b, c)
+    return y
+
+
+def newton_schulz(U: np.ndarray, steps: int, a: float, b: float, c: float,
+                  eps: float = 1e-7) -> np.ndarray:
+    """Approximate polar factor of ``U`` by the quintic Newton-Schulz iteration.
+
+    [MV] §2: X0 = U/||U||_F, then ``steps`` times A = X X^T,
+    X = a X + (b A + c A A) X.  [MC] §02: A is formed after choosing the
+    cheaper orientation, i.e. the short side first (m <= n); the result is
+    transposed back.  Returns an array of U's shape.
+    """
+    U = np.asarray(U, dtype=np.float64)
+    transposed = U.shape[0] > U.shape[1]
+    X = U.T if transposed else U
+    norm = np.sqrt(np.sum(X * X))
+    X = X / max(norm, eps)
+    for _ in range(steps):
+        A = X @ X.T
+        B = b * A + c * (A @ A)
+        X = a * X + B @ X
+    return X.T if transposed else X
+
+
+def muon_step(W, G, M, *, mu, nesterov, lr, wd, ns_steps, a, b, c, eps, rms_scale):
+    """One Muon step on one hidden 2D weight, in float64.
+
+    Follows [MC] §07's order: momentum, NS, scaled update with decoupled decay.
+
+      M_t   = mu * M_{t-1} + G                          ([MC] §02, [MV])
+      U     = G + mu * M_t  if nesterov else M_t         (reading, see module doc)
+      O     = NS_steps(U)                                ([MV] §2)
+      Upd   = rms_scale * sqrt(max(rows, cols)) * O      ([MC] §03, [MS])
+      W_t   = W_{t-1} - lr * (Upd + wd * W_{t-1})        ([MC] §03)
+
+    Returns (W_t, M_t, Upd, ||U||_F), all float64.
+    """
+    W = np.asarray(W, dtype=np.float64)
+    G = np.asarray(G, dtype=np.float64)
+    M = np.asarray(M, dtype=np.float64)
+    M_new = mu * M + G
+    U = G + mu * M_new if nesterov else M_new
+    O = newton_schulz(U, ns_steps, a, b, c, eps)
+    upd = rms_scale * np.sqrt(max(W.shape)) * O
+    W_new = W - lr * (upd + wd * W)
+    return W_new, M_new, upd, float(np.sqrt(np.sum(U * U)))
+
+
+def muon_step_many(Ws, Gs, Ms, hp: dict, workers: int = 1):
+    """``muon_step`` over a list of independent matrices (optionally in a
+    spawn-started process pool).  Returns lists (W_t, M_t, Upd, norm)."""
+    args = [(W, G, M) for W, G, M in zip(Ws, Gs, Ms)]
+    if workers <= 1 or len(args) <= 1:
+        outs = [muon_step(W, G, M, **hp) for (W, G, M) in args]
+    else:
+        import multiprocessing as mp
+        ctx = mp.get_context("spawn")
+        with ctx.Pool(workers) as pool:
+            outs = pool.starmap(_muon_step_kw, [(W, G, M, hp) for (W, G, M) in args])
+    return [list(t) for t in zip(*outs)]
+
+
+def _muon_step_kw(W, G, M, hp):
+    return muon_step(W, G, M, **hp)

@@ -1,0 +1,303 @@
+"""Pins for the fp64 oracle: each test ties an oracle function to something
+other than itself -- the odd-polynomial/SVD identity, numbers the pages print
+(tests/golden/printed_numbers.json, each entry cited), brute force on tiny
+inputs, limits with a textbook answer, or a third-party optimizer run as a
+library.  CPU only."""
+import json
+import os
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from matrix_orthogonalising_optimizer_step_b200 import workloads as wl
+
+GOLD = json.load(open(os.path.join(os.path.dirname(__file__), "golden", "printed_numbers.json")))
+TUNED = tuple(GOLD["tuned_coefficients"]["value"])
+
+
+def haar(rng, n, k):
+    q, r = np.linalg.qr(rng.standard_normal((n, k)))
+    return q * np.sign(np.diag(r))
+
+
+# ---------------------------------------------------------------- scalar map
+def test_scalar_map_printed_properties():
+    a, b, c = GOLD["simple_quintic"]["value"]
+    assert oracle.phi(1.0, a, b, c) == pytest.approx(GOLD["simple_quintic"]["phi_at_1"], abs=1e-15)
+    h = 1e-6
+    d = (oracle.phi(1 + h, a, b, c) - oracle.phi(1 - h, a, b, c)) / (2 * h)
+    assert d == pytest.approx(GOLD["simple_quintic"]["dphi_at_1"], abs=1e-8)
+    a3, b3, c3 = GOLD["classic_cubic"]["value"]
+    # The cubic converges to exactly 1 from inside (0, 1].
+    assert oracle.phi_iter(0.3, 60, a3, b3, c3) == pytest.approx(1.0, abs=1e-12)
+
+
+def test_scalar_map_polar_express_number():
+    g = GOLD["polar_express_vs_ns"]
+    y = oracle.phi_iter(g["x0"], g["steps"], *TUNED)
+    assert abs(y - g["printed"]) <= g["tol"]
+
+
+def test_scalar_map_overshoot_and_band():
+    xs = np.linspace(1e-6, 1.0, 400_001)
+    y = oracle.phi_iter(xs, 5, *TUNED)
+    g = GOLD["tuned_overshoot_max"]
+    assert abs(y.max() - g["printed"]) <= g["tol"]
+    band = GOLD["tuned_band"]
+    sel = xs >= band["x_from"]
+    assert y[sel].min() >= band["lo"] - band["slack"]
+    assert y[sel].max() <= band["hi"] + band["slack"]
+    jb = GOLD["jordan_band"]
+    assert jb["lo"] - 0.02 <= y[sel].min() and y.max() <= jb["hi"]
+
+
+def test_scalar_map_demo_numbers_are_consistent():
+    from scipy.optimize import brentq
+    g = GOLD["demo_consistency"]
+    x0 = brentq(lambda x: oracle.phi_iter(x, 5, *TUNED) - g["tuned_5"], 1e-5, 1e-2)
+    simple = tuple(GOLD["simple_quintic"]["value"])
+    assert abs(oracle.phi_iter(x0, 5, *simple) - g["simple_5"]) <= g["tol_simple_5"]
+    assert abs(oracle.phi_iter(x0, 10, *simple) - g["simple_10"]) <= g["tol_simple_10"]
+
+
+# ---------------------------------------------------------- matrix iteration
+@pytest.mark.parametrize("shape", [(24, 40), (40, 24), (32, 32), (7, 19)])
+def test_ns_equals_scalar_map_on_singular_values(shape):
+    """Odd-polynomial identity: NS(U diag(s) V^T) = U diag(phi^N(s/||s||)) V^T."""
+    r, c = shape
+    m = min(r, c)
+    rng = np.random.default_rng(11 + r * 100 + c)
+    U, V = haar(rng, r, m), haar(rng, c, m)
+    s = np.sort(rng.uniform(0.01, 3.0, m))[::-1]
+    G = (U * s) @ V.T
+    want = (U * oracle.phi_iter(s / np.linalg.norm(s), 5, *TUNED)) @ V.T
+    got = oracle.newton_schulz(G, 5, *TUNED)
+    assert np.linalg.norm(got - want) <= 1e-12 * np.linalg.norm(want)
+
+
+def test_ns_on_diagonal_is_scalar_map_entrywise():
+    d = np.array([3.0, -1.0, 0.5, 0.02, 0.0])
+    G = np.zeros((5, 9))
+    G[np.arange(5), np.arange(5)] = d
+    got = oracle.newton_schulz(G, 5, *TUNED)
+    want = np.zeros_like(G)
+    want[np.arange(5), np.arange(5)] = oracle.phi_iter(d / np.linalg.norm(d), 5, *TUNED)
+    assert np.max(np.abs(got - want)) <= 1e-14
+
+
+def test_ns_keeps_singular_vectors_and_band_and_approaches_polar():
+    rng = np.random.default_rng(5)
+    r, c = 48, 80
+    U, V = haar(rng, r, r), haar(rng, c, r)
+    s = np.linspace(1.0, 0.1, r)
+    G = (U * s) @ V.T
+    O = oracle.newton_schulz(G, 5, *TUNED)
+    D = U.T @ O @ V
+    off = D - np.diag(np.diag(D))
+    assert np.max(np.abs(off)) <= 1e-10
+    sv = np.diag(D)
+    assert sv.min() >= 0.68 and sv.max() <= 1.21
+    P = U @ V.T
+    assert np.linalg.norm(O - P) / np.linalg.norm(P) <= 0.32
+
+
+def test_ns_converges_to_svd_polar_factor_with_simple_quintic():
+    """With phi(1) = 1, phi'(1) = 0 the iteration converges to U V^T, the
+    polar factor that numpy's SVD gives (textbook limit)."""
+    rng = np.random.default_rng(6)
+    G = rng.standard_normal((30, 50)) + 3 * np.eye(30, 50)
+    u, _, vt = np.linalg.svd(G, full_matrices=False)
+    O = oracle.newton_schulz(G, 40, *GOLD["simple_quintic"]["value"])
+    assert np.linalg.norm(O - u @ vt) <= 1e-9 * np.linalg.norm(u @ vt)
+
+
+def test_ns_orientation_transpose_equivariant():
+    rng = np.random.default_rng(7)
+    G = rng.standard_normal((20, 33))
+    assert np.array_equal(oracle.newton_schulz(G.T, 5, *TUNED), oracle.newton_schulz(G, 5, *TUNED).T)
+
+
+def test_ns_zero_matrix_gives_zero():
+    assert np.array_equal(oracle.newton_schulz(np.zeros((4, 6)), 5, *TUNED), np.zeros((4, 6)))
+
+
+# ----------------------------------------------------------------- the step
+def test_update_rms_is_point_two_for_exact_polar_factor(hp):
+    """0.2 sqrt(max(m,n)) U V^T has entry RMS exactly 0.2 (printed target).
+    Uses the converging simple quintic so that NS reaches U V^T."""
+    rng = np.random.default_rng(8)
+    for (r, c) in [(40, 90), (90, 40), (64, 64)]:
+        G = rng.standard_normal((r, c)) + 2 * np.eye(r, c)
+        p = dict(hp, ns_steps=40, a=2.0, b=-1.5, c=0.5, lr=1.0, wd=0.0, mu=0.0, nesterov=False)
+        _, _, upd, _ = oracle.muon_step(np.zeros((r, c)), G, np.zeros((r, c)), **p)
+        rms = np.sqrt(np.mean(upd ** 2))
+        assert rms == pytest.approx(GOLD["rms_target"]["value"], rel=1e-10)
+
+
+def test_update_rms_closed_form_for_tuned_ns(hp):
+    """RMS of 0.2 sqrt(n) NS(G) = 0.2 sqrt(sum phi^5(s_i/||s||)^2 / m)."""
+    rng = np.random.default_rng(9)
+    r, c = 36, 100
+    U, V = haar(rng, r, r), haar(rng, c, r)
+    s = 1.0 / np.arange(1, r + 1)
+    G = (U * s) @ V.T
+    p = dict(hp, mu=0.0, nesterov=False)
+    _, _, upd, _ = oracle.muon_step(np.zeros((r, c)), G, np.zeros((r, c)), **p)
+    want = 0.2 * np.sqrt(np.sum(oracle.phi_iter(s / np.linalg.norm(s), 5, *TUNED) ** 2) / r)
+    assert np.sqrt(np.mean(upd ** 2)) == pytest.approx(want, rel=1e-12)
+
+
+def test_momentum_special_cases(hp):
+    rng = np.random.default_rng(10)
+    M0 = rng.standard_normal((6, 8))
+    G = rng.standard_normal((6, 8))
+    W = rng.standard_normal((6, 8))
+    _, M1, _, _ = oracle.muon_step(W, np.zeros_like(G), M0, **hp)
+    assert np.allclose(M1, hp["mu"] * M0, rtol=0, atol=0)
+    _, M1, _, _ = oracle.muon_step(W, G, np.zeros_like(M0), **hp)
+    assert np.array_equal(M1, G)
+
+
+def test_nesterov_lookahead_diagonal_pin(hp):
+    """With diagonal M0 = diag(p) and G = diag(q), Nesterov's NS input is
+    diagonal (1+mu) q + mu^2 p, the plain one q + mu p; the update is then the
+    scalar map on the normalised diagonal."""
+    mu = hp["mu"]
+    p_ = np.array([1.0, 0.2, 0.0, 0.05])
+    q_ = np.array([0.0, 0.3, 0.7, 0.01])
+    r, c = 4, 7
+    M0 = np.zeros((r, c)); M0[range(4), range(4)] = p_
+    G = np.zeros((r, c)); G[range(4), range(4)] = q_
+    for nesterov, u in [(True, (1 + mu) * q_ + mu * mu * p_), (False, q_ + mu * p_)]:
+        h = dict(hp, nesterov=nesterov)
+        _, _, upd, nrm = oracle.muon_step(np.zeros((r, c)), G, M0, **h)
+        want = np.zeros((r, c))
+        want[range(4), range(4)] = 0.2 * np.sqrt(c) * oracle.phi_iter(u / np.linalg.norm(u), 5, *TUNED)
+        assert np.max(np.abs(upd - want)) <= 1e-13
+        assert nrm == pytest.approx(np.linalg.norm(u), rel=1e-14)
+
+
+def test_first_step_independent_of_nesterov(hp):
+    W, G, M = wl.cfg0_matrix()
+    W, G, M = (t.double().numpy() for t in (W, G, M))
+    a = oracle.muon_step(W, G, M, **dict(hp, nesterov=True))
+    b = oracle.muon_step(W, G, M, **dict(hp, nesterov=False))
+    assert np.max(np.abs(a[2] - b[2])) <= 1e-13 * np.max(np.abs(a[2]))
+
+
+def test_decay_and_apply_special_cases(hp):
+    rng = np.random.default_rng(12)
+    W = rng.standard_normal((5, 9)); G = rng.standard_normal((5, 9)); M = rng.standard_normal((5, 9))
+    Wn, _, _, _ = oracle.muon_step(W, G, M, **dict(hp, lr=0.0))
+    assert np.array_equal(Wn, W)
+    Wn, _, upd, _ = oracle.muon_step(W, G, M, **dict(hp, wd=0.0))
+    assert np.allclose(Wn - W, -hp["lr"] * upd, rtol=1e-12, atol=1e-15)
+    Wn, _, upd, _ = oracle.muon_step(W, np.zeros_like(G), np.zeros_like(M), **hp)
+    assert np.array_equal(upd, np.zeros_like(upd))
+    assert np.allclose(Wn, (1 - hp["lr"] * hp["wd"]) * W, rtol=1e-15, atol=0)
+
+
+def test_cfg0_matches_torch_muon(hp):
+    """Third-party run: torch.optim.Muon with Moonshot's RMS matching on the
+    same cfg0 inputs (zero momentum, so its buffer convention does not matter
+    after normalisation).  torch runs its NS in bf16 whatever the parameter
+    dtype (measured: 2.08e-2 from this oracle with float32 and float64
+    parameters alike; a bf16-rounding emulation of the oracle's own NS sits
+    1.7e-2 away), so the bound is 3e-2.  It still separates the update scale
+    0.2*sqrt(max) from 0.2*sqrt(min) (41 %) and a missing transpose."""
+    W, G, M = wl.cfg0_matrix()
+    p = torch.nn.Parameter(W.clone())
+    opt = torch.optim.Muon([p], lr=hp["lr"], weight_decay=hp["wd"], momentum=hp["mu"],
+                           nesterov=True, ns_coefficients=TUNED, eps=hp["eps"],
+                           ns_steps=hp["ns_steps"], adjust_lr_fn="match_rms_adamw")
+    p.grad = G.clone()
+    opt.step()
+    dW_t = (p.detach().double() - W.double()).numpy()
+    Wn, _, _, _ = oracle.muon_step(W.double().numpy(), G.double().numpy(), M.double().numpy(), **hp)
+    dW_o = Wn - W.double().numpy()
+    assert np.linalg.norm(dW_t - dW_o) / np.linalg.norm(dW_o) <= 3e-2
+
+
+# ----------------------------------------------------------------- QK-Clip
+def test_smax_matches_bruteforce_and_planted_scores():
+    rng = np.random.default_rng(13)
+    B, S, D, H, dh = 2, 6, 5, 3, 2
+    X = rng.standard_normal((B, S, D))
+    Wq = rng.standard_normal((H * dh, D))
+    Wk = rng.standard_normal((H * dh, D))
+    for causal in (True, False):
+        got = oracle.qk_max_logit(X, Wq, Wk, H, dh, causal=causal)
+        want = oracle.qk_max_logit_bruteforce(X, Wq, Wk, H, dh, causal=causal)
+        assert np.allclose(got, want, rtol=1e-13, atol=1e-13)
+    # Planted pair: a large score between query 1 and key 4 (j > i) must not
+    # count under the causal mask; the same pair on the diagonal must count.
+    X = np.zeros((1, 5, 2)); X[0, :, 1] = 0.01
+    Wq = np.array([[1.0, 0.0], [0.0, 1.0]]); Wk = Wq.copy()
+    X[0, 1, 0] = 10.0; X[0, 4, 0] = 10.0
+    smax = oracle.qk_max_logit(X, Wq, Wk, 1, 2, causal=True)
+    assert smax[0] == pytest.approx(oracle.qk_max_logit_bruteforce(X, Wq, Wk, 1, 2)[0])
+    # query 4 sees key 4 (diagonal) -> 100.0001/sqrt(2); also query 4 sees key 1.
+    assert smax[0] == pytest.approx((100.0 + 1e-4) / np.sqrt(2), rel=1e-12)
+    X[0, 4, 0] = 0.0; X[0, 0, 0] = 10.0; X[0, 1, 0] = 0.0
+    # now only query 0 / key 0 is large: the diagonal of row 0 counts.
+    assert oracle.qk_max_logit(X, Wq, Wk, 1, 2)[0] == pytest.approx((100 + 1e-4) / np.sqrt(2), rel=1e-12)
+    X[0, 0, 0] = 0.0; X[0, 0, 1] = 0.01; X[0, 3, 0] = 10.0; X[0, 2, 0] = -10.0
+    # scores: q3.k3 = 100 counts; q2.k3 (j > i) = -100 would not anyway; signed max.
+    assert oracle.qk_max_logit(X, Wq, Wk, 1, 2)[0] == pytest.approx((100 + 1e-4) / np.sqrt(2), rel=1e-12)
+
+
+def test_smax_is_signed_max_not_abs():
+    X = np.array([[[1.0], [1.0]]])
+    Wq = np.array([[-3.0]]); Wk = np.array([[2.0]])
+    assert oracle.qk_max_logit(X, Wq, Wk, 1, 1)[0] == pytest.approx(-6.0)
+
+
+def test_clip_worked_example():
+    g = GOLD["qk_clip_example"]
+    H, dh, D = 2, 3, 4
+    rng = np.random.default_rng(14)
+    Wq = rng.standard_normal((H * dh, D)); Wk = rng.standard_normal((H * dh, D))
+    smax = np.array([g["smax"], g["smax_no_clip"]])
+    Wq2, Wk2, gamma, mask = oracle.qk_clip(Wq, Wk, smax, g["tau"], g["alpha"], H, dh)
+    assert gamma[0] == pytest.approx(g["gamma"], abs=1e-15) and gamma[1] == 1.0
+    assert list(mask) == [1, 0]
+    assert np.allclose(Wq2[:dh], g["side_scale"] * Wq[:dh], rtol=1e-15, atol=0)
+    assert np.allclose(Wk2[:dh], g["side_scale"] * Wk[:dh], rtol=1e-15, atol=0)
+    assert np.array_equal(Wq2[dh:], Wq[dh:]) and np.array_equal(Wk2[dh:], Wk[dh:])
+
+
+def test_clip_threshold_edges_leave_weights_bitwise():
+    Wq = np.arange(12.0).reshape(4, 3); Wk = -Wq
+    for s in (100.0, 99.999, -500.0, 0.0):
+        q2, k2, gamma, mask = oracle.qk_clip(Wq, Wk, np.array([s, s]), 100.0, 0.5, 2, 2)
+        assert np.array_equal(q2, Wq) and np.array_equal(k2, Wk)
+        assert mask.sum() == 0 and np.all(gamma == 1.0)
+
+
+@pytest.mark.parametrize("alpha", [0.5, 0.3, 1.0])
+def test_recomputed_smax_after_clip_equals_tau(alpha):
+    rng = np.random.default_rng(15)
+    B, S, D, H, dh = 2, 12, 16, 3, 4
+    X = rng.standard_normal((B, S, D))
+    Wq = rng.standard_normal((H * dh, D)) * np.array([4.0] * dh + [0.1] * dh + [5.0] * dh)[:, None]
+    Wk = rng.standard_normal((H * dh, D)) * np.array([4.0] * dh + [0.1] * dh + [5.0] * dh)[:, None]
+    tau = 5.0
+    s0 = oracle.qk_max_logit(X, Wq, Wk, H, dh)
+    q2, k2, gamma, mask = oracle.qk_clip(Wq, Wk, s0, tau, alpha, H, dh)
+    s1 = oracle.qk_max_logit(X, q2, k2, H, dh)
+    for h in range(H):
+        if s0[h] > tau:
+            assert s1[h] == pytest.approx(tau, rel=1e-12)
+            assert s1[h] <= tau * (1 + 1e-6)
+        else:
+            assert s1[h] == s0[h]
+    assert mask.sum() >= 1
+
+
+def test_round_bf16_matches_torch_cast():
+    rng = np.random.default_rng(16)
+    x = rng.standard_normal(10000) * np.exp(rng.uniform(-20, 20, 10000))
+    want = torch.from_numpy(x.astype(np.float32)).to(torch.bfloat16).double().numpy()
+    assert np.array_equal(oracle.round_bf16(x), want)
