@@ -1,0 +1,189 @@
+/*
+ * muonclip.h -- C ABI of the B200 (sm_100a) MuonClip step library.
+ *
+ * Three operations, as the MuonClip training step composes them
+ * ("MuonClip: speed, then stability", §07 "One complete training step"):
+ *
+ *   mc_muon_step     the Muon update of a list of hidden 2D weights
+ *   mc_qk_max_logit  per-head causal max of the pre-softmax logit (S_max)
+ *   mc_qk_clip       QK-Clip: rescale the W_q / W_k rows of heads with S_max > tau
+ *
+ * Conventions for every call
+ *   - All pointers named "device" are CUDA device pointers on the current
+ *     device; they must be 16-byte aligned.  The library never frees or
+ *     retains caller memory beyond the call (the call is asynchronous, so the
+ *     buffers must stay valid until the stream reaches that point).
+ *   - `stream` is a cudaStream_t (NULL = legacy default stream).  Calls only
+ *     enqueue work; none synchronises the host.
+ *   - Matrices are row-major and contiguous.  A weight of shape rows x cols
+ *     uses the nn.Linear layout: rows = out-features.
+ *   - Return value: MC_OK (0) or a negative MC_ERR_* code.  On an argument
+ *     error nothing is enqueued and no memory is touched.  The text of the last
+ *     error of the calling thread is available from mc_last_error().
+ *   - Requires a compute capability 10.0 device (B200); otherwise
+ *     MC_ERR_UNSUPPORTED.
+ */
+#ifndef MUONCLIP_H_
+#define MUONCLIP_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+enum {
+  MC_OK = 0,
+  MC_ERR_INVAL = -1,       /* null pointer, bad shape, bad hyper-parameter */
+  MC_ERR_ALIGN = -2,       /* a pointer is not 16-byte aligned */
+  MC_ERR_NOSPC = -3,       /* workspace smaller than the *_workspace_size query */
+  MC_ERR_CUDA = -4,        /* a CUDA runtime call failed (message in mc_last_error) */
+  MC_ERR_UNSUPPORTED = -5, /* not a compute capability 10.0 device */
+  MC_ERR_DEVICE = -6       /* mc_device_status: a kernel gave up on a bounded wait */
+};
+
+enum { MC_F32 = 0, MC_BF16 = 1 };
+
+/* One hidden 2D weight, its gradient and its momentum buffer. */
+typedef struct {
+  void* w;            /* device, rows x cols, dtype w_dtype; updated in place      */
+  const void* g;      /* device, rows x cols, dtype g_dtype; read only              */
+  float* m;           /* device, rows x cols fp32 momentum; updated in place        */
+  int64_t rows;       /* >= 1 */
+  int64_t cols;       /* >= 1 */
+  int32_t w_dtype;    /* MC_F32 or MC_BF16 */
+  int32_t g_dtype;    /* MC_F32 or MC_BF16 */
+  float* update_out;  /* optional device fp32 rows x cols: receives the applied
+                         update 0.2*sqrt(max(rows,cols))*NS(.) (diagnostics);
+                         NULL = not written */
+} mc_param;
+
+/* Hyper-parameters of the Muon step. */
+typedef struct {
+  float mu;           /* momentum coefficient (0.95) */
+  int32_t nesterov;   /* 1: NS input U = G + mu*M_t; 0: U = M_t */
+  float lr;           /* learning rate eta */
+  float wd;           /* decoupled weight decay lambda */
+  int32_t ns_steps;   /* Newton-Schulz iterations, 1 <= ns_steps < 100 (5) */
+  float a, b, c;      /* quintic coefficients (3.4445, -4.7750, 2.0315) */
+  float eps;          /* normalisation floor: X0 = U / max(||U||_F, eps) (1e-7) */
+  float rms_scale;    /* update scale factor: rms_scale*sqrt(max(rows,cols)) (0.2) */
+} mc_hparams;
+
+/*
+ * mc_muon_step -- one Muon step on every matrix of `params`.
+ *
+ * Per matrix, following "MuonClip: speed, then stability" §02-§03 and
+ * "Muon and MuonClip: orthogonalised updates for LLM training" §2:
+ *   M <- mu*M + G
+ *   U <- G + mu*M  (nesterov) or M
+ *   X0 <- U / max(||U||_F, eps), with the short side first (U^T when rows > cols)
+ *   ns_steps times:  A = X X^T;  B = b*A + c*A*A;  X <- a*X + B*X
+ *   O <- X in the weight's orientation
+ *   W <- W - lr*(rms_scale*sqrt(max(rows,cols))*O + wd*W)
+ * The Newton-Schulz products run on tcgen05 tensor cores with bf16 operands
+ * and fp32 accumulation; the iterate is also carried in fp32 for the a*X term.
+ * Matrices of equal shape and weight dtype are batched into one problem group.
+ *
+ * params/n      host array of n >= 0 entries (n == 0 is a no-op).  W, G, M of
+ *               one entry must not alias; G is left unchanged.
+ * hp            host pointer.
+ * workspace     device scratch of at least mc_muon_workspace_size(...) bytes,
+ *               or NULL to let the library allocate (and keep) its own.
+ *               Must not be used by anything else until the step completes.
+ * norms_out     optional device fp32 [n]: ||U||_F of each matrix (NULL = skip).
+ * Errors        MC_ERR_INVAL, MC_ERR_ALIGN, MC_ERR_NOSPC, MC_ERR_CUDA,
+ *               MC_ERR_UNSUPPORTED.
+ */
+size_t mc_muon_workspace_size(const mc_param* params, int n, const mc_hparams* hp);
+int mc_muon_step(const mc_param* params, int n, const mc_hparams* hp, void* workspace,
+                 size_t workspace_bytes, float* norms_out, void* stream);
+
+/*
+ * mc_qk_max_logit -- S_max[h] = max over b, i and j (j <= i when causal) of
+ * (q_{b,i,h} . k_{b,j,h}) / sqrt(dh), with Q = X W_q^T and K = X W_k^T.
+ * Definition: "Muon and MuonClip: orthogonalised updates for LLM training",
+ * "The exploding-logit problem"; "MuonClip: speed, then stability" §05.
+ * Q and K are formed on tensor cores (bf16 in, fp32 accumulate) and stored as
+ * bf16 in the workspace; the S x S score matrix is never stored.
+ *
+ * x             device bf16 [B][S][D]
+ * wq, wk        device bf16 [H*dh][D]; head h owns rows [h*dh, (h+1)*dh)
+ * causal        1: causal mask j <= i (diagonal included); 0: all pairs
+ * smax_out      device fp32 [H]
+ * workspace     device scratch of at least mc_qk_workspace_size(...) bytes, or NULL.
+ * Constraints   B, S, D, H, dh >= 1; D and dh multiples of 8.
+ */
+size_t mc_qk_workspace_size(int B, int S, int D, int H, int dh);
+int mc_qk_max_logit(const void* x, const void* wq, const void* wk, int B, int S, int D, int H, int dh,
+                    int causal, float* smax_out, void* workspace, size_t workspace_bytes, void* stream);
+
+/*
+ * mc_qk_clip -- QK-Clip for multi-head attention ("MuonClip: speed, then
+ * stability" §05; "About Muon: Muon At Scale", "When Softmax Collapses"):
+ *   gamma_h = tau / S_max[h] if S_max[h] > tau, else 1
+ *   rows [h*dh, (h+1)*dh) of W_q  *= gamma_h^alpha
+ *   rows [h*dh, (h+1)*dh) of W_k  *= gamma_h^(1-alpha)
+ * computed on the device from `smax` (no host round trip); rows of heads that
+ * are not clipped are left bit-for-bit unchanged.  The momentum buffers are
+ * never touched (§07).
+ *
+ * wq, wk        device bf16 [H*dh][D], updated in place
+ * smax          device fp32 [H] (e.g. from mc_qk_max_logit)
+ * gamma_out     optional device fp32 [H] (NULL = skip)
+ * mask_out      optional device int32 [H]: 1 where clipped (NULL = skip)
+ */
+int mc_qk_clip(void* wq, void* wk, int H, int dh, int D, const float* smax, float tau, float alpha,
+               float* gamma_out, int32_t* mask_out, void* stream);
+
+/* Text of the last error returned on the calling thread ("" if none). */
+const char* mc_last_error(void);
+
+/*
+ * mc_device_status -- synchronises the current device, then reads and clears
+ * the library's device error word.  Returns MC_OK, MC_ERR_DEVICE when a kernel
+ * abandoned a bounded wait (its outputs are then invalid), or MC_ERR_CUDA.
+ */
+int mc_device_status(void);
+
+/*
+ * Measurement support.  Between mc_profile_begin() and mc_profile_end(), every
+ * kernel this thread's calls enqueue is bracketed by two CUDA events recorded
+ * on the launch stream, and its algorithmic work is computed from the shapes.
+ * mc_profile_end() waits for those events and reports one row per kernel kind:
+ *
+ *   momentum        bytes = the momentum kernel's DRAM traffic by design:
+ *                   G (2 or 4) + M read/write (8) + fp32 and bf16 iterate (6)
+ *                   bytes per element
+ *   ns_gram, ns_poly, ns_apply, ns_apply_final
+ *                   flops = dense-equivalent Newton-Schulz FLOPs of that phase,
+ *                   2 m^2 n, 2 m^3, 2 m^2 n (their sum per iteration is the
+ *                   2(2nm^2 + m^3) of "Muon and MuonClip: orthogonalised updates
+ *                   for LLM training", §2); flops_executed = 2*128*256*K_padded
+ *                   per tile the tensor cores actually ran (symmetric phases
+ *                   skip about half of the tiles)
+ *   qk_proj         flops = 2 * B*S * H*dh * D * 2 (Q and K)
+ *   qk_causal_max   flops = 2 * dh * (score pairs inside the causal mask)
+ *   norm_finalize, qk_keys, qk_clip   (small kernels; counted, no work figure)
+ *
+ * The rows are written to `out` (up to `max_rows`), `*rows` receives the count.
+ * Recording events adds no synchronisation; the durations are device time.
+ */
+typedef struct {
+  char name[32];
+  int32_t launches;
+  double total_ms;
+  double flops;
+  double flops_executed;
+  double bytes;
+} mc_kernel_stat;
+
+int mc_profile_begin(void);
+int mc_profile_end(mc_kernel_stat* out, int max_rows, int* rows);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* MUONCLIP_H_ */

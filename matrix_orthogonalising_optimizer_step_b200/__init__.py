@@ -1,0 +1,279 @@
+"""B200-native MuonClip step: Python binding over the C ABI in include/muonclip.h.
+
+The binding only marshals arguments: every step of the Muon update and of
+QK-Clip runs in the sm_100a kernels of ``libmuonclip.so``.  PyTorch supplies
+device memory and the current stream.  There is no fallback: if the library is
+missing or the device is not a B200 the calls raise.
+
+    from matrix_orthogonalising_optimizer_step_b200 import muon_step, qk_max_logit, qk_clip
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from typing import Optional, Sequence
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "libmuonclip.so")
+
+MC_OK, MC_ERR_INVAL, MC_ERR_ALIGN, MC_ERR_NOSPC, MC_ERR_CUDA, MC_ERR_UNSUPPORTED, MC_ERR_DEVICE = (
+    0, -1, -2, -3, -4, -5, -6)
+MC_F32, MC_BF16 = 0, 1
+
+# Names the C ABI exports (include/muonclip.h).
+EXPORTS = ("mc_muon_workspace_size", "mc_muon_step", "mc_qk_workspace_size", "mc_qk_max_logit",
+           "mc_qk_clip", "mc_last_error", "mc_device_status", "mc_profile_begin", "mc_profile_end")
+
+
+class McParam(ctypes.Structure):
+    _fields_ = [("w", ctypes.c_void_p), ("g", ctypes.c_void_p), ("m", ctypes.c_void_p),
+                ("rows", ctypes.c_int64), ("cols", ctypes.c_int64),
+                ("w_dtype", ctypes.c_int32), ("g_dtype", ctypes.c_int32),
+                ("update_out", ctypes.c_void_p)]
+
+
+class McHparams(ctypes.Structure):
+    _fields_ = [("mu", ctypes.c_float), ("nesterov", ctypes.c_int32), ("lr", ctypes.c_float),
+                ("wd", ctypes.c_float), ("ns_steps", ctypes.c_int32), ("a", ctypes.c_float),
+                ("b", ctypes.c_float), ("c", ctypes.c_float), ("eps", ctypes.c_float),
+                ("rms_scale", ctypes.c_float)]
+
+
+class McKernelStat(ctypes.Structure):
+    _fields_ = [("name", ctypes.c_char * 32), ("launches", ctypes.c_int32), ("total_ms", ctypes.c_double),
+                ("flops", ctypes.c_double), ("flops_executed", ctypes.c_double), ("bytes", ctypes.c_double)]
+
+
+class MuonClipError(RuntimeError):
+    def __init__(self, code: int, msg: str):
+        super().__init__(f"[{code}] {msg}")
+        self.code = code
+
+
+_lib = None
+
+
+def load_library():
+    """Load libmuonclip.so (raises if it has not been built)."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(LIB_PATH):
+        raise RuntimeError(f"{LIB_PATH} is missing: build it with "
+                           "`python -m matrix_orthogonalising_optimizer_step_b200.build`")
+    lib = ctypes.CDLL(LIB_PATH)
+    P = ctypes.POINTER
+    vp, i32, sz = ctypes.c_void_p, ctypes.c_int, ctypes.c_size_t
+    lib.mc_muon_workspace_size.argtypes = [P(McParam), i32, P(McHparams)]
+    lib.mc_muon_workspace_size.restype = sz
+    lib.mc_muon_step.argtypes = [P(McParam), i32, P(McHparams), vp, sz, vp, vp]
+    lib.mc_muon_step.restype = i32
+    lib.mc_qk_workspace_size.argtypes = [i32] * 5
+    lib.mc_qk_workspace_size.restype = sz
+    lib.mc_qk_max_logit.argtypes = [vp, vp, vp, i32, i32, i32, i32, i32, i32, vp, vp, sz, vp]
+    lib.mc_qk_max_logit.restype = i32
+    lib.mc_qk_clip.argtypes = [vp, vp, i32, i32, i32, vp, ctypes.c_float, ctypes.c_float, vp, vp, vp]
+    lib.mc_qk_clip.restype = i32
+    lib.mc_last_error.argtypes = []
+    lib.mc_last_error.restype = ctypes.c_char_p
+    lib.mc_device_status.argtypes = []
+    lib.mc_device_status.restype = i32
+    lib.mc_profile_begin.argtypes = []
+    lib.mc_profile_begin.restype = i32
+    lib.mc_profile_end.argtypes = [P(McKernelStat), i32, P(ctypes.c_int)]
+    lib.mc_profile_end.restype = i32
+    _lib = lib
+    return lib
+
+
+def _check(rc: int):
+    if rc != MC_OK:
+        raise MuonClipError(rc, load_library().mc_last_error().decode())
+
+
+def last_error() -> str:
+    return load_library().mc_last_error().decode()
+
+
+def device_status() -> int:
+    """Synchronise the current device and return (and clear) the library's
+    device error word: MC_OK or MC_ERR_DEVICE."""
+    return load_library().mc_device_status()
+
+
+def profile_begin() -> None:
+    """Start bracketing every kernel this thread's calls launch with CUDA events."""
+    _check(load_library().mc_profile_begin())
+
+
+def profile_end() -> dict:
+    """Stop profiling; returns {kernel kind: {launches, total_ms, flops,
+    flops_executed, bytes}} of device time and algorithmic work."""
+    lib = load_library()
+    rows = (McKernelStat * 32)()
+    n = ctypes.c_int(0)
+    _check(lib.mc_profile_end(rows, 32, ctypes.byref(n)))
+    out = {}
+    for i in range(min(n.value, 32)):
+        r = rows[i]
+        out[r.name.decode()] = dict(launches=int(r.launches), total_ms=float(r.total_ms), flops=float(r.flops),
+                                    flops_executed=float(r.flops_executed), bytes=float(r.bytes))
+    return out
+
+
+# ----------------------------------------------------------------- helpers
+def _torch():
+    import torch
+    return torch
+
+
+def _stream_handle(stream) -> int:
+    torch = _torch()
+    s = stream if stream is not None else torch.cuda.current_stream()
+    return int(s.cuda_stream)
+
+
+def _dtype_code(t) -> int:
+    torch = _torch()
+    if t.dtype == torch.float32:
+        return MC_F32
+    if t.dtype == torch.bfloat16:
+        return MC_BF16
+    raise TypeError(f"unsupported dtype {t.dtype} (float32 or bfloat16)")
+
+
+def _ptr(t) -> Optional[int]:
+    return None if t is None else int(t.data_ptr())
+
+
+def _need_cuda_contig(t, name):
+    if not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+
+
+def make_hparams(mu=0.95, nesterov=True, lr=0.02, wd=0.1, ns_steps=5, a=3.4445, b=-4.7750,
+                 c=2.0315, eps=1e-7, rms_scale=0.2) -> McHparams:
+    return McHparams(float(mu), int(bool(nesterov)), float(lr), float(wd), int(ns_steps),
+                     float(a), float(b), float(c), float(eps), float(rms_scale))
+
+
+def make_params(weights, grads, moms, update_outs=None):
+    n = len(weights)
+    if not (len(grads) == n and len(moms) == n):
+        raise ValueError("weights, grads and moms must have the same length")
+    arr = (McParam * max(n, 1))()
+    for i in range(n):
+        W, G, M = weights[i], grads[i], moms[i]
+        for t, nm in ((W, "weight"), (G, "grad"), (M, "momentum")):
+            _need_cuda_contig(t, f"{nm}[{i}]")
+            if t.dim() != 2:
+                raise ValueError(f"{nm}[{i}] must be 2D")
+        if G.shape != W.shape or M.shape != W.shape:
+            raise ValueError(f"shape mismatch at index {i}")
+        if M.dtype != _torch().float32:
+            raise TypeError(f"momentum[{i}] must be float32")
+        U = update_outs[i] if update_outs is not None else None
+        if U is not None:
+            _need_cuda_contig(U, f"update_out[{i}]")
+            if U.shape != W.shape or U.dtype != _torch().float32:
+                raise ValueError(f"update_out[{i}] must be float32 of the weight's shape")
+        arr[i] = McParam(_ptr(W), _ptr(G), _ptr(M), int(W.shape[0]), int(W.shape[1]),
+                         _dtype_code(W), _dtype_code(G), _ptr(U))
+    return arr, n
+
+
+_workspaces = {}
+
+
+def _workspace(tag, device, nbytes):
+    """Device scratch owned by PyTorch's allocator, cached per (tag, device)."""
+    torch = _torch()
+    key = (tag, device)
+    ws = _workspaces.get(key)
+    if ws is None or ws.numel() < nbytes:
+        _workspaces.pop(key, None)
+        ws = torch.empty(max(int(nbytes), 1024), dtype=torch.uint8, device=device)
+        _workspaces[key] = ws
+    return ws
+
+
+def release_workspaces():
+    _workspaces.clear()
+
+
+# ----------------------------------------------------------------- the API
+def muon_workspace_size(weights, grads, moms, hparams: Optional[McHparams] = None, **hp) -> int:
+    lib = load_library()
+    arr, n = make_params(weights, grads, moms)
+    h = hparams if hparams is not None else make_hparams(**hp)
+    return int(lib.mc_muon_workspace_size(arr, n, ctypes.byref(h)))
+
+
+def muon_step(weights: Sequence, grads: Sequence, moms: Sequence, *, norms_out=None,
+              update_outs=None, workspace=None, stream=None, hparams: Optional[McHparams] = None,
+              **hp) -> None:
+    """One Muon step on every (W, G, M) triple, in place on W and M (see
+    mc_muon_step in include/muonclip.h).  Keyword hyper-parameters: mu,
+    nesterov, lr, wd, ns_steps, a, b, c, eps, rms_scale."""
+    lib = load_library()
+    arr, n = make_params(weights, grads, moms, update_outs)
+    h = hparams if hparams is not None else make_hparams(**hp)
+    if n == 0:
+        return
+    if norms_out is not None:
+        _need_cuda_contig(norms_out, "norms_out")
+    need = int(lib.mc_muon_workspace_size(arr, n, ctypes.byref(h)))
+    if need == 0:
+        _check(lib.mc_muon_step(arr, n, ctypes.byref(h), None, 0, None, None))
+    ws = workspace if workspace is not None else _workspace("muon", weights[0].device, need)
+    _check(lib.mc_muon_step(arr, n, ctypes.byref(h), _ptr(ws), int(ws.numel() * ws.element_size()),
+                            _ptr(norms_out), _stream_handle(stream)))
+
+
+def qk_workspace_size(B, S, D, H, dh) -> int:
+    return int(load_library().mc_qk_workspace_size(B, S, D, H, dh))
+
+
+def qk_max_logit(x, wq, wk, H: int, dh: int, *, causal: bool = True, smax_out=None,
+                 workspace=None, stream=None):
+    """Per-head S_max (fp32 [H]) of causal attention with Q = x Wq^T, K = x Wk^T."""
+    torch = _torch()
+    lib = load_library()
+    for t, nm in ((x, "x"), (wq, "wq"), (wk, "wk")):
+        _need_cuda_contig(t, nm)
+        if t.dtype != torch.bfloat16:
+            raise TypeError(f"{nm} must be bfloat16")
+    B, S, D = x.shape
+    if smax_out is None:
+        smax_out = torch.empty(H, dtype=torch.float32, device=x.device)
+    need = int(lib.mc_qk_workspace_size(B, S, D, H, dh))
+    if need == 0:
+        _check(lib.mc_qk_max_logit(None, None, None, B, S, D, H, dh, int(causal), None, None, 0, None))
+    ws = workspace if workspace is not None else _workspace("qk", x.device, need)
+    _check(lib.mc_qk_max_logit(_ptr(x), _ptr(wq), _ptr(wk), B, S, D, H, dh, int(causal),
+                               _ptr(smax_out), _ptr(ws), int(ws.numel() * ws.element_size()),
+                               _stream_handle(stream)))
+    return smax_out
+
+
+def qk_clip(wq, wk, smax, H: int, dh: int, *, tau: float = 100.0, alpha: float = 0.5,
+            gamma_out=None, mask_out=None, stream=None):
+    """QK-Clip in place on Wq/Wk rows of heads with S_max > tau.  Returns
+    (gamma [H] fp32, mask [H] int32)."""
+    torch = _torch()
+    lib = load_library()
+    for t, nm in ((wq, "wq"), (wk, "wk")):
+        _need_cuda_contig(t, nm)
+        if t.dtype != torch.bfloat16:
+            raise TypeError(f"{nm} must be bfloat16")
+    _need_cuda_contig(smax, "smax")
+    D = int(wq.shape[1])
+    if gamma_out is None:
+        gamma_out = torch.empty(H, dtype=torch.float32, device=wq.device)
+    if mask_out is None:
+        mask_out = torch.empty(H, dtype=torch.int32, device=wq.device)
+    _check(lib.mc_qk_clip(_ptr(wq), _ptr(wk), H, dh, D, _ptr(smax), float(tau), float(alpha),
+                          _ptr(gamma_out), _ptr(mask_out), _stream_handle(stream)))
+    return gamma_out, mask_out

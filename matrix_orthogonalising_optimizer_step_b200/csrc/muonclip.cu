@@ -1,0 +1,783 @@
+// Host engine and C ABI of the MuonClip step library (see include/muonclip.h).
+//
+// mc_muon_step enqueues, on the caller's stream:
+//   1. momentum_kernel       one launch over every matrix (momentum, Nesterov,
+//                            fp32 + bf16 iterate, ||U||^2 partials)
+//   2. norm_finalize_kernel  s = 1 / max(||U||_F, eps) per matrix
+//   3. ns_steps x { GRAM, POLY, APPLY } grouped tcgen05 GEMM launches; the last
+//      APPLY writes W directly (decay + scaled update), so the final iterate
+//      never goes to memory.
+// Matrices with equal (rows, cols, weight dtype) form one problem group; their
+// iterates sit back to back in the workspace so that one 3-D TMA descriptor
+// covers the whole group.  Tall matrices (rows > cols) are never transposed in
+// memory: the Gram product reads them MN-major and the apply multiplies from
+// the right (X B instead of B X), which is the oriented iteration transposed.
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <algorithm>
+#include <cmath>
+#include <cstring>
+#include <map>
+#include <mutex>
+#include <string>
+#include <vector>
+
+#include "muonclip.h"
+#include "ptx.cuh"
+#include "stream_kernels.cuh"
+#include "umma_gemm.cuh"
+
+#define MC_API extern "C" __attribute__((visibility("default")))
+
+namespace mc {
+__device__ int g_device_error = 0;
+}
+
+namespace {
+
+using namespace mc;
+
+thread_local std::string t_last_error;
+
+int fail(int code, const std::string& msg) {
+  t_last_error = msg;
+  return code;
+}
+
+#define MC_CUDA(expr)                                                                      \
+  do {                                                                                     \
+    cudaError_t e_ = (expr);                                                               \
+    if (e_ != cudaSuccess) return fail(MC_ERR_CUDA, std::string(#expr) + ": " + cudaGetErrorString(e_)); \
+  } while (0)
+
+using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                   const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                   CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+constexpr int kRing = 4;
+
+struct DeviceState {
+  bool init = false;
+  int sms = 0;
+  int cc_major = 0, cc_minor = 0;
+  int* err_ptr = nullptr;
+  void* own_ws = nullptr;
+  size_t own_ws_bytes = 0;
+  void* pinned[kRing] = {};
+  size_t pinned_bytes[kRing] = {};
+  cudaEvent_t ev[kRing] = {};
+  int next = 0;
+};
+
+std::mutex g_mu;
+std::map<int, DeviceState> g_devices;
+EncodeTiledFn g_encode = nullptr;
+
+inline size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+inline int64_t round8(int64_t x) { return (x + 7) / 8 * 8; }
+inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+template <int EPI>
+cudaError_t set_gemm_attr() {
+  return cudaFuncSetAttribute(umma_gemm_kernel<EPI>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                              static_cast<int>(GEMM_SMEM_BYTES));
+}
+
+// Caller holds g_mu.
+int device_state(DeviceState** out) {
+  int dev = 0;
+  MC_CUDA(cudaGetDevice(&dev));
+  DeviceState& st = g_devices[dev];
+  if (!st.init) {
+    MC_CUDA(cudaDeviceGetAttribute(&st.sms, cudaDevAttrMultiProcessorCount, dev));
+    MC_CUDA(cudaDeviceGetAttribute(&st.cc_major, cudaDevAttrComputeCapabilityMajor, dev));
+    MC_CUDA(cudaDeviceGetAttribute(&st.cc_minor, cudaDevAttrComputeCapabilityMinor, dev));
+    if (st.cc_major != 10 || st.cc_minor != 0)
+      return fail(MC_ERR_UNSUPPORTED, "device " + std::to_string(dev) + " has compute capability " +
+                                          std::to_string(st.cc_major) + "." + std::to_string(st.cc_minor) +
+                                          "; this library is built for sm_100a (B200)");
+    MC_CUDA(cudaGetSymbolAddress(reinterpret_cast<void**>(&st.err_ptr), g_device_error));
+    MC_CUDA(set_gemm_attr<EPI_GRAM>());
+    MC_CUDA(set_gemm_attr<EPI_POLY>());
+    MC_CUDA(set_gemm_attr<EPI_APPLY>());
+    MC_CUDA(set_gemm_attr<EPI_APPLY_FINAL>());
+    MC_CUDA(set_gemm_attr<EPI_STORE>());
+    MC_CUDA(set_gemm_attr<EPI_CAUSALMAX>());
+    if (!g_encode) {
+      void* fn = nullptr;
+      cudaDriverEntryPointQueryResult q;
+      MC_CUDA(cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q));
+      if (q != cudaDriverEntryPointSuccess || !fn)
+        return fail(MC_ERR_CUDA, "cuTensorMapEncodeTiled is not available from the driver");
+      g_encode = reinterpret_cast<EncodeTiledFn>(fn);
+    }
+    st.init = true;
+  }
+  *out = &st;
+  return MC_OK;
+}
+
+// Copy a small host table into device memory through a pinned staging ring
+// (so the copy is asynchronous and the host buffer can be reused at once).
+int upload(DeviceState& st, const void* host, size_t bytes, void* dst, cudaStream_t s) {
+  if (bytes == 0) return MC_OK;
+  const int i = st.next;
+  st.next = (st.next + 1) % kRing;
+  if (st.ev[i]) {
+    MC_CUDA(cudaEventSynchronize(st.ev[i]));
+  } else {
+    MC_CUDA(cudaEventCreateWithFlags(&st.ev[i], cudaEventDisableTiming));
+  }
+  if (st.pinned_bytes[i] < bytes) {
+    if (st.pinned[i]) MC_CUDA(cudaFreeHost(st.pinned[i]));
+    st.pinned[i] = nullptr;
+    st.pinned_bytes[i] = 0;
+    MC_CUDA(cudaMallocHost(&st.pinned[i], bytes));
+    st.pinned_bytes[i] = bytes;
+  }
+  std::memcpy(st.pinned[i], host, bytes);
+  MC_CUDA(cudaMemcpyAsync(dst, st.pinned[i], bytes, cudaMemcpyHostToDevice, s));
+  MC_CUDA(cudaEventRecord(st.ev[i], s));
+  return MC_OK;
+}
+
+int own_workspace(DeviceState& st, size_t bytes, void** ws) {
+  if (st.own_ws_bytes < bytes) {
+    if (st.own_ws) {
+      MC_CUDA(cudaDeviceSynchronize());
+      MC_CUDA(cudaFree(st.own_ws));
+      st.own_ws = nullptr;
+      st.own_ws_bytes = 0;
+    }
+    MC_CUDA(cudaMalloc(&st.own_ws, bytes));
+    st.own_ws_bytes = bytes;
+  }
+  *ws = st.own_ws;
+  return MC_OK;
+}
+
+// bf16 tensor map, 128-byte swizzle, zero fill out of bounds.
+int make_map(CUtensorMap* map, const void* base, int rank, const uint64_t* dims, const uint64_t* strides,
+             const uint32_t* box) {
+  cuuint64_t gd[5], gs[4];
+  cuuint32_t bx[5], es[5];
+  for (int i = 0; i < rank; ++i) {
+    gd[i] = dims[i];
+    bx[i] = box[i];
+    es[i] = 1;
+  }
+  for (int i = 0; i + 1 < rank; ++i) gs[i] = strides[i];
+  const CUresult r = g_encode(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, rank, const_cast<void*>(base), gd, gs, bx, es,
+                              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                              CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return fail(MC_ERR_CUDA, "cuTensorMapEncodeTiled failed with code " + std::to_string(r));
+  return MC_OK;
+}
+
+// [count][rows][ld] bf16, box {64, box_rows, 1}
+int map_batched(CUtensorMap* map, const void* base, int64_t count, int64_t rows, int64_t cols, int64_t ld,
+                uint32_t box_rows) {
+  const uint64_t dims[3] = {uint64_t(cols), uint64_t(rows), uint64_t(count)};
+  const uint64_t strides[2] = {uint64_t(ld) * 2, uint64_t(rows) * uint64_t(ld) * 2};
+  const uint32_t box[3] = {64, box_rows, 1};
+  return make_map(map, base, 3, dims, strides, box);
+}
+
+// ----------------------------------------------------------- profiling
+enum Kind : int { K_MOMENTUM, K_FINALIZE, K_GRAM, K_POLY, K_APPLY, K_APPLY_FINAL, K_QK_PROJ, K_QK_CMAX,
+                  K_QK_KEYS, K_QK_CLIP, K_COUNT };
+const char* const kKindNames[K_COUNT] = {"momentum", "norm_finalize", "ns_gram", "ns_poly", "ns_apply",
+                                         "ns_apply_final", "qk_proj", "qk_causal_max", "qk_keys", "qk_clip"};
+struct ProfRec {
+  int kind;
+  cudaEvent_t b, e;
+  double flops, flops_exec, bytes;
+};
+thread_local bool t_prof = false;
+thread_local std::vector<ProfRec> t_recs;
+
+// Brackets one launch with CUDA events on its stream while profiling is on.
+struct ProfScope {
+  bool on = false;
+  ProfRec r{};
+  cudaStream_t s;
+  ProfScope(int kind, cudaStream_t st, double flops = 0, double flops_exec = 0, double bytes = 0) : s(st) {
+    if (!t_prof) return;
+    r.kind = kind;
+    r.flops = flops;
+    r.flops_exec = flops_exec;
+    r.bytes = bytes;
+    if (cudaEventCreate(&r.b) != cudaSuccess) return;
+    if (cudaEventCreate(&r.e) != cudaSuccess) {
+      cudaEventDestroy(r.b);
+      return;
+    }
+    on = cudaEventRecord(r.b, s) == cudaSuccess;
+  }
+  ~ProfScope() {
+    if (!on) return;
+    cudaEventRecord(r.e, s);
+    t_recs.push_back(r);
+  }
+};
+
+double gemm_exec_flops(const GemmParams& p) {
+  double f = 0;
+  for (int i = 0; i < p.num_groups; ++i) {
+    const GemmGroup& G = p.g[i];
+    const double kpad = double((G.K + BK - 1) / BK) * BK;
+    f += double(G.tiles_per_prob) * G.count * 2.0 * BM * BN * kpad;
+  }
+  return f;
+}
+
+template <int EPI>
+int launch_gemm(const GemmParams& p, int sms, cudaStream_t s, int kind, double flops) {
+  if (p.total_tiles <= 0) return MC_OK;
+  const long long grid = std::min<long long>(sms, p.total_tiles);
+  ProfScope prof(kind, s, flops, gemm_exec_flops(p));
+  umma_gemm_kernel<EPI><<<static_cast<unsigned>(grid), GEMM_THREADS, GEMM_SMEM_BYTES, s>>>(p);
+  MC_CUDA(cudaGetLastError());
+  return MC_OK;
+}
+
+void finish_group(GemmParams& p, int gi, GemmGroup& G) {
+  G.tiles_m = (G.M + BM - 1) / BM;
+  G.tiles_n = (G.N + BN - 1) / BN;
+  G.tiles_per_prob = sched_tiles_per_prob(G.sched, G.tiles_m, G.tiles_n);
+  G.tile_start = p.total_tiles;
+  if (G.band <= 0) G.band = 8;
+  p.total_tiles += G.tiles_per_prob * G.count;
+  p.g[gi] = G;
+  p.num_groups = gi + 1;
+}
+
+// ------------------------------------------------------------------ muon plan
+struct NsGroup {
+  int64_t rows = 0, cols = 0;
+  int w_f32 = 0;
+  bool tall = false;
+  int64_t m = 0, n = 0;   // min, max
+  int64_t ld = 0;         // row stride of the iterate
+  int64_t ldm = 0;        // row stride of A and B
+  std::vector<int> members;
+  int prob_base = 0;
+  size_t off_xb[2] = {0, 0}, off_xf = 0, off_a = 0, off_b = 0, off_wptr = 0, off_uptr = 0;
+};
+
+struct MuonLayout {
+  std::vector<NsGroup> groups;
+  std::vector<int> order;   // workspace order -> caller index
+  std::vector<long long> cta_begin;
+  long long total_ctas = 0;
+  size_t off_tab = 0, tab_bytes = 0, off_partials = 0, off_scale = 0, total = 0;
+};
+
+int validate_muon(const mc_param* params, int n, const mc_hparams* hp) {
+  if (n < 0) return fail(MC_ERR_INVAL, "n must be >= 0");
+  if (n > 0 && !params) return fail(MC_ERR_INVAL, "params is NULL");
+  if (!hp) return fail(MC_ERR_INVAL, "hp is NULL");
+  if (hp->ns_steps < 1 || hp->ns_steps >= 100) return fail(MC_ERR_INVAL, "ns_steps must be in [1, 100)");
+  const float vals[] = {hp->mu, hp->lr, hp->wd, hp->a, hp->b, hp->c, hp->eps, hp->rms_scale};
+  for (float v : vals)
+    if (!std::isfinite(v)) return fail(MC_ERR_INVAL, "non-finite hyper-parameter");
+  if (!(hp->eps > 0.f)) return fail(MC_ERR_INVAL, "eps must be > 0");
+  for (int i = 0; i < n; ++i) {
+    const mc_param& q = params[i];
+    const std::string at = "params[" + std::to_string(i) + "]: ";
+    if (!q.w || !q.g || !q.m) return fail(MC_ERR_INVAL, at + "NULL w, g or m");
+    if (q.rows < 1 || q.cols < 1) return fail(MC_ERR_INVAL, at + "rows and cols must be >= 1");
+    if (q.rows > (1 << 24) || q.cols > (1 << 24) || q.rows * q.cols > (int64_t(1) << 36))
+      return fail(MC_ERR_INVAL, at + "matrix too large");
+    if ((q.w_dtype != MC_F32 && q.w_dtype != MC_BF16) || (q.g_dtype != MC_F32 && q.g_dtype != MC_BF16))
+      return fail(MC_ERR_INVAL, at + "dtype must be MC_F32 or MC_BF16");
+    if (q.w == static_cast<const void*>(q.g) || q.w == static_cast<void*>(q.m) ||
+        q.g == static_cast<const void*>(q.m))
+      return fail(MC_ERR_INVAL, at + "w, g and m must not alias");
+    if (!aligned16(q.w) || !aligned16(q.g) || !aligned16(q.m) || (q.update_out && !aligned16(q.update_out)))
+      return fail(MC_ERR_ALIGN, at + "pointers must be 16-byte aligned");
+  }
+  return MC_OK;
+}
+
+void plan_muon(const mc_param* params, int n, MuonLayout& L) {
+  std::map<std::tuple<int64_t, int64_t, int>, int> index;
+  for (int i = 0; i < n; ++i) {
+    const auto key = std::make_tuple(params[i].rows, params[i].cols, params[i].w_dtype == MC_F32 ? 1 : 0);
+    auto it = index.find(key);
+    if (it == index.end()) {
+      NsGroup g;
+      g.rows = params[i].rows;
+      g.cols = params[i].cols;
+      g.w_f32 = params[i].w_dtype == MC_F32;
+      g.tall = g.rows > g.cols;
+      g.m = std::min(g.rows, g.cols);
+      g.n = std::max(g.rows, g.cols);
+      g.ld = round8(g.cols);
+      g.ldm = round8(g.m);
+      index[key] = static_cast<int>(L.groups.size());
+      L.groups.push_back(g);
+      it = index.find(key);
+    }
+    L.groups[it->second].members.push_back(i);
+  }
+  size_t off = 0;
+  int pb = 0;
+  for (auto& g : L.groups) {
+    g.prob_base = pb;
+    pb += static_cast<int>(g.members.size());
+    for (int i : g.members) L.order.push_back(i);
+  }
+  // Momentum kernel CTA split, in workspace order.
+  L.cta_begin.resize(n);
+  long long ctas = 0;
+  for (int k = 0; k < n; ++k) {
+    const mc_param& q = params[L.order[k]];
+    L.cta_begin[k] = ctas;
+    ctas += (q.rows * q.cols + MOM_ELEMS_PER_CTA - 1) / MOM_ELEMS_PER_CTA;
+  }
+  L.total_ctas = ctas;
+  // Tables: MomEntry[n], then per group w_ptrs[count] and u_ptrs[count].
+  L.off_tab = 0;
+  off = align_up(sizeof(MomEntry) * n, 256);
+  for (auto& g : L.groups) {
+    g.off_wptr = off;
+    off += sizeof(void*) * g.members.size();
+    g.off_uptr = off;
+    off += sizeof(void*) * g.members.size();
+  }
+  L.tab_bytes = off;
+  off = align_up(off, 1024);
+  L.off_partials = off;
+  off = align_up(off + sizeof(double) * ctas, 1024);
+  L.off_scale = off;
+  off = align_up(off + sizeof(float) * n, 1024);
+  for (auto& g : L.groups) {
+    const size_t cnt = g.members.size();
+    const size_t xe = cnt * size_t(g.rows) * size_t(g.ld);
+    const size_t ae = cnt * size_t(g.m) * size_t(g.ldm);
+    g.off_xb[0] = off; off = align_up(off + 2 * xe, 1024);
+    g.off_xb[1] = off; off = align_up(off + 2 * xe, 1024);
+    g.off_xf = off;    off = align_up(off + 4 * xe, 1024);
+    g.off_a = off;     off = align_up(off + 2 * ae, 1024);
+    g.off_b = off;     off = align_up(off + 2 * ae, 1024);
+  }
+  L.total = std::max<size_t>(off, 1024);
+}
+
+struct GroupMaps {
+  CUtensorMap x_k128[2], x_k256[2], x_mn[2], a_k128, a_k256, b_k128, b_k256;
+};
+
+int build_group_maps(const NsGroup& g, uint8_t* ws, GroupMaps& M) {
+  const int64_t cnt = static_cast<int64_t>(g.members.size());
+  for (int par = 0; par < 2; ++par) {
+    const void* xb = ws + g.off_xb[par];
+    int rc;
+    if ((rc = map_batched(&M.x_k128[par], xb, cnt, g.rows, g.cols, g.ld, 128)) != MC_OK) return rc;
+    if ((rc = map_batched(&M.x_k256[par], xb, cnt, g.rows, g.cols, g.ld, 256)) != MC_OK) return rc;
+    if ((rc = map_batched(&M.x_mn[par], xb, cnt, g.rows, g.cols, g.ld, 64)) != MC_OK) return rc;
+  }
+  int rc;
+  if ((rc = map_batched(&M.a_k128, ws + g.off_a, cnt, g.m, g.m, g.ldm, 128)) != MC_OK) return rc;
+  if ((rc = map_batched(&M.a_k256, ws + g.off_a, cnt, g.m, g.m, g.ldm, 256)) != MC_OK) return rc;
+  if ((rc = map_batched(&M.b_k128, ws + g.off_b, cnt, g.m, g.m, g.ldm, 128)) != MC_OK) return rc;
+  if ((rc = map_batched(&M.b_k256, ws + g.off_b, cnt, g.m, g.m, g.ldm, 256)) != MC_OK) return rc;
+  return MC_OK;
+}
+
+GemmGroup base_group(const NsGroup& g) {
+  GemmGroup G;
+  std::memset(&G, 0, sizeof(G));
+  G.count = static_cast<int>(g.members.size());
+  G.layout = LAYOUT_BATCHED;
+  G.heads = 1;
+  G.prob_base = g.prob_base;
+  G.band = 8;
+  return G;
+}
+
+}  // namespace
+
+// =========================================================================
+MC_API const char* mc_last_error(void) { return t_last_error.c_str(); }
+
+MC_API size_t mc_muon_workspace_size(const mc_param* params, int n, const mc_hparams* hp) {
+  if (validate_muon(params, n, hp) != MC_OK) return 0;
+  MuonLayout L;
+  plan_muon(params, n, L);
+  return L.total;
+}
+
+MC_API int mc_muon_step(const mc_param* params, int n, const mc_hparams* hp, void* workspace,
+                        size_t workspace_bytes, float* norms_out, void* stream) {
+  int rc = validate_muon(params, n, hp);
+  if (rc != MC_OK) return rc;
+  if (n == 0) return MC_OK;
+  if (norms_out && !aligned16(norms_out)) return fail(MC_ERR_ALIGN, "norms_out must be 16-byte aligned");
+  if (workspace && !aligned16(workspace)) return fail(MC_ERR_ALIGN, "workspace must be 16-byte aligned");
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  std::lock_guard<std::mutex> lock(g_mu);
+  DeviceState* st = nullptr;
+  if ((rc = device_state(&st)) != MC_OK) return rc;
+
+  MuonLayout L;
+  plan_muon(params, n, L);
+  if (workspace) {
+    if (workspace_bytes < L.total)
+      return fail(MC_ERR_NOSPC, "workspace has " + std::to_string(workspace_bytes) + " bytes, needs " +
+                                    std::to_string(L.total));
+  } else if ((rc = own_workspace(*st, L.total, &workspace)) != MC_OK) {
+    return rc;
+  }
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+
+  // ---- device tables
+  std::vector<uint8_t> tab(L.tab_bytes, 0);
+  MomEntry* ent = reinterpret_cast<MomEntry*>(tab.data());
+  int k = 0;
+  for (const auto& g : L.groups) {
+    const size_t xe = size_t(g.rows) * size_t(g.ld);
+    for (size_t j = 0; j < g.members.size(); ++j, ++k) {
+      const mc_param& q = params[g.members[j]];
+      MomEntry& e = ent[k];
+      e.g = q.g;
+      e.m = q.m;
+      e.xf = reinterpret_cast<float*>(ws + g.off_xf) + j * xe;
+      e.xb = reinterpret_cast<__nv_bfloat16*>(ws + g.off_xb[0]) + j * xe;
+      e.rows = q.rows;
+      e.cols = q.cols;
+      e.ld = g.ld;
+      e.cta_begin = L.cta_begin[k];
+      e.g_f32 = q.g_dtype == MC_F32;
+      e.vec = (q.cols % 8) == 0;
+      e.orig = g.members[j];
+      void** wp = reinterpret_cast<void**>(tab.data() + g.off_wptr);
+      float** up = reinterpret_cast<float**>(tab.data() + g.off_uptr);
+      wp[j] = q.w;
+      up[j] = q.update_out;
+    }
+  }
+  if ((rc = upload(*st, tab.data(), tab.size(), ws + L.off_tab, s)) != MC_OK) return rc;
+
+  // ---- momentum, Nesterov, fp32/bf16 iterate, norm partials
+  const MomEntry* dtab = reinterpret_cast<const MomEntry*>(ws + L.off_tab);
+  double* partials = reinterpret_cast<double*>(ws + L.off_partials);
+  float* scale = reinterpret_cast<float*>(ws + L.off_scale);
+  double mom_bytes = 0;
+  for (int i = 0; i < n; ++i)
+    mom_bytes += double(params[i].rows) * double(params[i].cols) * ((params[i].g_dtype == MC_F32 ? 4 : 2) + 8 + 6);
+  {
+    ProfScope prof(K_MOMENTUM, s, 0, 0, mom_bytes);
+    momentum_kernel<<<static_cast<unsigned>(L.total_ctas), MOM_THREADS, 0, s>>>(dtab, n, partials, hp->mu,
+                                                                                 hp->nesterov ? 1 : 0);
+    MC_CUDA(cudaGetLastError());
+  }
+  {
+    ProfScope prof(K_FINALIZE, s);
+    norm_finalize_kernel<<<(n * 32 + 255) / 256, 256, 0, s>>>(dtab, n, partials, L.total_ctas, hp->eps, scale,
+                                                              norms_out);
+    MC_CUDA(cudaGetLastError());
+  }
+
+  // ---- tensor maps
+  std::vector<GroupMaps> maps(L.groups.size());
+  for (size_t gi = 0; gi < L.groups.size(); ++gi)
+    if ((rc = build_group_maps(L.groups[gi], ws, maps[gi])) != MC_OK) return rc;
+
+  // ---- Newton-Schulz iterations, MAX_GROUPS problem groups per launch
+  const int ng = static_cast<int>(L.groups.size());
+  for (int it = 0; it < hp->ns_steps; ++it) {
+    const int par = it & 1;
+    const bool first = it == 0, last = it + 1 == hp->ns_steps;
+    for (int g0 = 0; g0 < ng; g0 += MAX_GROUPS) {
+      const int g1 = std::min(ng, g0 + MAX_GROUPS);
+      GemmParams gram, poly, apply;
+      double f_gram = 0, f_poly = 0, f_apply = 0;
+      std::memset(&gram, 0, sizeof(gram));
+      std::memset(&poly, 0, sizeof(poly));
+      std::memset(&apply, 0, sizeof(apply));
+      gram.err = poly.err = apply.err = st->err_ptr;
+      for (int gi = g0; gi < g1; ++gi) {
+        const int slot = gi - g0;
+        const NsGroup& g = L.groups[gi];
+        const GroupMaps& Mp = maps[gi];
+        const double cnt = double(g.members.size()), dm = double(g.m), dn = double(g.n);
+        f_gram += 2.0 * dm * dm * dn * cnt;
+        f_poly += 2.0 * dm * dm * dm * cnt;
+        f_apply += 2.0 * dm * dm * dn * cnt;
+        // A = s^2 X X^T  (oriented; tall matrices read MN-major: X^T X)
+        GemmGroup G = base_group(g);
+        G.M = G.N = static_cast<int>(g.m);
+        G.K = static_cast<int>(g.n);
+        G.sched = SCHED_SYM;
+        G.a_mn = G.b_mn = g.tall ? 1 : 0;
+        G.d = ws + g.off_a;
+        G.d_ld = g.ldm;
+        G.d_bs = g.m * g.ldm;
+        G.scale = first ? scale : nullptr;
+        gram.map_a[slot] = g.tall ? Mp.x_mn[par] : Mp.x_k128[par];
+        gram.map_b[slot] = g.tall ? Mp.x_mn[par] : Mp.x_k256[par];
+        finish_group(gram, slot, G);
+        // B = b A + c A A
+        G = base_group(g);
+        G.M = G.N = G.K = static_cast<int>(g.m);
+        G.sched = SCHED_SYM;
+        G.src = ws + g.off_a;
+        G.src_ld = g.ldm;
+        G.src_bs = g.m * g.ldm;
+        G.d = ws + g.off_b;
+        G.d_ld = g.ldm;
+        G.d_bs = g.m * g.ldm;
+        G.coef_acc = hp->c;
+        G.coef_src = hp->b;
+        poly.map_a[slot] = Mp.a_k128;
+        poly.map_b[slot] = Mp.a_k256;
+        finish_group(poly, slot, G);
+        // X' = s (a X + B X)   (tall: s (a X + X B), in the stored layout)
+        G = base_group(g);
+        G.M = static_cast<int>(g.rows);
+        G.N = static_cast<int>(g.cols);
+        G.K = static_cast<int>(g.m);
+        G.sched = SCHED_DENSE;
+        if (g.tall) {
+          G.a_mn = 0;
+          G.b_mn = 0;
+          apply.map_a[slot] = Mp.x_k128[par];
+          apply.map_b[slot] = Mp.b_k256;
+        } else {
+          G.a_mn = 0;
+          G.b_mn = 1;
+          apply.map_a[slot] = Mp.b_k128;
+          apply.map_b[slot] = Mp.x_mn[par];
+        }
+        G.xf = reinterpret_cast<float*>(ws + g.off_xf);
+        G.xf_ld = g.ld;
+        G.xf_bs = g.rows * g.ld;
+        G.d = ws + g.off_xb[par ^ 1];
+        G.d_ld = g.ld;
+        G.d_bs = g.rows * g.ld;
+        G.scale = first ? scale : nullptr;
+        G.coef_src = hp->a;
+        if (last) {
+          G.w_ptrs = reinterpret_cast<void* const*>(ws + g.off_wptr);
+          bool any_u = false;
+          for (int i : g.members) any_u |= params[i].update_out != nullptr;
+          G.u_ptrs = any_u ? reinterpret_cast<float* const*>(ws + g.off_uptr) : nullptr;
+          G.w_f32 = g.w_f32;
+          G.w_vec = g.w_f32 ? (g.cols % 4 == 0) : (g.cols % 8 == 0);
+          G.rms = hp->rms_scale * std::sqrt(static_cast<float>(std::max(g.rows, g.cols)));
+          G.decay = 1.f - hp->lr * hp->wd;
+          G.step = -hp->lr * G.rms;
+        }
+        finish_group(apply, slot, G);
+      }
+      if ((rc = launch_gemm<EPI_GRAM>(gram, st->sms, s, K_GRAM, f_gram)) != MC_OK) return rc;
+      if ((rc = launch_gemm<EPI_POLY>(poly, st->sms, s, K_POLY, f_poly)) != MC_OK) return rc;
+      if (last) {
+        if ((rc = launch_gemm<EPI_APPLY_FINAL>(apply, st->sms, s, K_APPLY_FINAL, f_apply)) != MC_OK) return rc;
+      } else {
+        if ((rc = launch_gemm<EPI_APPLY>(apply, st->sms, s, K_APPLY, f_apply)) != MC_OK) return rc;
+      }
+    }
+  }
+  return MC_OK;
+}
+
+// =========================================================================
+namespace {
+struct QkLayout {
+  size_t off_q, off_k, off_keys, total;
+};
+QkLayout plan_qk(int B, int S, int H, int dh) {
+  QkLayout L;
+  const size_t qe = size_t(B) * size_t(S) * size_t(H) * size_t(dh);
+  L.off_q = 0;
+  L.off_k = align_up(2 * qe, 1024);
+  L.off_keys = align_up(L.off_k + 2 * qe, 1024);
+  L.total = align_up(L.off_keys + sizeof(int) * size_t(H), 1024);
+  return L;
+}
+int validate_qk_dims(int B, int S, int D, int H, int dh) {
+  if (B < 1 || S < 1 || D < 1 || H < 1 || dh < 1) return fail(MC_ERR_INVAL, "B, S, D, H, dh must be >= 1");
+  if (D % 8 || dh % 8) return fail(MC_ERR_INVAL, "D and dh must be multiples of 8");
+  if (int64_t(B) * S > (int64_t(1) << 31) - 1 || int64_t(H) * dh > (1 << 24) || D > (1 << 24))
+    return fail(MC_ERR_INVAL, "problem too large");
+  return MC_OK;
+}
+}  // namespace
+
+MC_API size_t mc_qk_workspace_size(int B, int S, int D, int H, int dh) {
+  if (validate_qk_dims(B, S, D, H, dh) != MC_OK) return 0;
+  return plan_qk(B, S, H, dh).total;
+}
+
+MC_API int mc_qk_max_logit(const void* x, const void* wq, const void* wk, int B, int S, int D, int H, int dh,
+                           int causal, float* smax_out, void* workspace, size_t workspace_bytes, void* stream) {
+  int rc = validate_qk_dims(B, S, D, H, dh);
+  if (rc != MC_OK) return rc;
+  if (!x || !wq || !wk || !smax_out) return fail(MC_ERR_INVAL, "NULL x, wq, wk or smax_out");
+  if (!aligned16(x) || !aligned16(wq) || !aligned16(wk) || !aligned16(smax_out) ||
+      (workspace && !aligned16(workspace)))
+    return fail(MC_ERR_ALIGN, "pointers must be 16-byte aligned");
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  std::lock_guard<std::mutex> lock(g_mu);
+  DeviceState* st = nullptr;
+  if ((rc = device_state(&st)) != MC_OK) return rc;
+  const QkLayout L = plan_qk(B, S, H, dh);
+  if (workspace) {
+    if (workspace_bytes < L.total)
+      return fail(MC_ERR_NOSPC, "workspace has " + std::to_string(workspace_bytes) + " bytes, needs " +
+                                    std::to_string(L.total));
+  } else if ((rc = own_workspace(*st, L.total, &workspace)) != MC_OK) {
+    return rc;
+  }
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  int* keys = reinterpret_cast<int*>(ws + L.off_keys);
+  const int HD = H * dh;
+  const int64_t BS = int64_t(B) * S;
+
+  {
+    ProfScope prof(K_QK_KEYS, s);
+    qk_keys_init_kernel<<<(H + 255) / 256, 256, 0, s>>>(keys, H);
+    MC_CUDA(cudaGetLastError());
+  }
+
+  // Q = X W_q^T and K = X W_k^T, bf16 out, one launch.
+  GemmParams proj;
+  std::memset(&proj, 0, sizeof(proj));
+  proj.err = st->err_ptr;
+  for (int which = 0; which < 2; ++which) {
+    if ((rc = map_batched(&proj.map_a[which], x, 1, BS, D, D, 128)) != MC_OK) return rc;
+    if ((rc = map_batched(&proj.map_b[which], which == 0 ? wq : wk, 1, HD, D, D, 256)) != MC_OK) return rc;
+    GemmGroup G;
+    std::memset(&G, 0, sizeof(G));
+    G.M = static_cast<int>(BS);
+    G.N = HD;
+    G.K = D;
+    G.count = 1;
+    G.sched = SCHED_DENSE;
+    G.layout = LAYOUT_BATCHED;
+    G.heads = 1;
+    G.band = 8;
+    G.d = ws + (which == 0 ? L.off_q : L.off_k);
+    G.d_ld = HD;
+    finish_group(proj, which, G);
+  }
+  if ((rc = launch_gemm<EPI_STORE>(proj, st->sms, s, K_QK_PROJ, 2.0 * 2.0 * double(BS) * HD * D)) != MC_OK)
+    return rc;
+
+  // Per-head causal max of Q K^T / sqrt(dh), scores never stored.
+  GemmParams cm;
+  std::memset(&cm, 0, sizeof(cm));
+  cm.err = st->err_ptr;
+  {
+    const uint64_t dims[4] = {uint64_t(dh), uint64_t(H), uint64_t(S), uint64_t(B)};
+    const uint64_t strides[3] = {uint64_t(dh) * 2, uint64_t(HD) * 2, uint64_t(S) * uint64_t(HD) * 2};
+    const uint32_t box_q[4] = {64, 1, 128, 1};
+    const uint32_t box_k[4] = {64, 1, 256, 1};
+    if ((rc = make_map(&cm.map_a[0], ws + L.off_q, 4, dims, strides, box_q)) != MC_OK) return rc;
+    if ((rc = make_map(&cm.map_b[0], ws + L.off_k, 4, dims, strides, box_k)) != MC_OK) return rc;
+    GemmGroup G;
+    std::memset(&G, 0, sizeof(G));
+    G.M = G.N = S;
+    G.K = dh;
+    G.count = B * H;
+    G.heads = H;
+    G.layout = LAYOUT_HEADS;
+    G.sched = causal ? SCHED_CAUSAL : SCHED_DENSE;
+    G.band = 8;
+    G.mask_causal = causal ? 1 : 0;
+    G.keys = keys;
+    G.out_scale = 1.f / std::sqrt(static_cast<float>(dh));
+    finish_group(cm, 0, G);
+  }
+  const double pairs = causal ? double(S) * (double(S) + 1) / 2 : double(S) * S;
+  if ((rc = launch_gemm<EPI_CAUSALMAX>(cm, st->sms, s, K_QK_CMAX, 2.0 * dh * pairs * B * H)) != MC_OK) return rc;
+  {
+    ProfScope prof(K_QK_KEYS, s);
+    qk_keys_decode_kernel<<<(H + 255) / 256, 256, 0, s>>>(keys, smax_out, H);
+    MC_CUDA(cudaGetLastError());
+  }
+  return MC_OK;
+}
+
+MC_API int mc_qk_clip(void* wq, void* wk, int H, int dh, int D, const float* smax, float tau, float alpha,
+                      float* gamma_out, int32_t* mask_out, void* stream) {
+  if (H < 1 || dh < 1 || D < 1) return fail(MC_ERR_INVAL, "H, dh, D must be >= 1");
+  if (int64_t(H) * dh > (1 << 24) || D > (1 << 24)) return fail(MC_ERR_INVAL, "problem too large");
+  if (!wq || !wk || !smax) return fail(MC_ERR_INVAL, "NULL wq, wk or smax");
+  if (wq == wk) return fail(MC_ERR_INVAL, "wq and wk must not alias");
+  if (!std::isfinite(tau) || !(tau > 0.f)) return fail(MC_ERR_INVAL, "tau must be finite and > 0");
+  if (!std::isfinite(alpha) || alpha < 0.f || alpha > 1.f) return fail(MC_ERR_INVAL, "alpha must be in [0, 1]");
+  if (!aligned16(wq) || !aligned16(wk) || !aligned16(smax) || (gamma_out && !aligned16(gamma_out)) ||
+      (mask_out && !aligned16(mask_out)))
+    return fail(MC_ERR_ALIGN, "pointers must be 16-byte aligned");
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  std::lock_guard<std::mutex> lock(g_mu);
+  DeviceState* st = nullptr;
+  int rc = device_state(&st);
+  if (rc != MC_OK) return rc;
+  const dim3 grid(static_cast<unsigned>(H * dh), 2);
+  ProfScope prof(K_QK_CLIP, s);
+  qk_clip_kernel<<<grid, 256, 0, s>>>(static_cast<__nv_bfloat16*>(wq), static_cast<__nv_bfloat16*>(wk), H, dh, D,
+                                      smax, tau, alpha, gamma_out, mask_out, D % 8 == 0 ? 1 : 0);
+  MC_CUDA(cudaGetLastError());
+  return MC_OK;
+}
+
+MC_API int mc_device_status(void) {
+  MC_CUDA(cudaDeviceSynchronize());
+  int v = 0;
+  MC_CUDA(cudaMemcpyFromSymbol(&v, g_device_error, sizeof(int)));
+  if (v != 0) {
+    const int zero = 0;
+    MC_CUDA(cudaMemcpyToSymbol(g_device_error, &zero, sizeof(int)));
+    return fail(MC_ERR_DEVICE, "a kernel abandoned a bounded wait (device error " + std::to_string(v) + ")");
+  }
+  return MC_OK;
+}
+
+MC_API int mc_profile_begin(void) {
+  for (auto& r : t_recs) {
+    cudaEventDestroy(r.b);
+    cudaEventDestroy(r.e);
+  }
+  t_recs.clear();
+  t_prof = true;
+  return MC_OK;
+}
+
+MC_API int mc_profile_end(mc_kernel_stat* out, int max_rows, int* rows) {
+  t_prof = false;
+  mc_kernel_stat acc[K_COUNT];
+  std::memset(acc, 0, sizeof(acc));
+  int rc = MC_OK;
+  for (auto& r : t_recs) {
+    float ms = 0.f;
+    if (cudaEventSynchronize(r.e) != cudaSuccess || cudaEventElapsedTime(&ms, r.b, r.e) != cudaSuccess) {
+      rc = fail(MC_ERR_CUDA, "profiling event could not be read");
+    }
+    mc_kernel_stat& a = acc[r.kind];
+    a.launches += 1;
+    a.total_ms += ms;
+    a.flops += r.flops;
+    a.flops_executed += r.flops_exec;
+    a.bytes += r.bytes;
+    cudaEventDestroy(r.b);
+    cudaEventDestroy(r.e);
+  }
+  t_recs.clear();
+  int k = 0;
+  for (int i = 0; i < K_COUNT; ++i) {
+    if (acc[i].launches == 0) continue;
+    if (out && k < max_rows) {
+      out[k] = acc[i];
+      std::strncpy(out[k].name, kKindNames[i], sizeof(out[k].name) - 1);
+    }
+    ++k;
+  }
+  if (rows) *rows = k;
+  return rc;
+}

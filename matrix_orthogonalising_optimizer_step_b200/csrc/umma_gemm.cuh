@@ -1,0 +1,550 @@
+// Grouped, persistent tcgen05 GEMM for sm_100a with the MuonClip epilogues.
+//
+// One kernel computes D = A * B^T tile by tile (128 x 256 fp32 accumulator in
+// TMEM) for up to MAX_GROUPS groups of equally shaped problems, and hands each
+// finished tile to a fused epilogue:
+//
+//   EPI_GRAM        A_k   = s^2 * X X^T            (symmetric: upper tiles only,
+//                                                  each element stored twice)
+//   EPI_POLY        B_k   = b*A + c*(A A)          (symmetric, mirrored store)
+//   EPI_APPLY       X_k+1 = s * (a*X + B X)        (fp32 iterate in place + bf16 copy)
+//   EPI_APPLY_FINAL W     = (1 - lr*wd) W - lr * rms * X_N   (last iteration; X_N
+//                                                  never touches memory)
+//   EPI_STORE       plain bf16 store (Q/K projection)
+//   EPI_CAUSALMAX   per-head max over j <= i of the score tile (QK-Clip's S_max);
+//                   the score tile is never stored
+//
+// The quintic Newton-Schulz step these epilogues implement is the one printed in
+// "Muon and MuonClip: orthogonalised updates for LLM training", §2 (A = X X^T,
+// X = aX + (bA + cA A)X) and "MuonClip: speed, then stability", §02; the apply
+// is §03's W <- W - eta (O + lambda W) with O scaled by 0.2 sqrt(max(m, n)).
+//
+// Warp roles (320 threads, one CTA per SM):
+//   warp 0      TMA producer: 4-stage ring of {A 128x64, B 256x64} bf16 tiles,
+//               128-byte swizzled, K-major or MN-major per group.
+//   warp 1      TMEM allocator + single-thread tcgen05.mma issuer (M=128, N=256,
+//               K=16 per instruction), commits to the ring and the accumulators.
+//   warps 2-9   epilogue: two accumulator buffers (2 x 256 TMEM columns) so the
+//               next tile's MMAs overlap this tile's epilogue.  Warp w reads TMEM
+//               lanes 32*(w%4)..+31 and column half (w-2)/4.
+#pragma once
+
+#include "ptx.cuh"
+
+namespace mc {
+
+constexpr int BM = 128, BN = 256, BK = 64, STAGES = 4;
+constexpr uint32_t A_STAGE_BYTES = BM * BK * 2;   // 16 KiB
+constexpr uint32_t B_STAGE_BYTES = BN * BK * 2;   // 32 KiB
+constexpr uint32_t STAGE_BYTES = A_STAGE_BYTES + B_STAGE_BYTES;
+constexpr uint32_t MN_BOX_BYTES = 64 * BK * 2;    // one {64 MN, 64 K} box: 8 KiB
+constexpr int NUM_EPI_WARPS = 8;
+constexpr int GEMM_THREADS = 64 + NUM_EPI_WARPS * 32;
+constexpr uint32_t TMEM_COLS = 2 * BN;
+constexpr int MAX_GROUPS = 4;
+constexpr int GEMM_BARRIER_BYTES = 256;
+constexpr size_t GEMM_SMEM_BYTES = 1024 + size_t(STAGES) * STAGE_BYTES + GEMM_BARRIER_BYTES;
+
+enum Sched : int { SCHED_DENSE = 0, SCHED_SYM = 1, SCHED_CAUSAL = 2 };
+enum Layout : int { LAYOUT_BATCHED = 0, LAYOUT_HEADS = 1 };
+enum Epi : int {
+  EPI_GRAM = 0,
+  EPI_POLY = 1,
+  EPI_APPLY = 2,
+  EPI_APPLY_FINAL = 3,
+  EPI_STORE = 4,
+  EPI_CAUSALMAX = 5
+};
+
+struct GemmGroup {
+  int M, N, K;             // D is M x N, contraction K
+  int count;               // independent problems in the group
+  int tiles_m, tiles_n;    // ceil(M / BM), ceil(N / BN)
+  long long tiles_per_prob;
+  long long tile_start;    // first global tile of this group
+  int sched, layout, heads;
+  int a_mn, b_mn;          // operand major-ness: 0 K-major, 1 MN-major
+  int prob_base;           // index of problem 0 in the per-matrix scale table
+  int band;                // dense raster: n-tiles per band
+  // ---- epilogue operands ----
+  void* d;                 // bf16 output [count][M][d_ld]
+  long long d_ld, d_bs;
+  const void* src;         // bf16 epilogue source (EPI_POLY)
+  long long src_ld, src_bs;
+  float* xf;               // fp32 iterate (EPI_APPLY*)
+  long long xf_ld, xf_bs;
+  void* const* w_ptrs;     // per-problem weight (EPI_APPLY_FINAL), row-major M x N
+  float* const* u_ptrs;    // per-problem update output, entries may be null
+  const float* scale;      // per-problem s, or null for 1
+  int w_f32;               // weight dtype: 1 fp32, 0 bf16
+  int w_vec;               // weight rows 16-byte aligned
+  int mask_causal;         // EPI_CAUSALMAX
+  int* keys;               // EPI_CAUSALMAX: order-preserving ints, one per head
+  float coef_acc, coef_src;
+  float decay, step, rms;  // EPI_APPLY_FINAL
+  float out_scale;         // EPI_CAUSALMAX: 1/sqrt(d_head)
+};
+
+struct GemmParams {
+  CUtensorMap map_a[MAX_GROUPS];
+  CUtensorMap map_b[MAX_GROUPS];
+  GemmGroup g[MAX_GROUPS];
+  int num_groups;
+  long long total_tiles;
+  int* err;
+};
+static_assert(sizeof(GemmParams) <= 4096, "kernel parameters must fit the classic 4 KiB limit");
+
+// ------------------------------------------------------------------ tiling
+// Tiles (i, j) of 128 rows x 256 columns.  SYM keeps the tiles that touch
+// the upper triangle (j >= floor(i/2)); CAUSAL keeps those that touch the
+// lower triangle including the diagonal (j <= floor(i/2)).
+__host__ __device__ inline long long sched_row_count(int sched, int i, int tiles_n) {
+  if (sched == SCHED_SYM) return tiles_n - i / 2;
+  if (sched == SCHED_CAUSAL) return (i / 2 + 1) < tiles_n ? (i / 2 + 1) : tiles_n;
+  return tiles_n;
+}
+__host__ __device__ inline long long sched_tiles_per_prob(int sched, int tiles_m, int tiles_n) {
+  if (sched == SCHED_DENSE) return (long long)tiles_m * tiles_n;
+  long long t = 0;
+  for (int i = 0; i < tiles_m; ++i) t += sched_row_count(sched, i, tiles_n);
+  return t;
+}
+
+struct TileInfo {
+  int g, prob, tm, tn, num_kb;
+};
+
+__host__ __device__ inline void decode_tile(const GemmGroup* groups, int num_groups, long long t,
+                                            TileInfo& ti) {
+  int g = 0;
+  while (g + 1 < num_groups && t >= groups[g + 1].tile_start) ++g;
+  const GemmGroup& G = groups[g];
+  long long local = t - G.tile_start;
+  const long long prob = local / G.tiles_per_prob;
+  long long tl = local - prob * G.tiles_per_prob;
+  int tm = 0, tn = 0;
+  if (G.sched == SCHED_DENSE) {
+    const int band = G.band;
+    const long long per_band = (long long)G.tiles_m * band;
+    const int bidx = (int)(tl / per_band);
+    const long long x = tl - (long long)bidx * per_band;
+    const int rem = G.tiles_n - bidx * band;
+    const int w = rem < band ? rem : band;
+    tm = (int)(x / w);
+    tn = bidx * band + (int)(x % w);
+  } else {
+    int i = 0;
+    while (true) {
+      const long long cnt = sched_row_count(G.sched, i, G.tiles_n);
+      if (tl < cnt) break;
+      tl -= cnt;
+      ++i;
+    }
+    tm = i;
+    tn = (G.sched == SCHED_SYM ? i / 2 : 0) + (int)tl;
+  }
+  ti.g = g;
+  ti.prob = (int)prob;
+  ti.tm = tm;
+  ti.tn = tn;
+  ti.num_kb = (G.K + BK - 1) / BK;
+}
+
+// -------------------------------------------------------------- epilogues
+__device__ __forceinline__ void load_bf16x16(const __nv_bfloat16* p, float (&x)[16]) {
+  const uint4* q = reinterpret_cast<const uint4*>(p);
+  uint4 a = q[0], b = q[1];
+  const uint32_t w[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    x[2 * i] = __uint_as_float(w[i] << 16);
+    x[2 * i + 1] = __uint_as_float(w[i] & 0xFFFF0000u);
+  }
+}
+__device__ __forceinline__ void store_bf16x16(__nv_bfloat16* p, const float (&x)[16]) {
+  uint4 a, b;
+  a.x = pack_bf16x2(x[0], x[1]);
+  a.y = pack_bf16x2(x[2], x[3]);
+  a.z = pack_bf16x2(x[4], x[5]);
+  a.w = pack_bf16x2(x[6], x[7]);
+  b.x = pack_bf16x2(x[8], x[9]);
+  b.y = pack_bf16x2(x[10], x[11]);
+  b.z = pack_bf16x2(x[12], x[13]);
+  b.w = pack_bf16x2(x[14], x[15]);
+  uint4* q = reinterpret_cast<uint4*>(p);
+  q[0] = a;
+  q[1] = b;
+}
+__device__ __forceinline__ void load_f32x16(const float* p, float (&x)[16]) {
+  const float4* q = reinterpret_cast<const float4*>(p);
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    float4 v = q[i];
+    x[4 * i] = v.x;
+    x[4 * i + 1] = v.y;
+    x[4 * i + 2] = v.z;
+    x[4 * i + 3] = v.w;
+  }
+}
+__device__ __forceinline__ void store_f32x16(float* p, const float (&x)[16]) {
+  float4* q = reinterpret_cast<float4*>(p);
+#pragma unroll
+  for (int i = 0; i < 4; ++i) q[i] = make_float4(x[4 * i], x[4 * i + 1], x[4 * i + 2], x[4 * i + 3]);
+}
+
+// Symmetric store of one 16-column chunk of row r: element (r, c) with c >= r
+// goes to (r, c) and, when c > r, also to (c, r).  Across a warp r runs over
+// 32 consecutive rows, so each mirrored store is one 64-byte segment.
+__device__ __forceinline__ void store_sym_chunk(__nv_bfloat16* D, long long ld, int M, int r, int c0,
+                                                const float (&v)[16]) {
+  if (r >= M) return;
+  if (c0 >= r && c0 + 16 <= M) {
+    store_bf16x16(D + (long long)r * ld + c0, v);
+  } else {
+#pragma unroll
+    for (int j = 0; j < 16; ++j) {
+      const int c = c0 + j;
+      if (c >= r && c < M) D[(long long)r * ld + c] = __float2bfloat16_rn(v[j]);
+    }
+  }
+#pragma unroll
+  for (int j = 0; j < 16; ++j) {
+    const int c = c0 + j;
+    if (c > r && c < M) D[(long long)c * ld + r] = __float2bfloat16_rn(v[j]);
+  }
+}
+
+template <int EPI>
+__device__ __forceinline__ void epilogue_chunk(const GemmGroup& G, int prob, int r, int c0,
+                                               float (&v)[16], float& run_max) {
+  const bool full = (r < G.M) && (c0 + 16 <= G.N);
+  if constexpr (EPI == EPI_GRAM) {
+    float s2 = 1.f;
+    if (G.scale) {
+      const float s = G.scale[G.prob_base + prob];
+      s2 = s * s;
+    }
+#pragma unroll
+    for (int j = 0; j < 16; ++j) v[j] *= s2;
+    __nv_bfloat16* D = static_cast<__nv_bfloat16*>(G.d) + (long long)prob * G.d_bs;
+    store_sym_chunk(D, G.d_ld, G.M, r, c0, v);
+  } else if constexpr (EPI == EPI_POLY) {
+    if (r >= G.M) return;
+    const __nv_bfloat16* S =
+        static_cast<const __nv_bfloat16*>(G.src) + (long long)prob * G.src_bs + (long long)r * G.src_ld;
+    float x[16];
+    if (full) {
+      load_bf16x16(S + c0, x);
+    } else {
+#pragma unroll
+      for (int j = 0; j < 16; ++j) x[j] = (c0 + j < G.N) ? __bfloat162float(S[c0 + j]) : 0.f;
+    }
+#pragma unroll
+    for (int j = 0; j < 16; ++j) v[j] = fmaf(G.coef_acc, v[j], G.coef_src * x[j]);
+    __nv_bfloat16* D = static_cast<__nv_bfloat16*>(G.d) + (long long)prob * G.d_bs;
+    store_sym_chunk(D, G.d_ld, G.M, r, c0, v);
+  } else if constexpr (EPI == EPI_APPLY || EPI == EPI_APPLY_FINAL) {
+    if (r >= G.M) return;
+    const float s = G.scale ? G.scale[G.prob_base + prob] : 1.f;
+    float* X = G.xf + (long long)prob * G.xf_bs + (long long)r * G.xf_ld;
+    float x[16];
+    if (full) {
+      load_f32x16(X + c0, x);
+    } else {
+#pragma unroll
+      for (int j = 0; j < 16; ++j) x[j] = (c0 + j < G.N) ? X[c0 + j] : 0.f;
+    }
+#pragma unroll
+    for (int j = 0; j < 16; ++j) v[j] = s * fmaf(G.coef_src, x[j], v[j]);
+    if constexpr (EPI == EPI_APPLY) {
+      __nv_bfloat16* D =
+          static_cast<__nv_bfloat16*>(G.d) + (long long)prob * G.d_bs + (long long)r * G.d_ld;
+      if (full) {
+        store_f32x16(X + c0, v);
+        store_bf16x16(D + c0, v);
+      } else {
+#pragma unroll
+        for (int j = 0; j < 16; ++j)
+          if (c0 + j < G.N) {
+            X[c0 + j] = v[j];
+            D[c0 + j] = __float2bfloat16_rn(v[j]);
+          }
+      }
+    } else {
+      float* U = G.u_ptrs ? G.u_ptrs[prob] : nullptr;
+      const long long row = (long long)r * G.N;
+      if (U) {
+        float u[16];
+#pragma unroll
+        for (int j = 0; j < 16; ++j) u[j] = G.rms * v[j];
+        if (full && (G.N % 4 == 0)) {
+          store_f32x16(U + row + c0, u);
+        } else {
+#pragma unroll
+          for (int j = 0; j < 16; ++j)
+            if (c0 + j < G.N) U[row + c0 + j] = u[j];
+        }
+      }
+      if (G.w_f32) {
+        float* W = static_cast<float*>(G.w_ptrs[prob]) + row;
+        if (full && G.w_vec) {
+          float w[16];
+          load_f32x16(W + c0, w);
+#pragma unroll
+          for (int j = 0; j < 16; ++j) w[j] = fmaf(G.step, v[j], G.decay * w[j]);
+          store_f32x16(W + c0, w);
+        } else {
+#pragma unroll
+          for (int j = 0; j < 16; ++j)
+            if (c0 + j < G.N) W[c0 + j] = fmaf(G.step, v[j], G.decay * W[c0 + j]);
+        }
+      } else {
+        __nv_bfloat16* W = static_cast<__nv_bfloat16*>(G.w_ptrs[prob]) + row;
+        if (full && G.w_vec) {
+          float w[16];
+          load_bf16x16(W + c0, w);
+#pragma unroll
+          for (int j = 0; j < 16; ++j) w[j] = fmaf(G.step, v[j], G.decay * w[j]);
+          store_bf16x16(W + c0, w);
+        } else {
+#pragma unroll
+          for (int j = 0; j < 16; ++j)
+            if (c0 + j < G.N)
+              W[c0 + j] = __float2bfloat16_rn(
+                  fmaf(G.step, v[j], G.decay * __bfloat162float(W[c0 + j])));
+        }
+      }
+    }
+  } else if constexpr (EPI == EPI_STORE) {
+    if (r >= G.M) return;
+    __nv_bfloat16* D =
+        static_cast<__nv_bfloat16*>(G.d) + (long long)prob * G.d_bs + (long long)r * G.d_ld;
+    if (full) {
+      store_bf16x16(D + c0, v);
+    } else {
+#pragma unroll
+      for (int j = 0; j < 16; ++j)
+        if (c0 + j < G.N) D[c0 + j] = __float2bfloat16_rn(v[j]);
+    }
+  } else if constexpr (EPI == EPI_CAUSALMAX) {
+    if (r >= G.M) return;
+#pragma unroll
+    for (int j = 0; j < 16; ++j) {
+      const int c = c0 + j;
+      const bool ok = (c < G.N) && (!G.mask_causal || c <= r);
+      if (ok) run_max = fmaxf(run_max, v[j]);
+    }
+  }
+}
+
+// ------------------------------------------------------------------ kernel
+template <int EPI>
+__global__ void __launch_bounds__(GEMM_THREADS, 1) umma_gemm_kernel(const __grid_constant__ GemmParams P) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + STAGES * STAGE_BYTES);
+  uint64_t* full_bar = bars;                    // [STAGES]
+  uint64_t* empty_bar = bars + STAGES;          // [STAGES]
+  uint64_t* tfull_bar = bars + 2 * STAGES;      // [2]
+  uint64_t* tempty_bar = bars + 2 * STAGES + 2; // [2]
+  uint64_t* drain_bar = bars + 2 * STAGES + 4;  // [1]
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2 * STAGES + 5);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < STAGES; ++s) {
+      mbar_init(smem_u32(&full_bar[s]), 1);
+      mbar_init(smem_u32(&empty_bar[s]), 1);
+    }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(smem_u32(&tfull_bar[b]), 1);
+      mbar_init(smem_u32(&tempty_bar[b]), NUM_EPI_WARPS);
+    }
+    mbar_init(smem_u32(drain_bar), 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 0 && lane == 0) {
+    for (int g = 0; g < P.num_groups; ++g) {
+      prefetch_tmap(&P.map_a[g]);
+      prefetch_tmap(&P.map_b[g]);
+    }
+  }
+  if (warp == 1) {
+    tmem_alloc(smem_u32(tmem_slot), TMEM_COLS);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+  const long long total = P.total_tiles;
+
+  if (warp == 0) {
+    // ------------------------------------------------------- TMA producer
+    if (lane == 0) {
+      int stage = 0;
+      uint32_t phase = 0;
+      uint32_t filled = 0;          // bit s: stage s was ever filled
+      uint32_t fill_parity = 0;     // bit s: parity of its latest fill
+      bool ok = true;
+      for (long long t = blockIdx.x; ok && t < total; t += gridDim.x) {
+        TileInfo ti;
+        decode_tile(P.g, P.num_groups, t, ti);
+        const GemmGroup& G = P.g[ti.g];
+        const CUtensorMap* ma = &P.map_a[ti.g];
+        const CUtensorMap* mb = &P.map_b[ti.g];
+        const int m0 = ti.tm * BM, n0 = ti.tn * BN;
+        for (int kb = 0; kb < ti.num_kb; ++kb) {
+          if (!wait_bounded(smem_u32(&empty_bar[stage]), phase ^ 1, abort_flag, P.err)) {
+            ok = false;
+            break;
+          }
+          const uint32_t fb = smem_u32(&full_bar[stage]);
+          mbar_arrive_expect_tx(fb, STAGE_BYTES);
+          filled |= 1u << stage;
+          fill_parity = (fill_parity & ~(1u << stage)) | (phase << stage);
+          const uint32_t sa = smem_u32(smem + stage * STAGE_BYTES);
+          const uint32_t sb = sa + A_STAGE_BYTES;
+          const int k0 = kb * BK;
+          if (G.layout == LAYOUT_HEADS) {
+            const int bb = ti.prob / G.heads, hh = ti.prob % G.heads;
+            tma_load_4d(sa, ma, fb, k0, hh, m0, bb);
+            tma_load_4d(sb, mb, fb, k0, hh, n0, bb);
+          } else {
+            if (!G.a_mn) {
+              tma_load_3d(sa, ma, fb, k0, m0, ti.prob);
+            } else {
+              tma_load_3d(sa, ma, fb, m0, k0, ti.prob);
+              tma_load_3d(sa + MN_BOX_BYTES, ma, fb, m0 + 64, k0, ti.prob);
+            }
+            if (!G.b_mn) {
+              tma_load_3d(sb, mb, fb, k0, n0, ti.prob);
+            } else {
+#pragma unroll
+              for (int q = 0; q < 4; ++q) tma_load_3d(sb + q * MN_BOX_BYTES, mb, fb, n0 + 64 * q, k0, ti.prob);
+            }
+          }
+          if (++stage == STAGES) {
+            stage = 0;
+            phase ^= 1;
+          }
+        }
+      }
+      // Do not leave while a copy may still be landing in shared memory.
+      for (int s = 0; s < STAGES; ++s)
+        if (filled & (1u << s)) {
+          volatile int no_abort = 0;
+          wait_bounded(smem_u32(&full_bar[s]), (fill_parity >> s) & 1u, &no_abort, nullptr,
+                       kDrainLimitCycles);
+        }
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------- MMA issuer
+    if (lane == 0) {
+      int stage = 0;
+      uint32_t phase = 0;
+      int acc = 0;
+      uint32_t acc_phase = 0;
+      bool ok = true;
+      for (long long t = blockIdx.x; ok && t < total; t += gridDim.x) {
+        TileInfo ti;
+        decode_tile(P.g, P.num_groups, t, ti);
+        const GemmGroup& G = P.g[ti.g];
+        const uint32_t idesc = idesc_bf16_f32(BM, BN, G.a_mn, G.b_mn);
+        const uint32_t a_lbo = G.a_mn ? MN_BOX_BYTES : 16u;
+        const uint32_t b_lbo = G.b_mn ? MN_BOX_BYTES : 16u;
+        const uint32_t a_kstep = G.a_mn ? 16u * 128u : 32u;
+        const uint32_t b_kstep = G.b_mn ? 16u * 128u : 32u;
+        if (!wait_bounded(smem_u32(&tempty_bar[acc]), acc_phase ^ 1, abort_flag, P.err)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        const uint32_t d_tmem = tmem_base + acc * BN;
+        for (int kb = 0; kb < ti.num_kb; ++kb) {
+          if (!wait_bounded(smem_u32(&full_bar[stage]), phase, abort_flag, P.err)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t sa = smem_u32(smem + stage * STAGE_BYTES);
+          const uint32_t sb = sa + A_STAGE_BYTES;
+#pragma unroll
+          for (int kk = 0; kk < BK / 16; ++kk) {
+            const uint64_t ad = smem_desc_sw128(sa + kk * a_kstep, a_lbo, 1024);
+            const uint64_t bd = smem_desc_sw128(sb + kk * b_kstep, b_lbo, 1024);
+            umma_bf16(d_tmem, ad, bd, idesc, (kb | kk) != 0);
+          }
+          umma_commit(smem_u32(&empty_bar[stage]));
+          if (++stage == STAGES) {
+            stage = 0;
+            phase ^= 1;
+          }
+        }
+        if (!ok) break;
+        umma_commit(smem_u32(&tfull_bar[acc]));
+        acc ^= 1;
+        if (acc == 0) acc_phase ^= 1;
+      }
+      // All MMAs issued by this thread complete before TMEM is released.
+      umma_commit(smem_u32(drain_bar));
+      volatile int no_abort = 0;
+      wait_bounded(smem_u32(drain_bar), 0, &no_abort, nullptr, kDrainLimitCycles);
+    }
+  } else {
+    // ------------------------------------------------------- epilogue
+    const int q = warp & 3;            // TMEM lane quarter this warp may read
+    const int half = (warp - 2) >> 2;  // column half of the 256-wide tile
+    int acc = 0;
+    uint32_t acc_phase = 0;
+    for (long long t = blockIdx.x; t < total; t += gridDim.x) {
+      TileInfo ti;
+      decode_tile(P.g, P.num_groups, t, ti);
+      const GemmGroup& G = P.g[ti.g];
+      // Every lane waits; the warp proceeds only if all lanes saw the phase
+      // complete, so a timeout can never split the warp before the
+      // warp-collective TMEM loads below.
+      const bool ok = wait_bounded(smem_u32(&tfull_bar[acc]), acc_phase, abort_flag, P.err);
+      if (!__all_sync(0xffffffffu, ok)) break;
+      tc_fence_after();
+      const int r = ti.tm * BM + q * 32 + lane;
+      const uint32_t t_row = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + acc * BN + half * 128;
+      float run_max = -INFINITY;
+#pragma unroll 1
+      for (int ch = 0; ch < 8; ++ch) {
+        float v[16];
+        tmem_ld16(t_row + ch * 16, v);
+        const int c0 = ti.tn * BN + half * 128 + ch * 16;
+        epilogue_chunk<EPI>(G, ti.prob, r, c0, v, run_max);
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(smem_u32(&tempty_bar[acc]));
+      if constexpr (EPI == EPI_CAUSALMAX) {
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) run_max = fmaxf(run_max, __shfl_xor_sync(0xffffffffu, run_max, o));
+        if (lane == 0 && run_max > -INFINITY) {
+          const int h = ti.prob % G.heads;
+          atomicMax(&G.keys[h], float_to_ordered(run_max * G.out_scale));
+        }
+      }
+      acc ^= 1;
+      if (acc == 0) acc_phase ^= 1;
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    __syncwarp();
+    tc_fence_after();
+    tmem_dealloc(tmem_base, TMEM_COLS);
+  }
+}
+
+}  // namespace mc

@@ -1,0 +1,120 @@
+"""CPU tests of the C-ABI library: it loads, exports every entry point that
+include/muonclip.h declares, rejects bad arguments before touching memory or the
+GPU, and its host-side tile scheduler covers every output element."""
+import ctypes
+import os
+import re
+import subprocess
+
+import pytest
+
+import matrix_orthogonalising_optimizer_step_b200 as mc
+from matrix_orthogonalising_optimizer_step_b200 import build as mcbuild
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "muonclip.h")
+
+
+@pytest.fixture(scope="module")
+def lib():
+    mcbuild.build()
+    return mc.load_library()
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(mc_\w+)\s*\(", text)))
+
+
+def test_header_declares_the_three_operations():
+    names = declared_functions()
+    for n in ("mc_muon_step", "mc_qk_max_logit", "mc_qk_clip"):
+        assert n in names
+
+
+def test_library_exports_every_declared_symbol(lib):
+    names = declared_functions()
+    assert set(names) == set(mc.EXPORTS)
+    out = subprocess.run(["nm", "-D", "--defined-only", mc.LIB_PATH], capture_output=True, text=True).stdout
+    exported = set(re.findall(r"\bT (mc_\w+)$", out, flags=re.M))
+    for n in names:
+        assert n in exported, n
+        assert hasattr(lib, n)
+    # internal symbols stay hidden
+    assert not any(s.startswith("_ZN2mc") for s in re.findall(r"\bT (\S+)$", out, flags=re.M))
+
+
+def _params(n, rows=64, cols=96, base=0x100000):
+    arr = (mc.McParam * max(n, 1))()
+    for i in range(n):
+        off = base + i * 0x10000
+        arr[i] = mc.McParam(off, off + 0x4000, off + 0x8000, rows, cols, mc.MC_BF16, mc.MC_BF16, None)
+    return arr
+
+
+def test_argument_errors_return_codes_without_a_gpu(lib):
+    hp = mc.make_hparams()
+    P = ctypes.byref
+    arr = _params(2)
+    # null params with n > 0
+    assert lib.mc_muon_step(None, 2, P(hp), None, 0, None, None) == mc.MC_ERR_INVAL
+    assert "params" in mc.last_error()
+    # negative n, null hp, bad ns_steps, bad eps
+    assert lib.mc_muon_step(arr, -1, P(hp), None, 0, None, None) == mc.MC_ERR_INVAL
+    assert lib.mc_muon_step(arr, 2, None, None, 0, None, None) == mc.MC_ERR_INVAL
+    for bad in (dict(ns_steps=0), dict(ns_steps=100), dict(eps=0.0), dict(lr=float("nan"))):
+        h = mc.make_hparams(**bad)
+        assert lib.mc_muon_step(arr, 2, P(h), None, 0, None, None) == mc.MC_ERR_INVAL
+    # bad shape, bad dtype, aliasing, misalignment
+    a = _params(1); a[0].rows = 0
+    assert lib.mc_muon_step(a, 1, P(hp), None, 0, None, None) == mc.MC_ERR_INVAL
+    a = _params(1); a[0].w_dtype = 7
+    assert lib.mc_muon_step(a, 1, P(hp), None, 0, None, None) == mc.MC_ERR_INVAL
+    a = _params(1); a[0].m = a[0].w
+    assert lib.mc_muon_step(a, 1, P(hp), None, 0, None, None) == mc.MC_ERR_INVAL
+    a = _params(1); a[0].g = a[0].g + 2
+    assert lib.mc_muon_step(a, 1, P(hp), None, 0, None, None) == mc.MC_ERR_ALIGN
+    # n == 0 is a no-op
+    assert lib.mc_muon_step(arr, 0, P(hp), None, 0, None, None) == mc.MC_OK
+    # QK
+    assert lib.mc_qk_max_logit(None, None, None, 1, 8, 64, 2, 64, 1, None, None, 0, None) == mc.MC_ERR_INVAL
+    assert lib.mc_qk_max_logit(16, 32, 48, 1, 8, 60, 2, 64, 1, 64, None, 0, None) == mc.MC_ERR_INVAL  # D % 8
+    assert lib.mc_qk_max_logit(16, 32, 48, 1, 8, 64, 2, 64, 1, 66, None, 0, None) == mc.MC_ERR_ALIGN
+    assert lib.mc_qk_clip(16, 32, 2, 8, 64, 48, 100.0, 1.5, None, None, None) == mc.MC_ERR_INVAL  # alpha
+    assert lib.mc_qk_clip(16, 32, 2, 8, 64, 48, -1.0, 0.5, None, None, None) == mc.MC_ERR_INVAL   # tau
+    assert lib.mc_qk_clip(16, 16, 2, 8, 64, 48, 100.0, 0.5, None, None, None) == mc.MC_ERR_INVAL  # alias
+    assert lib.mc_qk_clip(16, 32, 2, 8, 64, 50, 100.0, 0.5, None, None, None) == mc.MC_ERR_ALIGN
+
+
+def test_workspace_queries(lib):
+    hp = mc.make_hparams()
+    P = ctypes.byref
+    one = lib.mc_muon_workspace_size(_params(1), 1, P(hp))
+    two = lib.mc_muon_workspace_size(_params(2), 2, P(hp))
+    assert one > 0 and two > one
+    # 64 x 96 bf16: two bf16 iterates + fp32 iterate + A, B (64 x 64 bf16)
+    assert one >= 64 * 96 * (2 + 2 + 4) + 2 * 64 * 64 * 2
+    tall = _params(1, rows=96, cols=64)
+    assert lib.mc_muon_workspace_size(tall, 1, P(hp)) == one  # same bytes, stored layout
+    assert lib.mc_muon_workspace_size(_params(1), 1, P(mc.make_hparams(ns_steps=0))) == 0
+    q = lib.mc_qk_workspace_size(4, 4096, 4096, 32, 128)
+    assert q >= 2 * 4 * 4096 * 4096 * 2
+    assert lib.mc_qk_workspace_size(1, 8, 63, 1, 8) == 0
+
+
+def test_tile_scheduler_host_check(tmp_path):
+    src = os.path.join(ROOT, "tests", "host", "sched_check.cu")
+    exe = tmp_path / "sched_check"
+    cmd = [mcbuild.nvcc_path(), "-std=c++17", "-O1", "-gencode", "arch=compute_100a,code=sm_100a",
+           "-I", mcbuild.CSRC, "-o", str(exe), src]
+    subprocess.run(cmd, check=True, capture_output=True)
+    out = subprocess.run([str(exe)], capture_output=True, text=True)
+    assert out.returncode == 0 and out.stdout.strip() == "OK", out.stdout
+
+
+def test_python_binding_fails_loudly_without_library(monkeypatch, tmp_path):
+    monkeypatch.setattr(mc, "_lib", None)
+    monkeypatch.setattr(mc, "LIB_PATH", str(tmp_path / "missing.so"))
+    with pytest.raises(RuntimeError, match="missing"):
+        mc.load_library()
