@@ -33,6 +33,13 @@ WORKLOAD = ("7B-shaped Muon step (224 matrices, 7.78e9 params, bf16 W/G, fp32 M,
             "+ causal MHA S_max and QK-Clip (B4 S4096 H32 dh128)")
 
 
+# DRAM bytes per launch (dram__bytes_read.sum + dram__bytes_write.sum) of the
+# kernels as they stand, from one ncu capture: profiles/ns_gemm_1layer_full.md
+# (1-layer case, third NS iteration, scaled by the 32 layers processed at full
+# size).  None where no capture of the current kernel exists.
+KERNEL_TRAFFIC_BYTES = {"ns_apply": 51.9e9}
+
+
 def parse_args(argv=None):
     p = argparse.ArgumentParser()
     p.add_argument("--gpus", type=int, default=1)
@@ -293,8 +300,9 @@ def main(argv=None):
     d = kernels[dom]
     if d["flops"] > 0:
         ach = d["flops"] / (d["total_ms"] / 1e3) / 1e12
+        traffic = KERNEL_TRAFFIC_BYTES.get(dom) if args.layers == 32 else None
         roof = {"kernel": dom, "bound": "tensor", "achieved": ach, "peak": peaks["bf16_tflops_sustained"],
-                "unit": "TFLOP/s", "frac": ach / peaks["bf16_tflops_sustained"], "traffic": None,
+                "unit": "TFLOP/s", "frac": ach / peaks["bf16_tflops_sustained"], "traffic": traffic,
                 "peak_source": f"{peaks['source']} bf16_tflops_sustained (kernel timed inside a long step)"}
     else:
         ach = d["bytes"] / (d["total_ms"] / 1e3) / 1e9

@@ -83,7 +83,11 @@ typedef struct {
  *   O <- X in the weight's orientation
  *   W <- W - lr*(rms_scale*sqrt(max(rows,cols))*O + wd*W)
  * The Newton-Schulz products run on tcgen05 tensor cores with bf16 operands
- * and fp32 accumulation; the iterate is also carried in fp32 for the a*X term.
+ * and fp32 accumulation.  In the first two iterations the a*X term is taken
+ * from an fp32 copy of the iterate; from the third on, a*I is folded into B
+ * (X <- (aI + B) X), which amplifies the bf16 rounding of X less once the
+ * singular values have entered the polynomial's band.  The last iteration
+ * applies the update to W straight from the fp32 accumulator.
  * Matrices of equal shape and weight dtype are batched into one problem group.
  *
  * params/n      host array of n >= 0 entries (n == 0 is a no-op).  W, G, M of

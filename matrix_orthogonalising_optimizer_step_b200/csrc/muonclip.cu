@@ -56,6 +56,8 @@ using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t
                                    CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
 
 constexpr int kRing = 4;
+// Newton-Schulz iterations that take a*X from the fp32 iterate.
+constexpr int kMixedIters = 2;
 
 struct DeviceState {
   bool init = false;
@@ -486,11 +488,14 @@ MC_API int mc_muon_step(const mc_param* params, int n, const mc_hparams* hp, voi
   for (size_t gi = 0; gi < L.groups.size(); ++gi)
     if ((rc = build_group_maps(L.groups[gi], ws, maps[gi])) != MC_OK) return rc;
 
-  // ---- Newton-Schulz iterations, MAX_GROUPS problem groups per launch
+  // ---- Newton-Schulz iterations, MAX_GROUPS problem groups per launch.
+  // Iterations it < kMixedIters take a*X from the fp32 iterate; later ones
+  // fold a*I into B (see the precision note in umma_gemm.cuh).
   const int ng = static_cast<int>(L.groups.size());
   for (int it = 0; it < hp->ns_steps; ++it) {
     const int par = it & 1;
     const bool first = it == 0, last = it + 1 == hp->ns_steps;
+    const bool mixed = it < kMixedIters;
     for (int g0 = 0; g0 < ng; g0 += MAX_GROUPS) {
       const int g1 = std::min(ng, g0 + MAX_GROUPS);
       GemmParams gram, poly, apply;
@@ -532,6 +537,7 @@ MC_API int mc_muon_step(const mc_param* params, int n, const mc_hparams* hp, voi
         G.d_bs = g.m * g.ldm;
         G.coef_acc = hp->c;
         G.coef_src = hp->b;
+        G.diag = mixed ? 0.f : hp->a;
         poly.map_a[slot] = Mp.a_k128;
         poly.map_b[slot] = Mp.a_k256;
         finish_group(poly, slot, G);
@@ -555,6 +561,8 @@ MC_API int mc_muon_step(const mc_param* params, int n, const mc_hparams* hp, voi
         G.xf = reinterpret_cast<float*>(ws + g.off_xf);
         G.xf_ld = g.ld;
         G.xf_bs = g.rows * g.ld;
+        G.xf_read = mixed ? 1 : 0;
+        G.xf_write = (!last && it + 1 < kMixedIters) ? 1 : 0;
         G.d = ws + g.off_xb[par ^ 1];
         G.d_ld = g.ld;
         G.d_bs = g.rows * g.ld;

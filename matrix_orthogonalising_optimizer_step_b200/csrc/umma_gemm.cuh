@@ -6,10 +6,18 @@
 //
 //   EPI_GRAM        A_k   = s^2 * X X^T            (symmetric: upper tiles only,
 //                                                  each element stored twice)
-//   EPI_POLY        B_k   = b*A + c*(A A)          (symmetric, mirrored store)
-//   EPI_APPLY       X_k+1 = s * (a*X + B X)        (fp32 iterate in place + bf16 copy)
+//   EPI_POLY        B_k   = b*A + c*(A A) [+ a*I]  (symmetric, mirrored store)
+//   EPI_APPLY       X_k+1 = s * (a*X + B X)        (fp32 iterate read/written in
+//                           or  P X, P = aI+bA+cA^2  place when flagged + bf16 copy)
 //   EPI_APPLY_FINAL W     = (1 - lr*wd) W - lr * rms * X_N   (last iteration; X_N
 //                                                  never touches memory)
+//
+// Precision: operands are bf16, accumulation fp32.  While singular values are
+// still small (the first two iterations) the a*X term is taken from an fp32
+// copy of the iterate, so only B X sees a rounded X; afterwards a*I is folded
+// into B, because once the singular values sit in the polynomial's band
+// |a + b s^2 + c s^4| (the factor on a rounded X in P X) is smaller than
+// |b s^2 + c s^4| (the factor in B X).
 //   EPI_STORE       plain bf16 store (Q/K projection)
 //   EPI_CAUSALMAX   per-head max over j <= i of the score tile (QK-Clip's S_max);
 //                   the score tile is never stored
@@ -73,6 +81,7 @@ struct GemmGroup {
   long long src_ld, src_bs;
   float* xf;               // fp32 iterate (EPI_APPLY*)
   long long xf_ld, xf_bs;
+  int xf_read, xf_write;   // EPI_APPLY*: take a*X from xf; store the new iterate to xf
   void* const* w_ptrs;     // per-problem weight (EPI_APPLY_FINAL), row-major M x N
   float* const* u_ptrs;    // per-problem update output, entries may be null
   const float* scale;      // per-problem s, or null for 1
@@ -81,6 +90,7 @@ struct GemmGroup {
   int mask_causal;         // EPI_CAUSALMAX
   int* keys;               // EPI_CAUSALMAX: order-preserving ints, one per head
   float coef_acc, coef_src;
+  float diag;              // EPI_POLY: added on the diagonal (a for P = aI + B)
   float decay, step, rms;  // EPI_APPLY_FINAL
   float out_scale;         // EPI_CAUSALMAX: 1/sqrt(d_head)
 };
@@ -241,33 +251,38 @@ __device__ __forceinline__ void epilogue_chunk(const GemmGroup& G, int prob, int
       for (int j = 0; j < 16; ++j) x[j] = (c0 + j < G.N) ? __bfloat162float(S[c0 + j]) : 0.f;
     }
 #pragma unroll
-    for (int j = 0; j < 16; ++j) v[j] = fmaf(G.coef_acc, v[j], G.coef_src * x[j]);
+    for (int j = 0; j < 16; ++j) v[j] = fmaf(G.coef_acc, v[j], G.coef_src * x[j]) + (c0 + j == r ? G.diag : 0.f);
     __nv_bfloat16* D = static_cast<__nv_bfloat16*>(G.d) + (long long)prob * G.d_bs;
     store_sym_chunk(D, G.d_ld, G.M, r, c0, v);
   } else if constexpr (EPI == EPI_APPLY || EPI == EPI_APPLY_FINAL) {
     if (r >= G.M) return;
     const float s = G.scale ? G.scale[G.prob_base + prob] : 1.f;
-    float* X = G.xf + (long long)prob * G.xf_bs + (long long)r * G.xf_ld;
-    float x[16];
-    if (full) {
-      load_f32x16(X + c0, x);
+    float* X = G.xf ? G.xf + (long long)prob * G.xf_bs + (long long)r * G.xf_ld : nullptr;
+    if (G.xf_read) {
+      float x[16];
+      if (full) {
+        load_f32x16(X + c0, x);
+      } else {
+#pragma unroll
+        for (int j = 0; j < 16; ++j) x[j] = (c0 + j < G.N) ? X[c0 + j] : 0.f;
+      }
+#pragma unroll
+      for (int j = 0; j < 16; ++j) v[j] = s * fmaf(G.coef_src, x[j], v[j]);
     } else {
 #pragma unroll
-      for (int j = 0; j < 16; ++j) x[j] = (c0 + j < G.N) ? X[c0 + j] : 0.f;
+      for (int j = 0; j < 16; ++j) v[j] *= s;
     }
-#pragma unroll
-    for (int j = 0; j < 16; ++j) v[j] = s * fmaf(G.coef_src, x[j], v[j]);
     if constexpr (EPI == EPI_APPLY) {
       __nv_bfloat16* D =
           static_cast<__nv_bfloat16*>(G.d) + (long long)prob * G.d_bs + (long long)r * G.d_ld;
       if (full) {
-        store_f32x16(X + c0, v);
+        if (G.xf_write) store_f32x16(X + c0, v);
         store_bf16x16(D + c0, v);
       } else {
 #pragma unroll
         for (int j = 0; j < 16; ++j)
           if (c0 + j < G.N) {
-            X[c0 + j] = v[j];
+            if (G.xf_write) X[c0 + j] = v[j];
             D[c0 + j] = __float2bfloat16_rn(v[j]);
           }
       }

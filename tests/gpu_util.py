@@ -53,10 +53,24 @@ def check_muon_matrix(W0, G, M0, W1, M1, U1, nrm, hp, oracle_out, tag=""):
         assert rel_fro(w1 - w0, w_exp - w0) <= EW_TOL, f"{tag} apply"
     else:
         ulp = np.spacing(np.abs(round_like(w_exp, torch.bfloat16)).astype(np.float32)).astype(np.float64) * 65536
+        # fp32 evaluation of (1 - lr wd) w + (-lr) u: a few fp32 roundings of
+        # the operands, which matter where the two terms nearly cancel
+        slack = 4 * 2.0 ** -24 * (np.abs(w0) + lr * np.abs(to64(U1)))
         err = np.abs(w1 - w_exp)
-        assert np.all(err <= ulp + 1e-12), f"{tag} apply beyond 1 bf16 ulp"
+        assert np.all(err <= ulp + slack), f"{tag} apply beyond 1 bf16 ulp: {np.max(err - ulp - slack)}"
         assert np.mean(w1 == round_like(w_exp, W0.dtype)) >= 0.999, f"{tag} apply rounding"
     # end to end against the oracle, both rounded into the weight's dtype
-    e_dw = rel_fro(w1 - w0, round_like(Wo, W0.dtype) - w0)
-    assert e_dw <= NS_TOL, f"{tag} dW rel err {e_dw}"
+    wo = round_like(Wo, W0.dtype)
+    e_dw = rel_fro(w1 - w0, wo - w0)
+    if W0.dtype == torch.float32:
+        assert e_dw <= NS_TOL, f"{tag} dW rel err {e_dw}"
+    else:
+        # Rounding W_new to bf16 quantises dW in steps of one ulp of W, about
+        # 1/30 of dW here.  On large matrices that noise averages out far below
+        # NS_TOL; on matrices of a few elements it does not, so there the bound
+        # is NS_TOL plus the relative size q of one ulp against dW.
+        ulp_o = np.spacing(np.abs(wo).astype(np.float32)).astype(np.float64) * 65536
+        q = float(np.sqrt(np.mean(ulp_o ** 2)) / max(np.sqrt(np.mean((wo - w0) ** 2)), 1e-30))
+        bound = NS_TOL if w1.size >= 10000 else NS_TOL + q
+        assert e_dw <= bound, f"{tag} dW rel err {e_dw} (bound {bound})"
     return e_upd, e_dw
