@@ -141,6 +141,33 @@ int mc_qk_max_logit(const void* x, const void* wq, const void* wk, int B, int S,
 int mc_qk_clip(void* wq, void* wk, int H, int dh, int D, const float* smax, float tau, float alpha,
                float* gamma_out, int32_t* mask_out, void* stream);
 
+/*
+ * mc_qk_max_logit_static -- the same S_max as mc_qk_max_logit, but without a
+ * workspace argument and without allocating anything.  The pages have no
+ * counterpart: this exists for callers that cannot call cudaMalloc, e.g. a
+ * process whose device memory is entirely owned by another allocator's
+ * pre-reserved pool (so a cudaMalloc would fail or fragment it), or a code
+ * path that must not risk the implicit device synchronisation a cudaMalloc
+ * or cudaFree may perform.
+ *
+ * The Q and K projections live in one file-scope device array of
+ * MC_QK_STATIC_SCRATCH_BYTES (64 MiB + 16 KiB) that every GPU which loads this
+ * library holds until the process exits.  Limits: B*S*H*dh <= MC_QK_STATIC_MAX_ELEMS
+ * (2^24) and H <= MC_QK_STATIC_MAX_HEADS (4096); larger problems return
+ * MC_ERR_NOSPC before anything is enqueued.  The first call on a device looks
+ * up that device's address of the array (cudaGetSymbolAddress) and caches it,
+ * so make that first call before any stream capture.  All calls share the one
+ * array and it keeps the last call's contents (each call resets what must
+ * start fresh), so calls that can overlap on the GPU -- on different streams,
+ * or from different threads -- race and must be ordered by the caller.
+ * Arguments, layouts and the other errors are as for mc_qk_max_logit.
+ */
+#define MC_QK_STATIC_MAX_ELEMS (1u << 24)
+#define MC_QK_STATIC_MAX_HEADS 4096
+#define MC_QK_STATIC_SCRATCH_BYTES (4ull * MC_QK_STATIC_MAX_ELEMS + 4ull * MC_QK_STATIC_MAX_HEADS)
+int mc_qk_max_logit_static(const void* x, const void* wq, const void* wk, int B, int S, int D, int H, int dh,
+                           int causal, float* smax_out, void* stream);
+
 /* Text of the last error returned on the calling thread ("" if none). */
 const char* mc_last_error(void);
 

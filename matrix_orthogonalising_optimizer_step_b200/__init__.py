@@ -22,7 +22,10 @@ MC_F32, MC_BF16 = 0, 1
 
 # Names the C ABI exports (include/muonclip.h).
 EXPORTS = ("mc_muon_workspace_size", "mc_muon_step", "mc_qk_workspace_size", "mc_qk_max_logit",
-           "mc_qk_clip", "mc_last_error", "mc_device_status", "mc_profile_begin", "mc_profile_end")
+           "mc_qk_clip", "mc_last_error", "mc_device_status", "mc_profile_begin", "mc_profile_end",
+           "mc_qk_max_logit_static")
+MC_QK_STATIC_MAX_ELEMS = 1 << 24
+MC_QK_STATIC_MAX_HEADS = 4096
 
 
 class McParam(ctypes.Structure):
@@ -78,6 +81,8 @@ def load_library():
     lib.mc_last_error.restype = ctypes.c_char_p
     lib.mc_device_status.argtypes = []
     lib.mc_device_status.restype = i32
+    lib.mc_qk_max_logit_static.argtypes = [vp, vp, vp, i32, i32, i32, i32, i32, i32, vp, vp]
+    lib.mc_qk_max_logit_static.restype = i32
     lib.mc_profile_begin.argtypes = []
     lib.mc_profile_begin.restype = i32
     lib.mc_profile_end.argtypes = [P(McKernelStat), i32, P(ctypes.c_int)]
@@ -277,3 +282,24 @@ def qk_clip(wq, wk, smax, H: int, dh: int, *, tau: float = 100.0, alpha: float =
     _check(lib.mc_qk_clip(_ptr(wq), _ptr(wk), H, dh, D, _ptr(smax), float(tau), float(alpha),
                           _ptr(gamma_out), _ptr(mask_out), _stream_handle(stream)))
     return gamma_out, mask_out
+
+
+def qk_max_logit_static(x, wq, wk, H: int, dh: int, *, causal: bool = True, smax_out=None, stream=None):
+    """S_max like ``qk_max_logit`` but through the allocation-free entry point
+    (``mc_qk_max_logit_static``): no workspace is passed or allocated by the
+    library; it uses its own fixed 64 MiB device scratch, limited to
+    B*S*H*dh <= 2**24 and H <= 4096.  Calls that may overlap on the GPU race
+    on that scratch.  (``smax_out`` is created here with torch if not given;
+    pass it in to keep the whole call allocation-free.)"""
+    torch = _torch()
+    lib = load_library()
+    for t, nm in ((x, "x"), (wq, "wq"), (wk, "wk")):
+        _need_cuda_contig(t, nm)
+        if t.dtype != torch.bfloat16:
+            raise TypeError(f"{nm} must be bfloat16")
+    B, S, D = x.shape
+    if smax_out is None:
+        smax_out = torch.empty(H, dtype=torch.float32, device=x.device)
+    _check(lib.mc_qk_max_logit_static(_ptr(x), _ptr(wq), _ptr(wk), B, S, D, H, dh, int(causal),
+                                      _ptr(smax_out), _stream_handle(stream)))
+    return smax_out

@@ -789,3 +789,122 @@ MC_API int mc_profile_end(mc_kernel_stat* out, int max_rows, int* rows) {
   if (rows) *rows = k;
   return rc;
 }
+
+// =========================================================================
+// Allocation-free S_max (mc_qk_max_logit_static).  Its Q/K scratch is this
+// file-scope device array; host code must not pass the array's name to a
+// kernel (on the host it is only a stand-in), so each device's address is
+// looked up once with cudaGetSymbolAddress while that device is current.
+static __device__ __align__(256) uint8_t g_qk_static_scratch[MC_QK_STATIC_SCRATCH_BYTES];
+
+namespace {
+constexpr int kMaxDevices = 64;
+void* g_qk_static_addr[kMaxDevices] = {};  // guarded by g_mu
+
+int qk_static_scratch(void** out) {
+  int dev = 0;
+  MC_CUDA(cudaGetDevice(&dev));
+  if (dev < 0 || dev >= kMaxDevices) return fail(MC_ERR_UNSUPPORTED, "device ordinal out of range");
+  if (!g_qk_static_addr[dev]) {
+    void* p = nullptr;
+    const cudaError_t e = cudaGetSymbolAddress(&p, g_qk_static_scratch);
+    if (e != cudaSuccess || !p)
+      return fail(MC_ERR_CUDA, std::string("cudaGetSymbolAddress of the static scratch failed: ") +
+                                   cudaGetErrorString(e));
+    g_qk_static_addr[dev] = p;
+  }
+  *out = g_qk_static_addr[dev];
+  return MC_OK;
+}
+
+template <int EPI>
+int launch_gemm_unprofiled(const GemmParams& p, int sms, cudaStream_t s) {
+  if (p.total_tiles <= 0) return MC_OK;
+  const long long grid = std::min<long long>(sms, p.total_tiles);
+  umma_gemm_kernel<EPI><<<static_cast<unsigned>(grid), GEMM_THREADS, GEMM_SMEM_BYTES, s>>>(p);
+  MC_CUDA(cudaGetLastError());
+  return MC_OK;
+}
+}  // namespace
+
+MC_API int mc_qk_max_logit_static(const void* x, const void* wq, const void* wk, int B, int S, int D, int H,
+                                  int dh, int causal, float* smax_out, void* stream) {
+  int rc = validate_qk_dims(B, S, D, H, dh);
+  if (rc != MC_OK) return rc;
+  if (!x || !wq || !wk || !smax_out) return fail(MC_ERR_INVAL, "NULL x, wq, wk or smax_out");
+  if (!aligned16(x) || !aligned16(wq) || !aligned16(wk) || !aligned16(smax_out))
+    return fail(MC_ERR_ALIGN, "pointers must be 16-byte aligned");
+  const uint64_t elems = uint64_t(B) * uint64_t(S) * uint64_t(H) * uint64_t(dh);
+  if (elems > MC_QK_STATIC_MAX_ELEMS)
+    return fail(MC_ERR_NOSPC, "B*S*H*dh = " + std::to_string(elems) + " exceeds the static scratch limit of " +
+                                  std::to_string(MC_QK_STATIC_MAX_ELEMS) + " elements; use mc_qk_max_logit");
+  if (H > MC_QK_STATIC_MAX_HEADS)
+    return fail(MC_ERR_NOSPC, "H = " + std::to_string(H) + " exceeds the static scratch limit of " +
+                                  std::to_string(MC_QK_STATIC_MAX_HEADS) + " heads");
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  std::lock_guard<std::mutex> lock(g_mu);
+  DeviceState* st = nullptr;
+  if ((rc = device_state(&st)) != MC_OK) return rc;
+  void* scratch = nullptr;
+  if ((rc = qk_static_scratch(&scratch)) != MC_OK) return rc;
+  uint8_t* base = static_cast<uint8_t*>(scratch);
+  uint8_t* q = base;
+  uint8_t* k = base + 2ull * MC_QK_STATIC_MAX_ELEMS;
+  int* keys = reinterpret_cast<int*>(base + 4ull * MC_QK_STATIC_MAX_ELEMS);
+  const int HD = H * dh;
+  const int64_t BS = int64_t(B) * S;
+
+  // The keys carry the previous call's maxima: reset them first.
+  qk_keys_init_kernel<<<(H + 255) / 256, 256, 0, s>>>(keys, H);
+  MC_CUDA(cudaGetLastError());
+
+  GemmParams proj;
+  std::memset(&proj, 0, sizeof(proj));
+  proj.err = st->err_ptr;
+  for (int which = 0; which < 2; ++which) {
+    if ((rc = map_batched(&proj.map_a[which], x, 1, BS, D, D, 128)) != MC_OK) return rc;
+    if ((rc = map_batched(&proj.map_b[which], which == 0 ? wq : wk, 1, HD, D, D, 256)) != MC_OK) return rc;
+    GemmGroup G;
+    std::memset(&G, 0, sizeof(G));
+    G.M = static_cast<int>(BS);
+    G.N = HD;
+    G.K = D;
+    G.count = 1;
+    G.sched = SCHED_DENSE;
+    G.layout = LAYOUT_BATCHED;
+    G.heads = 1;
+    G.band = 8;
+    G.d = which == 0 ? q : k;
+    G.d_ld = HD;
+    finish_group(proj, which, G);
+  }
+  if ((rc = launch_gemm_unprofiled<EPI_STORE>(proj, st->sms, s)) != MC_OK) return rc;
+
+  GemmParams cm;
+  std::memset(&cm, 0, sizeof(cm));
+  cm.err = st->err_ptr;
+  const uint64_t dims[4] = {uint64_t(dh), uint64_t(H), uint64_t(S), uint64_t(B)};
+  const uint64_t strides[3] = {uint64_t(dh) * 2, uint64_t(HD) * 2, uint64_t(S) * uint64_t(HD) * 2};
+  const uint32_t box_q[4] = {64, 1, 128, 1};
+  const uint32_t box_k[4] = {64, 1, 256, 1};
+  if ((rc = make_map(&cm.map_a[0], q, 4, dims, strides, box_q)) != MC_OK) return rc;
+  if ((rc = make_map(&cm.map_b[0], k, 4, dims, strides, box_k)) != MC_OK) return rc;
+  GemmGroup G;
+  std::memset(&G, 0, sizeof(G));
+  G.M = G.N = S;
+  G.K = dh;
+  G.count = B * H;
+  G.heads = H;
+  G.layout = LAYOUT_HEADS;
+  G.sched = causal ? SCHED_CAUSAL : SCHED_DENSE;
+  G.band = 8;
+  G.mask_causal = causal ? 1 : 0;
+  G.keys = keys;
+  G.out_scale = 1.f / std::sqrt(static_cast<float>(dh));
+  finish_group(cm, 0, G);
+  if ((rc = launch_gemm_unprofiled<EPI_CAUSALMAX>(cm, st->sms, s)) != MC_OK) return rc;
+
+  qk_keys_decode_kernel<<<(H + 255) / 256, 256, 0, s>>>(keys, smax_out, H);
+  MC_CUDA(cudaGetLastError());
+  return MC_OK;
+}
