@@ -62,6 +62,7 @@ constexpr int kMixedIters = 2;
 struct DeviceState {
   bool init = false;
   int sms = 0;
+  int pair_clusters = 0;  // CTA pairs of the GEMM kernel that fit on the device at once
   int cc_major = 0, cc_minor = 0;
   int* err_ptr = nullptr;
   void* own_ws = nullptr;
@@ -106,6 +107,23 @@ int device_state(DeviceState** out) {
     MC_CUDA(set_gemm_attr<EPI_APPLY_FINAL>());
     MC_CUDA(set_gemm_attr<EPI_STORE>());
     MC_CUDA(set_gemm_attr<EPI_CAUSALMAX>());
+    {
+      cudaLaunchConfig_t cfg = {};
+      cudaLaunchAttribute attr[1];
+      attr[0].id = cudaLaunchAttributeClusterDimension;
+      attr[0].val.clusterDim.x = 2;
+      attr[0].val.clusterDim.y = 1;
+      attr[0].val.clusterDim.z = 1;
+      cfg.gridDim = dim3(static_cast<unsigned>(st.sms & ~1));
+      cfg.blockDim = dim3(GEMM_THREADS);
+      cfg.dynamicSmemBytes = GEMM_SMEM_BYTES;
+      cfg.attrs = attr;
+      cfg.numAttrs = 1;
+      int clusters = 0;
+      MC_CUDA(cudaOccupancyMaxActiveClusters(&clusters, umma_gemm_kernel<EPI_APPLY>, &cfg));
+      if (clusters < 1) return fail(MC_ERR_UNSUPPORTED, "no CTA pair of the GEMM kernel fits on this device");
+      st.pair_clusters = clusters;
+    }
     if (!g_encode) {
       void* fn = nullptr;
       cudaDriverEntryPointQueryResult q;
@@ -234,13 +252,31 @@ double gemm_exec_flops(const GemmParams& p) {
   return f;
 }
 
+// Persistent launch in clusters of two CTAs (one 2-SM MMA pair each), as
+// many pairs as fit on the device at once, at most one per tile.
 template <int EPI>
-int launch_gemm(const GemmParams& p, int sms, cudaStream_t s, int kind, double flops) {
+cudaError_t launch_pairs(const GemmParams& p, int pair_clusters, cudaStream_t s) {
+  const long long pairs = std::min<long long>(pair_clusters, p.total_tiles);
+  cudaLaunchConfig_t cfg = {};
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = 2;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.gridDim = dim3(static_cast<unsigned>(2 * pairs));
+  cfg.blockDim = dim3(GEMM_THREADS);
+  cfg.dynamicSmemBytes = GEMM_SMEM_BYTES;
+  cfg.stream = s;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, umma_gemm_kernel<EPI>, p);
+}
+
+template <int EPI>
+int launch_gemm(const GemmParams& p, const DeviceState& st, cudaStream_t s, int kind, double flops) {
   if (p.total_tiles <= 0) return MC_OK;
-  const long long grid = std::min<long long>(sms, p.total_tiles);
   ProfScope prof(kind, s, flops, gemm_exec_flops(p));
-  umma_gemm_kernel<EPI><<<static_cast<unsigned>(grid), GEMM_THREADS, GEMM_SMEM_BYTES, s>>>(p);
-  MC_CUDA(cudaGetLastError());
+  MC_CUDA(launch_pairs<EPI>(p, st.pair_clusters, s));
   return MC_OK;
 }
 
@@ -368,8 +404,10 @@ void plan_muon(const mc_param* params, int n, MuonLayout& L) {
   L.total = std::max<size_t>(off, 1024);
 }
 
+// K-major maps use 128-row boxes (each CTA of a pair stages 128 rows of an
+// operand); MN-major maps use {64, 64} boxes.
 struct GroupMaps {
-  CUtensorMap x_k128[2], x_k256[2], x_mn[2], a_k128, a_k256, b_k128, b_k256;
+  CUtensorMap x_k[2], x_mn[2], a_k, b_k;
 };
 
 int build_group_maps(const NsGroup& g, uint8_t* ws, GroupMaps& M) {
@@ -377,15 +415,12 @@ int build_group_maps(const NsGroup& g, uint8_t* ws, GroupMaps& M) {
   for (int par = 0; par < 2; ++par) {
     const void* xb = ws + g.off_xb[par];
     int rc;
-    if ((rc = map_batched(&M.x_k128[par], xb, cnt, g.rows, g.cols, g.ld, 128)) != MC_OK) return rc;
-    if ((rc = map_batched(&M.x_k256[par], xb, cnt, g.rows, g.cols, g.ld, 256)) != MC_OK) return rc;
+    if ((rc = map_batched(&M.x_k[par], xb, cnt, g.rows, g.cols, g.ld, HALF)) != MC_OK) return rc;
     if ((rc = map_batched(&M.x_mn[par], xb, cnt, g.rows, g.cols, g.ld, 64)) != MC_OK) return rc;
   }
   int rc;
-  if ((rc = map_batched(&M.a_k128, ws + g.off_a, cnt, g.m, g.m, g.ldm, 128)) != MC_OK) return rc;
-  if ((rc = map_batched(&M.a_k256, ws + g.off_a, cnt, g.m, g.m, g.ldm, 256)) != MC_OK) return rc;
-  if ((rc = map_batched(&M.b_k128, ws + g.off_b, cnt, g.m, g.m, g.ldm, 128)) != MC_OK) return rc;
-  if ((rc = map_batched(&M.b_k256, ws + g.off_b, cnt, g.m, g.m, g.ldm, 256)) != MC_OK) return rc;
+  if ((rc = map_batched(&M.a_k, ws + g.off_a, cnt, g.m, g.m, g.ldm, HALF)) != MC_OK) return rc;
+  if ((rc = map_batched(&M.b_k, ws + g.off_b, cnt, g.m, g.m, g.ldm, HALF)) != MC_OK) return rc;
   return MC_OK;
 }
 
@@ -522,8 +557,8 @@ MC_API int mc_muon_step(const mc_param* params, int n, const mc_hparams* hp, voi
         G.d_ld = g.ldm;
         G.d_bs = g.m * g.ldm;
         G.scale = first ? scale : nullptr;
-        gram.map_a[slot] = g.tall ? Mp.x_mn[par] : Mp.x_k128[par];
-        gram.map_b[slot] = g.tall ? Mp.x_mn[par] : Mp.x_k256[par];
+        gram.map_a[slot] = g.tall ? Mp.x_mn[par] : Mp.x_k[par];
+        gram.map_b[slot] = g.tall ? Mp.x_mn[par] : Mp.x_k[par];
         finish_group(gram, slot, G);
         // B = b A + c A A
         G = base_group(g);
@@ -538,8 +573,8 @@ MC_API int mc_muon_step(const mc_param* params, int n, const mc_hparams* hp, voi
         G.coef_acc = hp->c;
         G.coef_src = hp->b;
         G.diag = mixed ? 0.f : hp->a;
-        poly.map_a[slot] = Mp.a_k128;
-        poly.map_b[slot] = Mp.a_k256;
+        poly.map_a[slot] = Mp.a_k;
+        poly.map_b[slot] = Mp.a_k;
         finish_group(poly, slot, G);
         // X' = s (a X + B X)   (tall: s (a X + X B), in the stored layout)
         G = base_group(g);
@@ -550,12 +585,12 @@ MC_API int mc_muon_step(const mc_param* params, int n, const mc_hparams* hp, voi
         if (g.tall) {
           G.a_mn = 0;
           G.b_mn = 0;
-          apply.map_a[slot] = Mp.x_k128[par];
-          apply.map_b[slot] = Mp.b_k256;
+          apply.map_a[slot] = Mp.x_k[par];
+          apply.map_b[slot] = Mp.b_k;
         } else {
           G.a_mn = 0;
           G.b_mn = 1;
-          apply.map_a[slot] = Mp.b_k128;
+          apply.map_a[slot] = Mp.b_k;
           apply.map_b[slot] = Mp.x_mn[par];
         }
         G.xf = reinterpret_cast<float*>(ws + g.off_xf);
@@ -581,12 +616,12 @@ MC_API int mc_muon_step(const mc_param* params, int n, const mc_hparams* hp, voi
         }
         finish_group(apply, slot, G);
       }
-      if ((rc = launch_gemm<EPI_GRAM>(gram, st->sms, s, K_GRAM, f_gram)) != MC_OK) return rc;
-      if ((rc = launch_gemm<EPI_POLY>(poly, st->sms, s, K_POLY, f_poly)) != MC_OK) return rc;
+      if ((rc = launch_gemm<EPI_GRAM>(gram, *st, s, K_GRAM, f_gram)) != MC_OK) return rc;
+      if ((rc = launch_gemm<EPI_POLY>(poly, *st, s, K_POLY, f_poly)) != MC_OK) return rc;
       if (last) {
-        if ((rc = launch_gemm<EPI_APPLY_FINAL>(apply, st->sms, s, K_APPLY_FINAL, f_apply)) != MC_OK) return rc;
+        if ((rc = launch_gemm<EPI_APPLY_FINAL>(apply, *st, s, K_APPLY_FINAL, f_apply)) != MC_OK) return rc;
       } else {
-        if ((rc = launch_gemm<EPI_APPLY>(apply, st->sms, s, K_APPLY, f_apply)) != MC_OK) return rc;
+        if ((rc = launch_gemm<EPI_APPLY>(apply, *st, s, K_APPLY, f_apply)) != MC_OK) return rc;
       }
     }
   }
@@ -657,8 +692,8 @@ MC_API int mc_qk_max_logit(const void* x, const void* wq, const void* wk, int B,
   std::memset(&proj, 0, sizeof(proj));
   proj.err = st->err_ptr;
   for (int which = 0; which < 2; ++which) {
-    if ((rc = map_batched(&proj.map_a[which], x, 1, BS, D, D, 128)) != MC_OK) return rc;
-    if ((rc = map_batched(&proj.map_b[which], which == 0 ? wq : wk, 1, HD, D, D, 256)) != MC_OK) return rc;
+    if ((rc = map_batched(&proj.map_a[which], x, 1, BS, D, D, HALF)) != MC_OK) return rc;
+    if ((rc = map_batched(&proj.map_b[which], which == 0 ? wq : wk, 1, HD, D, D, HALF)) != MC_OK) return rc;
     GemmGroup G;
     std::memset(&G, 0, sizeof(G));
     G.M = static_cast<int>(BS);
@@ -673,7 +708,7 @@ MC_API int mc_qk_max_logit(const void* x, const void* wq, const void* wk, int B,
     G.d_ld = HD;
     finish_group(proj, which, G);
   }
-  if ((rc = launch_gemm<EPI_STORE>(proj, st->sms, s, K_QK_PROJ, 2.0 * 2.0 * double(BS) * HD * D)) != MC_OK)
+  if ((rc = launch_gemm<EPI_STORE>(proj, *st, s, K_QK_PROJ, 2.0 * 2.0 * double(BS) * HD * D)) != MC_OK)
     return rc;
 
   // Per-head causal max of Q K^T / sqrt(dh), scores never stored.
@@ -683,8 +718,8 @@ MC_API int mc_qk_max_logit(const void* x, const void* wq, const void* wk, int B,
   {
     const uint64_t dims[4] = {uint64_t(dh), uint64_t(H), uint64_t(S), uint64_t(B)};
     const uint64_t strides[3] = {uint64_t(dh) * 2, uint64_t(HD) * 2, uint64_t(S) * uint64_t(HD) * 2};
-    const uint32_t box_q[4] = {64, 1, 128, 1};
-    const uint32_t box_k[4] = {64, 1, 256, 1};
+    const uint32_t box_q[4] = {64, 1, HALF, 1};
+    const uint32_t box_k[4] = {64, 1, HALF, 1};
     if ((rc = make_map(&cm.map_a[0], ws + L.off_q, 4, dims, strides, box_q)) != MC_OK) return rc;
     if ((rc = make_map(&cm.map_b[0], ws + L.off_k, 4, dims, strides, box_k)) != MC_OK) return rc;
     GemmGroup G;
@@ -702,7 +737,7 @@ MC_API int mc_qk_max_logit(const void* x, const void* wq, const void* wk, int B,
     finish_group(cm, 0, G);
   }
   const double pairs = causal ? double(S) * (double(S) + 1) / 2 : double(S) * S;
-  if ((rc = launch_gemm<EPI_CAUSALMAX>(cm, st->sms, s, K_QK_CMAX, 2.0 * dh * pairs * B * H)) != MC_OK) return rc;
+  if ((rc = launch_gemm<EPI_CAUSALMAX>(cm, *st, s, K_QK_CMAX, 2.0 * dh * pairs * B * H)) != MC_OK) return rc;
   {
     ProfScope prof(K_QK_KEYS, s);
     qk_keys_decode_kernel<<<(H + 255) / 256, 256, 0, s>>>(keys, smax_out, H);
@@ -818,11 +853,9 @@ int qk_static_scratch(void** out) {
 }
 
 template <int EPI>
-int launch_gemm_unprofiled(const GemmParams& p, int sms, cudaStream_t s) {
+int launch_gemm_unprofiled(const GemmParams& p, const DeviceState& st, cudaStream_t s) {
   if (p.total_tiles <= 0) return MC_OK;
-  const long long grid = std::min<long long>(sms, p.total_tiles);
-  umma_gemm_kernel<EPI><<<static_cast<unsigned>(grid), GEMM_THREADS, GEMM_SMEM_BYTES, s>>>(p);
-  MC_CUDA(cudaGetLastError());
+  MC_CUDA(launch_pairs<EPI>(p, st.pair_clusters, s));
   return MC_OK;
 }
 }  // namespace
@@ -862,8 +895,8 @@ MC_API int mc_qk_max_logit_static(const void* x, const void* wq, const void* wk,
   std::memset(&proj, 0, sizeof(proj));
   proj.err = st->err_ptr;
   for (int which = 0; which < 2; ++which) {
-    if ((rc = map_batched(&proj.map_a[which], x, 1, BS, D, D, 128)) != MC_OK) return rc;
-    if ((rc = map_batched(&proj.map_b[which], which == 0 ? wq : wk, 1, HD, D, D, 256)) != MC_OK) return rc;
+    if ((rc = map_batched(&proj.map_a[which], x, 1, BS, D, D, HALF)) != MC_OK) return rc;
+    if ((rc = map_batched(&proj.map_b[which], which == 0 ? wq : wk, 1, HD, D, D, HALF)) != MC_OK) return rc;
     GemmGroup G;
     std::memset(&G, 0, sizeof(G));
     G.M = static_cast<int>(BS);
@@ -878,15 +911,15 @@ MC_API int mc_qk_max_logit_static(const void* x, const void* wq, const void* wk,
     G.d_ld = HD;
     finish_group(proj, which, G);
   }
-  if ((rc = launch_gemm_unprofiled<EPI_STORE>(proj, st->sms, s)) != MC_OK) return rc;
+  if ((rc = launch_gemm_unprofiled<EPI_STORE>(proj, *st, s)) != MC_OK) return rc;
 
   GemmParams cm;
   std::memset(&cm, 0, sizeof(cm));
   cm.err = st->err_ptr;
   const uint64_t dims[4] = {uint64_t(dh), uint64_t(H), uint64_t(S), uint64_t(B)};
   const uint64_t strides[3] = {uint64_t(dh) * 2, uint64_t(HD) * 2, uint64_t(S) * uint64_t(HD) * 2};
-  const uint32_t box_q[4] = {64, 1, 128, 1};
-  const uint32_t box_k[4] = {64, 1, 256, 1};
+  const uint32_t box_q[4] = {64, 1, HALF, 1};
+  const uint32_t box_k[4] = {64, 1, HALF, 1};
   if ((rc = make_map(&cm.map_a[0], q, 4, dims, strides, box_q)) != MC_OK) return rc;
   if ((rc = make_map(&cm.map_b[0], k, 4, dims, strides, box_k)) != MC_OK) return rc;
   GemmGroup G;
@@ -902,7 +935,7 @@ MC_API int mc_qk_max_logit_static(const void* x, const void* wq, const void* wk,
   G.keys = keys;
   G.out_scale = 1.f / std::sqrt(static_cast<float>(dh));
   finish_group(cm, 0, G);
-  if ((rc = launch_gemm_unprofiled<EPI_CAUSALMAX>(cm, st->sms, s)) != MC_OK) return rc;
+  if ((rc = launch_gemm_unprofiled<EPI_CAUSALMAX>(cm, *st, s)) != MC_OK) return rc;
 
   qk_keys_decode_kernel<<<(H + 255) / 256, 256, 0, s>>>(keys, smax_out, H);
   MC_CUDA(cudaGetLastError());

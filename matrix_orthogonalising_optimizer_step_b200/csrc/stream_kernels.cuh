@@ -53,6 +53,30 @@ __device__ __forceinline__ void load_g8(const void* g, long long idx, int g_f32,
   }
 }
 
+__device__ __forceinline__ void momentum8(const float (&g)[8], float4 ma, float4 mb, float mu, int nesterov,
+                                          float* m_out, float* xf_out, __nv_bfloat16* xb_out, double& acc) {
+  float m[8] = {ma.x, ma.y, ma.z, ma.w, mb.x, mb.y, mb.z, mb.w};
+  float u[8];
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    m[i] = fmaf(mu, m[i], g[i]);
+    u[i] = nesterov ? fmaf(mu, m[i], g[i]) : m[i];
+    acc += static_cast<double>(u[i]) * static_cast<double>(u[i]);
+  }
+  float4* mp = reinterpret_cast<float4*>(m_out);
+  mp[0] = make_float4(m[0], m[1], m[2], m[3]);
+  mp[1] = make_float4(m[4], m[5], m[6], m[7]);
+  float4* xp = reinterpret_cast<float4*>(xf_out);
+  xp[0] = make_float4(u[0], u[1], u[2], u[3]);
+  xp[1] = make_float4(u[4], u[5], u[6], u[7]);
+  uint4 b;
+  b.x = pack_bf16x2(u[0], u[1]);
+  b.y = pack_bf16x2(u[2], u[3]);
+  b.z = pack_bf16x2(u[4], u[5]);
+  b.w = pack_bf16x2(u[6], u[7]);
+  *reinterpret_cast<uint4*>(xb_out) = b;
+}
+
 __global__ void __launch_bounds__(MOM_THREADS) momentum_kernel(const MomEntry* __restrict__ tab, int n,
                                                                double* __restrict__ partials, float mu,
                                                                int nesterov) {
@@ -63,49 +87,49 @@ __global__ void __launch_bounds__(MOM_THREADS) momentum_kernel(const MomEntry* _
     const int mid = (lo + hi + 1) >> 1;
     if (tab[mid].cta_begin <= cta) lo = mid; else hi = mid - 1;
   }
-  const MomEntry e = tab[lo];
-  const long long total = e.rows * e.cols;
-  const long long e0 = (cta - e.cta_begin) * MOM_ELEMS_PER_CTA;
+  const MomEntry* e = tab + lo;
+  const void* gp = e->g;
+  float* mp = e->m;
+  float* xf = e->xf;
+  __nv_bfloat16* xb = e->xb;
+  const long long cols = e->cols, ld = e->ld;
+  const long long total = e->rows * cols;
+  const int g_f32 = e->g_f32;
+  const long long e0 = (cta - e->cta_begin) * MOM_ELEMS_PER_CTA;
   const long long e1 = (e0 + MOM_ELEMS_PER_CTA < total) ? e0 + MOM_ELEMS_PER_CTA : total;
   double acc = 0.0;
-  if (e.vec) {
-#pragma unroll 2
-    for (long long idx = e0 + threadIdx.x * 8; idx < e1; idx += MOM_THREADS * 8) {
-      float g[8];
-      load_g8(e.g, idx, e.g_f32, g);
-      float4* mp = reinterpret_cast<float4*>(e.m + idx);
-      float4 ma = mp[0], mb = mp[1];
-      float m[8] = {ma.x, ma.y, ma.z, ma.w, mb.x, mb.y, mb.z, mb.w};
-      float u[8];
-#pragma unroll
-      for (int i = 0; i < 8; ++i) {
-        m[i] = fmaf(mu, m[i], g[i]);
-        u[i] = nesterov ? fmaf(mu, m[i], g[i]) : m[i];
-        acc += static_cast<double>(u[i]) * static_cast<double>(u[i]);
+  if (e->vec) {
+    // Two groups of 8 elements per thread in flight: both groups' loads are
+    // issued before either is used.
+    constexpr long long STEP = MOM_THREADS * 8;
+    for (long long idx = e0 + threadIdx.x * 8; idx < e1; idx += 2 * STEP) {
+      const long long j = idx + STEP;
+      const bool two = j < e1;
+      float g0[8], g1[8];
+      load_g8(gp, idx, g_f32, g0);
+      const float4* m0p = reinterpret_cast<const float4*>(mp + idx);
+      const float4 m0a = m0p[0], m0b = m0p[1];
+      float4 m1a = make_float4(0.f, 0.f, 0.f, 0.f), m1b = m1a;
+      if (two) {
+        load_g8(gp, j, g_f32, g1);
+        const float4* m1p = reinterpret_cast<const float4*>(mp + j);
+        m1a = m1p[0];
+        m1b = m1p[1];
       }
-      mp[0] = make_float4(m[0], m[1], m[2], m[3]);
-      mp[1] = make_float4(m[4], m[5], m[6], m[7]);
-      float4* xp = reinterpret_cast<float4*>(e.xf + idx);
-      xp[0] = make_float4(u[0], u[1], u[2], u[3]);
-      xp[1] = make_float4(u[4], u[5], u[6], u[7]);
-      uint4 b;
-      b.x = pack_bf16x2(u[0], u[1]);
-      b.y = pack_bf16x2(u[2], u[3]);
-      b.z = pack_bf16x2(u[4], u[5]);
-      b.w = pack_bf16x2(u[6], u[7]);
-      *reinterpret_cast<uint4*>(e.xb + idx) = b;
+      momentum8(g0, m0a, m0b, mu, nesterov, mp + idx, xf + idx, xb + idx, acc);
+      if (two) momentum8(g1, m1a, m1b, mu, nesterov, mp + j, xf + j, xb + j, acc);
     }
   } else {
     for (long long idx = e0 + threadIdx.x; idx < e1; idx += MOM_THREADS) {
-      const float g = e.g_f32 ? static_cast<const float*>(e.g)[idx]
-                              : __bfloat162float(static_cast<const __nv_bfloat16*>(e.g)[idx]);
-      const float m = fmaf(mu, e.m[idx], g);
-      e.m[idx] = m;
+      const float g = g_f32 ? static_cast<const float*>(gp)[idx]
+                            : __bfloat162float(static_cast<const __nv_bfloat16*>(gp)[idx]);
+      const float m = fmaf(mu, mp[idx], g);
+      mp[idx] = m;
       const float u = nesterov ? fmaf(mu, m, g) : m;
       acc += static_cast<double>(u) * static_cast<double>(u);
-      const long long row = idx / e.cols, col = idx - row * e.cols;
-      e.xf[row * e.ld + col] = u;
-      e.xb[row * e.ld + col] = __float2bfloat16_rn(u);
+      const long long row = idx / cols, col = idx - row * cols;
+      xf[row * ld + col] = u;
+      xb[row * ld + col] = __float2bfloat16_rn(u);
     }
   }
   // Fixed-order block reduction (deterministic).

@@ -27,25 +27,37 @@
 // X = aX + (bA + cA A)X) and "MuonClip: speed, then stability", §02; the apply
 // is §03's W <- W - eta (O + lambda W) with O scaled by 0.2 sqrt(max(m, n)).
 //
-// Warp roles (320 threads, one CTA per SM):
-//   warp 0      TMA producer: 4-stage ring of {A 128x64, B 256x64} bf16 tiles,
-//               128-byte swizzled, K-major or MN-major per group.
-//   warp 1      TMEM allocator + single-thread tcgen05.mma issuer (M=128, N=256,
-//               K=16 per instruction), commits to the ring and the accumulators.
+// Execution: CTA pairs (clusters of 2, one CTA per SM) run 2-SM tensor-core
+// MMAs (tcgen05 cta_group::2): a 256 x 256 output tile per pair, of which each
+// CTA holds 128 rows in its own TMEM.  Each CTA stages its 128 rows of A and
+// its 128 rows of B (the pair's B is split between the two SMs), so an SM
+// pulls 32 KB per 512 tensor-core cycles instead of the 48 KB a one-SM
+// 128 x 256 tile needs.  No TMA multicast is used.
+//
+// Warp roles (320 threads per CTA):
+//   warp 0      TMA producer: 6-stage ring of {A 128x64, B 128x64} bf16 tiles,
+//               128-byte swizzled, K-major or MN-major per group.  Both CTAs'
+//               copies complete on the leader CTA's "full" barrier.
+//   warp 1      TMEM allocation (both CTAs, 2-SM form); in the leader CTA one
+//               thread issues tcgen05.mma (M=256, N=256, K=16) and commits to
+//               both CTAs' "empty" and "accumulator full" barriers.
 //   warps 2-9   epilogue: two accumulator buffers (2 x 256 TMEM columns) so the
 //               next tile's MMAs overlap this tile's epilogue.  Warp w reads TMEM
-//               lanes 32*(w%4)..+31 and column half (w-2)/4.
+//               lanes 32*(w%4)..+31 and column half (w-2)/4; the leader's
+//               "accumulator empty" barrier counts both CTAs' epilogue warps.
 #pragma once
 
 #include "ptx.cuh"
 
 namespace mc {
 
-constexpr int BM = 128, BN = 256, BK = 64, STAGES = 4;
-constexpr uint32_t A_STAGE_BYTES = BM * BK * 2;   // 16 KiB
-constexpr uint32_t B_STAGE_BYTES = BN * BK * 2;   // 32 KiB
+constexpr int BM = 256, BN = 256, BK = 64, STAGES = 6;
+constexpr int HALF = 128;                               // rows of A and of B per CTA
+constexpr uint32_t A_STAGE_BYTES = HALF * BK * 2;       // 16 KiB
+constexpr uint32_t B_STAGE_BYTES = HALF * BK * 2;       // 16 KiB
 constexpr uint32_t STAGE_BYTES = A_STAGE_BYTES + B_STAGE_BYTES;
-constexpr uint32_t MN_BOX_BYTES = 64 * BK * 2;    // one {64 MN, 64 K} box: 8 KiB
+constexpr uint32_t PAIR_STAGE_BYTES = 2 * STAGE_BYTES;  // what the leader's full barrier expects
+constexpr uint32_t MN_BOX_BYTES = 64 * BK * 2;          // one {64 MN, 64 K} box: 8 KiB
 constexpr int NUM_EPI_WARPS = 8;
 constexpr int GEMM_THREADS = 64 + NUM_EPI_WARPS * 32;
 constexpr uint32_t TMEM_COLS = 2 * BN;
@@ -106,12 +118,11 @@ struct GemmParams {
 static_assert(sizeof(GemmParams) <= 4096, "kernel parameters must fit the classic 4 KiB limit");
 
 // ------------------------------------------------------------------ tiling
-// Tiles (i, j) of 128 rows x 256 columns.  SYM keeps the tiles that touch
-// the upper triangle (j >= floor(i/2)); CAUSAL keeps those that touch the
-// lower triangle including the diagonal (j <= floor(i/2)).
+// Tiles (i, j) of 256 x 256.  SYM keeps the tiles on or above the diagonal
+// (j >= i); CAUSAL keeps those on or below it (j <= i).
 __host__ __device__ inline long long sched_row_count(int sched, int i, int tiles_n) {
-  if (sched == SCHED_SYM) return tiles_n - i / 2;
-  if (sched == SCHED_CAUSAL) return (i / 2 + 1) < tiles_n ? (i / 2 + 1) : tiles_n;
+  if (sched == SCHED_SYM) return tiles_n - i;
+  if (sched == SCHED_CAUSAL) return (i + 1) < tiles_n ? (i + 1) : tiles_n;
   return tiles_n;
 }
 __host__ __device__ inline long long sched_tiles_per_prob(int sched, int tiles_m, int tiles_n) {
@@ -152,7 +163,7 @@ __host__ __device__ inline void decode_tile(const GemmGroup* groups, int num_gro
       ++i;
     }
     tm = i;
-    tn = (G.sched == SCHED_SYM ? i / 2 : 0) + (int)tl;
+    tn = (G.sched == SCHED_SYM ? i : 0) + (int)tl;
   }
   ti.g = g;
   ti.prob = (int)prob;
@@ -359,16 +370,18 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1) umma_gemm_kernel(const __grid
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + STAGES * STAGE_BYTES);
-  uint64_t* full_bar = bars;                    // [STAGES]
-  uint64_t* empty_bar = bars + STAGES;          // [STAGES]
-  uint64_t* tfull_bar = bars + 2 * STAGES;      // [2]
-  uint64_t* tempty_bar = bars + 2 * STAGES + 2; // [2]
-  uint64_t* drain_bar = bars + 2 * STAGES + 4;  // [1]
+  uint64_t* full_bar = bars;                    // [STAGES]  used in the leader only
+  uint64_t* empty_bar = bars + STAGES;          // [STAGES]  every CTA
+  uint64_t* tfull_bar = bars + 2 * STAGES;      // [2]       every CTA
+  uint64_t* tempty_bar = bars + 2 * STAGES + 2; // [2]       used in the leader only
+  uint64_t* drain_bar = bars + 2 * STAGES + 4;  // [1]       leader
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2 * STAGES + 5);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
+  const uint32_t rank = cluster_ctarank();   // 0 = leader (issues the MMAs)
+  const bool leader = rank == 0;
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < STAGES; ++s) {
@@ -377,7 +390,7 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1) umma_gemm_kernel(const __grid
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(smem_u32(&tfull_bar[b]), 1);
-      mbar_init(smem_u32(&tempty_bar[b]), NUM_EPI_WARPS);
+      mbar_init(smem_u32(&tempty_bar[b]), 2 * NUM_EPI_WARPS);
     }
     mbar_init(smem_u32(drain_bar), 1);
     *abort_flag = 0;
@@ -390,58 +403,64 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1) umma_gemm_kernel(const __grid
     }
   }
   if (warp == 1) {
-    tmem_alloc(smem_u32(tmem_slot), TMEM_COLS);
-    tmem_relinquish();
+    tmem_alloc_pair(smem_u32(tmem_slot), TMEM_COLS);
+    tmem_relinquish_pair();
   }
   tc_fence_before();
-  __syncthreads();
+  cluster_sync();   // barriers initialised and TMEM allocated in both CTAs
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
   const long long total = P.total_tiles;
+  const long long first_tile = blockIdx.x >> 1;
+  const long long tile_step = gridDim.x >> 1;
 
   if (warp == 0) {
     // ------------------------------------------------------- TMA producer
     if (lane == 0) {
       int stage = 0;
       uint32_t phase = 0;
-      uint32_t filled = 0;          // bit s: stage s was ever filled
-      uint32_t fill_parity = 0;     // bit s: parity of its latest fill
+      uint32_t filled = 0;          // leader: bit s set once stage s was filled
+      uint32_t fill_parity = 0;     // leader: parity of stage s's latest fill
       bool ok = true;
-      for (long long t = blockIdx.x; ok && t < total; t += gridDim.x) {
+      for (long long t = first_tile; ok && t < total; t += tile_step) {
         TileInfo ti;
         decode_tile(P.g, P.num_groups, t, ti);
         const GemmGroup& G = P.g[ti.g];
         const CUtensorMap* ma = &P.map_a[ti.g];
         const CUtensorMap* mb = &P.map_b[ti.g];
-        const int m0 = ti.tm * BM, n0 = ti.tn * BN;
+        const int m0 = ti.tm * BM + HALF * static_cast<int>(rank);
+        const int n0 = ti.tn * BN + HALF * static_cast<int>(rank);
         for (int kb = 0; kb < ti.num_kb; ++kb) {
           if (!wait_bounded(smem_u32(&empty_bar[stage]), phase ^ 1, abort_flag, P.err)) {
             ok = false;
             break;
           }
-          const uint32_t fb = smem_u32(&full_bar[stage]);
-          mbar_arrive_expect_tx(fb, STAGE_BYTES);
-          filled |= 1u << stage;
-          fill_parity = (fill_parity & ~(1u << stage)) | (phase << stage);
+          const uint32_t fb_local = smem_u32(&full_bar[stage]);
+          if (leader) {
+            mbar_arrive_expect_tx(fb_local, PAIR_STAGE_BYTES);
+            filled |= 1u << stage;
+            fill_parity = (fill_parity & ~(1u << stage)) | (phase << stage);
+          }
+          const uint32_t fb = mapa_shared(fb_local, 0);
           const uint32_t sa = smem_u32(smem + stage * STAGE_BYTES);
           const uint32_t sb = sa + A_STAGE_BYTES;
           const int k0 = kb * BK;
           if (G.layout == LAYOUT_HEADS) {
             const int bb = ti.prob / G.heads, hh = ti.prob % G.heads;
-            tma_load_4d(sa, ma, fb, k0, hh, m0, bb);
-            tma_load_4d(sb, mb, fb, k0, hh, n0, bb);
+            tma_load_4d_pair(sa, ma, fb, k0, hh, m0, bb);
+            tma_load_4d_pair(sb, mb, fb, k0, hh, n0, bb);
           } else {
             if (!G.a_mn) {
-              tma_load_3d(sa, ma, fb, k0, m0, ti.prob);
+              tma_load_3d_pair(sa, ma, fb, k0, m0, ti.prob);
             } else {
-              tma_load_3d(sa, ma, fb, m0, k0, ti.prob);
-              tma_load_3d(sa + MN_BOX_BYTES, ma, fb, m0 + 64, k0, ti.prob);
+              tma_load_3d_pair(sa, ma, fb, m0, k0, ti.prob);
+              tma_load_3d_pair(sa + MN_BOX_BYTES, ma, fb, m0 + 64, k0, ti.prob);
             }
             if (!G.b_mn) {
-              tma_load_3d(sb, mb, fb, k0, n0, ti.prob);
+              tma_load_3d_pair(sb, mb, fb, k0, n0, ti.prob);
             } else {
-#pragma unroll
-              for (int q = 0; q < 4; ++q) tma_load_3d(sb + q * MN_BOX_BYTES, mb, fb, n0 + 64 * q, k0, ti.prob);
+              tma_load_3d_pair(sb, mb, fb, n0, k0, ti.prob);
+              tma_load_3d_pair(sb + MN_BOX_BYTES, mb, fb, n0 + 64, k0, ti.prob);
             }
           }
           if (++stage == STAGES) {
@@ -450,23 +469,24 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1) umma_gemm_kernel(const __grid
           }
         }
       }
-      // Do not leave while a copy may still be landing in shared memory.
-      for (int s = 0; s < STAGES; ++s)
-        if (filled & (1u << s)) {
-          volatile int no_abort = 0;
-          wait_bounded(smem_u32(&full_bar[s]), (fill_parity >> s) & 1u, &no_abort, nullptr,
-                       kDrainLimitCycles);
-        }
+      // The leader's full barriers count both CTAs' copies: wait for every
+      // copy of the pair to land before anyone leaves.
+      if (leader)
+        for (int s = 0; s < STAGES; ++s)
+          if (filled & (1u << s)) {
+            volatile int no_abort = 0;
+            wait_bounded(smem_u32(&full_bar[s]), (fill_parity >> s) & 1u, &no_abort, nullptr, kDrainLimitCycles);
+          }
     }
   } else if (warp == 1) {
-    // ------------------------------------------------------- MMA issuer
-    if (lane == 0) {
+    // ------------------------------------------------------- MMA issuer (leader)
+    if (leader && lane == 0) {
       int stage = 0;
       uint32_t phase = 0;
       int acc = 0;
       uint32_t acc_phase = 0;
       bool ok = true;
-      for (long long t = blockIdx.x; ok && t < total; t += gridDim.x) {
+      for (long long t = first_tile; ok && t < total; t += tile_step) {
         TileInfo ti;
         decode_tile(P.g, P.num_groups, t, ti);
         const GemmGroup& G = P.g[ti.g];
@@ -481,33 +501,39 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1) umma_gemm_kernel(const __grid
         }
         tc_fence_after();
         const uint32_t d_tmem = tmem_base + acc * BN;
+        // Descriptors of stage 0; stage s and k-step kk only move the start
+        // address field (address >> 4 in the low 14 bits, no carry out of it
+        // since shared memory ends below 2^18).
+        const uint32_t s0 = smem_u32(smem);
+        const uint64_t ad0 = smem_desc_sw128(s0, a_lbo, 1024);
+        const uint64_t bd0 = smem_desc_sw128(s0 + A_STAGE_BYTES, b_lbo, 1024);
         for (int kb = 0; kb < ti.num_kb; ++kb) {
+          // The TMA writes are made visible by the barrier's complete_tx; the
+          // MMAs read them through the same async proxy.
           if (!wait_bounded(smem_u32(&full_bar[stage]), phase, abort_flag, P.err)) {
             ok = false;
             break;
           }
-          tc_fence_after();
-          const uint32_t sa = smem_u32(smem + stage * STAGE_BYTES);
-          const uint32_t sb = sa + A_STAGE_BYTES;
+          const uint64_t soff = static_cast<uint64_t>((stage * STAGE_BYTES) >> 4);
 #pragma unroll
           for (int kk = 0; kk < BK / 16; ++kk) {
-            const uint64_t ad = smem_desc_sw128(sa + kk * a_kstep, a_lbo, 1024);
-            const uint64_t bd = smem_desc_sw128(sb + kk * b_kstep, b_lbo, 1024);
-            umma_bf16(d_tmem, ad, bd, idesc, (kb | kk) != 0);
+            const uint64_t ad = ad0 + soff + ((kk * a_kstep) >> 4);
+            const uint64_t bd = bd0 + soff + ((kk * b_kstep) >> 4);
+            umma_bf16_pair(d_tmem, ad, bd, idesc, (kb | kk) != 0);
           }
-          umma_commit(smem_u32(&empty_bar[stage]));
+          umma_commit_pair_mc(smem_u32(&empty_bar[stage]), 0x3);
           if (++stage == STAGES) {
             stage = 0;
             phase ^= 1;
           }
         }
         if (!ok) break;
-        umma_commit(smem_u32(&tfull_bar[acc]));
+        umma_commit_pair_mc(smem_u32(&tfull_bar[acc]), 0x3);
         acc ^= 1;
         if (acc == 0) acc_phase ^= 1;
       }
-      // All MMAs issued by this thread complete before TMEM is released.
-      umma_commit(smem_u32(drain_bar));
+      // Every MMA of the pair completes before TMEM is released.
+      umma_commit_pair(smem_u32(drain_bar));
       volatile int no_abort = 0;
       wait_bounded(smem_u32(drain_bar), 0, &no_abort, nullptr, kDrainLimitCycles);
     }
@@ -515,9 +541,11 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1) umma_gemm_kernel(const __grid
     // ------------------------------------------------------- epilogue
     const int q = warp & 3;            // TMEM lane quarter this warp may read
     const int half = (warp - 2) >> 2;  // column half of the 256-wide tile
+    const uint32_t tempty_leader0 = mapa_shared(smem_u32(&tempty_bar[0]), 0);
+    const uint32_t tempty_leader1 = mapa_shared(smem_u32(&tempty_bar[1]), 0);
     int acc = 0;
     uint32_t acc_phase = 0;
-    for (long long t = blockIdx.x; t < total; t += gridDim.x) {
+    for (long long t = first_tile; t < total; t += tile_step) {
       TileInfo ti;
       decode_tile(P.g, P.num_groups, t, ti);
       const GemmGroup& G = P.g[ti.g];
@@ -527,7 +555,7 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1) umma_gemm_kernel(const __grid
       const bool ok = wait_bounded(smem_u32(&tfull_bar[acc]), acc_phase, abort_flag, P.err);
       if (!__all_sync(0xffffffffu, ok)) break;
       tc_fence_after();
-      const int r = ti.tm * BM + q * 32 + lane;
+      const int r = ti.tm * BM + HALF * static_cast<int>(rank) + q * 32 + lane;
       const uint32_t t_row = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + acc * BN + half * 128;
       float run_max = -INFINITY;
 #pragma unroll 1
@@ -539,7 +567,7 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1) umma_gemm_kernel(const __grid
       }
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(smem_u32(&tempty_bar[acc]));
+      if (lane == 0) mbar_arrive_cluster(acc ? tempty_leader1 : tempty_leader0);
       if constexpr (EPI == EPI_CAUSALMAX) {
 #pragma unroll
         for (int o = 16; o > 0; o >>= 1) run_max = fmaxf(run_max, __shfl_xor_sync(0xffffffffu, run_max, o));
@@ -553,12 +581,15 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1) umma_gemm_kernel(const __grid
     }
   }
 
+  // Nobody leaves (or frees TMEM) while the peer may still signal this CTA's
+  // barriers or read its shared memory.
   tc_fence_before();
   __syncthreads();
+  cluster_sync();
   if (warp == 1) {
     __syncwarp();
     tc_fence_after();
-    tmem_dealloc(tmem_base, TMEM_COLS);
+    tmem_dealloc_pair(tmem_base, TMEM_COLS);
   }
 }
 

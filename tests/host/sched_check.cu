@@ -1,4 +1,4 @@
-// Host-only check of the GEMM tile scheduler in umma_gemm.cuh: enumerates every
+// Host-only check of the GEMM tile scheduler in umma_gemm.cuh (256 x 256 tiles): enumerates every
 // global tile index through decode_tile() and verifies coverage and uniqueness
 // for the dense (band raster), symmetric-upper and causal schedules, over
 // ragged sizes and multi-group launches.  Prints "OK" on success.
@@ -37,9 +37,9 @@ static void check_groups(std::vector<GemmGroup> gs) {
     auto key = std::make_tuple(ti.prob, ti.tm, ti.tn);
     CHECK(!seen[ti.g].count(key), "duplicate tile");
     seen[ti.g].insert(key);
-    if (G.sched == SCHED_SYM) CHECK(ti.tn >= ti.tm / 2, "sym tile below diagonal");
+    if (G.sched == SCHED_SYM) CHECK(ti.tn >= ti.tm, "sym tile below diagonal");
     if (G.sched == SCHED_CAUSAL) {
-      CHECK(ti.tn <= ti.tm / 2, "causal tile above diagonal");
+      CHECK(ti.tn <= ti.tm, "causal tile above diagonal");
       CHECK((long long)ti.tn * BN <= (long long)ti.tm * BM + BM - 1, "causal tile with no valid element");
     }
   }
@@ -79,10 +79,12 @@ int main() {
   check_groups({mk(4096, 14336, 4096, 2, SCHED_DENSE, 8), mk(14336, 4096, 4096, 1, SCHED_DENSE, 8),
                 mk(1024, 1024, 1024, 5, SCHED_DENSE, 8)});
   // the 7B-shaped symmetric launch size
+  // 16 x 16 tiles of 256: the upper (or lower) triangle with its diagonal
   GemmGroup a = mk(4096, 4096, 4096, 128, SCHED_SYM, 8);
-  CHECK(a.tiles_per_prob == 32 * 16 - (0 + 0 + 1 + 1 + 2 + 2 + 3 + 3 + 4 + 4 + 5 + 5 + 6 + 6 + 7 + 7 + 8 + 8 + 9 + 9 + 10 + 10 + 11 + 11 + 12 + 12 + 13 + 13 + 14 + 14 + 15 + 15), "sym count");
+  CHECK(a.tiles_per_prob == 136, "sym count %lld", a.tiles_per_prob);
   GemmGroup c = mk(4096, 4096, 128, 128, SCHED_CAUSAL, 8);
-  CHECK(c.tiles_per_prob == 272, "causal count %lld", c.tiles_per_prob);
+  CHECK(c.tiles_per_prob == 136, "causal count %lld", c.tiles_per_prob);
+  CHECK(BM == 256 && BN == 256, "tile shape");
   if (fails) { std::printf("FAILED %d checks\n", fails); return 1; }
   std::printf("OK\n");
   return 0;
