@@ -36,8 +36,8 @@ WORKLOAD = ("7B-shaped Muon step (224 matrices, 7.78e9 params, bf16 W/G, fp32 M,
 # DRAM bytes per launch (dram__bytes_read.sum + dram__bytes_write.sum) of the
 # kernels as they stand, from one ncu capture: profiles/ns_gemm_1layer_full.md
 # (1-layer case, third NS iteration, scaled by the 32 layers processed at full
-# size).  None where no capture of the current kernel exists.
-KERNEL_TRAFFIC_BYTES = {"ns_apply": 51.9e9}
+# size).  Kinds without a capture of the current kernel report null.
+KERNEL_TRAFFIC_BYTES = {"ns_gram": 35.9e9, "ns_apply": 55.4e9}
 
 
 def parse_args(argv=None):
@@ -283,7 +283,7 @@ def main(argv=None):
 
     # --- per-kernel figures from the CUDA events around each launch
     K = args.steps
-    ns_kinds = ("ns_gram", "ns_poly", "ns_apply", "ns_apply_final")
+    ns_kinds = ("ns_gram", "ns_poly", "ns_apply_mixed", "ns_apply", "ns_apply_final")
     muon_kinds = ("momentum", "norm_finalize") + ns_kinds
     per = {k: dict(v, ms_per_launch=v["total_ms"] / max(v["launches"], 1)) for k, v in kernels.items()}
     ns_ms = sum(kernels[k]["total_ms"] for k in ns_kinds if k in kernels) / K

@@ -187,13 +187,18 @@ int mc_device_status(void);
  *   momentum        bytes = the momentum kernel's DRAM traffic by design:
  *                   G (2 or 4) + M read/write (8) + fp32 and bf16 iterate (6)
  *                   bytes per element
- *   ns_gram, ns_poly, ns_apply, ns_apply_final
- *                   flops = dense-equivalent Newton-Schulz FLOPs of that phase,
- *                   2 m^2 n, 2 m^3, 2 m^2 n (their sum per iteration is the
+ *   ns_gram         A = X X^T: flops = m (m+1) n (the entries on and above the
+ *                   diagonal, 2n each), flops_dense_equiv = 2 m^2 n
+ *   ns_poly         B = bA + cA^2: flops = m^2 (m+1), flops_dense_equiv = 2 m^3
+ *   ns_apply_mixed  X <- s(aX + BX), iterations that read the fp32 iterate
+ *   ns_apply        X <- (aI + B) X, later iterations
+ *   ns_apply_final  last iteration fused with the weight update
+ *                   (apply rows: flops = flops_dense_equiv = 2 m^2 n.  Per
+ *                   iteration the dense-equivalent figures add up to the
  *                   2(2nm^2 + m^3) of "Muon and MuonClip: orthogonalised updates
- *                   for LLM training", §2); flops_executed = 2*128*256*K_padded
- *                   per tile the tensor cores actually ran (symmetric phases
- *                   skip about half of the tiles)
+ *                   for LLM training", §2.)
+ *                   flops_executed = 2*256*N_tile*K_padded per tile the tensor
+ *                   cores actually ran
  *   qk_proj         flops = 2 * B*S * H*dh * D * 2 (Q and K)
  *   qk_causal_max   flops = 2 * dh * (score pairs inside the causal mask)
  *   norm_finalize, qk_keys, qk_clip   (small kernels; counted, no work figure)
@@ -207,6 +212,7 @@ typedef struct {
   double total_ms;
   double flops;
   double flops_executed;
+  double flops_dense_equiv;
   double bytes;
 } mc_kernel_stat;
 

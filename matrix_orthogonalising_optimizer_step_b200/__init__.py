@@ -44,7 +44,8 @@ class McHparams(ctypes.Structure):
 
 class McKernelStat(ctypes.Structure):
     _fields_ = [("name", ctypes.c_char * 32), ("launches", ctypes.c_int32), ("total_ms", ctypes.c_double),
-                ("flops", ctypes.c_double), ("flops_executed", ctypes.c_double), ("bytes", ctypes.c_double)]
+                ("flops", ctypes.c_double), ("flops_executed", ctypes.c_double),
+                ("flops_dense_equiv", ctypes.c_double), ("bytes", ctypes.c_double)]
 
 
 class MuonClipError(RuntimeError):
@@ -113,7 +114,7 @@ def profile_begin() -> None:
 
 def profile_end() -> dict:
     """Stop profiling; returns {kernel kind: {launches, total_ms, flops,
-    flops_executed, bytes}} of device time and algorithmic work."""
+    flops_executed, flops_dense_equiv, bytes}} of device time and work."""
     lib = load_library()
     rows = (McKernelStat * 32)()
     n = ctypes.c_int(0)
@@ -122,7 +123,8 @@ def profile_end() -> dict:
     for i in range(min(n.value, 32)):
         r = rows[i]
         out[r.name.decode()] = dict(launches=int(r.launches), total_ms=float(r.total_ms), flops=float(r.flops),
-                                    flops_executed=float(r.flops_executed), bytes=float(r.bytes))
+                                    flops_executed=float(r.flops_executed),
+                                    flops_dense_equiv=float(r.flops_dense_equiv), bytes=float(r.bytes))
     return out
 
 

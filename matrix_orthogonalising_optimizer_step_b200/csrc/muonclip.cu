@@ -81,10 +81,10 @@ inline size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 inline int64_t round8(int64_t x) { return (x + 7) / 8 * 8; }
 inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
-template <int EPI>
+template <int EPI, int WIDE>
 cudaError_t set_gemm_attr() {
-  return cudaFuncSetAttribute(umma_gemm_kernel<EPI>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                              static_cast<int>(GEMM_SMEM_BYTES));
+  return cudaFuncSetAttribute(umma_gemm_kernel<EPI, WIDE>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                              static_cast<int>(TileCfg<WIDE>::SMEM_BYTES));
 }
 
 // Caller holds g_mu.
@@ -101,12 +101,14 @@ int device_state(DeviceState** out) {
                                           std::to_string(st.cc_major) + "." + std::to_string(st.cc_minor) +
                                           "; this library is built for sm_100a (B200)");
     MC_CUDA(cudaGetSymbolAddress(reinterpret_cast<void**>(&st.err_ptr), g_device_error));
-    MC_CUDA(set_gemm_attr<EPI_GRAM>());
-    MC_CUDA(set_gemm_attr<EPI_POLY>());
-    MC_CUDA(set_gemm_attr<EPI_APPLY>());
-    MC_CUDA(set_gemm_attr<EPI_APPLY_FINAL>());
-    MC_CUDA(set_gemm_attr<EPI_STORE>());
-    MC_CUDA(set_gemm_attr<EPI_CAUSALMAX>());
+    MC_CUDA((set_gemm_attr<EPI_GRAM, 1>()));
+    MC_CUDA((set_gemm_attr<EPI_POLY, 1>()));
+    MC_CUDA((set_gemm_attr<EPI_APPLY, 0>()));
+    MC_CUDA((set_gemm_attr<EPI_APPLY, 1>()));
+    MC_CUDA((set_gemm_attr<EPI_APPLY_FINAL, 0>()));
+    MC_CUDA((set_gemm_attr<EPI_APPLY_FINAL, 1>()));
+    MC_CUDA((set_gemm_attr<EPI_STORE, 1>()));
+    MC_CUDA((set_gemm_attr<EPI_CAUSALMAX, 0>()));
     {
       cudaLaunchConfig_t cfg = {};
       cudaLaunchAttribute attr[1];
@@ -120,7 +122,7 @@ int device_state(DeviceState** out) {
       cfg.attrs = attr;
       cfg.numAttrs = 1;
       int clusters = 0;
-      MC_CUDA(cudaOccupancyMaxActiveClusters(&clusters, umma_gemm_kernel<EPI_APPLY>, &cfg));
+      MC_CUDA(cudaOccupancyMaxActiveClusters(&clusters, umma_gemm_kernel<EPI_APPLY, 0>, &cfg));
       if (clusters < 1) return fail(MC_ERR_UNSUPPORTED, "no CTA pair of the GEMM kernel fits on this device");
       st.pair_clusters = clusters;
     }
@@ -205,14 +207,15 @@ int map_batched(CUtensorMap* map, const void* base, int64_t count, int64_t rows,
 }
 
 // ----------------------------------------------------------- profiling
-enum Kind : int { K_MOMENTUM, K_FINALIZE, K_GRAM, K_POLY, K_APPLY, K_APPLY_FINAL, K_QK_PROJ, K_QK_CMAX,
-                  K_QK_KEYS, K_QK_CLIP, K_COUNT };
-const char* const kKindNames[K_COUNT] = {"momentum", "norm_finalize", "ns_gram", "ns_poly", "ns_apply",
-                                         "ns_apply_final", "qk_proj", "qk_causal_max", "qk_keys", "qk_clip"};
+enum Kind : int { K_MOMENTUM, K_FINALIZE, K_GRAM, K_POLY, K_APPLY_MIXED, K_APPLY, K_APPLY_FINAL, K_QK_PROJ,
+                  K_QK_CMAX, K_QK_KEYS, K_QK_CLIP, K_COUNT };
+const char* const kKindNames[K_COUNT] = {"momentum",  "norm_finalize",  "ns_gram", "ns_poly",
+                                         "ns_apply_mixed", "ns_apply", "ns_apply_final", "qk_proj",
+                                         "qk_causal_max", "qk_keys", "qk_clip"};
 struct ProfRec {
   int kind;
   cudaEvent_t b, e;
-  double flops, flops_exec, bytes;
+  double flops, flops_exec, flops_dense, bytes;
 };
 thread_local bool t_prof = false;
 thread_local std::vector<ProfRec> t_recs;
@@ -222,11 +225,13 @@ struct ProfScope {
   bool on = false;
   ProfRec r{};
   cudaStream_t s;
-  ProfScope(int kind, cudaStream_t st, double flops = 0, double flops_exec = 0, double bytes = 0) : s(st) {
+  ProfScope(int kind, cudaStream_t st, double flops = 0, double flops_exec = 0, double bytes = 0,
+            double flops_dense = -1) : s(st) {
     if (!t_prof) return;
     r.kind = kind;
     r.flops = flops;
     r.flops_exec = flops_exec;
+    r.flops_dense = flops_dense < 0 ? flops : flops_dense;
     r.bytes = bytes;
     if (cudaEventCreate(&r.b) != cudaSuccess) return;
     if (cudaEventCreate(&r.e) != cudaSuccess) {
@@ -247,14 +252,14 @@ double gemm_exec_flops(const GemmParams& p) {
   for (int i = 0; i < p.num_groups; ++i) {
     const GemmGroup& G = p.g[i];
     const double kpad = double((G.K + BK - 1) / BK) * BK;
-    f += double(G.tiles_per_prob) * G.count * 2.0 * BM * BN * kpad;
+    f += double(G.tiles_per_prob) * G.count * 2.0 * BM * double(MMA_N << G.nshift) * kpad;
   }
   return f;
 }
 
 // Persistent launch in clusters of two CTAs (one 2-SM MMA pair each), as
 // many pairs as fit on the device at once, at most one per tile.
-template <int EPI>
+template <int EPI, int WIDE>
 cudaError_t launch_pairs(const GemmParams& p, int pair_clusters, cudaStream_t s) {
   const long long pairs = std::min<long long>(pair_clusters, p.total_tiles);
   cudaLaunchConfig_t cfg = {};
@@ -265,25 +270,29 @@ cudaError_t launch_pairs(const GemmParams& p, int pair_clusters, cudaStream_t s)
   attr[0].val.clusterDim.z = 1;
   cfg.gridDim = dim3(static_cast<unsigned>(2 * pairs));
   cfg.blockDim = dim3(GEMM_THREADS);
-  cfg.dynamicSmemBytes = GEMM_SMEM_BYTES;
+  cfg.dynamicSmemBytes = TileCfg<WIDE>::SMEM_BYTES;
   cfg.stream = s;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, umma_gemm_kernel<EPI>, p);
+  return cudaLaunchKernelEx(&cfg, umma_gemm_kernel<EPI, WIDE>, p);
 }
 
-template <int EPI>
-int launch_gemm(const GemmParams& p, const DeviceState& st, cudaStream_t s, int kind, double flops) {
+template <int EPI, int WIDE>
+int launch_gemm(const GemmParams& p, const DeviceState& st, cudaStream_t s, int kind, double flops,
+                double flops_dense = -1) {
   if (p.total_tiles <= 0) return MC_OK;
-  ProfScope prof(kind, s, flops, gemm_exec_flops(p));
-  MC_CUDA(launch_pairs<EPI>(p, st.pair_clusters, s));
+  ProfScope prof(kind, s, flops, gemm_exec_flops(p), 0, flops_dense);
+  MC_CUDA((launch_pairs<EPI, WIDE>(p, st.pair_clusters, s)));
   return MC_OK;
 }
 
-void finish_group(GemmParams& p, int gi, GemmGroup& G) {
+// `wide`: 1 for 256 x 512 tiles (TileCfg<1>), 0 for 256 x 256.
+void finish_group(GemmParams& p, int gi, GemmGroup& G, int wide) {
+  const int tile_n = MMA_N << wide;
+  G.nshift = wide;
   G.tiles_m = (G.M + BM - 1) / BM;
-  G.tiles_n = (G.N + BN - 1) / BN;
-  G.tiles_per_prob = sched_tiles_per_prob(G.sched, G.tiles_m, G.tiles_n);
+  G.tiles_n = (G.N + tile_n - 1) / tile_n;
+  G.tiles_per_prob = sched_tiles_per_prob(G.sched, G.tiles_m, G.tiles_n, G.nshift);
   G.tile_start = p.total_tiles;
   if (G.band <= 0) G.band = 8;
   p.total_tiles += G.tiles_per_prob * G.count;
@@ -534,7 +543,7 @@ MC_API int mc_muon_step(const mc_param* params, int n, const mc_hparams* hp, voi
     for (int g0 = 0; g0 < ng; g0 += MAX_GROUPS) {
       const int g1 = std::min(ng, g0 + MAX_GROUPS);
       GemmParams gram, poly, apply;
-      double f_gram = 0, f_poly = 0, f_apply = 0;
+      double f_gram = 0, f_poly = 0, f_apply = 0, fd_gram = 0, fd_poly = 0;
       std::memset(&gram, 0, sizeof(gram));
       std::memset(&poly, 0, sizeof(poly));
       std::memset(&apply, 0, sizeof(apply));
@@ -544,8 +553,10 @@ MC_API int mc_muon_step(const mc_param* params, int n, const mc_hparams* hp, voi
         const NsGroup& g = L.groups[gi];
         const GroupMaps& Mp = maps[gi];
         const double cnt = double(g.members.size()), dm = double(g.m), dn = double(g.n);
-        f_gram += 2.0 * dm * dm * dn * cnt;
-        f_poly += 2.0 * dm * dm * dm * cnt;
+        f_gram += dm * (dm + 1) * dn * cnt;  // symmetric: entries on and above the diagonal
+        fd_gram += 2.0 * dm * dm * dn * cnt;
+        f_poly += dm * dm * (dm + 1) * cnt;
+        fd_poly += 2.0 * dm * dm * dm * cnt;
         f_apply += 2.0 * dm * dm * dn * cnt;
         // A = s^2 X X^T  (oriented; tall matrices read MN-major: X^T X)
         GemmGroup G = base_group(g);
@@ -559,7 +570,7 @@ MC_API int mc_muon_step(const mc_param* params, int n, const mc_hparams* hp, voi
         G.scale = first ? scale : nullptr;
         gram.map_a[slot] = g.tall ? Mp.x_mn[par] : Mp.x_k[par];
         gram.map_b[slot] = g.tall ? Mp.x_mn[par] : Mp.x_k[par];
-        finish_group(gram, slot, G);
+        finish_group(gram, slot, G, 1);
         // B = b A + c A A
         G = base_group(g);
         G.M = G.N = G.K = static_cast<int>(g.m);
@@ -575,7 +586,7 @@ MC_API int mc_muon_step(const mc_param* params, int n, const mc_hparams* hp, voi
         G.diag = mixed ? 0.f : hp->a;
         poly.map_a[slot] = Mp.a_k;
         poly.map_b[slot] = Mp.a_k;
-        finish_group(poly, slot, G);
+        finish_group(poly, slot, G, 1);
         // X' = s (a X + B X)   (tall: s (a X + X B), in the stored layout)
         G = base_group(g);
         G.M = static_cast<int>(g.rows);
@@ -614,15 +625,20 @@ MC_API int mc_muon_step(const mc_param* params, int n, const mc_hparams* hp, voi
           G.decay = 1.f - hp->lr * hp->wd;
           G.step = -hp->lr * G.rms;
         }
-        finish_group(apply, slot, G);
+        finish_group(apply, slot, G, mixed ? 0 : 1);
       }
-      if ((rc = launch_gemm<EPI_GRAM>(gram, *st, s, K_GRAM, f_gram)) != MC_OK) return rc;
-      if ((rc = launch_gemm<EPI_POLY>(poly, *st, s, K_POLY, f_poly)) != MC_OK) return rc;
+      // Wide 256 x 512 tiles where the epilogue is light; the iterations whose
+      // apply reads and writes the fp32 iterate keep the double-buffered tile.
+      if ((rc = launch_gemm<EPI_GRAM, 1>(gram, *st, s, K_GRAM, f_gram, fd_gram)) != MC_OK) return rc;
+      if ((rc = launch_gemm<EPI_POLY, 1>(poly, *st, s, K_POLY, f_poly, fd_poly)) != MC_OK) return rc;
       if (last) {
-        if ((rc = launch_gemm<EPI_APPLY_FINAL>(apply, *st, s, K_APPLY_FINAL, f_apply)) != MC_OK) return rc;
+        rc = mixed ? launch_gemm<EPI_APPLY_FINAL, 0>(apply, *st, s, K_APPLY_FINAL, f_apply)
+                   : launch_gemm<EPI_APPLY_FINAL, 1>(apply, *st, s, K_APPLY_FINAL, f_apply);
       } else {
-        if ((rc = launch_gemm<EPI_APPLY>(apply, *st, s, K_APPLY, f_apply)) != MC_OK) return rc;
+        rc = mixed ? launch_gemm<EPI_APPLY, 0>(apply, *st, s, K_APPLY_MIXED, f_apply)
+                   : launch_gemm<EPI_APPLY, 1>(apply, *st, s, K_APPLY, f_apply);
       }
+      if (rc != MC_OK) return rc;
     }
   }
   return MC_OK;
@@ -706,9 +722,9 @@ MC_API int mc_qk_max_logit(const void* x, const void* wq, const void* wk, int B,
     G.band = 8;
     G.d = ws + (which == 0 ? L.off_q : L.off_k);
     G.d_ld = HD;
-    finish_group(proj, which, G);
+    finish_group(proj, which, G, 1);
   }
-  if ((rc = launch_gemm<EPI_STORE>(proj, *st, s, K_QK_PROJ, 2.0 * 2.0 * double(BS) * HD * D)) != MC_OK)
+  if ((rc = launch_gemm<EPI_STORE, 1>(proj, *st, s, K_QK_PROJ, 2.0 * 2.0 * double(BS) * HD * D)) != MC_OK)
     return rc;
 
   // Per-head causal max of Q K^T / sqrt(dh), scores never stored.
@@ -734,10 +750,10 @@ MC_API int mc_qk_max_logit(const void* x, const void* wq, const void* wk, int B,
     G.mask_causal = causal ? 1 : 0;
     G.keys = keys;
     G.out_scale = 1.f / std::sqrt(static_cast<float>(dh));
-    finish_group(cm, 0, G);
+    finish_group(cm, 0, G, 0);
   }
   const double pairs = causal ? double(S) * (double(S) + 1) / 2 : double(S) * S;
-  if ((rc = launch_gemm<EPI_CAUSALMAX>(cm, *st, s, K_QK_CMAX, 2.0 * dh * pairs * B * H)) != MC_OK) return rc;
+  if ((rc = launch_gemm<EPI_CAUSALMAX, 0>(cm, *st, s, K_QK_CMAX, 2.0 * dh * pairs * B * H)) != MC_OK) return rc;
   {
     ProfScope prof(K_QK_KEYS, s);
     qk_keys_decode_kernel<<<(H + 255) / 256, 256, 0, s>>>(keys, smax_out, H);
@@ -807,6 +823,7 @@ MC_API int mc_profile_end(mc_kernel_stat* out, int max_rows, int* rows) {
     a.total_ms += ms;
     a.flops += r.flops;
     a.flops_executed += r.flops_exec;
+    a.flops_dense_equiv += r.flops_dense;
     a.bytes += r.bytes;
     cudaEventDestroy(r.b);
     cudaEventDestroy(r.e);
@@ -852,10 +869,10 @@ int qk_static_scratch(void** out) {
   return MC_OK;
 }
 
-template <int EPI>
+template <int EPI, int WIDE>
 int launch_gemm_unprofiled(const GemmParams& p, const DeviceState& st, cudaStream_t s) {
   if (p.total_tiles <= 0) return MC_OK;
-  MC_CUDA(launch_pairs<EPI>(p, st.pair_clusters, s));
+  MC_CUDA((launch_pairs<EPI, WIDE>(p, st.pair_clusters, s)));
   return MC_OK;
 }
 }  // namespace
@@ -909,9 +926,9 @@ MC_API int mc_qk_max_logit_static(const void* x, const void* wq, const void* wk,
     G.band = 8;
     G.d = which == 0 ? q : k;
     G.d_ld = HD;
-    finish_group(proj, which, G);
+    finish_group(proj, which, G, 1);
   }
-  if ((rc = launch_gemm_unprofiled<EPI_STORE>(proj, *st, s)) != MC_OK) return rc;
+  if ((rc = launch_gemm_unprofiled<EPI_STORE, 1>(proj, *st, s)) != MC_OK) return rc;
 
   GemmParams cm;
   std::memset(&cm, 0, sizeof(cm));
@@ -934,8 +951,8 @@ MC_API int mc_qk_max_logit_static(const void* x, const void* wq, const void* wk,
   G.mask_causal = causal ? 1 : 0;
   G.keys = keys;
   G.out_scale = 1.f / std::sqrt(static_cast<float>(dh));
-  finish_group(cm, 0, G);
-  if ((rc = launch_gemm_unprofiled<EPI_CAUSALMAX>(cm, *st, s)) != MC_OK) return rc;
+  finish_group(cm, 0, G, 0);
+  if ((rc = launch_gemm_unprofiled<EPI_CAUSALMAX, 0>(cm, *st, s)) != MC_OK) return rc;
 
   qk_keys_decode_kernel<<<(H + 255) / 256, 256, 0, s>>>(keys, smax_out, H);
   MC_CUDA(cudaGetLastError());

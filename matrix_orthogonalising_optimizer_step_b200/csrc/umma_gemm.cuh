@@ -28,42 +28,61 @@
 // is §03's W <- W - eta (O + lambda W) with O scaled by 0.2 sqrt(max(m, n)).
 //
 // Execution: CTA pairs (clusters of 2, one CTA per SM) run 2-SM tensor-core
-// MMAs (tcgen05 cta_group::2): a 256 x 256 output tile per pair, of which each
-// CTA holds 128 rows in its own TMEM.  Each CTA stages its 128 rows of A and
-// its 128 rows of B (the pair's B is split between the two SMs), so an SM
-// pulls 32 KB per 512 tensor-core cycles instead of the 48 KB a one-SM
-// 128 x 256 tile needs.  No TMA multicast is used.
+// MMAs (tcgen05 cta_group::2): a 256 x 256 or 256 x 512 output tile per pair
+// (see TileCfg), of which each CTA holds 128 rows in its own TMEM.  Each CTA
+// stages its 128 rows of A and its 128 rows of every 256-column B block (the
+// pair's B is split between the two SMs).  No TMA multicast is used.
 //
 // Warp roles (320 threads per CTA):
-//   warp 0      TMA producer: 6-stage ring of {A 128x64, B 128x64} bf16 tiles,
+//   warp 0      TMA producer: ring of {A 128x64, one or two B 128x64} bf16 tiles,
 //               128-byte swizzled, K-major or MN-major per group.  Both CTAs'
 //               copies complete on the leader CTA's "full" barrier.
-//   warp 1      TMEM allocation (both CTAs, 2-SM form); in the leader CTA one
-//               thread issues tcgen05.mma (M=256, N=256, K=16) and commits to
-//               both CTAs' "empty" and "accumulator full" barriers.
-//   warps 2-9   epilogue: two accumulator buffers (2 x 256 TMEM columns) so the
-//               next tile's MMAs overlap this tile's epilogue.  Warp w reads TMEM
-//               lanes 32*(w%4)..+31 and column half (w-2)/4; the leader's
-//               "accumulator empty" barrier counts both CTAs' epilogue warps.
+//   warp 1      TMEM allocation (512 columns, both CTAs, 2-SM form); in the
+//               leader CTA one thread issues tcgen05.mma (M=256, N=256, K=16;
+//               two per k-step for WIDE tiles) and commits to both CTAs'
+//               "empty" and "accumulator full" barriers.
+//   warps 2-9   epilogue: warp w reads TMEM lanes 32*(w%4)..+31 and column
+//               half (w-2)/4 of the tile; the leader's "accumulator empty"
+//               barrier counts both CTAs' epilogue warps.
 #pragma once
 
 #include "ptx.cuh"
 
 namespace mc {
 
-constexpr int BM = 256, BN = 256, BK = 64, STAGES = 6;
-constexpr int HALF = 128;                               // rows of A and of B per CTA
+constexpr int BM = 256, BK = 64;
+constexpr int HALF = 128;                               // rows of A and of each B block per CTA
+constexpr int MMA_N = 256;                              // N of one MMA instruction
 constexpr uint32_t A_STAGE_BYTES = HALF * BK * 2;       // 16 KiB
-constexpr uint32_t B_STAGE_BYTES = HALF * BK * 2;       // 16 KiB
-constexpr uint32_t STAGE_BYTES = A_STAGE_BYTES + B_STAGE_BYTES;
-constexpr uint32_t PAIR_STAGE_BYTES = 2 * STAGE_BYTES;  // what the leader's full barrier expects
+constexpr uint32_t B_STAGE_BYTES = HALF * BK * 2;       // 16 KiB per B block
 constexpr uint32_t MN_BOX_BYTES = 64 * BK * 2;          // one {64 MN, 64 K} box: 8 KiB
 constexpr int NUM_EPI_WARPS = 8;
 constexpr int GEMM_THREADS = 64 + NUM_EPI_WARPS * 32;
-constexpr uint32_t TMEM_COLS = 2 * BN;
+constexpr uint32_t TMEM_COLS = 512;
 constexpr int MAX_GROUPS = 4;
 constexpr int GEMM_BARRIER_BYTES = 256;
-constexpr size_t GEMM_SMEM_BYTES = 1024 + size_t(STAGES) * STAGE_BYTES + GEMM_BARRIER_BYTES;
+
+// Two tile shapes per CTA pair:
+//   WIDE = 0: 256 x 256, two 256-column accumulators (the next tile's MMAs
+//             overlap this tile's epilogue), 6 stages of 32 KB per CTA;
+//   WIDE = 1: 256 x 512, one 512-column accumulator, 4 stages of 48 KB per
+//             CTA.  Sharing each A tile between two N=256 MMAs cuts the
+//             operand bytes per MMA cycle from 64 to 48 per SM, below the
+//             TMA feed limit; the epilogue is then not overlapped, so WIDE
+//             suits the phases whose epilogue is light.
+template <int WIDE>
+struct TileCfg {
+  static constexpr int N = MMA_N << WIDE;               // tile columns per pair
+  static constexpr int NB = 1 << WIDE;                  // B blocks (MMAs per k-step)
+  static constexpr int STAGES = WIDE ? 4 : 6;
+  static constexpr int NACC = WIDE ? 1 : 2;             // accumulator buffers
+  static constexpr uint32_t STAGE_BYTES = A_STAGE_BYTES + NB * B_STAGE_BYTES;
+  static constexpr uint32_t PAIR_STAGE_BYTES = 2 * STAGE_BYTES;
+  static constexpr size_t SMEM_BYTES = 1024 + size_t(STAGES) * STAGE_BYTES + GEMM_BARRIER_BYTES;
+  static_assert(NACC * N <= int(TMEM_COLS), "accumulators exceed TMEM");
+};
+constexpr size_t GEMM_SMEM_BYTES =
+    TileCfg<0>::SMEM_BYTES > TileCfg<1>::SMEM_BYTES ? TileCfg<0>::SMEM_BYTES : TileCfg<1>::SMEM_BYTES;
 
 enum Sched : int { SCHED_DENSE = 0, SCHED_SYM = 1, SCHED_CAUSAL = 2 };
 enum Layout : int { LAYOUT_BATCHED = 0, LAYOUT_HEADS = 1 };
@@ -86,6 +105,7 @@ struct GemmGroup {
   int a_mn, b_mn;          // operand major-ness: 0 K-major, 1 MN-major
   int prob_base;           // index of problem 0 in the per-matrix scale table
   int band;                // dense raster: n-tiles per band
+  int nshift;              // log2(tile columns / 256): 0 or 1 (WIDE tiles)
   // ---- epilogue operands ----
   void* d;                 // bf16 output [count][M][d_ld]
   long long d_ld, d_bs;
@@ -118,17 +138,18 @@ struct GemmParams {
 static_assert(sizeof(GemmParams) <= 4096, "kernel parameters must fit the classic 4 KiB limit");
 
 // ------------------------------------------------------------------ tiling
-// Tiles (i, j) of 256 x 256.  SYM keeps the tiles on or above the diagonal
-// (j >= i); CAUSAL keeps those on or below it (j <= i).
-__host__ __device__ inline long long sched_row_count(int sched, int i, int tiles_n) {
-  if (sched == SCHED_SYM) return tiles_n - i;
-  if (sched == SCHED_CAUSAL) return (i + 1) < tiles_n ? (i + 1) : tiles_n;
+// Tiles (i, j) of 256 rows x (256 << nshift) columns.  SYM keeps the tiles
+// that reach the upper triangle (j >= i >> nshift); CAUSAL keeps those that
+// reach the lower triangle including the diagonal (j <= i >> nshift).
+__host__ __device__ inline long long sched_row_count(int sched, int i, int tiles_n, int nshift) {
+  if (sched == SCHED_SYM) return tiles_n - (i >> nshift);
+  if (sched == SCHED_CAUSAL) return ((i >> nshift) + 1) < tiles_n ? ((i >> nshift) + 1) : tiles_n;
   return tiles_n;
 }
-__host__ __device__ inline long long sched_tiles_per_prob(int sched, int tiles_m, int tiles_n) {
+__host__ __device__ inline long long sched_tiles_per_prob(int sched, int tiles_m, int tiles_n, int nshift) {
   if (sched == SCHED_DENSE) return (long long)tiles_m * tiles_n;
   long long t = 0;
-  for (int i = 0; i < tiles_m; ++i) t += sched_row_count(sched, i, tiles_n);
+  for (int i = 0; i < tiles_m; ++i) t += sched_row_count(sched, i, tiles_n, nshift);
   return t;
 }
 
@@ -157,13 +178,13 @@ __host__ __device__ inline void decode_tile(const GemmGroup* groups, int num_gro
   } else {
     int i = 0;
     while (true) {
-      const long long cnt = sched_row_count(G.sched, i, G.tiles_n);
+      const long long cnt = sched_row_count(G.sched, i, G.tiles_n, G.nshift);
       if (tl < cnt) break;
       tl -= cnt;
       ++i;
     }
     tm = i;
-    tn = (G.sched == SCHED_SYM ? i : 0) + (int)tl;
+    tn = (G.sched == SCHED_SYM ? (i >> G.nshift) : 0) + (int)tl;
   }
   ti.g = g;
   ti.prob = (int)prob;
@@ -236,9 +257,99 @@ __device__ __forceinline__ void store_sym_chunk(__nv_bfloat16* D, long long ld, 
   }
 }
 
+// Each epilogue thread owns one row r of the tile and walks its columns in
+// chunks of 16: the global operands of a chunk are requested first
+// (epi_prefetch), then its accumulator columns are read from TMEM, so the two
+// latencies overlap, then the chunk is finished (epi_finish).
+
+// Global operands of one chunk, kept as raw 128-bit words until used:
+// x = the b*A source (EPI_POLY, bf16) or the fp32 iterate (EPI_APPLY* with
+// xf_read); w = the weight (EPI_APPLY_FINAL, bf16 or fp32).
+struct EpiPre {
+  uint4 x[4];
+  uint4 w[4];
+};
+
+// `valid` columns are in range; `vec`: the 16 elements may be read as two
+// 16-byte words (aligned row and full chunk), else element by element.
+__device__ __forceinline__ void raw_load_bf16x16(const __nv_bfloat16* p, int valid, bool vec, uint4 (&q)[4]) {
+  if (vec && valid >= 16) {
+    const uint4* s = reinterpret_cast<const uint4*>(p);
+    q[0] = s[0];
+    q[1] = s[1];
+  } else {
+    uint32_t w[8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      const uint32_t lo = (2 * i < valid) ? static_cast<uint32_t>(*reinterpret_cast<const uint16_t*>(p + 2 * i)) : 0u;
+      const uint32_t hi =
+          (2 * i + 1 < valid) ? static_cast<uint32_t>(*reinterpret_cast<const uint16_t*>(p + 2 * i + 1)) : 0u;
+      w[i] = lo | (hi << 16);
+    }
+    q[0] = make_uint4(w[0], w[1], w[2], w[3]);
+    q[1] = make_uint4(w[4], w[5], w[6], w[7]);
+  }
+}
+__device__ __forceinline__ void raw_load_f32x16(const float* p, int valid, bool vec, uint4 (&q)[4]) {
+  if (vec && valid >= 16) {
+    const uint4* s = reinterpret_cast<const uint4*>(p);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) q[i] = s[i];
+  } else {
+    uint32_t w[16];
+#pragma unroll
+    for (int i = 0; i < 16; ++i) w[i] = (i < valid) ? __float_as_uint(p[i]) : 0u;
+#pragma unroll
+    for (int i = 0; i < 4; ++i) q[i] = make_uint4(w[4 * i], w[4 * i + 1], w[4 * i + 2], w[4 * i + 3]);
+  }
+}
+__device__ __forceinline__ void raw_to_bf16x16(const uint4 (&q)[4], float (&x)[16]) {
+  const uint32_t w[8] = {q[0].x, q[0].y, q[0].z, q[0].w, q[1].x, q[1].y, q[1].z, q[1].w};
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    x[2 * i] = __uint_as_float(w[i] << 16);
+    x[2 * i + 1] = __uint_as_float(w[i] & 0xFFFF0000u);
+  }
+}
+__device__ __forceinline__ void raw_to_f32x16(const uint4 (&q)[4], float (&x)[16]) {
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    x[4 * i] = __uint_as_float(q[i].x);
+    x[4 * i + 1] = __uint_as_float(q[i].y);
+    x[4 * i + 2] = __uint_as_float(q[i].z);
+    x[4 * i + 3] = __uint_as_float(q[i].w);
+  }
+}
+
 template <int EPI>
-__device__ __forceinline__ void epilogue_chunk(const GemmGroup& G, int prob, int r, int c0,
-                                               float (&v)[16], float& run_max) {
+__device__ __forceinline__ void epi_prefetch(const GemmGroup& G, int prob, int r, int c0, EpiPre& pre) {
+  if (r >= G.M) return;
+  const int valid = G.N - c0;
+  if (valid <= 0) return;
+  if constexpr (EPI == EPI_POLY) {
+    const __nv_bfloat16* S =
+        static_cast<const __nv_bfloat16*>(G.src) + (long long)prob * G.src_bs + (long long)r * G.src_ld;
+    raw_load_bf16x16(S + c0, valid, true, pre.x);
+  } else if constexpr (EPI == EPI_APPLY || EPI == EPI_APPLY_FINAL) {
+    if (G.xf_read) {
+      const float* X = G.xf + (long long)prob * G.xf_bs + (long long)r * G.xf_ld;
+      raw_load_f32x16(X + c0, valid, true, pre.x);
+    }
+    if constexpr (EPI == EPI_APPLY_FINAL) {
+      const long long row = (long long)r * G.N;
+      if (G.w_f32) {
+        raw_load_f32x16(static_cast<const float*>(G.w_ptrs[prob]) + row + c0, valid, G.w_vec != 0, pre.w);
+      } else {
+        raw_load_bf16x16(static_cast<const __nv_bfloat16*>(G.w_ptrs[prob]) + row + c0, valid, G.w_vec != 0,
+                         pre.w);
+      }
+    }
+  }
+}
+
+template <int EPI>
+__device__ __forceinline__ void epi_finish(const GemmGroup& G, int prob, int r, int c0, float* v,
+                                           const EpiPre& pre, float& run_max) {
   const bool full = (r < G.M) && (c0 + 16 <= G.N);
   if constexpr (EPI == EPI_GRAM) {
     float s2 = 1.f;
@@ -246,64 +357,55 @@ __device__ __forceinline__ void epilogue_chunk(const GemmGroup& G, int prob, int
       const float s = G.scale[G.prob_base + prob];
       s2 = s * s;
     }
+    float o[16];
 #pragma unroll
-    for (int j = 0; j < 16; ++j) v[j] *= s2;
+    for (int j = 0; j < 16; ++j) o[j] = v[j] * s2;
     __nv_bfloat16* D = static_cast<__nv_bfloat16*>(G.d) + (long long)prob * G.d_bs;
-    store_sym_chunk(D, G.d_ld, G.M, r, c0, v);
+    store_sym_chunk(D, G.d_ld, G.M, r, c0, o);
   } else if constexpr (EPI == EPI_POLY) {
     if (r >= G.M) return;
-    const __nv_bfloat16* S =
-        static_cast<const __nv_bfloat16*>(G.src) + (long long)prob * G.src_bs + (long long)r * G.src_ld;
     float x[16];
-    if (full) {
-      load_bf16x16(S + c0, x);
-    } else {
+    raw_to_bf16x16(pre.x, x);
+    float o[16];
 #pragma unroll
-      for (int j = 0; j < 16; ++j) x[j] = (c0 + j < G.N) ? __bfloat162float(S[c0 + j]) : 0.f;
-    }
-#pragma unroll
-    for (int j = 0; j < 16; ++j) v[j] = fmaf(G.coef_acc, v[j], G.coef_src * x[j]) + (c0 + j == r ? G.diag : 0.f);
+    for (int j = 0; j < 16; ++j) o[j] = fmaf(G.coef_acc, v[j], G.coef_src * x[j]) + (c0 + j == r ? G.diag : 0.f);
     __nv_bfloat16* D = static_cast<__nv_bfloat16*>(G.d) + (long long)prob * G.d_bs;
-    store_sym_chunk(D, G.d_ld, G.M, r, c0, v);
+    store_sym_chunk(D, G.d_ld, G.M, r, c0, o);
   } else if constexpr (EPI == EPI_APPLY || EPI == EPI_APPLY_FINAL) {
     if (r >= G.M) return;
     const float s = G.scale ? G.scale[G.prob_base + prob] : 1.f;
-    float* X = G.xf ? G.xf + (long long)prob * G.xf_bs + (long long)r * G.xf_ld : nullptr;
+    float o[16];
     if (G.xf_read) {
       float x[16];
-      if (full) {
-        load_f32x16(X + c0, x);
-      } else {
+      raw_to_f32x16(pre.x, x);
 #pragma unroll
-        for (int j = 0; j < 16; ++j) x[j] = (c0 + j < G.N) ? X[c0 + j] : 0.f;
-      }
-#pragma unroll
-      for (int j = 0; j < 16; ++j) v[j] = s * fmaf(G.coef_src, x[j], v[j]);
+      for (int j = 0; j < 16; ++j) o[j] = s * fmaf(G.coef_src, x[j], v[j]);
     } else {
 #pragma unroll
-      for (int j = 0; j < 16; ++j) v[j] *= s;
+      for (int j = 0; j < 16; ++j) o[j] = s * v[j];
     }
     if constexpr (EPI == EPI_APPLY) {
+      float* X = G.xf ? G.xf + (long long)prob * G.xf_bs + (long long)r * G.xf_ld : nullptr;
       __nv_bfloat16* D =
           static_cast<__nv_bfloat16*>(G.d) + (long long)prob * G.d_bs + (long long)r * G.d_ld;
       if (full) {
-        if (G.xf_write) store_f32x16(X + c0, v);
-        store_bf16x16(D + c0, v);
+        if (G.xf_write) store_f32x16(X + c0, o);
+        store_bf16x16(D + c0, o);
       } else {
 #pragma unroll
         for (int j = 0; j < 16; ++j)
           if (c0 + j < G.N) {
-            if (G.xf_write) X[c0 + j] = v[j];
-            D[c0 + j] = __float2bfloat16_rn(v[j]);
+            if (G.xf_write) X[c0 + j] = o[j];
+            D[c0 + j] = __float2bfloat16_rn(o[j]);
           }
       }
     } else {
-      float* U = G.u_ptrs ? G.u_ptrs[prob] : nullptr;
       const long long row = (long long)r * G.N;
+      float* U = G.u_ptrs ? G.u_ptrs[prob] : nullptr;
       if (U) {
         float u[16];
 #pragma unroll
-        for (int j = 0; j < 16; ++j) u[j] = G.rms * v[j];
+        for (int j = 0; j < 16; ++j) u[j] = G.rms * o[j];
         if (full && (G.N % 4 == 0)) {
           store_f32x16(U + row + c0, u);
         } else {
@@ -312,33 +414,32 @@ __device__ __forceinline__ void epilogue_chunk(const GemmGroup& G, int prob, int
             if (c0 + j < G.N) U[row + c0 + j] = u[j];
         }
       }
+      float w[16];
+      if (G.w_f32) {
+        raw_to_f32x16(pre.w, w);
+      } else {
+        raw_to_bf16x16(pre.w, w);
+      }
+      float nw[16];
+#pragma unroll
+      for (int j = 0; j < 16; ++j) nw[j] = fmaf(G.step, o[j], G.decay * w[j]);
       if (G.w_f32) {
         float* W = static_cast<float*>(G.w_ptrs[prob]) + row;
         if (full && G.w_vec) {
-          float w[16];
-          load_f32x16(W + c0, w);
-#pragma unroll
-          for (int j = 0; j < 16; ++j) w[j] = fmaf(G.step, v[j], G.decay * w[j]);
-          store_f32x16(W + c0, w);
+          store_f32x16(W + c0, nw);
         } else {
 #pragma unroll
           for (int j = 0; j < 16; ++j)
-            if (c0 + j < G.N) W[c0 + j] = fmaf(G.step, v[j], G.decay * W[c0 + j]);
+            if (c0 + j < G.N) W[c0 + j] = nw[j];
         }
       } else {
         __nv_bfloat16* W = static_cast<__nv_bfloat16*>(G.w_ptrs[prob]) + row;
         if (full && G.w_vec) {
-          float w[16];
-          load_bf16x16(W + c0, w);
-#pragma unroll
-          for (int j = 0; j < 16; ++j) w[j] = fmaf(G.step, v[j], G.decay * w[j]);
-          store_bf16x16(W + c0, w);
+          store_bf16x16(W + c0, nw);
         } else {
 #pragma unroll
           for (int j = 0; j < 16; ++j)
-            if (c0 + j < G.N)
-              W[c0 + j] = __float2bfloat16_rn(
-                  fmaf(G.step, v[j], G.decay * __bfloat162float(W[c0 + j])));
+            if (c0 + j < G.N) W[c0 + j] = __float2bfloat16_rn(nw[j]);
         }
       }
     }
@@ -347,7 +448,7 @@ __device__ __forceinline__ void epilogue_chunk(const GemmGroup& G, int prob, int
     __nv_bfloat16* D =
         static_cast<__nv_bfloat16*>(G.d) + (long long)prob * G.d_bs + (long long)r * G.d_ld;
     if (full) {
-      store_bf16x16(D + c0, v);
+      store_bf16x16(D + c0, *reinterpret_cast<const float(*)[16]>(v));
     } else {
 #pragma unroll
       for (int j = 0; j < 16; ++j)
@@ -364,18 +465,30 @@ __device__ __forceinline__ void epilogue_chunk(const GemmGroup& G, int prob, int
   }
 }
 
-// ------------------------------------------------------------------ kernel
+// Chunks per batch.  One: measured against batches of four chunks (one
+// 64-column TMEM load, all global loads issued first) on the same GPU, the
+// single-chunk drain was as fast or faster in every phase.
 template <int EPI>
+struct EpiBatch {
+  static constexpr int CH = 1;
+};
+
+// ------------------------------------------------------------------ kernel
+template <int EPI, int WIDE>
 __global__ void __launch_bounds__(GEMM_THREADS, 1) umma_gemm_kernel(const __grid_constant__ GemmParams P) {
+  using T = TileCfg<WIDE>;
+  constexpr int STAGES = T::STAGES;
+  constexpr int NACC = T::NACC;
+  constexpr uint32_t STAGE_BYTES = T::STAGE_BYTES;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + STAGES * STAGE_BYTES);
-  uint64_t* full_bar = bars;                    // [STAGES]  used in the leader only
-  uint64_t* empty_bar = bars + STAGES;          // [STAGES]  every CTA
-  uint64_t* tfull_bar = bars + 2 * STAGES;      // [2]       every CTA
-  uint64_t* tempty_bar = bars + 2 * STAGES + 2; // [2]       used in the leader only
-  uint64_t* drain_bar = bars + 2 * STAGES + 4;  // [1]       leader
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2 * STAGES + 5);
+  uint64_t* full_bar = bars;                          // [STAGES]  used in the leader only
+  uint64_t* empty_bar = bars + STAGES;                // [STAGES]  every CTA
+  uint64_t* tfull_bar = bars + 2 * STAGES;            // [NACC]    every CTA
+  uint64_t* tempty_bar = bars + 2 * STAGES + NACC;    // [NACC]    used in the leader only
+  uint64_t* drain_bar = bars + 2 * STAGES + 2 * NACC; // [1]       leader
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain_bar + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
   const int warp = threadIdx.x >> 5;
@@ -388,7 +501,7 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1) umma_gemm_kernel(const __grid
       mbar_init(smem_u32(&full_bar[s]), 1);
       mbar_init(smem_u32(&empty_bar[s]), 1);
     }
-    for (int b = 0; b < 2; ++b) {
+    for (int b = 0; b < NACC; ++b) {
       mbar_init(smem_u32(&tfull_bar[b]), 1);
       mbar_init(smem_u32(&tempty_bar[b]), 2 * NUM_EPI_WARPS);
     }
@@ -429,7 +542,7 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1) umma_gemm_kernel(const __grid
         const CUtensorMap* ma = &P.map_a[ti.g];
         const CUtensorMap* mb = &P.map_b[ti.g];
         const int m0 = ti.tm * BM + HALF * static_cast<int>(rank);
-        const int n0 = ti.tn * BN + HALF * static_cast<int>(rank);
+        const int n0 = ti.tn * T::N + HALF * static_cast<int>(rank);
         for (int kb = 0; kb < ti.num_kb; ++kb) {
           if (!wait_bounded(smem_u32(&empty_bar[stage]), phase ^ 1, abort_flag, P.err)) {
             ok = false;
@@ -437,18 +550,19 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1) umma_gemm_kernel(const __grid
           }
           const uint32_t fb_local = smem_u32(&full_bar[stage]);
           if (leader) {
-            mbar_arrive_expect_tx(fb_local, PAIR_STAGE_BYTES);
+            mbar_arrive_expect_tx(fb_local, T::PAIR_STAGE_BYTES);
             filled |= 1u << stage;
             fill_parity = (fill_parity & ~(1u << stage)) | (phase << stage);
           }
           const uint32_t fb = mapa_shared(fb_local, 0);
           const uint32_t sa = smem_u32(smem + stage * STAGE_BYTES);
-          const uint32_t sb = sa + A_STAGE_BYTES;
           const int k0 = kb * BK;
           if (G.layout == LAYOUT_HEADS) {
             const int bb = ti.prob / G.heads, hh = ti.prob % G.heads;
             tma_load_4d_pair(sa, ma, fb, k0, hh, m0, bb);
-            tma_load_4d_pair(sb, mb, fb, k0, hh, n0, bb);
+#pragma unroll
+            for (int h = 0; h < T::NB; ++h)
+              tma_load_4d_pair(sa + A_STAGE_BYTES + h * B_STAGE_BYTES, mb, fb, k0, hh, n0 + h * MMA_N, bb);
           } else {
             if (!G.a_mn) {
               tma_load_3d_pair(sa, ma, fb, k0, m0, ti.prob);
@@ -456,11 +570,16 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1) umma_gemm_kernel(const __grid
               tma_load_3d_pair(sa, ma, fb, m0, k0, ti.prob);
               tma_load_3d_pair(sa + MN_BOX_BYTES, ma, fb, m0 + 64, k0, ti.prob);
             }
-            if (!G.b_mn) {
-              tma_load_3d_pair(sb, mb, fb, k0, n0, ti.prob);
-            } else {
-              tma_load_3d_pair(sb, mb, fb, n0, k0, ti.prob);
-              tma_load_3d_pair(sb + MN_BOX_BYTES, mb, fb, n0 + 64, k0, ti.prob);
+#pragma unroll
+            for (int h = 0; h < T::NB; ++h) {
+              const uint32_t sb = sa + A_STAGE_BYTES + h * B_STAGE_BYTES;
+              const int nh = n0 + h * MMA_N;
+              if (!G.b_mn) {
+                tma_load_3d_pair(sb, mb, fb, k0, nh, ti.prob);
+              } else {
+                tma_load_3d_pair(sb, mb, fb, nh, k0, ti.prob);
+                tma_load_3d_pair(sb + MN_BOX_BYTES, mb, fb, nh + 64, k0, ti.prob);
+              }
             }
           }
           if (++stage == STAGES) {
@@ -486,11 +605,12 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1) umma_gemm_kernel(const __grid
       int acc = 0;
       uint32_t acc_phase = 0;
       bool ok = true;
+      const uint32_t s0 = smem_u32(smem);
       for (long long t = first_tile; ok && t < total; t += tile_step) {
         TileInfo ti;
         decode_tile(P.g, P.num_groups, t, ti);
         const GemmGroup& G = P.g[ti.g];
-        const uint32_t idesc = idesc_bf16_f32(BM, BN, G.a_mn, G.b_mn);
+        const uint32_t idesc = idesc_bf16_f32(BM, MMA_N, G.a_mn, G.b_mn);
         const uint32_t a_lbo = G.a_mn ? MN_BOX_BYTES : 16u;
         const uint32_t b_lbo = G.b_mn ? MN_BOX_BYTES : 16u;
         const uint32_t a_kstep = G.a_mn ? 16u * 128u : 32u;
@@ -500,11 +620,10 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1) umma_gemm_kernel(const __grid
           break;
         }
         tc_fence_after();
-        const uint32_t d_tmem = tmem_base + acc * BN;
-        // Descriptors of stage 0; stage s and k-step kk only move the start
-        // address field (address >> 4 in the low 14 bits, no carry out of it
-        // since shared memory ends below 2^18).
-        const uint32_t s0 = smem_u32(smem);
+        const uint32_t d_tmem = tmem_base + acc * T::N;
+        // Descriptors of stage 0; the stage, the k-step and the B block only
+        // move the start-address field (address >> 4 in the low 14 bits, no
+        // carry out of it since shared memory ends below 2^18).
         const uint64_t ad0 = smem_desc_sw128(s0, a_lbo, 1024);
         const uint64_t bd0 = smem_desc_sw128(s0 + A_STAGE_BYTES, b_lbo, 1024);
         for (int kb = 0; kb < ti.num_kb; ++kb) {
@@ -518,8 +637,11 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1) umma_gemm_kernel(const __grid
 #pragma unroll
           for (int kk = 0; kk < BK / 16; ++kk) {
             const uint64_t ad = ad0 + soff + ((kk * a_kstep) >> 4);
-            const uint64_t bd = bd0 + soff + ((kk * b_kstep) >> 4);
-            umma_bf16_pair(d_tmem, ad, bd, idesc, (kb | kk) != 0);
+#pragma unroll
+            for (int h = 0; h < T::NB; ++h) {
+              const uint64_t bd = bd0 + soff + ((h * B_STAGE_BYTES + kk * b_kstep) >> 4);
+              umma_bf16_pair(d_tmem + h * MMA_N, ad, bd, idesc, (kb | kk) != 0);
+            }
           }
           umma_commit_pair_mc(smem_u32(&empty_bar[stage]), 0x3);
           if (++stage == STAGES) {
@@ -529,8 +651,10 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1) umma_gemm_kernel(const __grid
         }
         if (!ok) break;
         umma_commit_pair_mc(smem_u32(&tfull_bar[acc]), 0x3);
-        acc ^= 1;
-        if (acc == 0) acc_phase ^= 1;
+        if (++acc == NACC) {
+          acc = 0;
+          acc_phase ^= 1;
+        }
       }
       // Every MMA of the pair completes before TMEM is released.
       umma_commit_pair(smem_u32(drain_bar));
@@ -539,10 +663,12 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1) umma_gemm_kernel(const __grid
     }
   } else {
     // ------------------------------------------------------- epilogue
+    constexpr int WCOLS = T::N / 2;    // columns per epilogue warp
     const int q = warp & 3;            // TMEM lane quarter this warp may read
-    const int half = (warp - 2) >> 2;  // column half of the 256-wide tile
-    const uint32_t tempty_leader0 = mapa_shared(smem_u32(&tempty_bar[0]), 0);
-    const uint32_t tempty_leader1 = mapa_shared(smem_u32(&tempty_bar[1]), 0);
+    const int half = (warp - 2) >> 2;  // column half of the tile
+    uint32_t tempty_leader[NACC];
+#pragma unroll
+    for (int b = 0; b < NACC; ++b) tempty_leader[b] = mapa_shared(smem_u32(&tempty_bar[b]), 0);
     int acc = 0;
     uint32_t acc_phase = 0;
     for (long long t = first_tile; t < total; t += tile_step) {
@@ -556,18 +682,25 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1) umma_gemm_kernel(const __grid
       if (!__all_sync(0xffffffffu, ok)) break;
       tc_fence_after();
       const int r = ti.tm * BM + HALF * static_cast<int>(rank) + q * 32 + lane;
-      const uint32_t t_row = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + acc * BN + half * 128;
+      const uint32_t t_row = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + acc * T::N + half * WCOLS;
       float run_max = -INFINITY;
+      constexpr int CH = EpiBatch<EPI>::CH;
+      const int cbase = ti.tn * T::N + half * WCOLS;
 #pragma unroll 1
-      for (int ch = 0; ch < 8; ++ch) {
-        float v[16];
-        tmem_ld16(t_row + ch * 16, v);
-        const int c0 = ti.tn * BN + half * 128 + ch * 16;
-        epilogue_chunk<EPI>(G, ti.prob, r, c0, v, run_max);
+      for (int cb = 0; cb < WCOLS / 16; cb += CH) {
+        EpiPre pre[CH];
+#pragma unroll
+        for (int b = 0; b < CH; ++b) epi_prefetch<EPI>(G, ti.prob, r, cbase + (cb + b) * 16, pre[b]);
+        float v[CH * 16];
+        static_assert(CH == 1, "one 16-column TMEM load per chunk");
+        tmem_ld16(t_row + cb * 16, *reinterpret_cast<float(*)[16]>(v));
+#pragma unroll
+        for (int b = 0; b < CH; ++b)
+          epi_finish<EPI>(G, ti.prob, r, cbase + (cb + b) * 16, v + b * 16, pre[b], run_max);
       }
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive_cluster(acc ? tempty_leader1 : tempty_leader0);
+      if (lane == 0) mbar_arrive_cluster(tempty_leader[acc]);
       if constexpr (EPI == EPI_CAUSALMAX) {
 #pragma unroll
         for (int o = 16; o > 0; o >>= 1) run_max = fmaxf(run_max, __shfl_xor_sync(0xffffffffu, run_max, o));
@@ -576,8 +709,10 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1) umma_gemm_kernel(const __grid
           atomicMax(&G.keys[h], float_to_ordered(run_max * G.out_scale));
         }
       }
-      acc ^= 1;
-      if (acc == 0) acc_phase ^= 1;
+      if (++acc == NACC) {
+        acc = 0;
+        acc_phase ^= 1;
+      }
     }
   }
 

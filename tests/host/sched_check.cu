@@ -1,4 +1,4 @@
-// Host-only check of the GEMM tile scheduler in umma_gemm.cuh (256 x 256 tiles): enumerates every
+// Host-only check of the GEMM tile scheduler in umma_gemm.cuh (256 x 256 and 256 x 512 tiles): enumerates every
 // global tile index through decode_tile() and verifies coverage and uniqueness
 // for the dense (band raster), symmetric-upper and causal schedules, over
 // ragged sizes and multi-group launches.  Prints "OK" on success.
@@ -14,11 +14,12 @@ using namespace mc;
 static int fails = 0;
 #define CHECK(c, ...) do { if (!(c)) { ++fails; if (fails < 20) { std::printf(__VA_ARGS__); std::printf("\n"); } } } while (0)
 
-static GemmGroup mk(int M, int N, int K, int count, int sched, int band) {
+static GemmGroup mk(int M, int N, int K, int count, int sched, int band, int nshift = 0) {
   GemmGroup G{};
-  G.M = M; G.N = N; G.K = K; G.count = count; G.sched = sched; G.band = band;
-  G.tiles_m = (M + BM - 1) / BM; G.tiles_n = (N + BN - 1) / BN;
-  G.tiles_per_prob = sched_tiles_per_prob(sched, G.tiles_m, G.tiles_n);
+  G.M = M; G.N = N; G.K = K; G.count = count; G.sched = sched; G.band = band; G.nshift = nshift;
+  const int tn = MMA_N << nshift;
+  G.tiles_m = (M + BM - 1) / BM; G.tiles_n = (N + tn - 1) / tn;
+  G.tiles_per_prob = sched_tiles_per_prob(sched, G.tiles_m, G.tiles_n, nshift);
   return G;
 }
 
@@ -37,14 +38,19 @@ static void check_groups(std::vector<GemmGroup> gs) {
     auto key = std::make_tuple(ti.prob, ti.tm, ti.tn);
     CHECK(!seen[ti.g].count(key), "duplicate tile");
     seen[ti.g].insert(key);
-    if (G.sched == SCHED_SYM) CHECK(ti.tn >= ti.tm, "sym tile below diagonal");
+    const long long BNt = MMA_N << G.nshift;
+    if (G.sched == SCHED_SYM) {
+      CHECK(ti.tn >= (ti.tm >> G.nshift), "sym tile below diagonal");
+      CHECK((long long)ti.tn * BNt + BNt - 1 >= (long long)ti.tm * BM, "sym tile with no upper element");
+    }
     if (G.sched == SCHED_CAUSAL) {
-      CHECK(ti.tn <= ti.tm, "causal tile above diagonal");
-      CHECK((long long)ti.tn * BN <= (long long)ti.tm * BM + BM - 1, "causal tile with no valid element");
+      CHECK(ti.tn <= (ti.tm >> G.nshift), "causal tile above diagonal");
+      CHECK((long long)ti.tn * BNt <= (long long)ti.tm * BM + BM - 1, "causal tile with no valid element");
     }
   }
   for (size_t gi = 0; gi < gs.size(); ++gi) {
     const GemmGroup& G = gs[gi];
+    const int BN = MMA_N << G.nshift;
     for (int p = 0; p < G.count; ++p) {
       if (G.sched == SCHED_DENSE) {
         for (int i = 0; i < G.tiles_m; ++i)
@@ -65,14 +71,18 @@ static void check_groups(std::vector<GemmGroup> gs) {
 
 int main() {
   const int sizes[] = {1, 7, 64, 100, 128, 129, 255, 256, 257, 300, 384, 511, 640, 1000, 1024, 2048, 4096};
-  for (int M : sizes)
-    for (int N : sizes) {
-      check_groups({mk(M, N, 64, 2, SCHED_DENSE, 8)});
-      check_groups({mk(M, N, 300, 1, SCHED_DENSE, 3)});
+  for (int w = 0; w < 2; ++w) {
+    for (int M : sizes)
+      for (int N : sizes) {
+        check_groups({mk(M, N, 64, 2, SCHED_DENSE, 8, w)});
+        check_groups({mk(M, N, 300, 1, SCHED_DENSE, 3, w)});
+      }
+    for (int m : sizes) {
+      check_groups({mk(m, m, 77, 3, SCHED_SYM, 8, w)});
+      check_groups({mk(m, m, 128, 2, SCHED_CAUSAL, 8, w)});
     }
-  for (int m : sizes) {
-    check_groups({mk(m, m, 77, 3, SCHED_SYM, 8)});
-    check_groups({mk(m, m, 128, 2, SCHED_CAUSAL, 8)});
+    check_groups({mk(4096, 4096, 4096, 3, SCHED_SYM, 8, w), mk(4096, 4096, 14336, 2, SCHED_SYM, 8, w),
+                  mk(300, 300, 10, 4, SCHED_SYM, 8, w), mk(129, 129, 1, 1, SCHED_SYM, 8, w)});
   }
   check_groups({mk(4096, 4096, 4096, 3, SCHED_SYM, 8), mk(4096, 4096, 14336, 2, SCHED_SYM, 8),
                 mk(300, 300, 10, 4, SCHED_SYM, 8), mk(129, 129, 1, 1, SCHED_SYM, 8)});
@@ -84,7 +94,12 @@ int main() {
   CHECK(a.tiles_per_prob == 136, "sym count %lld", a.tiles_per_prob);
   GemmGroup c = mk(4096, 4096, 128, 128, SCHED_CAUSAL, 8);
   CHECK(c.tiles_per_prob == 136, "causal count %lld", c.tiles_per_prob);
-  CHECK(BM == 256 && BN == 256, "tile shape");
+  CHECK(BM == 256 && MMA_N == 256, "tile shape");
+  // 16 x 8 tiles of 256 x 512: rows i keep j >= i/2 (SYM) or j <= i/2 (CAUSAL)
+  GemmGroup aw = mk(4096, 4096, 4096, 1, SCHED_SYM, 8, 1);
+  CHECK(aw.tiles_per_prob == 72, "wide sym count %lld", aw.tiles_per_prob);
+  GemmGroup cw = mk(4096, 4096, 128, 1, SCHED_CAUSAL, 8, 1);
+  CHECK(cw.tiles_per_prob == 72, "wide causal count %lld", cw.tiles_per_prob);
   if (fails) { std::printf("FAILED %d checks\n", fails); return 1; }
   std::printf("OK\n");
   return 0;
