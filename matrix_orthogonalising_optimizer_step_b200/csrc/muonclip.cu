@@ -84,7 +84,7 @@ inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 
 template <int EPI, int WIDE>
 cudaError_t set_gemm_attr() {
   return cudaFuncSetAttribute(umma_gemm_kernel<EPI, WIDE>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                              static_cast<int>(TileCfg<WIDE>::SMEM_BYTES));
+                              static_cast<int>(gemm_smem_bytes<EPI, WIDE>()));
 }
 
 // Caller holds g_mu.
@@ -103,9 +103,7 @@ int device_state(DeviceState** out) {
     MC_CUDA(cudaGetSymbolAddress(reinterpret_cast<void**>(&st.err_ptr), g_device_error));
     MC_CUDA((set_gemm_attr<EPI_GRAM, 1>()));
     MC_CUDA((set_gemm_attr<EPI_POLY, 1>()));
-    MC_CUDA((set_gemm_attr<EPI_APPLY, 0>()));
     MC_CUDA((set_gemm_attr<EPI_APPLY, 1>()));
-    MC_CUDA((set_gemm_attr<EPI_APPLY_FINAL, 0>()));
     MC_CUDA((set_gemm_attr<EPI_APPLY_FINAL, 1>()));
     MC_CUDA((set_gemm_attr<EPI_STORE, 1>()));
     MC_CUDA((set_gemm_attr<EPI_CAUSALMAX, 0>()));
@@ -118,11 +116,11 @@ int device_state(DeviceState** out) {
       attr[0].val.clusterDim.z = 1;
       cfg.gridDim = dim3(static_cast<unsigned>(st.sms & ~1));
       cfg.blockDim = dim3(GEMM_THREADS);
-      cfg.dynamicSmemBytes = GEMM_SMEM_BYTES;
+      cfg.dynamicSmemBytes = gemm_smem_bytes<EPI_CAUSALMAX, 0>();
       cfg.attrs = attr;
       cfg.numAttrs = 1;
       int clusters = 0;
-      MC_CUDA(cudaOccupancyMaxActiveClusters(&clusters, umma_gemm_kernel<EPI_APPLY, 0>, &cfg));
+      MC_CUDA(cudaOccupancyMaxActiveClusters(&clusters, umma_gemm_kernel<EPI_CAUSALMAX, 0>, &cfg));
       if (clusters < 1) return fail(MC_ERR_UNSUPPORTED, "no CTA pair of the GEMM kernel fits on this device");
       st.pair_clusters = clusters;
     }
@@ -270,7 +268,7 @@ cudaError_t launch_pairs(const GemmParams& p, int pair_clusters, cudaStream_t s)
   attr[0].val.clusterDim.z = 1;
   cfg.gridDim = dim3(static_cast<unsigned>(2 * pairs));
   cfg.blockDim = dim3(GEMM_THREADS);
-  cfg.dynamicSmemBytes = TileCfg<WIDE>::SMEM_BYTES;
+  cfg.dynamicSmemBytes = gemm_smem_bytes<EPI, WIDE>();
   cfg.stream = s;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
@@ -625,18 +623,18 @@ MC_API int mc_muon_step(const mc_param* params, int n, const mc_hparams* hp, voi
           G.decay = 1.f - hp->lr * hp->wd;
           G.step = -hp->lr * G.rms;
         }
-        finish_group(apply, slot, G, mixed ? 0 : 1);
+        finish_group(apply, slot, G, 1);
       }
-      // Wide 256 x 512 tiles where the epilogue is light; the iterations whose
-      // apply reads and writes the fp32 iterate keep the double-buffered tile.
+      // All NS phases use the 256 x 512 tile.  For the apply iterations that
+      // read and write the fp32 iterate the exposed epilogue costs about what
+      // the narrower tile loses to the operand feed, and measured on one GPU
+      // the whole step was 2-3 % faster this way (the power cap).
       if ((rc = launch_gemm<EPI_GRAM, 1>(gram, *st, s, K_GRAM, f_gram, fd_gram)) != MC_OK) return rc;
       if ((rc = launch_gemm<EPI_POLY, 1>(poly, *st, s, K_POLY, f_poly, fd_poly)) != MC_OK) return rc;
       if (last) {
-        rc = mixed ? launch_gemm<EPI_APPLY_FINAL, 0>(apply, *st, s, K_APPLY_FINAL, f_apply)
-                   : launch_gemm<EPI_APPLY_FINAL, 1>(apply, *st, s, K_APPLY_FINAL, f_apply);
+        rc = launch_gemm<EPI_APPLY_FINAL, 1>(apply, *st, s, K_APPLY_FINAL, f_apply);
       } else {
-        rc = mixed ? launch_gemm<EPI_APPLY, 0>(apply, *st, s, K_APPLY_MIXED, f_apply)
-                   : launch_gemm<EPI_APPLY, 1>(apply, *st, s, K_APPLY, f_apply);
+        rc = launch_gemm<EPI_APPLY, 1>(apply, *st, s, mixed ? K_APPLY_MIXED : K_APPLY, f_apply);
       }
       if (rc != MC_OK) return rc;
     }

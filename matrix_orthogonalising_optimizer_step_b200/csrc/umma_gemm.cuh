@@ -41,10 +41,12 @@
 //               leader CTA one thread issues tcgen05.mma (M=256, N=256, K=16;
 //               two per k-step for WIDE tiles) and commits to both CTAs'
 //               "empty" and "accumulator full" barriers.
-//   warps 2-9   epilogue: warp w reads TMEM lanes 32*(w%4)..+31 and column
-//               half (w-2)/4 of the tile; the leader's "accumulator empty"
+//   warps 2..   epilogue: warp w reads TMEM lanes 32*(w%4)..+31 and column
+//               group (w-2)/4 of the tile; the leader's "accumulator empty"
 //               barrier counts both CTAs' epilogue warps.
 #pragma once
+
+#include <climits>
 
 #include "ptx.cuh"
 
@@ -56,8 +58,10 @@ constexpr int MMA_N = 256;                              // N of one MMA instruct
 constexpr uint32_t A_STAGE_BYTES = HALF * BK * 2;       // 16 KiB
 constexpr uint32_t B_STAGE_BYTES = HALF * BK * 2;       // 16 KiB per B block
 constexpr uint32_t MN_BOX_BYTES = 64 * BK * 2;          // one {64 MN, 64 K} box: 8 KiB
-constexpr int NUM_EPI_WARPS = 8;
+constexpr int NUM_EPI_WARPS = 8;                         // multiple of 4 (one per TMEM lane quarter)
+constexpr int EPI_COL_GROUPS = NUM_EPI_WARPS / 4;        // warps sharing a lane quarter split its columns
 constexpr int GEMM_THREADS = 64 + NUM_EPI_WARPS * 32;
+static_assert(NUM_EPI_WARPS % 4 == 0, "epilogue warps cover the four TMEM lane quarters evenly");
 constexpr uint32_t TMEM_COLS = 512;
 constexpr int MAX_GROUPS = 4;
 constexpr int GEMM_BARRIER_BYTES = 256;
@@ -70,6 +74,10 @@ constexpr int GEMM_BARRIER_BYTES = 256;
 //             operand bytes per MMA cycle from 64 to 48 per SM, below the
 //             TMA feed limit; the epilogue is then not overlapped, so WIDE
 //             suits the phases whose epilogue is light.
+// EPI_CAUSALMAX keeps one running maximum per head in shared memory (for up to
+// this many heads) and flushes it to global memory once, at the end.
+constexpr int SMEM_HEADS = 4096;
+
 template <int WIDE>
 struct TileCfg {
   static constexpr int N = MMA_N << WIDE;               // tile columns per pair
@@ -79,10 +87,12 @@ struct TileCfg {
   static constexpr uint32_t STAGE_BYTES = A_STAGE_BYTES + NB * B_STAGE_BYTES;
   static constexpr uint32_t PAIR_STAGE_BYTES = 2 * STAGE_BYTES;
   static constexpr size_t SMEM_BYTES = 1024 + size_t(STAGES) * STAGE_BYTES + GEMM_BARRIER_BYTES;
+  static constexpr size_t SMEM_BYTES_HEADS = SMEM_BYTES + 4 * size_t(SMEM_HEADS);
   static_assert(NACC * N <= int(TMEM_COLS), "accumulators exceed TMEM");
 };
 constexpr size_t GEMM_SMEM_BYTES =
     TileCfg<0>::SMEM_BYTES > TileCfg<1>::SMEM_BYTES ? TileCfg<0>::SMEM_BYTES : TileCfg<1>::SMEM_BYTES;
+static_assert(TileCfg<0>::SMEM_BYTES_HEADS <= 232448, "shared memory per CTA");
 
 enum Sched : int { SCHED_DENSE = 0, SCHED_SYM = 1, SCHED_CAUSAL = 2 };
 enum Layout : int { LAYOUT_BATCHED = 0, LAYOUT_HEADS = 1 };
@@ -94,6 +104,11 @@ enum Epi : int {
   EPI_STORE = 4,
   EPI_CAUSALMAX = 5
 };
+
+template <int EPI, int WIDE>
+constexpr size_t gemm_smem_bytes() {
+  return EPI == EPI_CAUSALMAX ? TileCfg<WIDE>::SMEM_BYTES_HEADS : TileCfg<WIDE>::SMEM_BYTES;
+}
 
 struct GemmGroup {
   int M, N, K;             // D is M x N, contraction K
@@ -456,21 +471,32 @@ __device__ __forceinline__ void epi_finish(const GemmGroup& G, int prob, int r, 
     }
   } else if constexpr (EPI == EPI_CAUSALMAX) {
     if (r >= G.M) return;
+    if (c0 + 16 <= G.N && (!G.mask_causal || c0 + 15 <= r)) {
+      // Whole chunk inside the mask and the bounds: a max tree, no compares.
+      float m[8];
 #pragma unroll
-    for (int j = 0; j < 16; ++j) {
-      const int c = c0 + j;
-      const bool ok = (c < G.N) && (!G.mask_causal || c <= r);
-      if (ok) run_max = fmaxf(run_max, v[j]);
+      for (int j = 0; j < 8; ++j) m[j] = fmaxf(v[2 * j], v[2 * j + 1]);
+#pragma unroll
+      for (int j = 0; j < 4; ++j) m[j] = fmaxf(m[2 * j], m[2 * j + 1]);
+      run_max = fmaxf(run_max, fmaxf(fmaxf(m[0], m[1]), fmaxf(m[2], m[3])));
+    } else {
+#pragma unroll
+      for (int j = 0; j < 16; ++j) {
+        const int c = c0 + j;
+        const bool ok = (c < G.N) && (!G.mask_causal || c <= r);
+        if (ok) run_max = fmaxf(run_max, v[j]);
+      }
     }
   }
 }
 
-// Chunks per batch.  One: measured against batches of four chunks (one
-// 64-column TMEM load, all global loads issued first) on the same GPU, the
-// single-chunk drain was as fast or faster in every phase.
+// Chunks per batch.  One for the NS phases: measured against batches of four
+// chunks (one 64-column TMEM load, all global loads issued first) on the same
+// GPU, the single-chunk drain was as fast or faster.  Four for the causal max,
+// whose epilogue has no global operands and is bound by the TMEM load latency.
 template <int EPI>
 struct EpiBatch {
-  static constexpr int CH = 1;
+  static constexpr int CH = (EPI == EPI_CAUSALMAX) ? 4 : 1;
 };
 
 // ------------------------------------------------------------------ kernel
@@ -490,6 +516,9 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1) umma_gemm_kernel(const __grid
   uint64_t* drain_bar = bars + 2 * STAGES + 2 * NACC; // [1]       leader
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain_bar + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+  int* head_max = reinterpret_cast<int*>(smem + STAGES * STAGE_BYTES + GEMM_BARRIER_BYTES);  // EPI_CAUSALMAX
+  const int nheads_smem = (EPI == EPI_CAUSALMAX && P.g[0].heads <= SMEM_HEADS) ? P.g[0].heads : 0;
+  for (int i = threadIdx.x; i < nheads_smem; i += blockDim.x) head_max[i] = INT_MIN;
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -663,9 +692,9 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1) umma_gemm_kernel(const __grid
     }
   } else {
     // ------------------------------------------------------- epilogue
-    constexpr int WCOLS = T::N / 2;    // columns per epilogue warp
-    const int q = warp & 3;            // TMEM lane quarter this warp may read
-    const int half = (warp - 2) >> 2;  // column half of the tile
+    constexpr int WCOLS = T::N / EPI_COL_GROUPS;  // columns per epilogue warp
+    const int q = warp & 3;                       // TMEM lane quarter this warp may read
+    const int half = (warp - 2) >> 2;             // which column group of the tile
     uint32_t tempty_leader[NACC];
 #pragma unroll
     for (int b = 0; b < NACC; ++b) tempty_leader[b] = mapa_shared(smem_u32(&tempty_bar[b]), 0);
@@ -686,14 +715,24 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1) umma_gemm_kernel(const __grid
       float run_max = -INFINITY;
       constexpr int CH = EpiBatch<EPI>::CH;
       const int cbase = ti.tn * T::N + half * WCOLS;
+      // Last row of this warp: a chunk that starts beyond it lies above the
+      // diagonal for every lane, as do all later chunks (causal max only).
+      const int r_warp_last = ti.tm * BM + HALF * static_cast<int>(rank) + q * 32 + 31;
 #pragma unroll 1
       for (int cb = 0; cb < WCOLS / 16; cb += CH) {
+        if constexpr (EPI == EPI_CAUSALMAX) {
+          if (G.mask_causal && cbase + cb * 16 > r_warp_last) break;
+        }
         EpiPre pre[CH];
 #pragma unroll
         for (int b = 0; b < CH; ++b) epi_prefetch<EPI>(G, ti.prob, r, cbase + (cb + b) * 16, pre[b]);
         float v[CH * 16];
-        static_assert(CH == 1, "one 16-column TMEM load per chunk");
-        tmem_ld16(t_row + cb * 16, *reinterpret_cast<float(*)[16]>(v));
+        if constexpr (CH == 4) {
+          tmem_ld64(t_row + cb * 16, v);
+        } else {
+          static_assert(CH == 1, "one 16- or 64-column TMEM load per batch");
+          tmem_ld16(t_row + cb * 16, *reinterpret_cast<float(*)[16]>(v));
+        }
 #pragma unroll
         for (int b = 0; b < CH; ++b)
           epi_finish<EPI>(G, ti.prob, r, cbase + (cb + b) * 16, v + b * 16, pre[b], run_max);
@@ -706,7 +745,12 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1) umma_gemm_kernel(const __grid
         for (int o = 16; o > 0; o >>= 1) run_max = fmaxf(run_max, __shfl_xor_sync(0xffffffffu, run_max, o));
         if (lane == 0 && run_max > -INFINITY) {
           const int h = ti.prob % G.heads;
-          atomicMax(&G.keys[h], float_to_ordered(run_max * G.out_scale));
+          const int key = float_to_ordered(run_max * G.out_scale);
+          if (nheads_smem) {
+            atomicMax(&head_max[h], key);
+          } else {
+            atomicMax(&G.keys[h], key);
+          }
         }
       }
       if (++acc == NACC) {
@@ -720,6 +764,10 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1) umma_gemm_kernel(const __grid
   // barriers or read its shared memory.
   tc_fence_before();
   __syncthreads();
+  if constexpr (EPI == EPI_CAUSALMAX) {
+    for (int i = threadIdx.x; i < nheads_smem; i += blockDim.x)
+      if (head_max[i] != INT_MIN) atomicMax(&P.g[0].keys[i], head_max[i]);
+  }
   cluster_sync();
   if (warp == 1) {
     __syncwarp();
