@@ -16,5 +16,5 @@ Pins (tests/test_oracle_pins.py) tie each function to something other than
 itself: the odd-polynomial/SVD identity, numbers the pages print, brute force
 on tiny inputs, limits with a textbook answer, and a third-party optimizer.
 """
-from .muon import phi, phi_iter, newton_schulz, muon_step, muon_step_many  # noqa: F401
+from .muon import phi, phi_iter, phi_schedule, newton_schulz, muon_step, muon_step_many  # noqa: F401
 from .qk import qk_max_logit, qk_max_logit_bruteforce, qk_clip, round_bf16  # noqa: F401

@@ -46,28 +46,41 @@ def phi_iter(x, steps: int, a: float, b: float, c: float):
     return y
 
 
+def phi_schedule(x, coeffs):
+    """phi_{(a_k, b_k, c_k)} applied in order, one step per coefficient triple."""
+    y = np.asarray(x, dtype=np.float64)
+    for (a, b, c) in coeffs:
+        y = phi(y, a, b, c)
+    return y
+
+
 def newton_schulz(U: np.ndarray, steps: int, a: float, b: float, c: float,
-                  eps: float = 1e-7) -> np.ndarray:
+                  eps: float = 1e-7, coeffs=None) -> np.ndarray:
     """Approximate polar factor of ``U`` by the quintic Newton-Schulz iteration.
 
     [MV] §2: X0 = U/||U||_F, then ``steps`` times A = X X^T,
     X = a X + (b A + c A A) X.  [MC] §02: A is formed after choosing the
     cheaper orientation, i.e. the short side first (m <= n); the result is
-    transposed back.  Returns an array of U's shape.
+    transposed back.  ``coeffs``, if given, is a list of ``steps`` triples
+    (a_k, b_k, c_k) used in iteration k instead of (a, b, c): the per-step
+    coefficient schedules [MV] §2 compares (cubic, simple and tuned quintic)
+    and that "About Muon: Muon At Scale" mentions for Polar Express.  Returns
+    an array of U's shape.
     """
     U = np.asarray(U, dtype=np.float64)
     transposed = U.shape[0] > U.shape[1]
     X = U.T if transposed else U
     norm = np.sqrt(np.sum(X * X))
     X = X / max(norm, eps)
-    for _ in range(steps):
+    for k in range(steps):
+        ak, bk, ck = coeffs[k] if coeffs is not None else (a, b, c)
         A = X @ X.T
-        B = b * A + c * (A @ A)
-        X = a * X + B @ X
+        B = bk * A + ck * (A @ A)
+        X = ak * X + B @ X
     return X.T if transposed else X
 
 
-def muon_step(W, G, M, *, mu, nesterov, lr, wd, ns_steps, a, b, c, eps, rms_scale):
+def muon_step(W, G, M, *, mu, nesterov, lr, wd, ns_steps, a, b, c, eps, rms_scale, coeffs=None):
     """One Muon step on one hidden 2D weight, in float64.
 
     Follows [MC] §07's order: momentum, NS, scaled update with decoupled decay.
@@ -78,6 +91,7 @@ def muon_step(W, G, M, *, mu, nesterov, lr, wd, ns_steps, a, b, c, eps, rms_scal
       Upd   = rms_scale * sqrt(max(rows, cols)) * O      ([MC] §03, [MS])
       W_t   = W_{t-1} - lr * (Upd + wd * W_{t-1})        ([MC] §03)
 
+    ``coeffs``: optional per-iteration (a_k, b_k, c_k) list (see newton_schulz).
     Returns (W_t, M_t, Upd, ||U||_F), all float64.
     """
     W = np.asarray(W, dtype=np.float64)
@@ -85,7 +99,7 @@ def muon_step(W, G, M, *, mu, nesterov, lr, wd, ns_steps, a, b, c, eps, rms_scal
     M = np.asarray(M, dtype=np.float64)
     M_new = mu * M + G
     U = G + mu * M_new if nesterov else M_new
-    O = newton_schulz(U, ns_steps, a, b, c, eps)
+    O = newton_schulz(U, ns_steps, a, b, c, eps, coeffs)
     upd = rms_scale * np.sqrt(max(W.shape)) * O
     W_new = W - lr * (upd + wd * W)
     return W_new, M_new, upd, float(np.sqrt(np.sum(U * U)))

@@ -301,3 +301,32 @@ def test_round_bf16_matches_torch_cast():
     x = rng.standard_normal(10000) * np.exp(rng.uniform(-20, 20, 10000))
     want = torch.from_numpy(x.astype(np.float32)).to(torch.bfloat16).double().numpy()
     assert np.array_equal(oracle.round_bf16(x), want)
+
+
+# ------------------------------------------------ per-step coefficient tables
+def test_ns_coefficient_schedule_equals_composed_scalar_maps():
+    """With a per-iteration schedule, the odd-polynomial identity composes:
+    NS(U diag(s) V^T) = U diag(phi_N o ... o phi_1 (s/||s||)) V^T."""
+    rng = np.random.default_rng(21)
+    r, c = 30, 52
+    U, V = haar(rng, r, r), haar(rng, c, r)
+    s = np.sort(rng.uniform(0.02, 2.0, r))[::-1]
+    G = (U * s) @ V.T
+    sched = [tuple(GOLD["classic_cubic"]["value"])] * 2 + [tuple(GOLD["simple_quintic"]["value"])] * 3 + [TUNED] * 2
+    got = oracle.newton_schulz(G, len(sched), *TUNED, coeffs=sched)
+    want = (U * oracle.phi_schedule(s / np.linalg.norm(s), sched)) @ V.T
+    assert np.linalg.norm(got - want) <= 1e-12 * np.linalg.norm(want)
+    # a schedule of one repeated triple is the plain iteration
+    same = oracle.newton_schulz(G, 5, *TUNED, coeffs=[TUNED] * 5)
+    assert np.array_equal(same, oracle.newton_schulz(G, 5, *TUNED))
+
+
+def test_cubic_schedule_converges_to_polar_factor():
+    """The classic cubic (1.5, -0.5, 0) converges to exactly U V^T (printed:
+    converges to exactly 1); numpy's SVD gives the polar factor."""
+    rng = np.random.default_rng(22)
+    G = rng.standard_normal((20, 35)) + 2 * np.eye(20, 35)
+    u, _, vt = np.linalg.svd(G, full_matrices=False)
+    cubic = tuple(GOLD["classic_cubic"]["value"])
+    O = oracle.newton_schulz(G, 60, *TUNED, coeffs=[cubic] * 60)
+    assert np.linalg.norm(O - u @ vt) <= 1e-9 * np.linalg.norm(u @ vt)
