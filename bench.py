@@ -49,6 +49,8 @@ def parse_args(argv=None):
     p.add_argument("--layers", type=int, default=32, help="layers of the 7B-shaped set (32 = full size)")
     p.add_argument("--no-e2e", action="store_true")
     p.add_argument("--no-cpu-baseline", action="store_true")
+    p.add_argument("--no-extras", action="store_true",
+                   help="skip the separately timed MLA QK-Clip layer and coefficient-table step")
     return p.parse_args(argv)
 
 
@@ -198,6 +200,85 @@ def run_reference(args, rank, world):
 
 
 # --------------------------------------------------------------- our arm
+def time_extras(mc, wl, dev, stream, hp, steps, peaks, barrier, max_over_ranks):
+    """Work outside the step, timed on its own after the step's timed region:
+    (1) S_max and the slice-map QK-Clip of a multi-head latent attention layer
+    (B 4, S 4096, D 4096, H 32, content 128 + rotary 64 per head); (2) the
+    64 x 1024^2 batched Muon step with its five NS coefficient triples passed
+    as a per-iteration table, beside the same step with scalar coefficients."""
+    import torch
+
+    out = {}
+    c = wl.MLA
+    B, S, D, H, dc, dr = c["B"], c["S"], c["D"], c["H"], c["dc"], c["dr"]
+    X, w = wl.mla_layer_inputs()
+    x = X.to(dev)
+    d = {k: v.to(dev) for k, v in w.items()}
+    smax = torch.empty(H, dtype=torch.float32, device=dev)
+    gamma = torch.empty(H, dtype=torch.float32, device=dev)
+    mask = torch.empty(H, dtype=torch.int32, device=dev)
+    slices = mc.mla_slices(d["W_qC"], d["W_kC"], d["W_qR"], H, dc, dr)
+
+    def mla_step():
+        mc.mla_max_logit(x, d["W_qC"], d["W_kC"], d["W_qR"], d["W_kR"], H, dc, dr, causal=True, smax_out=smax,
+                         stream=stream)
+        mc.qk_clip_slices(slices, smax, H, tau=wl.QK_TAU, gamma_out=gamma, mask_out=mask, stream=stream)
+
+    def timed(fn, reps):
+        for _ in range(3):
+            fn()
+        barrier()
+        torch.cuda.synchronize()
+        mc.profile_begin()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        for _ in range(reps):
+            fn()
+        b.record(stream)
+        torch.cuda.synchronize()
+        k = mc.profile_end()
+        assert mc.device_status() == mc.MC_OK, mc.last_error()
+        barrier()
+        return max_over_ranks(a.elapsed_time(b)) / reps, k
+
+    reps = max(steps, 5)
+    ms, k = timed(mla_step, reps)
+    cm = k["mla_causal_max"]
+    pr = k["mla_proj"]
+    cm_tf = cm["flops"] / (cm["total_ms"] / 1e3) / 1e12
+    out["mla_qk_clip"] = {
+        "workload": f"MLA layer B{B} S{S} D{D} H{H} dc{dc} dr{dr}, causal, bf16; S_max then slice-map clip",
+        "ms_per_layer": ms, "tokens_per_s": B * S / (ms / 1e3),
+        "mla_causal_max_ms": cm["total_ms"] / reps, "mla_causal_max_tflops": cm_tf,
+        "mla_causal_max_pct_bf16_peak": 100.0 * cm_tf / peaks["bf16_tflops"],
+        "mla_proj_ms": pr["total_ms"] / reps,
+        "mla_proj_tflops": pr["flops"] / (pr["total_ms"] / 1e3) / 1e12,
+        "qk_clip_slices_ms": k["qk_clip_slices"]["total_ms"] / reps if "qk_clip_slices" in k else None,
+        "launches_per_layer": sum(v["launches"] for v in k.values()) / reps}
+    del x, d, X, w
+    mc.release_workspaces()
+    torch.cuda.empty_cache()
+
+    mats = [wl.cfg1_matrix(i) for i in range(64)]
+    Ws = [W.to(dev) for W, _, _ in mats]
+    Gs = [G.to(dev) for _, G, _ in mats]
+    Ms = [M.to(dev) for _, _, M in mats]
+    table = [(hp["a"], hp["b"], hp["c"])] * hp["ns_steps"]
+    res = {}
+    for name, h in (("scalar", dict(hp)), ("table", dict(hp, coeffs=table))):
+        ms, _ = timed(lambda: mc.muon_step(Ws, Gs, Ms, stream=stream, **h), reps)
+        res[name] = ms
+    flops = 64 * hp["ns_steps"] * (4 * 1024 ** 3 + 2 * 1024 ** 3)
+    out["ns_coefficient_table"] = {
+        "workload": "64 x 1024^2 bf16 Muon step, 5 NS iterations given as a per-iteration table",
+        "ms_table": res["table"], "ms_scalar": res["scalar"],
+        "tflops_dense_equiv_table": flops / (res["table"] / 1e3) / 1e12}
+    del Ws, Gs, Ms
+    mc.release_workspaces()
+    torch.cuda.empty_cache()
+    return out
+
+
 def main(argv=None):
     args = parse_args(argv)
     world = int(os.environ.get("WORLD_SIZE", "1"))
@@ -343,6 +424,10 @@ def main(argv=None):
                "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h)}
         del g_host, x_host
 
+    extras = None
+    if not args.no_extras:
+        extras = time_extras(mc, wl, dev, stream, hp, args.steps, peaks, barrier, max_over_ranks)
+
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         ts, f = oracle_sample_seconds(1)
@@ -368,6 +453,7 @@ def main(argv=None):
                 "elementwise_pct_hbm": (100.0 * elem_gbs / peaks["hbm_gbs"]) if elem_gbs else None,
                 "qk_max_tokens_per_s": qk_tokens},
             "kernels": per,
+            "extras": extras,
             "roofline": roof,
             "cpu_baseline": cpu,
             "e2e": e2e,

@@ -7,6 +7,9 @@
  *   mc_muon_step     the Muon update of a list of hidden 2D weights
  *   mc_qk_max_logit  per-head causal max of the pre-softmax logit (S_max)
  *   mc_qk_clip       QK-Clip: rescale the W_q / W_k rows of heads with S_max > tau
+ *   mc_qk_clip_slices   QK-Clip over an explicit slice map (multi-head latent
+ *                       attention, fused projection layouts)
+ *   mc_mla_max_logit    S_max of multi-head latent attention (content + rotary parts)
  *
  * Conventions for every call
  *   - All pointers named "device" are CUDA device pointers on the current
@@ -69,6 +72,11 @@ typedef struct {
   float a, b, c;      /* quintic coefficients (3.4445, -4.7750, 2.0315) */
   float eps;          /* normalisation floor: X0 = U / max(||U||_F, eps) (1e-7) */
   float rms_scale;    /* update scale factor: rms_scale*sqrt(max(rows,cols)) (0.2) */
+  const float* coeffs; /* optional host array of 3*ns_steps floats: (a_k, b_k, c_k)
+                          for iteration k, e.g. the classic cubic (1.5, -0.5, 0) or
+                          the simple quintic (2, -1.5, 0.5) of "Muon and MuonClip:
+                          orthogonalised updates for LLM training" §2, or a
+                          per-step schedule; NULL = (a, b, c) in every iteration */
 } mc_hparams;
 
 /*
@@ -80,6 +88,7 @@ typedef struct {
  *   U <- G + mu*M  (nesterov) or M
  *   X0 <- U / max(||U||_F, eps), with the short side first (U^T when rows > cols)
  *   ns_steps times:  A = X X^T;  B = b*A + c*A*A;  X <- a*X + B*X
+ *                    (with (a, b, c) taken from hp->coeffs per iteration if set)
  *   O <- X in the weight's orientation
  *   W <- W - lr*(rms_scale*sqrt(max(rows,cols))*O + wd*W)
  * The Newton-Schulz products run on tcgen05 tensor cores with bf16 operands
@@ -140,6 +149,79 @@ int mc_qk_max_logit(const void* x, const void* wq, const void* wk, int B, int S,
  */
 int mc_qk_clip(void* wq, void* wk, int H, int dh, int D, const float* smax, float tau, float alpha,
                float* gamma_out, int32_t* mask_out, void* stream);
+
+/*
+ * mc_clip_slice -- one block of weight rows that QK-Clip rescales with the
+ * factor of one head.  Rows [row_begin, row_end) of the row-major matrix at
+ * `w` (`cols` elements per row, dtype MC_BF16 or MC_F32) are multiplied by
+ * gamma_head ^ exponent when head `head` clips.
+ */
+typedef struct mc_clip_slice {
+  void* w;            /* device, 16-byte aligned base of the matrix */
+  int64_t row_begin;  /* first row, >= 0 */
+  int64_t row_end;    /* one past the last row, > row_begin */
+  int64_t cols;       /* elements per row (the row stride), >= 1 */
+  int32_t dtype;      /* MC_BF16 or MC_F32 */
+  int32_t head;       /* index into smax, in [0, H) */
+  float exponent;     /* in [0, 1] */
+  int32_t reserved;   /* set to 0 */
+} mc_clip_slice;
+
+/*
+ * mc_qk_clip_slices -- QK-Clip where the rescaled tensors are named by an
+ * explicit map ("MuonClip: speed, then stability" §06, and its §12 item on
+ * identifying the physical slices; "Muon and MuonClip: orthogonalised updates
+ * for LLM training", "MuonClip: QK-clip, per head, adapted to MLA"):
+ *   gamma_h = tau / S_max[h] if S_max[h] > tau, else 1
+ *   for every slice: its rows *= gamma_head ^ exponent
+ * For multi-head latent attention the map holds, per head h, the rows of the
+ * head-specific content query q^C_h and content key k^C_h with exponent 1/2
+ * and the rows of the head-specific rotary query q^R_h with exponent 1; the
+ * rotary key that every head shares is not in the map and is never written.
+ * Plain MHA is the map {W_q rows of h: alpha, W_k rows of h: 1 - alpha}.
+ * Slices may live in different matrices, in one fused projection matrix
+ * (e.g. per-head [content | rotary] row blocks) or in both; rows outside
+ * every slice and rows of heads that do not clip are left bit-for-bit
+ * unchanged.  Computed on the device from `smax`; rows are rescaled in fp32
+ * and rounded to nearest-even into their dtype.
+ *
+ * slices     HOST array of n entries (read during the call only); no two
+ *            slices may overlap in memory (MC_ERR_INVAL otherwise)
+ * smax       device fp32 [H]
+ * gamma_out  optional device fp32 [H] (NULL = skip)
+ * mask_out   optional device int32 [H]: 1 where clipped (NULL = skip)
+ * Errors: MC_ERR_INVAL (bad slice, head out of range, exponent outside
+ * [0, 1], overlap, tau not finite and > 0), MC_ERR_ALIGN.
+ */
+int mc_qk_clip_slices(const mc_clip_slice* slices, int n, const float* smax, int H, float tau,
+                      float* gamma_out, int32_t* mask_out, void* stream);
+
+/*
+ * mc_mla_max_logit -- per-head max pre-softmax logit of multi-head latent
+ * attention, whose score splits into a content part with a head-specific
+ * query and key and a rotary part whose key is shared by all heads
+ * ("MuonClip: speed, then stability" §06):
+ *   s_h(b, i, j) = (q^C_{b,i,h} . k^C_{b,j,h} + q^R_{b,i,h} . k^R_{b,j}) / sqrt(dc + dr)
+ *   q^C = X W_qC^T, k^C = X W_kC^T, q^R = X W_qR^T, k^R = X W_kR^T
+ *   S_max[h] = max over b, i and j <= i (all j when causal == 0)
+ * Position rotation is not applied (it does not change how the clip factors
+ * enter the score); pass already-rotated projections' weights if needed.
+ * The score matrix is never stored: the two parts are one tensor-core
+ * contraction of length dc + dr.  q^C, k^C, q^R and k^R are kept in bf16.
+ *
+ * x         device bf16 [B][S][D]
+ * wqc, wkc  device bf16 [H*dc][D]     (head h owns rows [h*dc, (h+1)*dc))
+ * wqr       device bf16 [H*dr][D]     (head h owns rows [h*dr, (h+1)*dr))
+ * wkr       device bf16 [dr][D]       (shared by every head)
+ * smax_out  device fp32 [H]
+ * workspace device, >= mc_mla_workspace_size(...) bytes, or NULL for an
+ *           engine-owned buffer
+ * Requirements: D and dr multiples of 8, dc a multiple of 64.
+ */
+size_t mc_mla_workspace_size(int B, int S, int D, int H, int dc, int dr);
+int mc_mla_max_logit(const void* x, const void* wqc, const void* wkc, const void* wqr, const void* wkr, int B,
+                     int S, int D, int H, int dc, int dr, int causal, float* smax_out, void* workspace,
+                     size_t workspace_bytes, void* stream);
 
 /*
  * mc_qk_max_logit_static -- the same S_max as mc_qk_max_logit, but without a

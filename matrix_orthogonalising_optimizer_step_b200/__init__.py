@@ -23,7 +23,7 @@ MC_F32, MC_BF16 = 0, 1
 # Names the C ABI exports (include/muonclip.h).
 EXPORTS = ("mc_muon_workspace_size", "mc_muon_step", "mc_qk_workspace_size", "mc_qk_max_logit",
            "mc_qk_clip", "mc_last_error", "mc_device_status", "mc_profile_begin", "mc_profile_end",
-           "mc_qk_max_logit_static")
+           "mc_qk_max_logit_static", "mc_qk_clip_slices", "mc_mla_workspace_size", "mc_mla_max_logit")
 MC_QK_STATIC_MAX_ELEMS = 1 << 24
 MC_QK_STATIC_MAX_HEADS = 4096
 
@@ -39,7 +39,13 @@ class McHparams(ctypes.Structure):
     _fields_ = [("mu", ctypes.c_float), ("nesterov", ctypes.c_int32), ("lr", ctypes.c_float),
                 ("wd", ctypes.c_float), ("ns_steps", ctypes.c_int32), ("a", ctypes.c_float),
                 ("b", ctypes.c_float), ("c", ctypes.c_float), ("eps", ctypes.c_float),
-                ("rms_scale", ctypes.c_float)]
+                ("rms_scale", ctypes.c_float), ("coeffs", ctypes.c_void_p)]
+
+
+class McClipSlice(ctypes.Structure):
+    _fields_ = [("w", ctypes.c_void_p), ("row_begin", ctypes.c_int64), ("row_end", ctypes.c_int64),
+                ("cols", ctypes.c_int64), ("dtype", ctypes.c_int32), ("head", ctypes.c_int32),
+                ("exponent", ctypes.c_float), ("reserved", ctypes.c_int32)]
 
 
 class McKernelStat(ctypes.Structure):
@@ -84,6 +90,12 @@ def load_library():
     lib.mc_device_status.restype = i32
     lib.mc_qk_max_logit_static.argtypes = [vp, vp, vp, i32, i32, i32, i32, i32, i32, vp, vp]
     lib.mc_qk_max_logit_static.restype = i32
+    lib.mc_qk_clip_slices.argtypes = [P(McClipSlice), i32, vp, i32, ctypes.c_float, vp, vp, vp]
+    lib.mc_qk_clip_slices.restype = i32
+    lib.mc_mla_workspace_size.argtypes = [i32] * 6
+    lib.mc_mla_workspace_size.restype = sz
+    lib.mc_mla_max_logit.argtypes = [vp, vp, vp, vp, vp] + [i32] * 7 + [vp, vp, sz, vp]
+    lib.mc_mla_max_logit.restype = i32
     lib.mc_profile_begin.argtypes = []
     lib.mc_profile_begin.restype = i32
     lib.mc_profile_end.argtypes = [P(McKernelStat), i32, P(ctypes.c_int)]
@@ -161,9 +173,20 @@ def _need_cuda_contig(t, name):
 
 
 def make_hparams(mu=0.95, nesterov=True, lr=0.02, wd=0.1, ns_steps=5, a=3.4445, b=-4.7750,
-                 c=2.0315, eps=1e-7, rms_scale=0.2) -> McHparams:
-    return McHparams(float(mu), int(bool(nesterov)), float(lr), float(wd), int(ns_steps),
-                     float(a), float(b), float(c), float(eps), float(rms_scale))
+                 c=2.0315, eps=1e-7, rms_scale=0.2, coeffs=None) -> McHparams:
+    """``coeffs``: optional list of ns_steps (a_k, b_k, c_k) triples, one per
+    Newton-Schulz iteration.  The returned struct keeps the coefficient array
+    alive (as ``_coeff_buf``)."""
+    h = McHparams(float(mu), int(bool(nesterov)), float(lr), float(wd), int(ns_steps),
+                  float(a), float(b), float(c), float(eps), float(rms_scale), None)
+    if coeffs is not None:
+        flat = [float(v) for t in coeffs for v in t]
+        if len(flat) != 3 * int(ns_steps):
+            raise ValueError("coeffs must hold one (a, b, c) triple per Newton-Schulz step")
+        buf = (ctypes.c_float * len(flat))(*flat)
+        h._coeff_buf = buf
+        h.coeffs = ctypes.cast(buf, ctypes.c_void_p)
+    return h
 
 
 def make_params(weights, grads, moms, update_outs=None):
@@ -284,6 +307,74 @@ def qk_clip(wq, wk, smax, H: int, dh: int, *, tau: float = 100.0, alpha: float =
     _check(lib.mc_qk_clip(_ptr(wq), _ptr(wk), H, dh, D, _ptr(smax), float(tau), float(alpha),
                           _ptr(gamma_out), _ptr(mask_out), _stream_handle(stream)))
     return gamma_out, mask_out
+
+
+def make_clip_slices(slices):
+    """ctypes array of McClipSlice from (weight, head, row_begin, row_end,
+    exponent) tuples; each weight is a contiguous 2D CUDA tensor (bf16 or fp32)."""
+    arr = (McClipSlice * max(len(slices), 1))()
+    for i, (w, head, r0, r1, e) in enumerate(slices):
+        _need_cuda_contig(w, f"slices[{i}] weight")
+        if w.dim() != 2:
+            raise ValueError(f"slices[{i}]: weight must be 2D")
+        arr[i] = McClipSlice(_ptr(w), int(r0), int(r1), int(w.shape[1]), _dtype_code(w), int(head), float(e), 0)
+    return arr, len(slices)
+
+
+def mla_slices(wqc, wkc, wqr, H: int, dc: int, dr: int):
+    """The MLA slice map: per head h, rows of the content query and key with
+    exponent 1/2 and rows of the rotary query with exponent 1 (the shared
+    rotary key has no entry, so it is never written)."""
+    out = []
+    for h in range(H):
+        out += [(wqc, h, h * dc, (h + 1) * dc, 0.5), (wkc, h, h * dc, (h + 1) * dc, 0.5),
+                (wqr, h, h * dr, (h + 1) * dr, 1.0)]
+    return out
+
+
+def qk_clip_slices(slices, smax, H: int, *, tau: float = 100.0, gamma_out=None, mask_out=None, stream=None):
+    """QK-Clip in place over an explicit slice map (see mc_qk_clip_slices).
+    Returns (gamma [H] fp32, mask [H] int32)."""
+    torch = _torch()
+    lib = load_library()
+    _need_cuda_contig(smax, "smax")
+    arr, n = make_clip_slices(slices)
+    if gamma_out is None:
+        gamma_out = torch.empty(H, dtype=torch.float32, device=smax.device)
+    if mask_out is None:
+        mask_out = torch.empty(H, dtype=torch.int32, device=smax.device)
+    _check(lib.mc_qk_clip_slices(arr, n, _ptr(smax), H, float(tau), _ptr(gamma_out), _ptr(mask_out),
+                                 _stream_handle(stream)))
+    return gamma_out, mask_out
+
+
+def mla_workspace_size(B, S, D, H, dc, dr) -> int:
+    return int(load_library().mc_mla_workspace_size(B, S, D, H, dc, dr))
+
+
+def mla_max_logit(x, wqc, wkc, wqr, wkr, H: int, dc: int, dr: int, *, causal: bool = True, smax_out=None,
+                  workspace=None, stream=None):
+    """Per-head S_max (fp32 [H]) of multi-head latent attention: content part
+    x W_qC^T . x W_kC^T per head plus rotary part x W_qR^T . x W_kR^T with one
+    shared rotary key, over sqrt(dc + dr) (see mc_mla_max_logit)."""
+    torch = _torch()
+    lib = load_library()
+    for t, nm in ((x, "x"), (wqc, "wqc"), (wkc, "wkc"), (wqr, "wqr"), (wkr, "wkr")):
+        _need_cuda_contig(t, nm)
+        if t.dtype != torch.bfloat16:
+            raise TypeError(f"{nm} must be bfloat16")
+    B, S, D = x.shape
+    if smax_out is None:
+        smax_out = torch.empty(H, dtype=torch.float32, device=x.device)
+    need = int(lib.mc_mla_workspace_size(B, S, D, H, dc, dr))
+    if need == 0:
+        _check(lib.mc_mla_max_logit(None, None, None, None, None, B, S, D, H, dc, dr, int(causal), None, None, 0,
+                                    None))
+    ws = workspace if workspace is not None else _workspace("mla", x.device, need)
+    _check(lib.mc_mla_max_logit(_ptr(x), _ptr(wqc), _ptr(wkc), _ptr(wqr), _ptr(wkr), B, S, D, H, dc, dr,
+                                int(causal), _ptr(smax_out), _ptr(ws), int(ws.numel() * ws.element_size()),
+                                _stream_handle(stream)))
+    return smax_out
 
 
 def qk_max_logit_static(x, wq, wk, H: int, dh: int, *, causal: bool = True, smax_out=None, stream=None):

@@ -206,10 +206,11 @@ int map_batched(CUtensorMap* map, const void* base, int64_t count, int64_t rows,
 
 // ----------------------------------------------------------- profiling
 enum Kind : int { K_MOMENTUM, K_FINALIZE, K_GRAM, K_POLY, K_APPLY_MIXED, K_APPLY, K_APPLY_FINAL, K_QK_PROJ,
-                  K_QK_CMAX, K_QK_KEYS, K_QK_CLIP, K_COUNT };
+                  K_QK_CMAX, K_QK_KEYS, K_QK_CLIP, K_MLA_PROJ, K_MLA_CMAX, K_QK_CLIP_SLICES, K_COUNT };
 const char* const kKindNames[K_COUNT] = {"momentum",  "norm_finalize",  "ns_gram", "ns_poly",
                                          "ns_apply_mixed", "ns_apply", "ns_apply_final", "qk_proj",
-                                         "qk_causal_max", "qk_keys", "qk_clip"};
+                                         "qk_causal_max", "qk_keys", "qk_clip", "mla_proj",
+                                         "mla_causal_max", "qk_clip_slices"};
 struct ProfRec {
   int kind;
   cudaEvent_t b, e;
@@ -327,6 +328,9 @@ int validate_muon(const mc_param* params, int n, const mc_hparams* hp) {
   const float vals[] = {hp->mu, hp->lr, hp->wd, hp->a, hp->b, hp->c, hp->eps, hp->rms_scale};
   for (float v : vals)
     if (!std::isfinite(v)) return fail(MC_ERR_INVAL, "non-finite hyper-parameter");
+  if (hp->coeffs)
+    for (int i = 0; i < 3 * hp->ns_steps; ++i)
+      if (!std::isfinite(hp->coeffs[i])) return fail(MC_ERR_INVAL, "non-finite coefficient in hp->coeffs");
   if (!(hp->eps > 0.f)) return fail(MC_ERR_INVAL, "eps must be > 0");
   for (int i = 0; i < n; ++i) {
     const mc_param& q = params[i];
@@ -538,6 +542,9 @@ MC_API int mc_muon_step(const mc_param* params, int n, const mc_hparams* hp, voi
     const int par = it & 1;
     const bool first = it == 0, last = it + 1 == hp->ns_steps;
     const bool mixed = it < kMixedIters;
+    const float ca = hp->coeffs ? hp->coeffs[3 * it] : hp->a;
+    const float cb = hp->coeffs ? hp->coeffs[3 * it + 1] : hp->b;
+    const float cc = hp->coeffs ? hp->coeffs[3 * it + 2] : hp->c;
     for (int g0 = 0; g0 < ng; g0 += MAX_GROUPS) {
       const int g1 = std::min(ng, g0 + MAX_GROUPS);
       GemmParams gram, poly, apply;
@@ -579,9 +586,9 @@ MC_API int mc_muon_step(const mc_param* params, int n, const mc_hparams* hp, voi
         G.d = ws + g.off_b;
         G.d_ld = g.ldm;
         G.d_bs = g.m * g.ldm;
-        G.coef_acc = hp->c;
-        G.coef_src = hp->b;
-        G.diag = mixed ? 0.f : hp->a;
+        G.coef_acc = cc;
+        G.coef_src = cb;
+        G.diag = mixed ? 0.f : ca;
         poly.map_a[slot] = Mp.a_k;
         poly.map_b[slot] = Mp.a_k;
         finish_group(poly, slot, G, 1);
@@ -611,7 +618,7 @@ MC_API int mc_muon_step(const mc_param* params, int n, const mc_hparams* hp, voi
         G.d_ld = g.ld;
         G.d_bs = g.rows * g.ld;
         G.scale = first ? scale : nullptr;
-        G.coef_src = hp->a;
+        G.coef_src = ca;
         if (last) {
           G.w_ptrs = reinterpret_cast<void* const*>(ws + g.off_wptr);
           bool any_u = false;
@@ -781,6 +788,230 @@ MC_API int mc_qk_clip(void* wq, void* wk, int H, int dh, int D, const float* sma
   qk_clip_kernel<<<grid, 256, 0, s>>>(static_cast<__nv_bfloat16*>(wq), static_cast<__nv_bfloat16*>(wk), H, dh, D,
                                       smax, tau, alpha, gamma_out, mask_out, D % 8 == 0 ? 1 : 0);
   MC_CUDA(cudaGetLastError());
+  return MC_OK;
+}
+
+// =========================================================================
+// QK-Clip over an explicit slice map (MLA and fused projection layouts).
+MC_API int mc_qk_clip_slices(const mc_clip_slice* slices, int n, const float* smax, int H, float tau,
+                             float* gamma_out, int32_t* mask_out, void* stream) {
+  if (n < 0 || (n > 0 && !slices)) return fail(MC_ERR_INVAL, "slices must be non-NULL when n > 0, and n >= 0");
+  if (H < 1 || H > (1 << 24)) return fail(MC_ERR_INVAL, "H must be in [1, 2^24]");
+  if (!smax) return fail(MC_ERR_INVAL, "NULL smax");
+  if (!std::isfinite(tau) || !(tau > 0.f)) return fail(MC_ERR_INVAL, "tau must be finite and > 0");
+  if (!aligned16(smax) || (gamma_out && !aligned16(gamma_out)) || (mask_out && !aligned16(mask_out)))
+    return fail(MC_ERR_ALIGN, "pointers must be 16-byte aligned");
+  struct Span {
+    uintptr_t lo, hi;
+    int idx;
+  };
+  std::vector<Span> spans;
+  spans.reserve(static_cast<size_t>(n));
+  for (int i = 0; i < n; ++i) {
+    const mc_clip_slice& c = slices[i];
+    const std::string at = "slices[" + std::to_string(i) + "]: ";
+    if (!c.w) return fail(MC_ERR_INVAL, at + "NULL w");
+    if (c.dtype != MC_F32 && c.dtype != MC_BF16) return fail(MC_ERR_INVAL, at + "dtype must be MC_F32 or MC_BF16");
+    if (c.reserved != 0) return fail(MC_ERR_INVAL, at + "reserved must be 0");
+    if (c.cols < 1 || c.row_begin < 0 || c.row_end <= c.row_begin)
+      return fail(MC_ERR_INVAL, at + "need cols >= 1 and 0 <= row_begin < row_end");
+    if (c.row_end > (int64_t(1) << 40) / c.cols || c.row_end - c.row_begin > INT_MAX)
+      return fail(MC_ERR_INVAL, at + "slice too large");
+    if (c.head < 0 || c.head >= H) return fail(MC_ERR_INVAL, at + "head out of [0, H)");
+    if (!std::isfinite(c.exponent) || c.exponent < 0.f || c.exponent > 1.f)
+      return fail(MC_ERR_INVAL, at + "exponent must be in [0, 1]");
+    if (!aligned16(c.w)) return fail(MC_ERR_ALIGN, at + "w must be 16-byte aligned");
+    const uintptr_t es = c.dtype == MC_F32 ? 4 : 2;
+    const uintptr_t base = reinterpret_cast<uintptr_t>(c.w);
+    spans.push_back({base + uintptr_t(c.row_begin) * uintptr_t(c.cols) * es,
+                     base + uintptr_t(c.row_end) * uintptr_t(c.cols) * es, i});
+  }
+  std::sort(spans.begin(), spans.end(), [](const Span& a, const Span& b) { return a.lo < b.lo; });
+  for (size_t i = 1; i < spans.size(); ++i)
+    if (spans[i].lo < spans[i - 1].hi)
+      return fail(MC_ERR_INVAL, "slices[" + std::to_string(spans[i - 1].idx) + "] and slices[" +
+                                    std::to_string(spans[i].idx) + "] overlap in memory");
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  std::lock_guard<std::mutex> lock(g_mu);
+  DeviceState* st = nullptr;
+  int rc = device_state(&st);
+  if (rc != MC_OK) return rc;
+  if (gamma_out || mask_out) {
+    ProfScope prof(K_QK_KEYS, s);
+    qk_gamma_kernel<<<(H + 255) / 256, 256, 0, s>>>(smax, H, tau, gamma_out, mask_out);
+    MC_CUDA(cudaGetLastError());
+  }
+  ClipTable T;
+  std::memset(&T, 0, sizeof(T));
+  double bytes = 0;
+  auto flush = [&]() -> int {
+    if (T.n == 0) return MC_OK;
+    ProfScope prof(K_QK_CLIP_SLICES, s, 0, 0, bytes);
+    qk_clip_slices_kernel<<<static_cast<unsigned>(T.row_end[T.n - 1]), 256, 0, s>>>(T, smax, tau);
+    MC_CUDA(cudaGetLastError());
+    std::memset(&T, 0, sizeof(T));
+    bytes = 0;
+    return MC_OK;
+  };
+  for (int i = 0; i < n; ++i) {
+    const mc_clip_slice& c = slices[i];
+    if (c.exponent == 0.f) continue;  // gamma^0 = 1: nothing to write
+    const long long rows = c.row_end - c.row_begin;
+    const long long prev = T.n ? T.row_end[T.n - 1] : 0;
+    if (T.n == CLIP_MAX_SLICES || prev + rows > INT_MAX) {
+      if ((rc = flush()) != MC_OK) return rc;
+    }
+    const long long base = T.n ? T.row_end[T.n - 1] : 0;
+    const int es = c.dtype == MC_F32 ? 4 : 2;
+    ClipSlice& d = T.s[T.n];
+    d.w = c.w;
+    d.row_begin = c.row_begin;
+    d.cols = c.cols;
+    d.exponent = c.exponent;
+    d.head = c.head;
+    d.f32 = c.dtype == MC_F32 ? 1 : 0;
+    d.vec = (c.cols * es) % 16 == 0 ? 1 : 0;
+    T.row_end[T.n] = base + rows;
+    ++T.n;
+    bytes += 2.0 * double(rows) * double(c.cols) * es;  // read + write if the head clips
+  }
+  return flush();
+}
+
+// =========================================================================
+// Per-head causal max logit of multi-head latent attention.
+namespace {
+struct MlaLayout {
+  size_t off_qc, off_kc, off_qr, off_kr, off_keys, total;
+};
+MlaLayout plan_mla(int B, int S, int H, int dc, int dr) {
+  MlaLayout L;
+  const size_t bs = size_t(B) * size_t(S);
+  L.off_qc = 0;
+  L.off_kc = align_up(L.off_qc + 2 * bs * size_t(H) * size_t(dc), 1024);
+  L.off_qr = align_up(L.off_kc + 2 * bs * size_t(H) * size_t(dc), 1024);
+  L.off_kr = align_up(L.off_qr + 2 * bs * size_t(H) * size_t(dr), 1024);
+  L.off_keys = align_up(L.off_kr + 2 * bs * size_t(dr), 1024);
+  L.total = align_up(L.off_keys + sizeof(int) * size_t(H), 1024);
+  return L;
+}
+int validate_mla_dims(int B, int S, int D, int H, int dc, int dr) {
+  if (B < 1 || S < 1 || D < 1 || H < 1 || dc < 1 || dr < 1)
+    return fail(MC_ERR_INVAL, "B, S, D, H, dc, dr must be >= 1");
+  if (D % 8 || dr % 8) return fail(MC_ERR_INVAL, "D and dr must be multiples of 8");
+  if (dc % BK) return fail(MC_ERR_INVAL, "dc must be a multiple of 64");
+  if (int64_t(B) * S > (int64_t(1) << 31) - 1 || int64_t(H) * dc > (1 << 24) || int64_t(H) * dr > (1 << 24) ||
+      D > (1 << 24))
+    return fail(MC_ERR_INVAL, "problem too large");
+  return MC_OK;
+}
+}  // namespace
+
+MC_API size_t mc_mla_workspace_size(int B, int S, int D, int H, int dc, int dr) {
+  if (validate_mla_dims(B, S, D, H, dc, dr) != MC_OK) return 0;
+  return plan_mla(B, S, H, dc, dr).total;
+}
+
+MC_API int mc_mla_max_logit(const void* x, const void* wqc, const void* wkc, const void* wqr, const void* wkr,
+                            int B, int S, int D, int H, int dc, int dr, int causal, float* smax_out,
+                            void* workspace, size_t workspace_bytes, void* stream) {
+  int rc = validate_mla_dims(B, S, D, H, dc, dr);
+  if (rc != MC_OK) return rc;
+  if (!x || !wqc || !wkc || !wqr || !wkr || !smax_out)
+    return fail(MC_ERR_INVAL, "NULL x, wqc, wkc, wqr, wkr or smax_out");
+  if (!aligned16(x) || !aligned16(wqc) || !aligned16(wkc) || !aligned16(wqr) || !aligned16(wkr) ||
+      !aligned16(smax_out) || (workspace && !aligned16(workspace)))
+    return fail(MC_ERR_ALIGN, "pointers must be 16-byte aligned");
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  std::lock_guard<std::mutex> lock(g_mu);
+  DeviceState* st = nullptr;
+  if ((rc = device_state(&st)) != MC_OK) return rc;
+  const MlaLayout L = plan_mla(B, S, H, dc, dr);
+  if (workspace) {
+    if (workspace_bytes < L.total)
+      return fail(MC_ERR_NOSPC, "workspace has " + std::to_string(workspace_bytes) + " bytes, needs " +
+                                    std::to_string(L.total));
+  } else if ((rc = own_workspace(*st, L.total, &workspace)) != MC_OK) {
+    return rc;
+  }
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  int* keys = reinterpret_cast<int*>(ws + L.off_keys);
+  const int64_t BS = int64_t(B) * S;
+  {
+    ProfScope prof(K_QK_KEYS, s);
+    qk_keys_init_kernel<<<(H + 255) / 256, 256, 0, s>>>(keys, H);
+    MC_CUDA(cudaGetLastError());
+  }
+
+  // q^C = X W_qC^T, k^C = X W_kC^T, q^R = X W_qR^T, k^R = X W_kR^T: one launch.
+  GemmParams proj;
+  std::memset(&proj, 0, sizeof(proj));
+  proj.err = st->err_ptr;
+  const void* wts[4] = {wqc, wkc, wqr, wkr};
+  const int outs[4] = {H * dc, H * dc, H * dr, dr};
+  const size_t offs[4] = {L.off_qc, L.off_kc, L.off_qr, L.off_kr};
+  double proj_flops = 0;
+  for (int which = 0; which < 4; ++which) {
+    if ((rc = map_batched(&proj.map_a[which], x, 1, BS, D, D, HALF)) != MC_OK) return rc;
+    if ((rc = map_batched(&proj.map_b[which], wts[which], 1, outs[which], D, D, HALF)) != MC_OK) return rc;
+    GemmGroup G;
+    std::memset(&G, 0, sizeof(G));
+    G.M = static_cast<int>(BS);
+    G.N = outs[which];
+    G.K = D;
+    G.count = 1;
+    G.sched = SCHED_DENSE;
+    G.layout = LAYOUT_BATCHED;
+    G.heads = 1;
+    G.band = 8;
+    G.d = ws + offs[which];
+    G.d_ld = outs[which];
+    finish_group(proj, which, G, 1);
+    proj_flops += 2.0 * double(BS) * outs[which] * D;
+  }
+  if ((rc = launch_gemm<EPI_STORE, 1>(proj, *st, s, K_MLA_PROJ, proj_flops)) != MC_OK) return rc;
+
+  // s_h(i, j) = (q^C_hi . k^C_hj + q^R_hi . k^R_j) / sqrt(dc + dr): one contraction
+  // of length dc + dr whose first dc columns come from the content pair and
+  // the rest from the rotary pair (the rotary key has a single shared head).
+  GemmParams cm;
+  std::memset(&cm, 0, sizeof(cm));
+  cm.err = st->err_ptr;
+  {
+    const uint32_t box[4] = {64, 1, HALF, 1};
+    const uint64_t dc_dims[4] = {uint64_t(dc), uint64_t(H), uint64_t(S), uint64_t(B)};
+    const uint64_t dc_str[3] = {uint64_t(dc) * 2, uint64_t(H) * dc * 2, uint64_t(S) * H * dc * 2};
+    const uint64_t qr_dims[4] = {uint64_t(dr), uint64_t(H), uint64_t(S), uint64_t(B)};
+    const uint64_t qr_str[3] = {uint64_t(dr) * 2, uint64_t(H) * dr * 2, uint64_t(S) * H * dr * 2};
+    const uint64_t kr_dims[4] = {uint64_t(dr), 1, uint64_t(S), uint64_t(B)};
+    const uint64_t kr_str[3] = {uint64_t(dr) * 2, uint64_t(dr) * 2, uint64_t(S) * dr * 2};
+    if ((rc = make_map(&cm.map_a[0], ws + L.off_qc, 4, dc_dims, dc_str, box)) != MC_OK) return rc;
+    if ((rc = make_map(&cm.map_b[0], ws + L.off_kc, 4, dc_dims, dc_str, box)) != MC_OK) return rc;
+    if ((rc = make_map(&cm.map_a[1], ws + L.off_qr, 4, qr_dims, qr_str, box)) != MC_OK) return rc;
+    if ((rc = make_map(&cm.map_b[1], ws + L.off_kr, 4, kr_dims, kr_str, box)) != MC_OK) return rc;
+    GemmGroup G;
+    std::memset(&G, 0, sizeof(G));
+    G.M = G.N = S;
+    G.K = dc + dr;
+    G.k_split = dc;
+    G.count = B * H;
+    G.heads = H;
+    G.layout = LAYOUT_HEADS;
+    G.sched = causal ? SCHED_CAUSAL : SCHED_DENSE;
+    G.band = 8;
+    G.mask_causal = causal ? 1 : 0;
+    G.keys = keys;
+    G.out_scale = 1.f / std::sqrt(static_cast<float>(dc + dr));
+    finish_group(cm, 0, G, 0);
+  }
+  const double pairs = causal ? double(S) * (double(S) + 1) / 2 : double(S) * S;
+  if ((rc = launch_gemm<EPI_CAUSALMAX, 0>(cm, *st, s, K_MLA_CMAX, 2.0 * (dc + dr) * pairs * B * H)) != MC_OK)
+    return rc;
+  {
+    ProfScope prof(K_QK_KEYS, s);
+    qk_keys_decode_kernel<<<(H + 255) / 256, 256, 0, s>>>(keys, smax_out, H);
+    MC_CUDA(cudaGetLastError());
+  }
   return MC_OK;
 }
 

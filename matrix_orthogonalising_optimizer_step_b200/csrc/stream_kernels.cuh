@@ -12,6 +12,16 @@
 //  qk_clip_kernel    gamma_h = tau / S_max_h when S_max_h > tau; rows of head h
 //                    in W_q scaled by gamma^alpha, in W_k by gamma^(1-alpha)
 //                    ("MuonClip: speed, then stability", §05).
+//  qk_gamma_kernel   gamma_h and the clipped-head mask alone.
+//  qk_clip_slices_kernel
+//                    the same rescale over an explicit map of weight slices,
+//                    each with its head and exponent: multi-head latent
+//                    attention scales the head's content query and content key
+//                    by gamma^(1/2) and its rotary query by gamma, and leaves
+//                    the rotary key that all heads share alone ("MuonClip:
+//                    speed, then stability", §06; "Muon and MuonClip:
+//                    orthogonalised updates for LLM training", "MuonClip:
+//                    QK-clip, per head, adapted to MLA").
 #pragma once
 
 #include <climits>
@@ -208,6 +218,78 @@ __global__ void qk_clip_kernel(__nv_bfloat16* __restrict__ wq, __nv_bfloat16* __
     }
   } else {
     for (int c = threadIdx.x; c < D; c += blockDim.x) w[c] = __float2bfloat16_rn(__bfloat162float(w[c]) * f);
+  }
+}
+
+__global__ void qk_gamma_kernel(const float* __restrict__ smax, int H, float tau, float* __restrict__ gamma_out,
+                                int* __restrict__ mask_out) {
+  const int h = blockIdx.x * blockDim.x + threadIdx.x;
+  if (h >= H) return;
+  const float s = smax[h];
+  const bool clip = s > tau;
+  if (gamma_out) gamma_out[h] = clip ? tau / s : 1.f;
+  if (mask_out) mask_out[h] = clip ? 1 : 0;
+}
+
+// One launch covers up to CLIP_MAX_SLICES slices; CTA b rescales one row,
+// the row of the slice whose cumulative row range holds b.
+constexpr int CLIP_MAX_SLICES = 48;
+struct ClipSlice {
+  void* w;               // row-major matrix, `cols` elements per row
+  long long row_begin;   // first row of the slice
+  long long cols;
+  float exponent;        // rows *= gamma_head ^ exponent
+  int head;
+  int f32;               // 1 fp32, 0 bf16
+  int vec;               // rows are 16-byte aligned and a whole number of 16-byte chunks
+};
+struct ClipTable {
+  ClipSlice s[CLIP_MAX_SLICES];
+  long long row_end[CLIP_MAX_SLICES];  // cumulative: slice i owns CTAs [row_end[i-1], row_end[i])
+  int n;
+};
+static_assert(sizeof(ClipTable) + 64 <= 4096, "clip table must fit the classic 4 KiB parameter limit");
+
+__global__ void qk_clip_slices_kernel(const __grid_constant__ ClipTable T, const float* __restrict__ smax,
+                                      float tau) {
+  const long long b = blockIdx.x;
+  int lo = 0, hi = T.n - 1;
+  while (lo < hi) {
+    const int mid = (lo + hi) >> 1;
+    if (T.row_end[mid] > b) hi = mid;
+    else lo = mid + 1;
+  }
+  const ClipSlice& S = T.s[lo];
+  const float sm = smax[S.head];
+  if (!(sm > tau)) return;  // S_max == tau (or NaN) does not clip: rows stay bit-for-bit
+  const float gamma = tau / sm;
+  const float f = S.exponent == 0.5f ? sqrtf(gamma) : (S.exponent == 1.f ? gamma : powf(gamma, S.exponent));
+  const long long row = S.row_begin + (b - (lo ? T.row_end[lo - 1] : 0));
+  if (S.f32) {
+    float* w = static_cast<float*>(S.w) + row * S.cols;
+    if (S.vec) {
+      for (long long c = threadIdx.x * 4; c < S.cols; c += blockDim.x * 4) {
+        float4 a = *reinterpret_cast<float4*>(w + c);
+        a.x *= f; a.y *= f; a.z *= f; a.w *= f;
+        *reinterpret_cast<float4*>(w + c) = a;
+      }
+    } else {
+      for (long long c = threadIdx.x; c < S.cols; c += blockDim.x) w[c] *= f;
+    }
+  } else {
+    __nv_bfloat16* w = static_cast<__nv_bfloat16*>(S.w) + row * S.cols;
+    if (S.vec) {
+      for (long long c = threadIdx.x * 8; c < S.cols; c += blockDim.x * 8) {
+        uint4 a = *reinterpret_cast<uint4*>(w + c);
+        uint32_t x[4] = {a.x, a.y, a.z, a.w};
+#pragma unroll
+        for (int i = 0; i < 4; ++i)
+          x[i] = pack_bf16x2(__uint_as_float(x[i] << 16) * f, __uint_as_float(x[i] & 0xFFFF0000u) * f);
+        *reinterpret_cast<uint4*>(w + c) = make_uint4(x[0], x[1], x[2], x[3]);
+      }
+    } else {
+      for (long long c = threadIdx.x; c < S.cols; c += blockDim.x) w[c] = __float2bfloat16_rn(__bfloat162float(w[c]) * f);
+    }
   }
 }
 

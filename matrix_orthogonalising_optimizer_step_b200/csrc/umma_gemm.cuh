@@ -117,6 +117,8 @@ struct GemmGroup {
   long long tiles_per_prob;
   long long tile_start;    // first global tile of this group
   int sched, layout, heads;
+  int k_split;             // LAYOUT_HEADS: contraction columns [0, k_split) come from
+                           // maps slot 0, the rest from slot 1 (0 = no split)
   int a_mn, b_mn;          // operand major-ness: 0 K-major, 1 MN-major
   int prob_base;           // index of problem 0 in the per-matrix scale table
   int band;                // dense raster: n-tiles per band
@@ -588,10 +590,18 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1) umma_gemm_kernel(const __grid
           const int k0 = kb * BK;
           if (G.layout == LAYOUT_HEADS) {
             const int bb = ti.prob / G.heads, hh = ti.prob % G.heads;
-            tma_load_4d_pair(sa, ma, fb, k0, hh, m0, bb);
+            // A split contraction concatenates two per-head operand pairs along K
+            // (MLA's content and rotary parts); the second key operand has one
+            // head shared by all query heads.
+            const bool second = G.k_split > 0 && k0 >= G.k_split;
+            const CUtensorMap* qa = second ? &P.map_a[1] : ma;
+            const CUtensorMap* kb_map = second ? &P.map_b[1] : mb;
+            const int kk = second ? k0 - G.k_split : k0;
+            const int hk = second ? 0 : hh;
+            tma_load_4d_pair(sa, qa, fb, kk, hh, m0, bb);
 #pragma unroll
             for (int h = 0; h < T::NB; ++h)
-              tma_load_4d_pair(sa + A_STAGE_BYTES + h * B_STAGE_BYTES, mb, fb, k0, hh, n0 + h * MMA_N, bb);
+              tma_load_4d_pair(sa + A_STAGE_BYTES + h * B_STAGE_BYTES, kb_map, fb, kk, hk, n0 + h * MMA_N, bb);
           } else {
             if (!G.a_mn) {
               tma_load_3d_pair(sa, ma, fb, k0, m0, ti.prob);

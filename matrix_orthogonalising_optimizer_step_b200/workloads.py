@@ -87,6 +87,10 @@ def cfg4_shapes(experts: int = 64, d_model: int = 2048, d_ff: int = 7168):
 
 
 CFG3 = dict(B=4, S=4096, D=4096, H=32, dh=128, hot_heads=(3, 17, 29), hot_scale=8.0)
+# Multi-head latent attention layer at the same scale: each head's 192-wide
+# query/key split into a 128-wide content part and a 64-wide rotary part (the
+# rotary key shared by all heads).
+MLA = dict(B=4, S=4096, D=4096, H=32, dc=128, dr=64, hot_heads=(3, 17, 29), hot_scale=8.0)
 
 
 # --------------------------------------------------------------------------
@@ -165,6 +169,33 @@ def qk_inputs(B: int, S: int, D: int, H: int, dh: int, *, seed: int = 3,
         Wk[h * dh:(h + 1) * dh] *= hot_scale
     return (to_dtype(X, torch.bfloat16), to_dtype(Wq, torch.bfloat16),
             to_dtype(Wk, torch.bfloat16))
+
+
+def mla_inputs(B: int, S: int, D: int, H: int, dc: int, dr: int, *, seed: int = 5,
+               hot_heads=(), hot_scale: float = 8.0, w_std: float = 0.02):
+    """X [B, S, D] and the MLA projection weights, all bf16 (nn.Linear layout):
+    W_qC, W_kC [H*dc, D], W_qR [H*dr, D], W_kR [dr, D].  The head-specific rows
+    (W_qC, W_kC, W_qR) of every head in ``hot_heads`` are multiplied by
+    ``hot_scale``; the shared W_kR is not."""
+    rng = rng_for(5, seed, B, S, D, H, dc, dr)
+    X = rng.standard_normal((B, S, D))
+    Wqc = rng.normal(0.0, w_std, (H * dc, D))
+    Wkc = rng.normal(0.0, w_std, (H * dc, D))
+    Wqr = rng.normal(0.0, w_std, (H * dr, D))
+    Wkr = rng.normal(0.0, w_std, (dr, D))
+    for h in hot_heads:
+        Wqc[h * dc:(h + 1) * dc] *= hot_scale
+        Wkc[h * dc:(h + 1) * dc] *= hot_scale
+        Wqr[h * dr:(h + 1) * dr] *= hot_scale
+    bf = torch.bfloat16
+    return (to_dtype(X, bf), {"W_qC": to_dtype(Wqc, bf), "W_kC": to_dtype(Wkc, bf),
+                              "W_qR": to_dtype(Wqr, bf), "W_kR": to_dtype(Wkr, bf)})
+
+
+def mla_layer_inputs():
+    c = MLA
+    return mla_inputs(c["B"], c["S"], c["D"], c["H"], c["dc"], c["dr"], seed=5,
+                      hot_heads=c["hot_heads"], hot_scale=c["hot_scale"])
 
 
 def cfg3_inputs():

@@ -11,6 +11,11 @@ Sources (page title, then section):
   "The exploding-logit problem" (S_max^h = (1/sqrt(d)) max_{samples,i,j} q_i.k_j),
   "MuonClip: QK-clip, per head, adapted to MLA" (MHA rule, alpha = 0.5).
 * [MS] "About Muon: Muon At Scale" -- "When Softmax Collapses" (same rule).
+* Multi-head latent attention: [MC] §06 "Multi-head latent attention changes
+  the surgery" and [MV] "MuonClip: QK-clip, per head, adapted to MLA" (the
+  head-specific content query q^C and content key k^C scale by sqrt(gamma_h),
+  the head-specific rotary query q^R by gamma_h, the shared rotary key k^R is
+  left untouched; [MC] §12 asks implementers to name the physical slices).
 
 Readings (also in DESIGN.md):
 
@@ -116,3 +121,71 @@ def qk_clip(Wq, Wk, smax, tau: float, alpha: float, H: int, dh: int):
             Wq[h * dh:(h + 1) * dh] *= gamma[h] ** alpha
             Wk[h * dh:(h + 1) * dh] *= gamma[h] ** (1.0 - alpha)
     return Wq, Wk, gamma, mask
+
+
+def qk_clip_slices(weights: dict, slices, smax, tau: float):
+    """QK-Clip over an explicit map of weight slices ([MC] §06, §12.5).
+
+    ``weights``: name -> 2D array (rows are output features).  ``slices``: list
+    of (name, head, row_begin, row_end, exponent); rows [row_begin, row_end) of
+    weights[name] are multiplied by gamma_head**exponent when that head clips.
+    MHA is the map {W_q rows of h: alpha, W_k rows of h: 1 - alpha}; MLA is
+    {q^C rows of h: 1/2, k^C rows of h: 1/2, q^R rows of h: 1} with the shared
+    k^R absent.  gamma_h = tau / S_max_h if S_max_h > tau else 1.  Returns
+    (new weights dict, gamma [H], mask [H]).
+    """
+    smax = np.asarray(smax, dtype=np.float64)
+    H = len(smax)
+    gamma = np.ones(H)
+    mask = np.zeros(H, dtype=np.int32)
+    for h in range(H):
+        if smax[h] > tau:
+            gamma[h] = tau / smax[h]
+            mask[h] = 1
+    out = {k: np.array(v, dtype=np.float64, copy=True) for k, v in weights.items()}
+    for (name, h, r0, r1, e) in slices:
+        if mask[h]:
+            out[name][r0:r1] *= gamma[h] ** e
+    return out, gamma, mask
+
+
+def mla_max_logit(X, w: dict, H: int, dc: int, dr: int, causal: bool = True,
+                  qk_bf16: bool = False) -> np.ndarray:
+    """Per-head max logit of a (simplified, uncompressed) multi-head latent
+    attention score, split into a content and a rotary part:
+
+      s_h(i, j) = (q^C_{h,i} . k^C_{h,j} + q^R_{h,i} . k^R_j) / sqrt(dc + dr)
+
+    with q^C = x W_qC[h], k^C = x W_kC[h], q^R = x W_qR[h] (head-specific rows)
+    and k^R = x W_kR (one rotary key shared by every head).  Positional
+    rotation is omitted: it does not change how the clip factors enter.
+    X is [B, S, D]; W_qC, W_kC are [H*dc, D], W_qR is [H*dr, D], W_kR [dr, D].
+    ``qk_bf16`` rounds the four projections to bf16, as ``qk_max_logit`` does.
+    """
+    X = np.asarray(X, dtype=np.float64)
+    B, S, _ = X.shape
+    keep = np.tril(np.ones((S, S), dtype=bool)) if causal else np.ones((S, S), dtype=bool)
+    scale = 1.0 / np.sqrt(dc + dr)
+    out = np.full(H, -np.inf)
+    for b in range(B):
+        qc = X[b] @ np.asarray(w["W_qC"], dtype=np.float64).T
+        kc = X[b] @ np.asarray(w["W_kC"], dtype=np.float64).T
+        qr = X[b] @ np.asarray(w["W_qR"], dtype=np.float64).T
+        kr = X[b] @ np.asarray(w["W_kR"], dtype=np.float64).T
+        if qk_bf16:
+            qc, kc, qr, kr = (round_bf16(t) for t in (qc, kc, qr, kr))
+        for h in range(H):
+            s = (qc[:, h * dc:(h + 1) * dc] @ kc[:, h * dc:(h + 1) * dc].T
+                 + qr[:, h * dr:(h + 1) * dr] @ kr.T) * scale
+            out[h] = max(out[h], float(np.max(np.where(keep, s, -np.inf))))
+    return out
+
+
+def mla_slices(H: int, dc: int, dr: int):
+    """The MLA slice map of [MC] §06: (name, head, row_begin, row_end, exponent)."""
+    sl = []
+    for h in range(H):
+        sl.append(("W_qC", h, h * dc, (h + 1) * dc, 0.5))
+        sl.append(("W_kC", h, h * dc, (h + 1) * dc, 0.5))
+        sl.append(("W_qR", h, h * dr, (h + 1) * dr, 1.0))
+    return sl

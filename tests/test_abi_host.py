@@ -118,3 +118,69 @@ def test_python_binding_fails_loudly_without_library(monkeypatch, tmp_path):
     monkeypatch.setattr(mc, "LIB_PATH", str(tmp_path / "missing.so"))
     with pytest.raises(RuntimeError, match="missing"):
         mc.load_library()
+
+
+def test_coefficient_table_validation(lib):
+    P = ctypes.byref
+    bad = mc.make_hparams(ns_steps=2, coeffs=[(1.5, float("nan"), 0.0), (2.0, -1.5, 0.5)])
+    assert lib.mc_muon_step(_params(1), 1, P(bad), None, 0, None, None) == mc.MC_ERR_INVAL
+    assert "coeffs" in mc.last_error()
+    with pytest.raises(ValueError):
+        mc.make_hparams(ns_steps=3, coeffs=[(1.5, -0.5, 0.0)])
+
+
+def _slice(w=0x100000, r0=0, r1=8, cols=64, dtype=mc.MC_BF16, head=0, e=0.5, reserved=0):
+    return mc.McClipSlice(w, r0, r1, cols, dtype, head, e, reserved)
+
+
+def test_clip_slices_argument_errors(lib):
+    def call(slices, n=None, smax=0x200000, H=4, tau=100.0):
+        arr = (mc.McClipSlice * max(len(slices), 1))(*slices)
+        return lib.mc_qk_clip_slices(arr, len(slices) if n is None else n, smax, H, tau, None, None, None)
+
+    ok = _slice()
+    assert lib.mc_qk_clip_slices(None, 1, 0x200000, 4, 100.0, None, None, None) == mc.MC_ERR_INVAL
+    assert call([ok], n=-1) == mc.MC_ERR_INVAL
+    assert call([ok], smax=0) == mc.MC_ERR_INVAL
+    assert call([ok], H=0) == mc.MC_ERR_INVAL
+    assert call([ok], tau=0.0) == mc.MC_ERR_INVAL
+    assert call([ok], tau=float("inf")) == mc.MC_ERR_INVAL
+    assert call([_slice(w=0)]) == mc.MC_ERR_INVAL
+    assert call([_slice(dtype=5)]) == mc.MC_ERR_INVAL
+    assert call([_slice(r0=8, r1=8)]) == mc.MC_ERR_INVAL
+    assert call([_slice(r0=-1)]) == mc.MC_ERR_INVAL
+    assert call([_slice(cols=0)]) == mc.MC_ERR_INVAL
+    assert call([_slice(head=4)]) == mc.MC_ERR_INVAL
+    assert call([_slice(head=-1)]) == mc.MC_ERR_INVAL
+    assert call([_slice(e=1.5)]) == mc.MC_ERR_INVAL
+    assert call([_slice(e=float("nan"))]) == mc.MC_ERR_INVAL
+    assert call([_slice(reserved=1)]) == mc.MC_ERR_INVAL
+    assert call([_slice(w=0x100008)]) == mc.MC_ERR_ALIGN
+    assert lib.mc_qk_clip_slices((mc.McClipSlice * 1)(ok), 1, 0x200004, 4, 100.0, None, None, None) == mc.MC_ERR_ALIGN
+    # overlapping rows of one matrix, and two base pointers whose ranges meet
+    assert call([_slice(r0=0, r1=8), _slice(r0=7, r1=9, head=1)]) == mc.MC_ERR_INVAL
+    assert "overlap" in mc.last_error()
+    assert call([_slice(r0=0, r1=8), _slice(w=0x100000 + 7 * 128, r0=0, r1=1, head=1)]) == mc.MC_ERR_INVAL
+    # smax is required even for an empty map
+    assert call([], n=0, smax=0) == mc.MC_ERR_INVAL
+
+
+def test_mla_argument_errors_and_workspace(lib):
+    a = (0x100000, 0x200000, 0x300000, 0x400000, 0x500000)
+    args = lambda **k: dict(dict(B=1, S=64, D=64, H=2, dc=64, dr=32, causal=1), **k)
+
+    def call(ptrs=a, smax=0x600000, **k):
+        d = args(**k)
+        return lib.mc_mla_max_logit(*ptrs, d["B"], d["S"], d["D"], d["H"], d["dc"], d["dr"], d["causal"],
+                                    smax, None, 0, None)
+    assert call(dc=32) == mc.MC_ERR_INVAL          # dc must be a multiple of 64
+    assert call(dr=12) == mc.MC_ERR_INVAL          # dr multiple of 8
+    assert call(dr=0) == mc.MC_ERR_INVAL
+    assert call(D=60) == mc.MC_ERR_INVAL
+    assert call(ptrs=(0,) + a[1:]) == mc.MC_ERR_INVAL
+    assert call(smax=0) == mc.MC_ERR_INVAL
+    assert call(ptrs=a[:4] + (0x500008,)) == mc.MC_ERR_ALIGN
+    n = lib.mc_mla_workspace_size(2, 128, 64, 4, 128, 64)
+    bs = 2 * 128
+    assert n >= 2 * bs * (2 * 4 * 128 + 4 * 64 + 64) + 4 * 4
+    assert lib.mc_mla_workspace_size(2, 128, 64, 4, 96, 64) == 0

@@ -54,6 +54,23 @@ def test_hparam_variants(hp, nesterov, ns_steps):
     check_all(mats, h, run_step(mats, h), f"nest{nesterov}-ns{ns_steps}")
 
 
+CUBIC = (1.5, -0.5, 0.0)          # "Muon and MuonClip: orthogonalised updates for LLM training", §2
+SIMPLE = (2.0, -1.5, 0.5)
+TUNED = (3.4445, -4.7750, 2.0315)
+
+
+@pytest.mark.parametrize("name,sched", [
+    ("cubic x12", [CUBIC] * 12),
+    ("simple quintic x8", [SIMPLE] * 8),
+    ("tuned x3 then simple x4", [TUNED] * 3 + [SIMPLE] * 4),
+])
+def test_coefficient_schedules(hp, name, sched):
+    h = dict(hp, ns_steps=len(sched), coeffs=sched)
+    mats = [wl.generic_matrix(256, 768, seed=31), wl.generic_matrix(768, 256, seed=32),
+            wl.cfg1_matrix(0, n=512)]
+    check_all(mats, h, run_step(mats, h), name)
+
+
 RAGGED = [(1, 1), (3, 5), (5, 3), (8, 1), (64, 64), (100, 37), (37, 100), (129, 129),
           (256, 256), (300, 520), (520, 300), (129, 1000), (1000, 129), (640, 384)]
 

@@ -330,3 +330,89 @@ def test_cubic_schedule_converges_to_polar_factor():
     cubic = tuple(GOLD["classic_cubic"]["value"])
     O = oracle.newton_schulz(G, 60, *TUNED, coeffs=[cubic] * 60)
     assert np.linalg.norm(O - u @ vt) <= 1e-9 * np.linalg.norm(u @ vt)
+
+
+# ------------------------------------------------------------ MLA QK-Clip
+def _mla_setup(seed=23, B=2, S=10, D=12, H=3, dc=4, dr=2):
+    rng = np.random.default_rng(seed)
+    X = rng.standard_normal((B, S, D))
+    w = {"W_qC": rng.standard_normal((H * dc, D)), "W_kC": rng.standard_normal((H * dc, D)),
+         "W_qR": rng.standard_normal((H * dr, D)), "W_kR": rng.standard_normal((dr, D))}
+    return X, w, H, dc, dr
+
+
+def test_mla_clip_worked_example():
+    g = GOLD["mla_clip_example"]
+    X, w, H, dc, dr = _mla_setup()
+    smax = np.array([g["smax"], 50.0, 80.0])
+    out, gamma, mask = oracle.qk_clip_slices(w, oracle.mla_slices(H, dc, dr), smax, g["tau"])
+    assert gamma[0] == pytest.approx(g["gamma"], abs=1e-15) and list(mask) == [1, 0, 0]
+    assert np.allclose(out["W_qC"][:dc], g["content_scale"] * w["W_qC"][:dc], rtol=1e-15, atol=0)
+    assert np.allclose(out["W_kC"][:dc], g["content_scale"] * w["W_kC"][:dc], rtol=1e-15, atol=0)
+    assert np.allclose(out["W_qR"][:dr], g["rotary_query_scale"] * w["W_qR"][:dr], rtol=1e-15, atol=0)
+    assert np.array_equal(out["W_kR"], w["W_kR"])          # shared rotary key untouched
+    for k in ("W_qC", "W_kC"):
+        assert np.array_equal(out[k][dc:], w[k][dc:])      # other heads untouched
+    assert np.array_equal(out["W_qR"][dr:], w["W_qR"][dr:])
+
+
+def test_mla_recomputed_max_logit_equals_tau():
+    """Both parts of the MLA score (content and rotary) scale by gamma, so a
+    clipped head comes back to exactly tau; unclipped heads are unchanged."""
+    X, w, H, dc, dr = _mla_setup(seed=24)
+    w["W_qC"][:4] *= 6.0
+    w["W_kC"][:4] *= 6.0
+    w["W_qR"][:2] *= 20.0
+    s0 = oracle.mla_max_logit(X, w, H, dc, dr)
+    tau = float(np.sort(s0)[-1]) / 3
+    out, gamma, mask = oracle.qk_clip_slices(w, oracle.mla_slices(H, dc, dr), s0, tau)
+    s1 = oracle.mla_max_logit(X, out, H, dc, dr)
+    assert mask.sum() >= 1
+    for h in range(H):
+        if mask[h]:
+            assert s1[h] == pytest.approx(tau, rel=1e-12)
+        else:
+            assert s1[h] == pytest.approx(s0[h], rel=1e-14)
+
+
+def test_mha_as_a_slice_map_equals_qk_clip():
+    rng = np.random.default_rng(25)
+    H, dh, D = 4, 3, 5
+    Wq, Wk = rng.standard_normal((H * dh, D)), rng.standard_normal((H * dh, D))
+    smax = np.array([300.0, 90.0, 101.0, -4.0])
+    alpha = 0.3
+    q2, k2, g1, m1 = oracle.qk_clip(Wq, Wk, smax, 100.0, alpha, H, dh)
+    sl = [s for h in range(H) for s in (("q", h, h * dh, (h + 1) * dh, alpha), ("k", h, h * dh, (h + 1) * dh, 1 - alpha))]
+    out, g2, m2 = oracle.qk_clip_slices({"q": Wq, "k": Wk}, sl, smax, 100.0)
+    assert np.array_equal(out["q"], q2) and np.array_equal(out["k"], k2)
+    assert np.array_equal(g1, g2) and np.array_equal(m1, m2)
+
+
+def test_mla_max_logit_bruteforce_tiny():
+    """The content + rotary split, with the rotary key shared by all heads,
+    equals an explicit loop over every pair and feature on a tiny case."""
+    X, w, H, dc, dr = _mla_setup(seed=26, B=1, S=5, D=4, H=2, dc=3, dr=2)
+    got = oracle.mla_max_logit(X, w, H, dc, dr)
+    want = np.full(H, -np.inf)
+    for h in range(H):
+        for i in range(5):
+            for j in range(i + 1):
+                s = 0.0
+                for e in range(dc):
+                    r = h * dc + e
+                    s += (X[0, i] @ w["W_qC"][r]) * (X[0, j] @ w["W_kC"][r])
+                for e in range(dr):
+                    s += (X[0, i] @ w["W_qR"][h * dr + e]) * (X[0, j] @ w["W_kR"][e])
+                want[h] = max(want[h], s / np.sqrt(dc + dr))
+    assert np.allclose(got, want, rtol=1e-12)
+
+
+def test_mla_with_zero_rotary_part_is_mha():
+    """With the rotary weights zero, the MLA statistic is the MHA one over the
+    content projections, rescaled from 1/sqrt(dc) to 1/sqrt(dc + dr)."""
+    X, w, H, dc, dr = _mla_setup(seed=27)
+    w["W_qR"][:] = 0.0
+    w["W_kR"][:] = 0.0
+    got = oracle.mla_max_logit(X, w, H, dc, dr)
+    mha = oracle.qk_max_logit(X, w["W_qC"], w["W_kC"], H, dc)
+    assert np.allclose(got, mha * np.sqrt(dc) / np.sqrt(dc + dr), rtol=1e-12)
