@@ -12,7 +12,10 @@ Sources (page title, then section):
   A = X X^T, X = aX + (bA + cA A)X, phi(x) = ax + bx^3 + cx^5, m <= n cost
   rule), "The Muon optimizer" (M <- mu M + G; Moonlight form of the update).
 * [MS] "About Muon: Muon At Scale" -- "Why Not Bernstein's Multiplier?"
-  (update snippet: p *= 1 - lr*wd; p += -lr*scale*u, scale = 0.2*sqrt(max)).
+  (update snippet: p *= 1 - lr*wd; p += -lr*scale*u, scale = 0.2*sqrt(max)),
+  and "Certain Neurons Still Dominate" (NorMuon: one second-moment scalar per
+  row, each row of the orthogonalised update divided by the square root of it,
+  then the whole matrix rescaled to the Frobenius norm it had before).
 
 Readings where the pages are silent (each also listed in the design doc):
 
@@ -25,6 +28,10 @@ Readings where the pages are silent (each also listed in the design doc):
   matrix gives a zero update ([MV] prints U/||U||_F with no eps).
 * Scale: 0.2*sqrt(max(rows, cols)) ([MC] §03, [MV], [MS]); weight decay acts
   on the pre-update W.
+* NorMuon ([MS]): a "row" is an output feature (a row of the stored r x c
+  weight); its second moment is an exponential average, v <- beta2*v +
+  (1 - beta2)*mean_j(O_ij^2), with no bias correction; the row is divided by
+  sqrt(v) + eps_v; the RMS-matching scale and decay then act as in Muon.
 """
 from __future__ import annotations
 
@@ -121,3 +128,38 @@ def muon_step_many(Ws, Gs, Ms, hp: dict, workers: int = 1):
 
 def _muon_step_kw(W, G, M, hp):
     return muon_step(W, G, M, **hp)
+
+
+def normuon_rows(O: np.ndarray, v: np.ndarray, beta2: float, eps_v: float):
+    """The NorMuon step after orthogonalisation ([MS] "Certain Neurons Still
+    Dominate"): per-row second moment, row division, and the rescale back to
+    the Frobenius norm of O.  Returns (O_hat, v_new)."""
+    O = np.asarray(O, dtype=np.float64)
+    rows, cols = O.shape
+    v_new = np.empty(rows)
+    O_hat = np.empty_like(O)
+    for i in range(rows):
+        v_new[i] = beta2 * float(v[i]) + (1.0 - beta2) * float(np.sum(O[i] * O[i])) / cols
+        O_hat[i] = O[i] / (np.sqrt(v_new[i]) + eps_v)
+    n_in = np.sqrt(np.sum(O * O))
+    n_out = np.sqrt(np.sum(O_hat * O_hat))
+    if n_out > 0:
+        O_hat *= n_in / n_out
+    return O_hat, v_new
+
+
+def normuon_step(W, G, M, v, *, beta2, eps_v, mu, nesterov, lr, wd, ns_steps, a, b, c, eps, rms_scale,
+                 coeffs=None):
+    """One NorMuon step on one hidden 2D weight, in float64: the Muon step of
+    ``muon_step`` with ``normuon_rows`` between Newton-Schulz and the scale.
+    ``v`` is the per-row state (length rows).  Returns (W_t, M_t, Upd, v_t)."""
+    W = np.asarray(W, dtype=np.float64)
+    G = np.asarray(G, dtype=np.float64)
+    M = np.asarray(M, dtype=np.float64)
+    M_new = mu * M + G
+    U = G + mu * M_new if nesterov else M_new
+    O = newton_schulz(U, ns_steps, a, b, c, eps, coeffs)
+    O_hat, v_new = normuon_rows(O, np.asarray(v, dtype=np.float64), beta2, eps_v)
+    upd = rms_scale * np.sqrt(max(W.shape)) * O_hat
+    W_new = W - lr * (upd + wd * W)
+    return W_new, M_new, upd, v_new

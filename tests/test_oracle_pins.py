@@ -416,3 +416,66 @@ def test_mla_with_zero_rotary_part_is_mha():
     got = oracle.mla_max_logit(X, w, H, dc, dr)
     mha = oracle.qk_max_logit(X, w["W_qC"], w["W_kC"], H, dc)
     assert np.allclose(got, mha * np.sqrt(dc) / np.sqrt(dc + dr), rtol=1e-12)
+
+
+# ------------------------------------------------------------ NorMuon
+def _nm_hp(**kw):
+    h = dict(wl.HPARAMS)
+    h.update(beta2=0.95, eps_v=1e-8)
+    h.update(kw)
+    return h
+
+
+def test_normuon_keeps_the_frobenius_norm_and_equalises_rows():
+    """The two facts the page states: the update is rescaled to the Frobenius
+    norm it had going in, and (with a fresh state) every row then carries the
+    same share of it."""
+    rng = np.random.default_rng(40)
+    r, c = 24, 40
+    W, G, M = rng.normal(0, 0.02, (r, c)), rng.normal(0, 1, (r, c)) * np.exp(rng.normal(0, 1, (r, 1))), np.zeros((r, c))
+    h = _nm_hp(beta2=0.0, eps_v=0.0)
+    _, _, upd_mu, _ = oracle.muon_step(W, G, M, **{k: v for k, v in h.items() if k not in ("beta2", "eps_v")})
+    _, _, upd, v = oracle.normuon_step(W, G, M, np.zeros(r), **h)
+    assert np.linalg.norm(upd) == pytest.approx(np.linalg.norm(upd_mu), rel=1e-12)
+    rn = np.linalg.norm(upd, axis=1)
+    assert np.allclose(rn, rn[0], rtol=1e-12)
+    # the Muon update itself does not have equal rows here (the row scaling of G survives)
+    rm = np.linalg.norm(upd_mu, axis=1)
+    assert rm.max() / rm.min() > 1.01
+    # the state holds the row mean squares of the NS output
+    O = upd_mu / (h["rms_scale"] * np.sqrt(max(r, c)))
+    assert np.allclose(v, np.mean(O * O, axis=1), rtol=1e-12)
+
+
+def test_normuon_reduces_to_muon_when_rows_are_already_equal():
+    """An exactly orthogonal square NS output (simple quintic run to
+    convergence) has unit rows, so the row division is uniform and NorMuon is
+    Muon; likewise with a large uniform state, whatever the rows."""
+    rng = np.random.default_rng(41)
+    n = 32
+    Q, _ = np.linalg.qr(rng.standard_normal((n, n)))
+    G = Q @ np.diag(np.linspace(1.0, 0.5, n)) @ np.linalg.qr(rng.standard_normal((n, n)))[0].T
+    W, M = rng.normal(0, 0.02, (n, n)), np.zeros((n, n))
+    simple = [(2.0, -1.5, 0.5)] * 40
+    base = {k: v for k, v in _nm_hp().items() if k not in ("beta2", "eps_v")}
+    base.update(ns_steps=40, coeffs=simple)
+    W_mu, _, _, _ = oracle.muon_step(W, G, M, **base)
+    W_nm, _, _, _ = oracle.normuon_step(W, G, M, np.zeros(n), beta2=0.95, eps_v=1e-8, **base)
+    assert np.allclose(W_nm, W_mu, rtol=0, atol=1e-12)
+    # any shape, large uniform prior state: v ~ beta2 * 1e6 on every row
+    W, G, M = rng.normal(0, 0.02, (20, 36)), rng.normal(0, 1, (20, 36)), np.zeros((20, 36))
+    base = {k: v for k, v in _nm_hp().items() if k not in ("beta2", "eps_v")}
+    W_mu, _, _, _ = oracle.muon_step(W, G, M, **base)
+    W_nm, _, _, _ = oracle.normuon_step(W, G, M, np.full(20, 1e6), beta2=0.95, eps_v=0.0, **base)
+    assert np.allclose(W_nm, W_mu, rtol=0, atol=1e-9)
+
+
+def test_normuon_fresh_state_is_independent_of_beta2():
+    """With v0 = 0 the first state is (1 - beta2) times the row mean squares,
+    a common factor that the Frobenius rescale removes."""
+    rng = np.random.default_rng(42)
+    W, G, M = rng.normal(0, 0.02, (30, 18)), rng.normal(0, 1, (30, 18)), rng.normal(0, 0.1, (30, 18))
+    outs = [oracle.normuon_step(W, G, M, np.zeros(30), **_nm_hp(beta2=b2, eps_v=0.0)) for b2 in (0.0, 0.5, 0.95)]
+    for o in outs[1:]:
+        assert np.allclose(o[0], outs[0][0], rtol=0, atol=1e-13)
+        assert np.allclose(o[2], outs[0][2], rtol=1e-10, atol=1e-13)
