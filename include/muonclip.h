@@ -7,6 +7,7 @@
  *   mc_muon_step     the Muon update of a list of hidden 2D weights
  *   mc_qk_max_logit  per-head causal max of the pre-softmax logit (S_max)
  *   mc_qk_clip       QK-Clip: rescale the W_q / W_k rows of heads with S_max > tau
+ *   mc_normuon_step  the Muon update with NorMuon's per-row normalisation
  *   mc_qk_clip_slices   QK-Clip over an explicit slice map (multi-head latent
  *                       attention, fused projection layouts)
  *   mc_mla_max_logit    S_max of multi-head latent attention (content + rotary parts)
@@ -151,6 +152,35 @@ int mc_qk_clip(void* wq, void* wk, int H, int dh, int D, const float* smax, floa
                float* gamma_out, int32_t* mask_out, void* stream);
 
 /*
+ * mc_normuon -- the per-row state and constants of NorMuon ("About Muon: Muon
+ * At Scale", "Certain Neurons Still Dominate").
+ */
+typedef struct mc_normuon {
+  float beta2;       /* exponential-average factor of the row second moment, in [0, 1) */
+  float eps;         /* added to sqrt(v) before dividing, finite and >= 0 */
+  float* const* v;   /* HOST array of n device pointers; v[i] is fp32 [params[i].rows],
+                        16-byte aligned, updated in place (start from zeros) */
+} mc_normuon;
+
+/*
+ * mc_normuon_step -- the Muon step of mc_muon_step with NorMuon's per-row
+ * normalisation between Newton-Schulz and the scale.  With O the un-oriented
+ * NS output of a rows x cols weight:
+ *   v_i   <- beta2 v_i + (1 - beta2) mean_j O_ij^2          (row = out-feature)
+ *   Ohat_i = O_i / (sqrt(v_i) + eps)
+ *   Ohat  <- Ohat * ||O||_F / ||Ohat||_F                     (0 if ||Ohat||_F = 0)
+ *   W     <- (1 - lr wd) W - lr * rms_scale * sqrt(max(rows, cols)) * Ohat
+ * update_out (if set) receives rms_scale * sqrt(max(rows, cols)) * Ohat.
+ * Everything else (arguments, momentum, workspace ownership, errors) is as
+ * for mc_muon_step; the workspace is larger (mc_normuon_workspace_size).
+ * Errors also: MC_ERR_INVAL for a NULL nm or v, beta2 outside [0, 1), a
+ * negative or non-finite eps, or a v that aliases w, g or m; MC_ERR_ALIGN.
+ */
+size_t mc_normuon_workspace_size(const mc_param* params, int n, const mc_hparams* hp);
+int mc_normuon_step(const mc_param* params, int n, const mc_hparams* hp, const mc_normuon* nm, void* workspace,
+                    size_t workspace_bytes, float* norms_out, void* stream);
+
+/*
  * mc_clip_slice -- one block of weight rows that QK-Clip rescales with the
  * factor of one head.  Rows [row_begin, row_end) of the row-major matrix at
  * `w` (`cols` elements per row, dtype MC_BF16 or MC_F32) are multiplied by
@@ -249,6 +279,27 @@ int mc_mla_max_logit(const void* x, const void* wqc, const void* wkc, const void
 #define MC_QK_STATIC_SCRATCH_BYTES (4ull * MC_QK_STATIC_MAX_ELEMS + 4ull * MC_QK_STATIC_MAX_HEADS)
 int mc_qk_max_logit_static(const void* x, const void* wq, const void* wk, int B, int S, int D, int H, int dh,
                            int causal, float* smax_out, void* stream);
+
+/*
+ * mc_shard_plan -- host-only: assign whole matrices to the ranks of an
+ * ownership-sharded data-parallel step ("MuonClip: speed, then stability" §08:
+ * orthogonalising a shard of a matrix is not orthogonalising the matrix, so
+ * the unit of work is a whole matrix).  Each matrix costs its Newton-Schulz
+ * work ns_steps * (4 m^2 n + 2 m^3), m = min(rows, cols), n = max(rows, cols).
+ * Matrices are taken in decreasing cost (ties: lower index first) and each is
+ * given to the rank with the least cost so far (ties: lower rank): the
+ * longest-processing-time rule, whose largest load is within
+ * 4/3 - 1/(3 world) of the best possible.  The result depends only on the
+ * arguments, so every rank computes the same plan.
+ *
+ * rows, cols  HOST int64 [n], each >= 1
+ * owner_out   HOST int32 [n]: rank in [0, world)
+ * load_out    optional HOST double [world]: summed cost per rank
+ * Errors: MC_ERR_INVAL (NULL arrays with n > 0, n < 0, world < 1,
+ * ns_steps < 1, a dimension < 1).  Touches no device.
+ */
+int mc_shard_plan(const int64_t* rows, const int64_t* cols, int n, int ns_steps, int world, int32_t* owner_out,
+                  double* load_out);
 
 /* Text of the last error returned on the calling thread ("" if none). */
 const char* mc_last_error(void);

@@ -23,7 +23,8 @@ MC_F32, MC_BF16 = 0, 1
 # Names the C ABI exports (include/muonclip.h).
 EXPORTS = ("mc_muon_workspace_size", "mc_muon_step", "mc_qk_workspace_size", "mc_qk_max_logit",
            "mc_qk_clip", "mc_last_error", "mc_device_status", "mc_profile_begin", "mc_profile_end",
-           "mc_qk_max_logit_static", "mc_qk_clip_slices", "mc_mla_workspace_size", "mc_mla_max_logit")
+           "mc_qk_max_logit_static", "mc_qk_clip_slices", "mc_mla_workspace_size", "mc_mla_max_logit",
+           "mc_shard_plan")
 MC_QK_STATIC_MAX_ELEMS = 1 << 24
 MC_QK_STATIC_MAX_HEADS = 4096
 
@@ -96,6 +97,9 @@ def load_library():
     lib.mc_mla_workspace_size.restype = sz
     lib.mc_mla_max_logit.argtypes = [vp, vp, vp, vp, vp] + [i32] * 7 + [vp, vp, sz, vp]
     lib.mc_mla_max_logit.restype = i32
+    lib.mc_shard_plan.argtypes = [P(ctypes.c_int64), P(ctypes.c_int64), i32, i32, i32, P(ctypes.c_int32),
+                                  P(ctypes.c_double)]
+    lib.mc_shard_plan.restype = i32
     lib.mc_profile_begin.argtypes = []
     lib.mc_profile_begin.restype = i32
     lib.mc_profile_end.argtypes = [P(McKernelStat), i32, P(ctypes.c_int)]
@@ -375,6 +379,19 @@ def mla_max_logit(x, wqc, wkc, wqr, wkr, H: int, dc: int, dr: int, *, causal: bo
                                 int(causal), _ptr(smax_out), _ptr(ws), int(ws.numel() * ws.element_size()),
                                 _stream_handle(stream)))
     return smax_out
+
+
+def shard_plan(shapes, world: int, ns_steps: int = 5):
+    """Owner rank of each (rows, cols) matrix and the per-rank Newton-Schulz
+    cost (see mc_shard_plan).  Host only."""
+    lib = load_library()
+    n = len(shapes)
+    rows = (ctypes.c_int64 * max(n, 1))(*[int(r) for r, _ in shapes])
+    cols = (ctypes.c_int64 * max(n, 1))(*[int(c) for _, c in shapes])
+    owner = (ctypes.c_int32 * max(n, 1))()
+    load = (ctypes.c_double * max(world, 1))()
+    _check(lib.mc_shard_plan(rows, cols, n, ns_steps, world, owner, load))
+    return [int(owner[i]) for i in range(n)], [float(load[r]) for r in range(world)]
 
 
 def qk_max_logit_static(x, wq, wk, H: int, dh: int, *, causal: bool = True, smax_out=None, stream=None):

@@ -206,11 +206,13 @@ int map_batched(CUtensorMap* map, const void* base, int64_t count, int64_t rows,
 
 // ----------------------------------------------------------- profiling
 enum Kind : int { K_MOMENTUM, K_FINALIZE, K_GRAM, K_POLY, K_APPLY_MIXED, K_APPLY, K_APPLY_FINAL, K_QK_PROJ,
-                  K_QK_CMAX, K_QK_KEYS, K_QK_CLIP, K_MLA_PROJ, K_MLA_CMAX, K_QK_CLIP_SLICES, K_COUNT };
+                  K_QK_CMAX, K_QK_KEYS, K_QK_CLIP, K_MLA_PROJ, K_MLA_CMAX, K_QK_CLIP_SLICES, K_NORM_ROWS,
+                  K_NORM_APPLY, K_COUNT };
 const char* const kKindNames[K_COUNT] = {"momentum",  "norm_finalize",  "ns_gram", "ns_poly",
                                          "ns_apply_mixed", "ns_apply", "ns_apply_final", "qk_proj",
                                          "qk_causal_max", "qk_keys", "qk_clip", "mla_proj",
-                                         "mla_causal_max", "qk_clip_slices"};
+                                         "mla_causal_max", "qk_clip_slices", "normuon_rows",
+                                         "normuon_apply"};
 struct ProfRec {
   int kind;
   cudaEvent_t b, e;
@@ -318,6 +320,10 @@ struct MuonLayout {
   std::vector<long long> cta_begin;
   long long total_ctas = 0;
   size_t off_tab = 0, tab_bytes = 0, off_partials = 0, off_scale = 0, total = 0;
+  // NorMuon only: NormEntry[n] inside the table block, and two fp32 row arrays
+  bool normuon = false;
+  size_t off_ntab = 0, off_rowsq = 0, off_rowf = 0;
+  long long total_rows = 0;
 };
 
 int validate_muon(const mc_param* params, int n, const mc_hparams* hp) {
@@ -350,7 +356,8 @@ int validate_muon(const mc_param* params, int n, const mc_hparams* hp) {
   return MC_OK;
 }
 
-void plan_muon(const mc_param* params, int n, MuonLayout& L) {
+void plan_muon(const mc_param* params, int n, MuonLayout& L, bool normuon = false) {
+  L.normuon = normuon;
   std::map<std::tuple<int64_t, int64_t, int>, int> index;
   for (int i = 0; i < n; ++i) {
     const auto key = std::make_tuple(params[i].rows, params[i].cols, params[i].w_dtype == MC_F32 ? 1 : 0);
@@ -396,6 +403,11 @@ void plan_muon(const mc_param* params, int n, MuonLayout& L) {
     g.off_uptr = off;
     off += sizeof(void*) * g.members.size();
   }
+  if (normuon) {
+    off = align_up(off, 256);
+    L.off_ntab = off;
+    off += sizeof(NormEntry) * n;
+  }
   L.tab_bytes = off;
   off = align_up(off, 1024);
   L.off_partials = off;
@@ -411,6 +423,13 @@ void plan_muon(const mc_param* params, int n, MuonLayout& L) {
     g.off_xf = off;    off = align_up(off + 4 * xe, 1024);
     g.off_a = off;     off = align_up(off + 2 * ae, 1024);
     g.off_b = off;     off = align_up(off + 2 * ae, 1024);
+  }
+  if (normuon) {
+    for (int i = 0; i < n; ++i) L.total_rows += params[i].rows;
+    L.off_rowsq = off;
+    off = align_up(off + sizeof(float) * size_t(L.total_rows), 1024);
+    L.off_rowf = off;
+    off = align_up(off + sizeof(float) * size_t(L.total_rows), 1024);
   }
   L.total = std::max<size_t>(off, 1024);
 }
@@ -458,20 +477,66 @@ MC_API size_t mc_muon_workspace_size(const mc_param* params, int n, const mc_hpa
   return L.total;
 }
 
+namespace {
+int validate_normuon(const mc_param* params, int n, const mc_normuon* nm) {
+  if (!nm) return fail(MC_ERR_INVAL, "nm is NULL");
+  if (!std::isfinite(nm->beta2) || nm->beta2 < 0.f || nm->beta2 >= 1.f)
+    return fail(MC_ERR_INVAL, "nm->beta2 must be in [0, 1)");
+  if (!std::isfinite(nm->eps) || nm->eps < 0.f) return fail(MC_ERR_INVAL, "nm->eps must be finite and >= 0");
+  if (n > 0 && !nm->v) return fail(MC_ERR_INVAL, "nm->v is NULL");
+  for (int i = 0; i < n; ++i) {
+    const float* v = nm->v[i];
+    const std::string at = "nm->v[" + std::to_string(i) + "]: ";
+    if (!v) return fail(MC_ERR_INVAL, at + "NULL");
+    if (!aligned16(v)) return fail(MC_ERR_ALIGN, at + "must be 16-byte aligned");
+    if (static_cast<const void*>(v) == params[i].w || static_cast<const void*>(v) == params[i].g ||
+        v == params[i].m)
+      return fail(MC_ERR_INVAL, at + "aliases w, g or m");
+  }
+  return MC_OK;
+}
+
+int run_muon(const mc_param* params, int n, const mc_hparams* hp, const mc_normuon* nm, void* workspace,
+             size_t workspace_bytes, float* norms_out, cudaStream_t s);
+}  // namespace
+
+MC_API size_t mc_normuon_workspace_size(const mc_param* params, int n, const mc_hparams* hp) {
+  if (validate_muon(params, n, hp) != MC_OK || n == 0) return 0;
+  MuonLayout L;
+  plan_muon(params, n, L, true);
+  return L.total;
+}
+
+MC_API int mc_normuon_step(const mc_param* params, int n, const mc_hparams* hp, const mc_normuon* nm,
+                           void* workspace, size_t workspace_bytes, float* norms_out, void* stream) {
+  int rc = validate_muon(params, n, hp);
+  if (rc != MC_OK) return rc;
+  if ((rc = validate_normuon(params, n, nm)) != MC_OK) return rc;
+  if (n == 0) return MC_OK;
+  return run_muon(params, n, hp, nm, workspace, workspace_bytes, norms_out, static_cast<cudaStream_t>(stream));
+}
+
 MC_API int mc_muon_step(const mc_param* params, int n, const mc_hparams* hp, void* workspace,
                         size_t workspace_bytes, float* norms_out, void* stream) {
   int rc = validate_muon(params, n, hp);
   if (rc != MC_OK) return rc;
   if (n == 0) return MC_OK;
+  return run_muon(params, n, hp, nullptr, workspace, workspace_bytes, norms_out,
+                  static_cast<cudaStream_t>(stream));
+}
+
+namespace {
+int run_muon(const mc_param* params, int n, const mc_hparams* hp, const mc_normuon* nm, void* workspace,
+             size_t workspace_bytes, float* norms_out, cudaStream_t s) {
+  int rc = MC_OK;
   if (norms_out && !aligned16(norms_out)) return fail(MC_ERR_ALIGN, "norms_out must be 16-byte aligned");
   if (workspace && !aligned16(workspace)) return fail(MC_ERR_ALIGN, "workspace must be 16-byte aligned");
-  cudaStream_t s = static_cast<cudaStream_t>(stream);
   std::lock_guard<std::mutex> lock(g_mu);
   DeviceState* st = nullptr;
   if ((rc = device_state(&st)) != MC_OK) return rc;
 
   MuonLayout L;
-  plan_muon(params, n, L);
+  plan_muon(params, n, L, nm != nullptr);
   if (workspace) {
     if (workspace_bytes < L.total)
       return fail(MC_ERR_NOSPC, "workspace has " + std::to_string(workspace_bytes) + " bytes, needs " +
@@ -505,6 +570,27 @@ MC_API int mc_muon_step(const mc_param* params, int n, const mc_hparams* hp, voi
       float** up = reinterpret_cast<float**>(tab.data() + g.off_uptr);
       wp[j] = q.w;
       up[j] = q.update_out;
+    }
+  }
+  if (nm) {
+    NormEntry* ne = reinterpret_cast<NormEntry*>(tab.data() + L.off_ntab);
+    long long rb = 0;
+    for (int kk = 0; kk < n; ++kk) {
+      const mc_param& q = params[ent[kk].orig];
+      NormEntry& e = ne[kk];
+      e.o = ent[kk].xf;
+      e.v = nm->v[ent[kk].orig];
+      e.w = q.w;
+      e.u = q.update_out;
+      e.rows = q.rows;
+      e.cols = q.cols;
+      e.ld = ent[kk].ld;
+      e.row_base = rb;
+      e.cta_begin = L.cta_begin[kk];
+      e.rms = hp->rms_scale * std::sqrt(static_cast<float>(std::max(q.rows, q.cols)));
+      e.w_f32 = q.w_dtype == MC_F32;
+      e.vec = (q.cols % 8) == 0;
+      rb += q.rows;
     }
   }
   if ((rc = upload(*st, tab.data(), tab.size(), ws + L.off_tab, s)) != MC_OK) return rc;
@@ -613,13 +699,14 @@ MC_API int mc_muon_step(const mc_param* params, int n, const mc_hparams* hp, voi
         G.xf_ld = g.ld;
         G.xf_bs = g.rows * g.ld;
         G.xf_read = mixed ? 1 : 0;
-        G.xf_write = (!last && it + 1 < kMixedIters) ? 1 : 0;
+        // NorMuon keeps the last iterate (the NS output O) in fp32 for the row pass.
+        G.xf_write = ((!last && it + 1 < kMixedIters) || (last && nm)) ? 1 : 0;
         G.d = ws + g.off_xb[par ^ 1];
         G.d_ld = g.ld;
         G.d_bs = g.rows * g.ld;
         G.scale = first ? scale : nullptr;
         G.coef_src = ca;
-        if (last) {
+        if (last && !nm) {
           G.w_ptrs = reinterpret_cast<void* const*>(ws + g.off_wptr);
           bool any_u = false;
           for (int i : g.members) any_u |= params[i].update_out != nullptr;
@@ -638,7 +725,7 @@ MC_API int mc_muon_step(const mc_param* params, int n, const mc_hparams* hp, voi
       // the whole step was 2-3 % faster this way (the power cap).
       if ((rc = launch_gemm<EPI_GRAM, 1>(gram, *st, s, K_GRAM, f_gram, fd_gram)) != MC_OK) return rc;
       if ((rc = launch_gemm<EPI_POLY, 1>(poly, *st, s, K_POLY, f_poly, fd_poly)) != MC_OK) return rc;
-      if (last) {
+      if (last && !nm) {
         rc = launch_gemm<EPI_APPLY_FINAL, 1>(apply, *st, s, K_APPLY_FINAL, f_apply);
       } else {
         rc = launch_gemm<EPI_APPLY, 1>(apply, *st, s, mixed ? K_APPLY_MIXED : K_APPLY, f_apply);
@@ -646,8 +733,37 @@ MC_API int mc_muon_step(const mc_param* params, int n, const mc_hparams* hp, voi
       if (rc != MC_OK) return rc;
     }
   }
+  if (nm) {
+    // NorMuon: row sums of squares of O, then the row factors, then the update.
+    const NormEntry* ntab = reinterpret_cast<const NormEntry*>(ws + L.off_tab + L.off_ntab);
+    float* rowsq = reinterpret_cast<float*>(ws + L.off_rowsq);
+    float* rowf = reinterpret_cast<float*>(ws + L.off_rowf);
+    double o_bytes = 0, w_bytes = 0;
+    for (int i = 0; i < n; ++i) {
+      const double el = double(params[i].rows) * double(params[i].cols);
+      o_bytes += 4.0 * el;
+      w_bytes += el * (4.0 + 2.0 * (params[i].w_dtype == MC_F32 ? 4 : 2) + (params[i].update_out ? 4 : 0));
+    }
+    {
+      ProfScope prof(K_NORM_ROWS, s, 0, 0, o_bytes);
+      const long long rows_per_cta = NORM_THREADS / 32;
+      normuon_rowsq_kernel<<<static_cast<unsigned>((L.total_rows + rows_per_cta - 1) / rows_per_cta),
+                             NORM_THREADS, 0, s>>>(ntab, n, L.total_rows, rowsq);
+      MC_CUDA(cudaGetLastError());
+      normuon_finalize_kernel<<<static_cast<unsigned>(n), NORM_THREADS, 0, s>>>(ntab, rowsq, rowf, nm->beta2,
+                                                                                nm->eps);
+      MC_CUDA(cudaGetLastError());
+    }
+    {
+      ProfScope prof(K_NORM_APPLY, s, 0, 0, w_bytes);
+      normuon_apply_kernel<<<static_cast<unsigned>(L.total_ctas), NORM_THREADS, 0, s>>>(
+          ntab, n, rowf, 1.f - hp->lr * hp->wd, -hp->lr);
+      MC_CUDA(cudaGetLastError());
+    }
+  }
   return MC_OK;
 }
+}  // namespace
 
 // =========================================================================
 namespace {
@@ -1024,6 +1140,35 @@ MC_API int mc_device_status(void) {
     MC_CUDA(cudaMemcpyToSymbol(g_device_error, &zero, sizeof(int)));
     return fail(MC_ERR_DEVICE, "a kernel abandoned a bounded wait (device error " + std::to_string(v) + ")");
   }
+  return MC_OK;
+}
+
+// =========================================================================
+// Ownership plan for the sharded data-parallel step (host only).
+MC_API int mc_shard_plan(const int64_t* rows, const int64_t* cols, int n, int ns_steps, int world,
+                         int32_t* owner_out, double* load_out) {
+  if (n < 0 || world < 1 || ns_steps < 1) return fail(MC_ERR_INVAL, "need n >= 0, world >= 1, ns_steps >= 1");
+  if (n > 0 && (!rows || !cols || !owner_out)) return fail(MC_ERR_INVAL, "NULL rows, cols or owner_out");
+  std::vector<double> cost(static_cast<size_t>(n));
+  for (int i = 0; i < n; ++i) {
+    if (rows[i] < 1 || cols[i] < 1) return fail(MC_ERR_INVAL, "matrix " + std::to_string(i) + " has a dimension < 1");
+    const double m = static_cast<double>(std::min(rows[i], cols[i]));
+    const double nn = static_cast<double>(std::max(rows[i], cols[i]));
+    cost[static_cast<size_t>(i)] = ns_steps * (4.0 * m * m * nn + 2.0 * m * m * m);
+  }
+  std::vector<int> order(static_cast<size_t>(n));
+  for (int i = 0; i < n; ++i) order[static_cast<size_t>(i)] = i;
+  std::stable_sort(order.begin(), order.end(), [&](int a, int b) { return cost[size_t(a)] > cost[size_t(b)]; });
+  std::vector<double> load(static_cast<size_t>(world), 0.0);
+  for (int i : order) {
+    int best = 0;
+    for (int r = 1; r < world; ++r)
+      if (load[size_t(r)] < load[size_t(best)]) best = r;
+    owner_out[i] = best;
+    load[size_t(best)] += cost[size_t(i)];
+  }
+  if (load_out)
+    for (int r = 0; r < world; ++r) load_out[r] = load[size_t(r)];
   return MC_OK;
 }
 

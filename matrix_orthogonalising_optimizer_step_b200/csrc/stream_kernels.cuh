@@ -22,6 +22,12 @@
 //                    speed, then stability", §06; "Muon and MuonClip:
 //                    orthogonalised updates for LLM training", "MuonClip:
 //                    QK-clip, per head, adapted to MLA").
+//  normuon_rowsq_kernel, normuon_finalize_kernel, normuon_apply_kernel
+//                    NorMuon after Newton-Schulz ("About Muon: Muon At Scale",
+//                    "Certain Neurons Still Dominate"): per-row sums of
+//                    squares of O, the per-row second moment and row factors
+//                    (with the rescale to ||O||_F folded in), then the scaled
+//                    update with decoupled decay.
 #pragma once
 
 #include <climits>
@@ -218,6 +224,157 @@ __global__ void qk_clip_kernel(__nv_bfloat16* __restrict__ wq, __nv_bfloat16* __
     }
   } else {
     for (int c = threadIdx.x; c < D; c += blockDim.x) w[c] = __float2bfloat16_rn(__bfloat162float(w[c]) * f);
+  }
+}
+
+// ---------------------------------------------------------------- NorMuon
+struct NormEntry {
+  const float* o;        // NS output, rows x ld fp32 (stored, un-oriented layout)
+  float* v;              // per-row second moment [rows], updated in place
+  void* w;               // weight rows x cols (bf16 or fp32)
+  float* u;              // optional update output rows x cols
+  long long rows, cols, ld;
+  long long row_base;    // first slot of this matrix in the row arrays
+  long long cta_begin;   // first CTA of this matrix in the apply launch
+  float rms;             // rms_scale * sqrt(max(rows, cols))
+  int w_f32;
+  int vec;               // cols % 8 == 0 (then ld == cols)
+  int pad_;
+};
+
+constexpr int NORM_THREADS = 256;
+
+// First entry whose `key` field exceeds x, minus one (entries sorted by key).
+template <typename F>
+__device__ __forceinline__ int find_entry(int n, long long x, F key) {
+  int lo = 0, hi = n - 1;
+  while (lo < hi) {
+    const int mid = (lo + hi + 1) >> 1;
+    if (key(mid) <= x) lo = mid;
+    else hi = mid - 1;
+  }
+  return lo;
+}
+
+// One warp per row: sum of squares of the row of O, fixed lane order and a
+// fixed shuffle tree (deterministic).
+__global__ void normuon_rowsq_kernel(const NormEntry* __restrict__ tab, int n, long long total_rows,
+                                     float* __restrict__ rowsq) {
+  const long long gr = (long long)blockIdx.x * (NORM_THREADS / 32) + (threadIdx.x >> 5);
+  if (gr >= total_rows) return;
+  const int lane = threadIdx.x & 31;
+  const int k = find_entry(n, gr, [&](int i) { return tab[i].row_base; });
+  const NormEntry& E = tab[k];
+  const long long i = gr - E.row_base;
+  const float* o = E.o + i * E.ld;
+  float acc = 0.f;
+  const long long c4 = E.cols & ~3LL;
+  for (long long j = 4 * lane; j < c4; j += 128) {
+    const float4 x = *reinterpret_cast<const float4*>(o + j);
+    acc = fmaf(x.x, x.x, acc);
+    acc = fmaf(x.y, x.y, acc);
+    acc = fmaf(x.z, x.z, acc);
+    acc = fmaf(x.w, x.w, acc);
+  }
+  for (long long j = c4 + lane; j < E.cols; j += 32) acc = fmaf(o[j], o[j], acc);
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
+  if (lane == 0) rowsq[E.row_base + i] = acc;
+}
+
+// One CTA per matrix: v <- beta2 v + (1 - beta2) rowsq / cols, f = 1/(sqrt(v)+eps),
+// then every row factor times ||O||_F / ||f o O||_F (fp64 sums, fixed order).
+__global__ void normuon_finalize_kernel(const NormEntry* __restrict__ tab, const float* __restrict__ rowsq,
+                                        float* __restrict__ rowf, float beta2, float eps) {
+  const NormEntry& E = tab[blockIdx.x];
+  __shared__ double red_a[NORM_THREADS], red_b[NORM_THREADS];
+  __shared__ float g_sh;
+  double a = 0.0, b = 0.0;
+  const float inv_cols = 1.f / static_cast<float>(E.cols);
+  for (long long i = threadIdx.x; i < E.rows; i += NORM_THREADS) {
+    const float q = rowsq[E.row_base + i];
+    const float vn = fmaf(beta2, E.v[i], (1.f - beta2) * (q * inv_cols));
+    E.v[i] = vn;
+    const float f = 1.f / (sqrtf(vn) + eps);
+    rowf[E.row_base + i] = f;
+    a += static_cast<double>(q);
+    b += static_cast<double>(f) * static_cast<double>(f) * static_cast<double>(q);
+  }
+  red_a[threadIdx.x] = a;
+  red_b[threadIdx.x] = b;
+  __syncthreads();
+  for (int w = NORM_THREADS / 2; w > 0; w >>= 1) {
+    if (threadIdx.x < w) {
+      red_a[threadIdx.x] += red_a[threadIdx.x + w];
+      red_b[threadIdx.x] += red_b[threadIdx.x + w];
+    }
+    __syncthreads();
+  }
+  if (threadIdx.x == 0) g_sh = red_b[0] > 0.0 ? static_cast<float>(sqrt(red_a[0] / red_b[0])) : 0.f;
+  __syncthreads();
+  const float g = g_sh;
+  for (long long i = threadIdx.x; i < E.rows; i += NORM_THREADS) rowf[E.row_base + i] *= g;
+}
+
+// W <- decay W + step * (rowf_i O_ij), update_out = rms * rowf_i O_ij;
+// MOM_ELEMS_PER_CTA elements of one matrix per CTA, 8 at a time when rows are
+// 16-byte multiples.
+__global__ void normuon_apply_kernel(const NormEntry* __restrict__ tab, int n, const float* __restrict__ rowf,
+                                     float decay, float neg_lr) {
+  const int k = find_entry(n, blockIdx.x, [&](int i) { return tab[i].cta_begin; });
+  const NormEntry& E = tab[k];
+  const long long total = E.rows * E.cols;
+  const long long e0 = (blockIdx.x - E.cta_begin) * MOM_ELEMS_PER_CTA;
+  const long long e1 = e0 + MOM_ELEMS_PER_CTA < total ? e0 + MOM_ELEMS_PER_CTA : total;
+  const float step = neg_lr * E.rms;
+  const float* rf = rowf + E.row_base;
+  if (E.vec) {
+    for (long long e = e0 + 8LL * threadIdx.x; e < e1; e += 8LL * NORM_THREADS) {
+      const long long i = e / E.cols;
+      const float f = rf[i];
+      const float4 o0 = *reinterpret_cast<const float4*>(E.o + e);
+      const float4 o1 = *reinterpret_cast<const float4*>(E.o + e + 4);
+      const float x[8] = {f * o0.x, f * o0.y, f * o0.z, f * o0.w, f * o1.x, f * o1.y, f * o1.z, f * o1.w};
+      if (E.u) {
+        float4* U = reinterpret_cast<float4*>(E.u + e);
+        U[0] = make_float4(E.rms * x[0], E.rms * x[1], E.rms * x[2], E.rms * x[3]);
+        U[1] = make_float4(E.rms * x[4], E.rms * x[5], E.rms * x[6], E.rms * x[7]);
+      }
+      if (E.w_f32) {
+        float4* W = reinterpret_cast<float4*>(static_cast<float*>(E.w) + e);
+        float4 a = W[0], b = W[1];
+        a = make_float4(fmaf(step, x[0], decay * a.x), fmaf(step, x[1], decay * a.y),
+                        fmaf(step, x[2], decay * a.z), fmaf(step, x[3], decay * a.w));
+        b = make_float4(fmaf(step, x[4], decay * b.x), fmaf(step, x[5], decay * b.y),
+                        fmaf(step, x[6], decay * b.z), fmaf(step, x[7], decay * b.w));
+        W[0] = a;
+        W[1] = b;
+      } else {
+        uint4* W = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(E.w) + e);
+        uint4 a = *W;
+        uint32_t wv[4] = {a.x, a.y, a.z, a.w};
+#pragma unroll
+        for (int t = 0; t < 4; ++t) {
+          const float lo = fmaf(step, x[2 * t], decay * __uint_as_float(wv[t] << 16));
+          const float hi = fmaf(step, x[2 * t + 1], decay * __uint_as_float(wv[t] & 0xFFFF0000u));
+          wv[t] = pack_bf16x2(lo, hi);
+        }
+        *W = make_uint4(wv[0], wv[1], wv[2], wv[3]);
+      }
+    }
+  } else {
+    for (long long e = e0 + threadIdx.x; e < e1; e += NORM_THREADS) {
+      const long long i = e / E.cols, j = e - i * E.cols;
+      const float x = rf[i] * E.o[i * E.ld + j];
+      if (E.u) E.u[e] = E.rms * x;
+      if (E.w_f32) {
+        float* W = static_cast<float*>(E.w) + e;
+        *W = fmaf(step, x, decay * *W);
+      } else {
+        __nv_bfloat16* W = static_cast<__nv_bfloat16*>(E.w) + e;
+        *W = __float2bfloat16_rn(fmaf(step, x, decay * __bfloat162float(*W)));
+      }
+    }
   }
 }
 
