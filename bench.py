@@ -200,12 +200,14 @@ def run_reference(args, rank, world):
 
 
 # --------------------------------------------------------------- our arm
-def time_extras(mc, wl, dev, stream, hp, steps, peaks, barrier, max_over_ranks):
+def time_extras(mc, wl, dev, stream, hp, steps, peaks, barrier, max_over_ranks, muon_set=None):
     """Work outside the step, timed on its own after the step's timed region:
     (1) S_max and the slice-map QK-Clip of a multi-head latent attention layer
     (B 4, S 4096, D 4096, H 32, content 128 + rotary 64 per head); (2) the
     64 x 1024^2 batched Muon step with its five NS coefficient triples passed
-    as a per-iteration table, beside the same step with scalar coefficients."""
+    as a per-iteration table, beside the same step with scalar coefficients;
+    (3) a NorMuon step over the whole 7B-shaped set (``muon_set``: its W, G,
+    M lists), whose row pass adds two bandwidth-bound kernels."""
     import torch
 
     out = {}
@@ -276,6 +278,25 @@ def time_extras(mc, wl, dev, stream, hp, steps, peaks, barrier, max_over_ranks):
     del Ws, Gs, Ms
     mc.release_workspaces()
     torch.cuda.empty_cache()
+
+    if muon_set is not None:
+        Ws, Gs, Ms = muon_set
+        Vs = [torch.zeros(w.shape[0], dtype=torch.float32, device=dev) for w in Ws]
+        ms, k = timed(lambda: mc.normuon_step(Ws, Gs, Ms, Vs, beta2=0.95, eps_v=1e-8, stream=stream, **hp),
+                      max(2, min(steps, 3)))
+        reps = max(2, min(steps, 3))
+        rows, app = k["normuon_rows"], k["normuon_apply"]
+        out["normuon_7b"] = {
+            "workload": "NorMuon step over the 7B-shaped set (224 matrices), beta2 0.95",
+            "ms_per_step": ms,
+            "normuon_rows_ms": rows["total_ms"] / reps,
+            "normuon_rows_gbs": rows["bytes"] / (rows["total_ms"] / 1e3) / 1e9,
+            "normuon_apply_ms": app["total_ms"] / reps,
+            "normuon_apply_gbs": app["bytes"] / (app["total_ms"] / 1e3) / 1e9,
+            "normuon_apply_pct_hbm": 100.0 * app["bytes"] / (app["total_ms"] / 1e3) / 1e9 / peaks["hbm_gbs"]}
+        del Vs
+        mc.release_workspaces()
+        torch.cuda.empty_cache()
     return out
 
 
@@ -426,7 +447,8 @@ def main(argv=None):
 
     extras = None
     if not args.no_extras:
-        extras = time_extras(mc, wl, dev, stream, hp, args.steps, peaks, barrier, max_over_ranks)
+        extras = time_extras(mc, wl, dev, stream, hp, args.steps, peaks, barrier, max_over_ranks,
+                             muon_set=(Ws, Gs, Ms))
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:

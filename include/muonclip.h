@@ -281,6 +281,28 @@ int mc_qk_max_logit_static(const void* x, const void* wq, const void* wk, int B,
                            int causal, float* smax_out, void* stream);
 
 /*
+ * mc_polar_express_coeffs -- host-only: a per-iteration coefficient table
+ * (for mc_hparams.coeffs) built the Polar Express way.  "About Muon: Muon At
+ * Scale" ("Which Norm for Which Layer") cites it as a better polynomial for
+ * UV^T, whose ten steps take a singular value of 1e-4 to 0.994, but does not
+ * print the coefficients.  This restates the published construction (Amsel,
+ * Persson, Musco and Gower, "The Polar Express", 2025):
+ *   l_0 = l0, u_0 = 1; step t uses the odd quintic p_t closest to 1 in the
+ *   max norm on [l_t, u_t] (found by the Remez exchange), then
+ *   l_{t+1} = p_t(l_t), u_{t+1} = 2 - l_{t+1}; once u_t - l_t < 1e-3 the step
+ *   is the limit 15/8 x - 5/4 x^3 + 3/8 x^5; finally every polynomial but the
+ *   last is replaced by p(x / (1 + safety)).
+ * With steps = 10, l0 = 1e-3 and safety = 0.01 the composed map takes 1e-4 to
+ * 0.9942.
+ *
+ * coeffs_out  HOST float [3 * steps]: (a_t, b_t, c_t) for t = 0 .. steps-1
+ * Errors: MC_ERR_INVAL (steps outside [1, 100), l0 outside (0, 1), safety
+ * negative or not finite, NULL coeffs_out), MC_ERR_UNSUPPORTED if the
+ * exchange does not converge.  Touches no device.
+ */
+int mc_polar_express_coeffs(int steps, double l0, double safety, float* coeffs_out);
+
+/*
  * mc_shard_plan -- host-only: assign whole matrices to the ranks of an
  * ownership-sharded data-parallel step ("MuonClip: speed, then stability" §08:
  * orthogonalising a shard of a matrix is not orthogonalising the matrix, so

@@ -24,7 +24,7 @@ MC_F32, MC_BF16 = 0, 1
 EXPORTS = ("mc_muon_workspace_size", "mc_muon_step", "mc_qk_workspace_size", "mc_qk_max_logit",
            "mc_qk_clip", "mc_last_error", "mc_device_status", "mc_profile_begin", "mc_profile_end",
            "mc_qk_max_logit_static", "mc_qk_clip_slices", "mc_mla_workspace_size", "mc_mla_max_logit",
-           "mc_shard_plan")
+           "mc_shard_plan", "mc_normuon_workspace_size", "mc_normuon_step", "mc_polar_express_coeffs")
 MC_QK_STATIC_MAX_ELEMS = 1 << 24
 MC_QK_STATIC_MAX_HEADS = 4096
 
@@ -41,6 +41,10 @@ class McHparams(ctypes.Structure):
                 ("wd", ctypes.c_float), ("ns_steps", ctypes.c_int32), ("a", ctypes.c_float),
                 ("b", ctypes.c_float), ("c", ctypes.c_float), ("eps", ctypes.c_float),
                 ("rms_scale", ctypes.c_float), ("coeffs", ctypes.c_void_p)]
+
+
+class McNormuon(ctypes.Structure):
+    _fields_ = [("beta2", ctypes.c_float), ("eps", ctypes.c_float), ("v", ctypes.c_void_p)]
 
 
 class McClipSlice(ctypes.Structure):
@@ -97,6 +101,12 @@ def load_library():
     lib.mc_mla_workspace_size.restype = sz
     lib.mc_mla_max_logit.argtypes = [vp, vp, vp, vp, vp] + [i32] * 7 + [vp, vp, sz, vp]
     lib.mc_mla_max_logit.restype = i32
+    lib.mc_normuon_workspace_size.argtypes = [P(McParam), i32, P(McHparams)]
+    lib.mc_normuon_workspace_size.restype = sz
+    lib.mc_normuon_step.argtypes = [P(McParam), i32, P(McHparams), P(McNormuon), vp, sz, vp, vp]
+    lib.mc_normuon_step.restype = i32
+    lib.mc_polar_express_coeffs.argtypes = [i32, ctypes.c_double, ctypes.c_double, P(ctypes.c_float)]
+    lib.mc_polar_express_coeffs.restype = i32
     lib.mc_shard_plan.argtypes = [P(ctypes.c_int64), P(ctypes.c_int64), i32, i32, i32, P(ctypes.c_int32),
                                   P(ctypes.c_double)]
     lib.mc_shard_plan.restype = i32
@@ -266,6 +276,49 @@ def muon_step(weights: Sequence, grads: Sequence, moms: Sequence, *, norms_out=N
                             _ptr(norms_out), _stream_handle(stream)))
 
 
+def make_normuon(vs, beta2: float = 0.95, eps: float = 1e-8) -> McNormuon:
+    """McNormuon over per-matrix row-state tensors ``vs`` (fp32 [rows], CUDA).
+    The host pointer array is kept alive on the returned struct."""
+    torch = _torch()
+    ptrs = (ctypes.c_void_p * max(len(vs), 1))()
+    for i, v in enumerate(vs):
+        _need_cuda_contig(v, f"vs[{i}]")
+        if v.dtype != torch.float32:
+            raise TypeError(f"vs[{i}] must be float32")
+        ptrs[i] = _ptr(v)
+    nm = McNormuon(float(beta2), float(eps), ctypes.cast(ptrs, ctypes.c_void_p).value)
+    nm._ptrs = ptrs
+    return nm
+
+
+def normuon_step(weights: Sequence, grads: Sequence, moms: Sequence, vs: Sequence, *, beta2: float = 0.95,
+                 eps_v: float = 1e-8, norms_out=None, update_outs=None, workspace=None, stream=None,
+                 hparams: Optional[McHparams] = None, **hp) -> None:
+    """One NorMuon step (see mc_normuon_step in include/muonclip.h): the Muon
+    step with each row of the orthogonalised update divided by the square root
+    of its running second moment ``vs[i]`` (fp32 [rows], updated in place),
+    then rescaled to the Frobenius norm it had."""
+    lib = load_library()
+    arr, n = make_params(weights, grads, moms, update_outs)
+    if len(vs) != n:
+        raise ValueError("one row-state tensor per matrix")
+    for i, (v, w) in enumerate(zip(vs, weights)):
+        if v.shape != (w.shape[0],):
+            raise ValueError(f"vs[{i}] must have shape ({w.shape[0]},)")
+    h = hparams if hparams is not None else make_hparams(**hp)
+    nm = make_normuon(vs, beta2, eps_v)
+    if n == 0:
+        return
+    if norms_out is not None:
+        _need_cuda_contig(norms_out, "norms_out")
+    need = int(lib.mc_normuon_workspace_size(arr, n, ctypes.byref(h)))
+    if need == 0:
+        _check(lib.mc_normuon_step(arr, n, ctypes.byref(h), ctypes.byref(nm), None, 0, None, None))
+    ws = workspace if workspace is not None else _workspace("muon", weights[0].device, need)
+    _check(lib.mc_normuon_step(arr, n, ctypes.byref(h), ctypes.byref(nm), _ptr(ws),
+                               int(ws.numel() * ws.element_size()), _ptr(norms_out), _stream_handle(stream)))
+
+
 def qk_workspace_size(B, S, D, H, dh) -> int:
     return int(load_library().mc_qk_workspace_size(B, S, D, H, dh))
 
@@ -379,6 +432,16 @@ def mla_max_logit(x, wqc, wkc, wqr, wkr, H: int, dc: int, dr: int, *, causal: bo
                                 int(causal), _ptr(smax_out), _ptr(ws), int(ws.numel() * ws.element_size()),
                                 _stream_handle(stream)))
     return smax_out
+
+
+def polar_express_coeffs(steps: int = 10, l0: float = 1e-3, safety: float = 0.01):
+    """Per-iteration (a, b, c) triples of a Polar Express schedule, for
+    ``muon_step(..., ns_steps=steps, coeffs=...)`` (see mc_polar_express_coeffs).
+    Host only."""
+    lib = load_library()
+    out = (ctypes.c_float * (3 * max(int(steps), 1)))()
+    _check(lib.mc_polar_express_coeffs(int(steps), float(l0), float(safety), out))
+    return [(float(out[3 * i]), float(out[3 * i + 1]), float(out[3 * i + 2])) for i in range(int(steps))]
 
 
 def shard_plan(shapes, world: int, ns_steps: int = 5):

@@ -1144,6 +1144,104 @@ MC_API int mc_device_status(void) {
 }
 
 // =========================================================================
+// Polar Express coefficient schedule (host only).
+namespace {
+// Gaussian elimination with partial pivoting on an augmented 4 x 5 system.
+bool solve4(double (&m)[4][5], double (&x)[4]) {
+  for (int col = 0; col < 4; ++col) {
+    int piv = col;
+    for (int r = col + 1; r < 4; ++r)
+      if (std::fabs(m[r][col]) > std::fabs(m[piv][col])) piv = r;
+    if (!(std::fabs(m[piv][col]) > 1e-300)) return false;
+    if (piv != col)
+      for (int k = 0; k < 5; ++k) std::swap(m[col][k], m[piv][k]);
+    for (int r = col + 1; r < 4; ++r) {
+      const double f = m[r][col] / m[col][col];
+      for (int k = col; k < 5; ++k) m[r][k] -= f * m[col][k];
+    }
+  }
+  for (int r = 3; r >= 0; --r) {
+    double acc = m[r][4];
+    for (int k = r + 1; k < 4; ++k) acc -= m[r][k] * x[k];
+    x[r] = acc / m[r][r];
+  }
+  return true;
+}
+
+// Odd quintic closest to 1 in the max norm on [lo, hi]: Remez exchange over
+// four alternation points (the two ends and the two interior extrema).
+bool minimax_quintic(double lo, double hi, double& a, double& b, double& c) {
+  const double kPi = 3.14159265358979323846;
+  double pts[4];
+  for (int k = 0; k < 4; ++k) pts[k] = lo + (hi - lo) * 0.5 * (1.0 - std::cos(kPi * k / 3.0));
+  for (int it = 0; it < 200; ++it) {
+    double m[4][5], sol[4];
+    for (int i = 0; i < 4; ++i) {
+      const double x = pts[i], x2 = x * x;
+      m[i][0] = x;
+      m[i][1] = x * x2;
+      m[i][2] = x * x2 * x2;
+      m[i][3] = (i & 1) ? -1.0 : 1.0;
+      m[i][4] = 1.0;
+    }
+    if (!solve4(m, sol)) return false;
+    a = sol[0];
+    b = sol[1];
+    c = sol[2];
+    // p'(x) = a + 3b x^2 + 5c x^4 = 0: a quadratic in y = x^2
+    const double disc = 9.0 * b * b - 20.0 * a * c;
+    // No two interior extrema: the points cannot move, keep this solution.
+    if (disc < 0.0 || c == 0.0) return true;
+    const double sq = std::sqrt(disc);
+    double ys[2] = {(-3.0 * b - sq) / (10.0 * c), (-3.0 * b + sq) / (10.0 * c)};
+    double inner[2];
+    int cnt = 0;
+    for (double y : ys)
+      if (y > 0.0) {
+        const double x = std::sqrt(y);
+        if (x > lo && x < hi && cnt < 2) inner[cnt++] = x;
+      }
+    if (cnt != 2) return true;
+    if (inner[0] > inner[1]) std::swap(inner[0], inner[1]);
+    const double next[4] = {lo, inner[0], inner[1], hi};
+    double moved = 0.0;
+    for (int k = 0; k < 4; ++k) moved = std::max(moved, std::fabs(next[k] - pts[k]));
+    for (int k = 0; k < 4; ++k) pts[k] = next[k];
+    if (moved <= 1e-15 * hi) return true;
+  }
+  return true;
+}
+}  // namespace
+
+MC_API int mc_polar_express_coeffs(int steps, double l0, double safety, float* coeffs_out) {
+  if (steps < 1 || steps >= 100) return fail(MC_ERR_INVAL, "steps must be in [1, 100)");
+  if (!(l0 > 0.0 && l0 < 1.0)) return fail(MC_ERR_INVAL, "l0 must be in (0, 1)");
+  if (!std::isfinite(safety) || safety < 0.0) return fail(MC_ERR_INVAL, "safety must be finite and >= 0");
+  if (!coeffs_out) return fail(MC_ERR_INVAL, "NULL coeffs_out");
+  std::vector<double> co(3 * static_cast<size_t>(steps));
+  double lo = l0, hi = 1.0;
+  for (int t = 0; t < steps; ++t) {
+    double a = 15.0 / 8.0, b = -10.0 / 8.0, c = 3.0 / 8.0;
+    if (hi - lo >= 1e-3 && !minimax_quintic(lo, hi, a, b, c))
+      return fail(MC_ERR_UNSUPPORTED, "the Remez exchange did not converge at step " + std::to_string(t));
+    co[3 * t] = a;
+    co[3 * t + 1] = b;
+    co[3 * t + 2] = c;
+    const double l2 = lo * lo;
+    lo = a * lo + b * lo * l2 + c * lo * l2 * l2;
+    hi = 2.0 - lo;
+  }
+  const double s = 1.0 + safety;
+  for (int t = 0; t < steps; ++t) {
+    const bool last = t + 1 == steps;
+    coeffs_out[3 * t] = static_cast<float>(last ? co[3 * t] : co[3 * t] / s);
+    coeffs_out[3 * t + 1] = static_cast<float>(last ? co[3 * t + 1] : co[3 * t + 1] / (s * s * s));
+    coeffs_out[3 * t + 2] = static_cast<float>(last ? co[3 * t + 2] : co[3 * t + 2] / (s * s * s * s * s));
+  }
+  return MC_OK;
+}
+
+// =========================================================================
 // Ownership plan for the sharded data-parallel step (host only).
 MC_API int mc_shard_plan(const int64_t* rows, const int64_t* cols, int n, int ns_steps, int world,
                          int32_t* owner_out, double* load_out) {

@@ -18,6 +18,6 @@ itself: the odd-polynomial/SVD identity, numbers the pages print, brute force
 on tiny inputs, limits with a textbook answer, and a third-party optimizer.
 """
 from .muon import (phi, phi_iter, phi_schedule, newton_schulz, muon_step, muon_step_many,  # noqa: F401
-                   normuon_rows, normuon_step)
+                   normuon_rows, normuon_step, minimax_odd_quintic, polar_express_schedule)
 from .qk import (qk_max_logit, qk_max_logit_bruteforce, qk_clip, qk_clip_slices, mla_max_logit,  # noqa: F401
                  mla_slices, round_bf16)

@@ -28,6 +28,13 @@ Readings where the pages are silent (each also listed in the design doc):
   matrix gives a zero update ([MV] prints U/||U||_F with no eps).
 * Scale: 0.2*sqrt(max(rows, cols)) ([MC] §03, [MV], [MS]); weight decay acts
   on the pre-update W.
+* Polar Express ([MS] "Which Norm for Which Layer"): the pages print only its
+  effect (ten steps take 1e-4 to 0.994).  The schedule is read as the
+  published construction: step t uses the odd quintic that is closest to 1 in
+  the max norm on [l_t, u_t] (l_0 = 1e-3, u_0 = 1), then l_{t+1} = p_t(l_t),
+  u_{t+1} = 2 - l_{t+1}; once the interval is narrower than 1e-3 the step is
+  the limit of that polynomial, 15/8 x - 5/4 x^3 + 3/8 x^5; every polynomial
+  but the last is then evaluated at x / 1.01 (a safety factor).
 * NorMuon ([MS]): a "row" is an output feature (a row of the stored r x c
   weight); its second moment is an exponential average, v <- beta2*v +
   (1 - beta2)*mean_j(O_ij^2), with no bias correction; the row is divided by
@@ -163,3 +170,48 @@ def normuon_step(W, G, M, v, *, beta2, eps_v, mu, nesterov, lr, wd, ns_steps, a,
     upd = rms_scale * np.sqrt(max(W.shape)) * O_hat
     W_new = W - lr * (upd + wd * W)
     return W_new, M_new, upd, v_new
+
+
+def minimax_odd_quintic(lo: float, hi: float, iters: int = 200):
+    """The odd quintic p(x) = a x + b x^3 + c x^5 minimising max |1 - p(x)| on
+    [lo, hi] (0 < lo < hi), by the Remez exchange: solve for equal and
+    alternating errors at four points, move the points to the extrema of the
+    error (the ends and the two interior zeros of p'), repeat.  Returns
+    ((a, b, c), E) with E the minimax error."""
+    k = np.arange(4)
+    xs = lo + (hi - lo) * (1.0 - np.cos(np.pi * k / 3.0)) / 2.0
+    a = b = c = E = 0.0
+    for _ in range(iters):
+        A = np.stack([xs, xs ** 3, xs ** 5, (-1.0) ** k], axis=1)
+        a, b, c, E = np.linalg.solve(A, np.ones(4))
+        y = np.roots([5.0 * c, 3.0 * b, a])          # p'(x) = 0 with y = x^2
+        inner = sorted(float(np.sqrt(r.real)) for r in y
+                       if abs(r.imag) < 1e-12 and r.real > 0 and lo < np.sqrt(r.real) < hi)
+        if len(inner) != 2:
+            break
+        new = np.array([lo, inner[0], inner[1], hi])
+        if np.max(np.abs(new - xs)) <= 1e-15 * hi:
+            break
+        xs = new
+    return (float(a), float(b), float(c)), float(abs(E))
+
+
+def polar_express_schedule(steps: int, l0: float = 1e-3, safety: float = 0.01):
+    """Per-iteration (a_k, b_k, c_k) of the Polar Express construction (see the
+    module readings).  The safety factor maps p(x) to p(x / (1 + safety)) for
+    all but the last step."""
+    lo, hi = l0, 1.0
+    out = []
+    for _ in range(steps):
+        if hi - lo < 1e-3:
+            # the interval has shrunk onto 1, where the exchange is ill-conditioned
+            # (and the minimax error below 1e-9): take the limit of the minimax
+            # polynomial, the odd quintic with p(1) = 1 and p'(1) = p''(1) = 0
+            (a, b, c), E = (15.0 / 8.0, -10.0 / 8.0, 3.0 / 8.0), 0.0
+        else:
+            (a, b, c), E = minimax_odd_quintic(lo, hi)
+        out.append((a, b, c))
+        lo = a * lo + b * lo ** 3 + c * lo ** 5
+        hi = 2.0 - lo
+    s = 1.0 + safety
+    return [(a / s, b / s ** 3, c / s ** 5) for (a, b, c) in out[:-1]] + [out[-1]]

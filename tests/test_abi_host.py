@@ -184,3 +184,43 @@ def test_mla_argument_errors_and_workspace(lib):
     bs = 2 * 128
     assert n >= 2 * bs * (2 * 4 * 128 + 4 * 64 + 64) + 4 * 4
     assert lib.mc_mla_workspace_size(2, 128, 64, 4, 96, 64) == 0
+
+
+def test_normuon_argument_errors(lib):
+    P = ctypes.byref
+    hp = mc.make_hparams()
+    arr = _params(2)
+    vptrs = (ctypes.c_void_p * 2)(0x900000, 0x910000)
+    good = mc.McNormuon(0.95, 1e-8, ctypes.cast(vptrs, ctypes.c_void_p).value)
+    call = lambda nm: lib.mc_normuon_step(arr, 2, P(hp), nm, None, 0, None, None)
+    assert call(None) == mc.MC_ERR_INVAL
+    for b2, eps in ((1.0, 1e-8), (-0.1, 1e-8), (float("nan"), 1e-8), (0.9, -1.0), (0.9, float("inf"))):
+        assert call(P(mc.McNormuon(b2, eps, good.v))) == mc.MC_ERR_INVAL
+    assert call(P(mc.McNormuon(0.95, 1e-8, None))) == mc.MC_ERR_INVAL
+    bad = (ctypes.c_void_p * 2)(0x900000, 0)
+    assert call(P(mc.McNormuon(0.95, 1e-8, ctypes.cast(bad, ctypes.c_void_p).value))) == mc.MC_ERR_INVAL
+    alias = (ctypes.c_void_p * 2)(arr[0].m, 0x910000)
+    assert call(P(mc.McNormuon(0.95, 1e-8, ctypes.cast(alias, ctypes.c_void_p).value))) == mc.MC_ERR_INVAL
+    mis = (ctypes.c_void_p * 2)(0x900004, 0x910000)
+    assert call(P(mc.McNormuon(0.95, 1e-8, ctypes.cast(mis, ctypes.c_void_p).value))) == mc.MC_ERR_ALIGN
+    # the workspace adds two fp32 row arrays and the row table to the Muon plan
+    a = lib.mc_muon_workspace_size(arr, 2, P(hp))
+    b = lib.mc_normuon_workspace_size(arr, 2, P(hp))
+    assert b >= a + 2 * 4 * (64 + 64)
+
+
+def test_polar_express_coeffs_match_the_oracle(lib):
+    import numpy as np
+    import oracle
+    for steps, l0, safety in ((10, 1e-3, 0.01), (5, 1e-3, 0.01), (8, 1e-2, 0.0), (3, 0.3, 0.02)):
+        got = np.array(mc.polar_express_coeffs(steps, l0, safety))
+        want = np.array(oracle.polar_express_schedule(steps, l0, safety))
+        assert got.shape == (steps, 3)
+        assert np.allclose(got, want, rtol=1e-6, atol=1e-6), (steps, l0, safety)
+    # the printed effect, through the library's own table
+    assert float(oracle.phi_schedule(1e-4, mc.polar_express_coeffs(10))) == pytest.approx(0.994, abs=5e-4)
+    out = (ctypes.c_float * 3)()
+    assert lib.mc_polar_express_coeffs(0, 1e-3, 0.01, out) == mc.MC_ERR_INVAL
+    assert lib.mc_polar_express_coeffs(5, 1.0, 0.01, out) == mc.MC_ERR_INVAL
+    assert lib.mc_polar_express_coeffs(5, 1e-3, -0.1, out) == mc.MC_ERR_INVAL
+    assert lib.mc_polar_express_coeffs(5, 1e-3, 0.01, None) == mc.MC_ERR_INVAL

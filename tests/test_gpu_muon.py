@@ -71,6 +71,21 @@ def test_coefficient_schedules(hp, name, sched):
     check_all(mats, h, run_step(mats, h), name)
 
 
+def test_polar_express_schedule(hp):
+    """Ten Polar Express steps (the library's own table) against the oracle
+    running its own table: the first polynomial's slope of about 8 makes the
+    first two iterations the hardest for bf16 operands."""
+    sched = mc.polar_express_coeffs(10)
+    ref_sched = oracle.polar_express_schedule(10)
+    h = dict(hp, ns_steps=10, coeffs=sched)
+    h_ref = dict(hp, ns_steps=10, coeffs=ref_sched)
+    mats = [wl.generic_matrix(256, 768, seed=33), wl.generic_matrix(768, 256, seed=34), wl.cfg1_matrix(1, n=512)]
+    W1, M1, U1, nrm = run_step(mats, h)
+    for i, (W0, G, M0) in enumerate(mats):
+        ref = oracle.muon_step(to64(W0), to64(G), to64(M0), **h_ref)
+        check_muon_matrix(W0, G, M0, W1[i], M1[i], U1[i], nrm[i], h_ref, ref, f"polar express[{i}]")
+
+
 RAGGED = [(1, 1), (3, 5), (5, 3), (8, 1), (64, 64), (100, 37), (37, 100), (129, 129),
           (256, 256), (300, 520), (520, 300), (129, 1000), (1000, 129), (640, 384)]
 

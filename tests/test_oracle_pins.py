@@ -479,3 +479,48 @@ def test_normuon_fresh_state_is_independent_of_beta2():
     for o in outs[1:]:
         assert np.allclose(o[0], outs[0][0], rtol=0, atol=1e-13)
         assert np.allclose(o[2], outs[0][2], rtol=1e-10, atol=1e-13)
+
+
+# ------------------------------------------------------------ Polar Express
+def test_polar_express_ten_steps_printed_value():
+    g = GOLD["polar_express_10"]
+    sched = oracle.polar_express_schedule(g["steps"])
+    assert len(sched) == 10
+    assert float(oracle.phi_schedule(g["x0"], sched)) == pytest.approx(g["printed"], abs=g["tol"])
+    # the five-step tuned quintic stays far below (the printed 0.05 of the same bullet)
+    tuned = GOLD["tuned_coefficients"]["value"]
+    assert float(oracle.phi_iter(g["x0"], 5, *tuned)) < 0.06
+
+
+def test_minimax_quintic_is_optimal_against_a_linear_program():
+    """The Remez result equioscillates at four points, and no odd quintic does
+    better on a fine grid (an LP over (a, b, c, E), solved independently)."""
+    from scipy.optimize import linprog
+    for lo, hi in ((1e-3, 1.0), (0.3, 1.7), (0.05, 1.0)):
+        (a, b, c), E = oracle.minimax_odd_quintic(lo, hi)
+        x = np.linspace(lo, hi, 20001)
+        err = 1.0 - (a * x + b * x ** 3 + c * x ** 5)
+        assert np.max(np.abs(err)) == pytest.approx(E, rel=1e-6)
+        # sign changes of the error at its extrema: at least 3 (4 alternation points)
+        ext = np.r_[0, np.nonzero(np.diff(np.sign(np.diff(err))))[0] + 1, len(x) - 1]
+        assert np.sum(np.diff(np.sign(err[ext])) != 0) >= 3
+        # LP: minimise E s.t. |1 - (a x + b x^3 + c x^5)| <= E on the grid
+        xg = np.linspace(lo, hi, 4001)
+        V = np.stack([xg, xg ** 3, xg ** 5], axis=1)
+        A_ub = np.block([[V, -np.ones((len(xg), 1))], [-V, -np.ones((len(xg), 1))]])
+        b_ub = np.r_[np.ones(len(xg)), -np.ones(len(xg))]
+        lp = linprog(c=[0, 0, 0, 1], A_ub=A_ub, b_ub=b_ub, bounds=[(None, None)] * 4, method="highs")
+        assert lp.status == 0
+        assert lp.fun == pytest.approx(E, rel=1e-4)
+        assert E <= lp.fun * (1 + 1e-4)
+
+
+def test_minimax_limit_polynomial_on_a_shrinking_interval():
+    """On [1 - d, 1 + d] the minimax quintic tends to the odd quintic with
+    p(1) = 1 and p'(1) = p''(1) = 0, which the schedule uses once the
+    interval is too narrow to resolve."""
+    (a, b, c), E = oracle.minimax_odd_quintic(1 - 1e-3, 1 + 1e-3)
+    assert (a, b, c) == pytest.approx((15 / 8, -10 / 8, 3 / 8), abs=1e-4)
+    assert oracle.phi(1.0, 15 / 8, -10 / 8, 3 / 8) == pytest.approx(1.0, abs=1e-15)
+    assert 15 / 8 - 3 * 10 / 8 + 5 * 3 / 8 == pytest.approx(0.0, abs=1e-15)     # p'(1)
+    assert -6 * 10 / 8 + 20 * 3 / 8 == pytest.approx(0.0, abs=1e-15)            # p''(1)
