@@ -39,6 +39,9 @@ WORKLOAD = ("7B-shaped Muon step (224 matrices, 7.78e9 params, bf16 W/G, fp32 M,
 # size).  Kinds without a capture of the current kernel report null.
 KERNEL_TRAFFIC_BYTES = {"ns_gram": 35.9e9, "ns_apply": 55.4e9}
 
+# Pieces the end-to-end step splits the gradient upload into.
+E2E_CHUNKS = 8
+
 
 def parse_args(argv=None):
     p = argparse.ArgumentParser()
@@ -421,11 +424,20 @@ def main(argv=None):
         outs_host = [torch.empty(t.shape, dtype=t.dtype).pin_memory() for t in (norms, smax, gamma, mask)]
         h2d = g_host.numel() * g_host.element_size() + x_host.numel() * x_host.element_size()
         d2h = sum(t.numel() * t.element_size() for t in outs_host)
+        g_host_views, off = [], 0
+        for (r, c) in shapes:
+            g_host_views.append(g_host[off:off + r * c].view(r, c))
+            off += r * c
 
         def e2e_step():
-            Gf.copy_(g_host, non_blocking=True)
+            # the gradient upload overlaps the Muon step of the pieces already
+            # on the device (mc_muon_step_host_grads); X goes up on the stream
+            mc.muon_step_host_grads(Ws, Gs, g_host_views, Ms, chunks=E2E_CHUNKS, norms_out=norms,
+                                    stream=stream, **hp)
             x.copy_(x_host, non_blocking=True)
-            step()
+            mc.qk_max_logit(x, wq, wk, H, dh, causal=True, smax_out=smax, stream=stream)
+            mc.qk_clip(wq, wk, smax, H, dh, tau=wl.QK_TAU, alpha=wl.QK_ALPHA, gamma_out=gamma, mask_out=mask,
+                       stream=stream)
             for dst, src in zip(outs_host, (norms, smax, gamma, mask)):
                 dst.copy_(src, non_blocking=True)
 
@@ -442,7 +454,9 @@ def main(argv=None):
         barrier()
         e2e_ms = max_over_ranks(f0.elapsed_time(f1)) / args.steps
         e2e = {"value": world * step_flops / (e2e_ms / 1e3) / 1e12, "unit": "TFLOP/s", "ms_per_step": e2e_ms,
-               "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h)}
+               "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h),
+               "api": f"muon_step_host_grads (gradient upload in {E2E_CHUNKS} pieces under the step), "
+                      "qk_max_logit, qk_clip"}
         del g_host, x_host
 
     extras = None

@@ -5,6 +5,7 @@
  * ("MuonClip: speed, then stability", §07 "One complete training step"):
  *
  *   mc_muon_step     the Muon update of a list of hidden 2D weights
+ *   mc_muon_step_host_grads  the same, with the gradient upload overlapped
  *   mc_qk_max_logit  per-head causal max of the pre-softmax logit (S_max)
  *   mc_qk_clip       QK-Clip: rescale the W_q / W_k rows of heads with S_max > tau
  *   mc_normuon_step  the Muon update with NorMuon's per-row normalisation
@@ -113,6 +114,26 @@ typedef struct {
 size_t mc_muon_workspace_size(const mc_param* params, int n, const mc_hparams* hp);
 int mc_muon_step(const mc_param* params, int n, const mc_hparams* hp, void* workspace,
                  size_t workspace_bytes, float* norms_out, void* stream);
+
+/*
+ * mc_muon_step_host_grads -- mc_muon_step for gradients that still sit in
+ * host memory.  g_host[i] (HOST, page-locked for the copies to overlap,
+ * rows*cols elements of params[i].g_dtype) is copied into params[i].g
+ * (device) on the library's own copy stream.  The list is split in order into
+ * `chunks` pieces of about equal bytes; the step of piece k runs on `stream`
+ * once piece k has landed, so the transfer of later pieces runs under the
+ * Newton-Schulz GEMMs of earlier ones.  Every result is bit-for-bit that of
+ * mc_muon_step (a matrix's update does not depend on the other matrices of a
+ * call).  The copies start after the work already queued on `stream`, and
+ * everything this call enqueues is ordered before later work on `stream`.
+ * Workspace: >= mc_muon_host_grads_workspace_size(...) (the largest piece's
+ * mc_muon_workspace_size), or NULL for an engine-owned buffer.
+ * Errors: as mc_muon_step, plus MC_ERR_INVAL for chunks < 1 or a NULL host
+ * pointer.
+ */
+size_t mc_muon_host_grads_workspace_size(const mc_param* params, int n, const mc_hparams* hp, int chunks);
+int mc_muon_step_host_grads(const mc_param* params, const void* const* g_host, int n, const mc_hparams* hp,
+                            int chunks, void* workspace, size_t workspace_bytes, float* norms_out, void* stream);
 
 /*
  * mc_qk_max_logit -- S_max[h] = max over b, i and j (j <= i when causal) of

@@ -24,7 +24,8 @@ MC_F32, MC_BF16 = 0, 1
 EXPORTS = ("mc_muon_workspace_size", "mc_muon_step", "mc_qk_workspace_size", "mc_qk_max_logit",
            "mc_qk_clip", "mc_last_error", "mc_device_status", "mc_profile_begin", "mc_profile_end",
            "mc_qk_max_logit_static", "mc_qk_clip_slices", "mc_mla_workspace_size", "mc_mla_max_logit",
-           "mc_shard_plan", "mc_normuon_workspace_size", "mc_normuon_step", "mc_polar_express_coeffs")
+           "mc_shard_plan", "mc_normuon_workspace_size", "mc_normuon_step", "mc_polar_express_coeffs",
+           "mc_muon_host_grads_workspace_size", "mc_muon_step_host_grads")
 MC_QK_STATIC_MAX_ELEMS = 1 << 24
 MC_QK_STATIC_MAX_HEADS = 4096
 
@@ -105,6 +106,10 @@ def load_library():
     lib.mc_normuon_workspace_size.restype = sz
     lib.mc_normuon_step.argtypes = [P(McParam), i32, P(McHparams), P(McNormuon), vp, sz, vp, vp]
     lib.mc_normuon_step.restype = i32
+    lib.mc_muon_host_grads_workspace_size.argtypes = [P(McParam), i32, P(McHparams), i32]
+    lib.mc_muon_host_grads_workspace_size.restype = sz
+    lib.mc_muon_step_host_grads.argtypes = [P(McParam), vp, i32, P(McHparams), i32, vp, sz, vp, vp]
+    lib.mc_muon_step_host_grads.restype = i32
     lib.mc_polar_express_coeffs.argtypes = [i32, ctypes.c_double, ctypes.c_double, P(ctypes.c_float)]
     lib.mc_polar_express_coeffs.restype = i32
     lib.mc_shard_plan.argtypes = [P(ctypes.c_int64), P(ctypes.c_int64), i32, i32, i32, P(ctypes.c_int32),
@@ -274,6 +279,36 @@ def muon_step(weights: Sequence, grads: Sequence, moms: Sequence, *, norms_out=N
     ws = workspace if workspace is not None else _workspace("muon", weights[0].device, need)
     _check(lib.mc_muon_step(arr, n, ctypes.byref(h), _ptr(ws), int(ws.numel() * ws.element_size()),
                             _ptr(norms_out), _stream_handle(stream)))
+
+
+def muon_step_host_grads(weights: Sequence, grads: Sequence, grads_host: Sequence, moms: Sequence, *,
+                         chunks: int = 8, norms_out=None, update_outs=None, workspace=None, stream=None,
+                         hparams: Optional[McHparams] = None, **hp) -> None:
+    """``muon_step`` whose gradients start in (page-locked) host memory:
+    ``grads_host[i]`` is copied into the device tensor ``grads[i]`` piece by
+    piece, overlapped with the step of the pieces already on the device (see
+    mc_muon_step_host_grads).  Results are those of ``muon_step``."""
+    lib = load_library()
+    arr, n = make_params(weights, grads, moms, update_outs)
+    if len(grads_host) != n:
+        raise ValueError("one host gradient per matrix")
+    hptr = (ctypes.c_void_p * max(n, 1))()
+    for i, (gh, g) in enumerate(zip(grads_host, grads)):
+        if gh.is_cuda or not gh.is_contiguous() or gh.dtype != g.dtype or gh.shape != g.shape:
+            raise ValueError(f"grads_host[{i}] must be a contiguous CPU tensor shaped and typed like grads[{i}]")
+        hptr[i] = _ptr(gh)
+    h = hparams if hparams is not None else make_hparams(**hp)
+    if n == 0:
+        return
+    if norms_out is not None:
+        _need_cuda_contig(norms_out, "norms_out")
+    need = int(lib.mc_muon_host_grads_workspace_size(arr, n, ctypes.byref(h), int(chunks)))
+    if need == 0:
+        _check(lib.mc_muon_step_host_grads(arr, hptr, n, ctypes.byref(h), int(chunks), None, 0, None, None))
+    ws = workspace if workspace is not None else _workspace("muon", weights[0].device, need)
+    _check(lib.mc_muon_step_host_grads(arr, hptr, n, ctypes.byref(h), int(chunks), _ptr(ws),
+                                       int(ws.numel() * ws.element_size()), _ptr(norms_out),
+                                       _stream_handle(stream)))
 
 
 def make_normuon(vs, beta2: float = 0.95, eps: float = 1e-8) -> McNormuon:

@@ -71,6 +71,10 @@ struct DeviceState {
   size_t pinned_bytes[kRing] = {};
   cudaEvent_t ev[kRing] = {};
   int next = 0;
+  // mc_muon_step_host_grads: a non-blocking stream for the gradient copies and
+  // events that order each chunk's compute after its copies
+  cudaStream_t copy_stream = nullptr;
+  std::vector<cudaEvent_t> chunk_ev;
 };
 
 std::mutex g_mu;
@@ -497,7 +501,9 @@ int validate_normuon(const mc_param* params, int n, const mc_normuon* nm) {
 }
 
 int run_muon(const mc_param* params, int n, const mc_hparams* hp, const mc_normuon* nm, void* workspace,
-             size_t workspace_bytes, float* norms_out, cudaStream_t s);
+             size_t workspace_bytes, float* norms_out, cudaStream_t s, uint8_t* tab_dev = nullptr);
+void build_muon_table(const mc_param* params, int n, const mc_hparams* hp, const mc_normuon* nm, uint8_t* ws,
+                      const MuonLayout& L, uint8_t* tab);
 }  // namespace
 
 MC_API size_t mc_normuon_workspace_size(const mc_param* params, int n, const mc_hparams* hp) {
@@ -507,11 +513,35 @@ MC_API size_t mc_normuon_workspace_size(const mc_param* params, int n, const mc_
   return L.total;
 }
 
+int check_out_align(const float* norms_out, const void* workspace) {
+  if (norms_out && !aligned16(norms_out)) return fail(MC_ERR_ALIGN, "norms_out must be 16-byte aligned");
+  if (workspace && !aligned16(workspace)) return fail(MC_ERR_ALIGN, "workspace must be 16-byte aligned");
+  return MC_OK;
+}
+
+// Split params[0, n) in order into at most `chunks` pieces of about equal
+// gradient bytes; returns the piece boundaries (first entry 0, last n).
+std::vector<int> split_chunks(const mc_param* params, int n, int chunks) {
+  double total = 0;
+  for (int i = 0; i < n; ++i)
+    total += double(params[i].rows) * double(params[i].cols) * (params[i].g_dtype == MC_F32 ? 4 : 2);
+  std::vector<int> b{0};
+  double acc = 0;
+  for (int i = 0; i < n; ++i) {
+    acc += double(params[i].rows) * double(params[i].cols) * (params[i].g_dtype == MC_F32 ? 4 : 2);
+    const int k = static_cast<int>(b.size());
+    if (i + 1 < n && k < chunks && acc >= total * k / chunks) b.push_back(i + 1);
+  }
+  b.push_back(n);
+  return b;
+}
+
 MC_API int mc_normuon_step(const mc_param* params, int n, const mc_hparams* hp, const mc_normuon* nm,
                            void* workspace, size_t workspace_bytes, float* norms_out, void* stream) {
   int rc = validate_muon(params, n, hp);
   if (rc != MC_OK) return rc;
   if ((rc = validate_normuon(params, n, nm)) != MC_OK) return rc;
+  if ((rc = check_out_align(norms_out, workspace)) != MC_OK) return rc;
   if (n == 0) return MC_OK;
   return run_muon(params, n, hp, nm, workspace, workspace_bytes, norms_out, static_cast<cudaStream_t>(stream));
 }
@@ -520,35 +550,124 @@ MC_API int mc_muon_step(const mc_param* params, int n, const mc_hparams* hp, voi
                         size_t workspace_bytes, float* norms_out, void* stream) {
   int rc = validate_muon(params, n, hp);
   if (rc != MC_OK) return rc;
+  if ((rc = check_out_align(norms_out, workspace)) != MC_OK) return rc;
   if (n == 0) return MC_OK;
   return run_muon(params, n, hp, nullptr, workspace, workspace_bytes, norms_out,
                   static_cast<cudaStream_t>(stream));
 }
 
-namespace {
-int run_muon(const mc_param* params, int n, const mc_hparams* hp, const mc_normuon* nm, void* workspace,
-             size_t workspace_bytes, float* norms_out, cudaStream_t s) {
-  int rc = MC_OK;
-  if (norms_out && !aligned16(norms_out)) return fail(MC_ERR_ALIGN, "norms_out must be 16-byte aligned");
-  if (workspace && !aligned16(workspace)) return fail(MC_ERR_ALIGN, "workspace must be 16-byte aligned");
-  std::lock_guard<std::mutex> lock(g_mu);
-  DeviceState* st = nullptr;
-  if ((rc = device_state(&st)) != MC_OK) return rc;
+// Workspace of mc_muon_step_host_grads: one compute region that every piece
+// reuses in turn, then every piece's tables, all uploaded before the first
+// gradient copy.  (A table upload queued behind the gradient copies would
+// wait for all of them in the copy engine, and so would the first piece.)
+struct HostGradsPlan {
+  std::vector<int> bounds;
+  std::vector<MuonLayout> layouts;
+  std::vector<size_t> tab_off;
+  size_t compute = 0, total = 0;
+};
 
-  MuonLayout L;
-  plan_muon(params, n, L, nm != nullptr);
-  if (workspace) {
-    if (workspace_bytes < L.total)
-      return fail(MC_ERR_NOSPC, "workspace has " + std::to_string(workspace_bytes) + " bytes, needs " +
-                                    std::to_string(L.total));
-  } else if ((rc = own_workspace(*st, L.total, &workspace)) != MC_OK) {
-    return rc;
+void plan_host_grads(const mc_param* params, int n, int chunks, HostGradsPlan& P) {
+  P.bounds = split_chunks(params, n, chunks);
+  const int nch = static_cast<int>(P.bounds.size()) - 1;
+  P.layouts.resize(static_cast<size_t>(nch));
+  for (int k = 0; k < nch; ++k) {
+    plan_muon(params + P.bounds[k], P.bounds[k + 1] - P.bounds[k], P.layouts[size_t(k)]);
+    P.compute = std::max(P.compute, P.layouts[size_t(k)].total);
   }
-  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  size_t off = align_up(P.compute, 1024);
+  for (int k = 0; k < nch; ++k) {
+    P.tab_off.push_back(off);
+    off = align_up(off + P.layouts[size_t(k)].tab_bytes, 256);
+  }
+  P.total = align_up(off, 1024);
+}
 
-  // ---- device tables
-  std::vector<uint8_t> tab(L.tab_bytes, 0);
-  MomEntry* ent = reinterpret_cast<MomEntry*>(tab.data());
+MC_API size_t mc_muon_host_grads_workspace_size(const mc_param* params, int n, const mc_hparams* hp, int chunks) {
+  if (validate_muon(params, n, hp) != MC_OK || n == 0 || chunks < 1) return 0;
+  HostGradsPlan P;
+  plan_host_grads(params, n, chunks, P);
+  return P.total;
+}
+
+MC_API int mc_muon_step_host_grads(const mc_param* params, const void* const* g_host, int n, const mc_hparams* hp,
+                                   int chunks, void* workspace, size_t workspace_bytes, float* norms_out,
+                                   void* stream) {
+  int rc = validate_muon(params, n, hp);
+  if (rc != MC_OK) return rc;
+  if ((rc = check_out_align(norms_out, workspace)) != MC_OK) return rc;
+  if (chunks < 1) return fail(MC_ERR_INVAL, "chunks must be >= 1");
+  if (n > 0 && !g_host) return fail(MC_ERR_INVAL, "g_host is NULL");
+  for (int i = 0; i < n; ++i)
+    if (!g_host[i]) return fail(MC_ERR_INVAL, "g_host[" + std::to_string(i) + "] is NULL");
+  if (n == 0) return MC_OK;
+  HostGradsPlan P;
+  plan_host_grads(params, n, chunks, P);
+  const std::vector<int>& b = P.bounds;
+  const int nch = static_cast<int>(b.size()) - 1;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  std::vector<cudaEvent_t> done(static_cast<size_t>(nch));
+  uint8_t* ws = nullptr;
+  {
+    std::lock_guard<std::mutex> lock(g_mu);
+    DeviceState* st = nullptr;
+    if ((rc = device_state(&st)) != MC_OK) return rc;
+    if (workspace) {
+      if (workspace_bytes < P.total)
+        return fail(MC_ERR_NOSPC, "workspace has " + std::to_string(workspace_bytes) + " bytes, needs " +
+                                      std::to_string(P.total));
+    } else if ((rc = own_workspace(*st, P.total, &workspace)) != MC_OK) {
+      return rc;
+    }
+    ws = static_cast<uint8_t*>(workspace);
+    // every piece's tables, in one upload, ahead of the gradient copies
+    const size_t t0 = P.tab_off.front();
+    std::vector<uint8_t> tabs(P.total - t0, 0);
+    for (int k = 0; k < nch; ++k)
+      build_muon_table(params + b[k], b[k + 1] - b[k], hp, nullptr, ws, P.layouts[size_t(k)],
+                       tabs.data() + (P.tab_off[size_t(k)] - t0));
+    if ((rc = upload(*st, tabs.data(), tabs.size(), ws + t0, s)) != MC_OK) return rc;
+    if (!st->copy_stream) MC_CUDA(cudaStreamCreateWithFlags(&st->copy_stream, cudaStreamNonBlocking));
+    while (static_cast<int>(st->chunk_ev.size()) < nch + 1) {
+      cudaEvent_t e;
+      MC_CUDA(cudaEventCreateWithFlags(&e, cudaEventDisableTiming));
+      st->chunk_ev.push_back(e);
+    }
+    // Copies start only after the work already queued on `stream` (which may
+    // still read the previous gradients, and includes the table upload); each
+    // piece's step waits for its own copies.
+    MC_CUDA(cudaEventRecord(st->chunk_ev[nch], s));
+    MC_CUDA(cudaStreamWaitEvent(st->copy_stream, st->chunk_ev[nch], 0));
+    for (int k = 0; k < nch; ++k) {
+      for (int i = b[k]; i < b[k + 1]; ++i) {
+        const size_t bytes = size_t(params[i].rows) * size_t(params[i].cols) * (params[i].g_dtype == MC_F32 ? 4 : 2);
+        MC_CUDA(cudaMemcpyAsync(const_cast<void*>(params[i].g), g_host[i], bytes, cudaMemcpyHostToDevice,
+                                st->copy_stream));
+      }
+      MC_CUDA(cudaEventRecord(st->chunk_ev[k], st->copy_stream));
+      done[static_cast<size_t>(k)] = st->chunk_ev[k];
+    }
+  }
+  // Piece k's step waits only for piece k's copies, so the copies of later
+  // pieces run under the GEMMs of earlier ones.  Its tables are already on
+  // the device, so it queues no copy of its own.
+  for (int k = 0; k < nch; ++k) {
+    MC_CUDA(cudaStreamWaitEvent(s, done[static_cast<size_t>(k)], 0));
+    if ((rc = run_muon(params + b[k], b[k + 1] - b[k], hp, nullptr, ws, P.compute,
+                       norms_out ? norms_out + b[k] : nullptr, s, ws + P.tab_off[size_t(k)])) != MC_OK)
+      return rc;
+  }
+  return MC_OK;
+}
+
+namespace {
+// Host image of the device tables of one call (MomEntry[n], the per-group
+// weight and update pointer arrays, NormEntry[n] for NorMuon), for a layout
+// whose workspace starts at `ws`.
+void build_muon_table(const mc_param* params, int n, const mc_hparams* hp, const mc_normuon* nm, uint8_t* ws,
+                      const MuonLayout& L, uint8_t* tab) {
+  std::memset(tab, 0, L.tab_bytes);
+  MomEntry* ent = reinterpret_cast<MomEntry*>(tab);
   int k = 0;
   for (const auto& g : L.groups) {
     const size_t xe = size_t(g.rows) * size_t(g.ld);
@@ -566,14 +685,14 @@ int run_muon(const mc_param* params, int n, const mc_hparams* hp, const mc_normu
       e.g_f32 = q.g_dtype == MC_F32;
       e.vec = (q.cols % 8) == 0;
       e.orig = g.members[j];
-      void** wp = reinterpret_cast<void**>(tab.data() + g.off_wptr);
-      float** up = reinterpret_cast<float**>(tab.data() + g.off_uptr);
+      void** wp = reinterpret_cast<void**>(tab + g.off_wptr);
+      float** up = reinterpret_cast<float**>(tab + g.off_uptr);
       wp[j] = q.w;
       up[j] = q.update_out;
     }
   }
   if (nm) {
-    NormEntry* ne = reinterpret_cast<NormEntry*>(tab.data() + L.off_ntab);
+    NormEntry* ne = reinterpret_cast<NormEntry*>(tab + L.off_ntab);
     long long rb = 0;
     for (int kk = 0; kk < n; ++kk) {
       const mc_param& q = params[ent[kk].orig];
@@ -593,10 +712,40 @@ int run_muon(const mc_param* params, int n, const mc_hparams* hp, const mc_normu
       rb += q.rows;
     }
   }
-  if ((rc = upload(*st, tab.data(), tab.size(), ws + L.off_tab, s)) != MC_OK) return rc;
+}
+
+// `tab_dev`: where the tables already are (uploaded by the caller), or NULL to
+// upload them to the start of the workspace here.
+int run_muon(const mc_param* params, int n, const mc_hparams* hp, const mc_normuon* nm, void* workspace,
+             size_t workspace_bytes, float* norms_out, cudaStream_t s, uint8_t* tab_dev) {
+  int rc = MC_OK;
+  std::lock_guard<std::mutex> lock(g_mu);
+  DeviceState* st = nullptr;
+  if ((rc = device_state(&st)) != MC_OK) return rc;
+
+  MuonLayout L;
+  plan_muon(params, n, L, nm != nullptr);
+  if (workspace) {
+    if (workspace_bytes < L.total)
+      return fail(MC_ERR_NOSPC, "workspace has " + std::to_string(workspace_bytes) + " bytes, needs " +
+                                    std::to_string(L.total));
+  } else if ((rc = own_workspace(*st, L.total, &workspace)) != MC_OK) {
+    return rc;
+  }
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+
+  // ---- device tables
+  uint8_t* tb = tab_dev;
+  if (!tb) {
+    tb = ws + L.off_tab;
+    std::vector<uint8_t> tab(L.tab_bytes, 0);
+    build_muon_table(params, n, hp, nm, ws, L, tab.data());
+    if ((rc = upload(*st, tab.data(), tab.size(), tb, s)) != MC_OK) return rc;
+  }
+
 
   // ---- momentum, Nesterov, fp32/bf16 iterate, norm partials
-  const MomEntry* dtab = reinterpret_cast<const MomEntry*>(ws + L.off_tab);
+  const MomEntry* dtab = reinterpret_cast<const MomEntry*>(tb);
   double* partials = reinterpret_cast<double*>(ws + L.off_partials);
   float* scale = reinterpret_cast<float*>(ws + L.off_scale);
   double mom_bytes = 0;
@@ -707,10 +856,10 @@ int run_muon(const mc_param* params, int n, const mc_hparams* hp, const mc_normu
         G.scale = first ? scale : nullptr;
         G.coef_src = ca;
         if (last && !nm) {
-          G.w_ptrs = reinterpret_cast<void* const*>(ws + g.off_wptr);
+          G.w_ptrs = reinterpret_cast<void* const*>(tb + g.off_wptr);
           bool any_u = false;
           for (int i : g.members) any_u |= params[i].update_out != nullptr;
-          G.u_ptrs = any_u ? reinterpret_cast<float* const*>(ws + g.off_uptr) : nullptr;
+          G.u_ptrs = any_u ? reinterpret_cast<float* const*>(tb + g.off_uptr) : nullptr;
           G.w_f32 = g.w_f32;
           G.w_vec = g.w_f32 ? (g.cols % 4 == 0) : (g.cols % 8 == 0);
           G.rms = hp->rms_scale * std::sqrt(static_cast<float>(std::max(g.rows, g.cols)));
@@ -735,7 +884,7 @@ int run_muon(const mc_param* params, int n, const mc_hparams* hp, const mc_normu
   }
   if (nm) {
     // NorMuon: row sums of squares of O, then the row factors, then the update.
-    const NormEntry* ntab = reinterpret_cast<const NormEntry*>(ws + L.off_tab + L.off_ntab);
+    const NormEntry* ntab = reinterpret_cast<const NormEntry*>(tb + L.off_ntab);
     float* rowsq = reinterpret_cast<float*>(ws + L.off_rowsq);
     float* rowf = reinterpret_cast<float*>(ws + L.off_rowf);
     double o_bytes = 0, w_bytes = 0;

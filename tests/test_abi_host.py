@@ -224,3 +224,22 @@ def test_polar_express_coeffs_match_the_oracle(lib):
     assert lib.mc_polar_express_coeffs(5, 1.0, 0.01, out) == mc.MC_ERR_INVAL
     assert lib.mc_polar_express_coeffs(5, 1e-3, -0.1, out) == mc.MC_ERR_INVAL
     assert lib.mc_polar_express_coeffs(5, 1e-3, 0.01, None) == mc.MC_ERR_INVAL
+
+
+def test_host_grads_entry_arguments_and_workspace(lib):
+    P = ctypes.byref
+    hp = mc.make_hparams()
+    arr = _params(6, rows=128, cols=256)
+    hptr = (ctypes.c_void_p * 6)(*[0x7000000 + i * 0x100000 for i in range(6)])
+    assert lib.mc_muon_step_host_grads(arr, hptr, 6, P(hp), 0, None, 0, None, None) == mc.MC_ERR_INVAL
+    assert lib.mc_muon_step_host_grads(arr, None, 6, P(hp), 2, None, 0, None, None) == mc.MC_ERR_INVAL
+    bad = (ctypes.c_void_p * 6)(*([0x7000000] * 5 + [0]))
+    assert lib.mc_muon_step_host_grads(arr, bad, 6, P(hp), 2, None, 0, None, None) == mc.MC_ERR_INVAL
+    # one compute region reused by every piece, plus every piece's own tables
+    full = lib.mc_muon_workspace_size(arr, 6, P(hp))
+    one = lib.mc_muon_host_grads_workspace_size(arr, 6, P(hp), 1)
+    assert full < one <= full + 64 * 1024
+    three = lib.mc_muon_host_grads_workspace_size(arr, 6, P(hp), 3)
+    two = lib.mc_muon_workspace_size(arr, 2, P(hp))                  # six equal matrices in pieces of two
+    assert two < three <= two + 64 * 1024 and three < one
+    assert lib.mc_muon_host_grads_workspace_size(arr, 6, P(hp), 0) == 0
