@@ -33,11 +33,14 @@ WORKLOAD = ("7B-shaped Muon step (224 matrices, 7.78e9 params, bf16 W/G, fp32 M,
             "+ causal MHA S_max and QK-Clip (B4 S4096 H32 dh128)")
 
 
-# DRAM bytes per launch (dram__bytes_read.sum + dram__bytes_write.sum) of the
-# kernels as they stand, from one ncu capture: profiles/ns_gemm_1layer_full.md
-# (1-layer case, third NS iteration, scaled by the 32 layers processed at full
-# size).  Kinds without a capture of the current kernel report null.
-KERNEL_TRAFFIC_BYTES = {"ns_gram": 35.9e9, "ns_apply": 55.4e9}
+# DRAM bytes (dram__bytes_read.sum + dram__bytes_write.sum) of one launch of a
+# kernel kind over ONE layer of the 7B-shaped set, from the ncu capture in
+# profiles/ns_gemm_1layer_full.md (third NS iteration).  A launch at full size
+# covers several layers (the engine runs the list in pieces), and traffic is
+# proportional to the matrices processed, so the per-launch figure is this
+# times the layers one launch covers.  Kinds without a capture of the kernel
+# as it stands are absent (reported as null).
+KERNEL_TRAFFIC_PER_LAYER = {"ns_gram": 1.117e9, "ns_apply": 1.724e9}
 
 # Pieces the end-to-end step splits the gradient upload into.
 E2E_CHUNKS = 8
@@ -405,7 +408,13 @@ def main(argv=None):
     d = kernels[dom]
     if d["flops"] > 0:
         ach = d["flops"] / (d["total_ms"] / 1e3) / 1e12
-        traffic = KERNEL_TRAFFIC_BYTES.get(dom) if args.layers == 32 else None
+        traffic = None
+        per_layer = KERNEL_TRAFFIC_PER_LAYER.get(dom)
+        iters = {"ns_gram": hp["ns_steps"], "ns_poly": hp["ns_steps"], "ns_apply_final": 1,
+                 "ns_apply_mixed": min(2, hp["ns_steps"] - 1), "ns_apply": max(hp["ns_steps"] - 3, 0)}.get(dom)
+        if per_layer and iters:
+            launches_per_step = d["launches"] / K
+            traffic = per_layer * args.layers * iters / launches_per_step
         roof = {"kernel": dom, "bound": "tensor", "achieved": ach, "peak": peaks["bf16_tflops_sustained"],
                 "unit": "TFLOP/s", "frac": ach / peaks["bf16_tflops_sustained"], "traffic": traffic,
                 "peak_source": f"{peaks['source']} bf16_tflops_sustained (kernel timed inside a long step)"}

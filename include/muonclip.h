@@ -95,17 +95,22 @@ typedef struct {
  *   W <- W - lr*(rms_scale*sqrt(max(rows,cols))*O + wd*W)
  * The Newton-Schulz products run on tcgen05 tensor cores with bf16 operands
  * and fp32 accumulation.  In the first two iterations the a*X term is taken
- * from an fp32 copy of the iterate; from the third on, a*I is folded into B
+ * from a two-part copy of the iterate (bf16 hi + bf16 lo, about 16
+ * significant bits); from the third on, a*I is folded into B
  * (X <- (aI + B) X), which amplifies the bf16 rounding of X less once the
  * singular values have entered the polynomial's band.  The last iteration
  * applies the update to W straight from the fp32 accumulator.
- * Matrices of equal shape and weight dtype are batched into one problem group.
+ * The list is processed in consecutive pieces of at most 2^30 elements (at
+ * least one matrix each), all reusing one workspace; inside a piece, matrices
+ * of equal shape and weight dtype are batched into one problem group.  A
+ * matrix's result does not depend on the other matrices of the call.
  *
  * params/n      host array of n >= 0 entries (n == 0 is a no-op).  W, G, M of
  *               one entry must not alias; G is left unchanged.
  * hp            host pointer.
- * workspace     device scratch of at least mc_muon_workspace_size(...) bytes,
- *               or NULL to let the library allocate (and keep) its own.
+ * workspace     device scratch of at least mc_muon_workspace_size(...) bytes
+ *               (what the largest piece needs), or NULL to let the library
+ *               allocate (and keep) its own.
  *               Must not be used by anything else until the step completes.
  * norms_out     optional device fp32 [n]: ||U||_F of each matrix (NULL = skip).
  * Errors        MC_ERR_INVAL, MC_ERR_ALIGN, MC_ERR_NOSPC, MC_ERR_CUDA,
@@ -361,12 +366,12 @@ int mc_device_status(void);
  * mc_profile_end() waits for those events and reports one row per kernel kind:
  *
  *   momentum        bytes = the momentum kernel's DRAM traffic by design:
- *                   G (2 or 4) + M read/write (8) + fp32 and bf16 iterate (6)
- *                   bytes per element
+ *                   G (2 or 4) + M read/write (8) + the iterate's two bf16
+ *                   halves, hi and lo (4) bytes per element
  *   ns_gram         A = X X^T: flops = m (m+1) n (the entries on and above the
  *                   diagonal, 2n each), flops_dense_equiv = 2 m^2 n
  *   ns_poly         B = bA + cA^2: flops = m^2 (m+1), flops_dense_equiv = 2 m^3
- *   ns_apply_mixed  X <- s(aX + BX), iterations that read the fp32 iterate
+ *   ns_apply_mixed  X <- s(aX + BX), iterations that read the iterate's hi + lo halves
  *   ns_apply        X <- (aI + B) X, later iterations
  *   ns_apply_final  last iteration fused with the weight update
  *                   (apply rows: flops = flops_dense_equiv = 2 m^2 n.  Per

@@ -1,8 +1,9 @@
 // Bandwidth-bound kernels of the MuonClip step (CUDA cores, 128-bit accesses).
 //
 //  momentum_kernel   M <- mu*M + G;  U = G + mu*M (Nesterov) or M;  writes U as
-//                    the fp32 iterate and its bf16 copy (same row-major layout as
-//                    the weight), and one fp64 partial of ||U||_F^2 per CTA.
+//                    two bf16 halves, hi = bf16(U) (the first MMA operand) and
+//                    lo = bf16(U - hi) (same row-major layout as the weight), and
+//                    one fp64 partial of ||U||_F^2 per CTA.
 //                    ("MuonClip: speed, then stability", §02 momentum; "Muon and
 //                    MuonClip: orthogonalised updates for LLM training", §2
 //                    Frobenius normalisation.)
@@ -42,8 +43,8 @@ constexpr long long MOM_ELEMS_PER_CTA = 32768;
 struct MomEntry {
   const void* g;        // gradient, rows x cols row-major (bf16 or fp32)
   float* m;             // momentum, rows x cols row-major, updated in place
-  float* xf;            // fp32 iterate [rows][ld]
-  __nv_bfloat16* xb;    // bf16 iterate [rows][ld]
+  __nv_bfloat16* xl;    // lo half of the iterate, bf16(U - bf16(U)) [rows][ld]
+  __nv_bfloat16* xb;    // bf16 iterate (its hi half) [rows][ld]
   long long rows, cols, ld;
   long long cta_begin;  // first CTA of this matrix in the launch
   int g_f32;
@@ -70,7 +71,8 @@ __device__ __forceinline__ void load_g8(const void* g, long long idx, int g_f32,
 }
 
 __device__ __forceinline__ void momentum8(const float (&g)[8], float4 ma, float4 mb, float mu, int nesterov,
-                                          float* m_out, float* xf_out, __nv_bfloat16* xb_out, double& acc) {
+                                          float* m_out, __nv_bfloat16* xl_out, __nv_bfloat16* xb_out,
+                                          double& acc) {
   float m[8] = {ma.x, ma.y, ma.z, ma.w, mb.x, mb.y, mb.z, mb.w};
   float u[8];
 #pragma unroll
@@ -82,15 +84,21 @@ __device__ __forceinline__ void momentum8(const float (&g)[8], float4 ma, float4
   float4* mp = reinterpret_cast<float4*>(m_out);
   mp[0] = make_float4(m[0], m[1], m[2], m[3]);
   mp[1] = make_float4(m[4], m[5], m[6], m[7]);
-  float4* xp = reinterpret_cast<float4*>(xf_out);
-  xp[0] = make_float4(u[0], u[1], u[2], u[3]);
-  xp[1] = make_float4(u[4], u[5], u[6], u[7]);
+  float lo[8];
+#pragma unroll
+  for (int i = 0; i < 8; ++i) lo[i] = u[i] - __bfloat162float(__float2bfloat16_rn(u[i]));
   uint4 b;
   b.x = pack_bf16x2(u[0], u[1]);
   b.y = pack_bf16x2(u[2], u[3]);
   b.z = pack_bf16x2(u[4], u[5]);
   b.w = pack_bf16x2(u[6], u[7]);
   *reinterpret_cast<uint4*>(xb_out) = b;
+  uint4 l;
+  l.x = pack_bf16x2(lo[0], lo[1]);
+  l.y = pack_bf16x2(lo[2], lo[3]);
+  l.z = pack_bf16x2(lo[4], lo[5]);
+  l.w = pack_bf16x2(lo[6], lo[7]);
+  *reinterpret_cast<uint4*>(xl_out) = l;
 }
 
 __global__ void __launch_bounds__(MOM_THREADS) momentum_kernel(const MomEntry* __restrict__ tab, int n,
@@ -106,7 +114,7 @@ __global__ void __launch_bounds__(MOM_THREADS) momentum_kernel(const MomEntry* _
   const MomEntry* e = tab + lo;
   const void* gp = e->g;
   float* mp = e->m;
-  float* xf = e->xf;
+  __nv_bfloat16* xl = e->xl;
   __nv_bfloat16* xb = e->xb;
   const long long cols = e->cols, ld = e->ld;
   const long long total = e->rows * cols;
@@ -132,8 +140,8 @@ __global__ void __launch_bounds__(MOM_THREADS) momentum_kernel(const MomEntry* _
         m1a = m1p[0];
         m1b = m1p[1];
       }
-      momentum8(g0, m0a, m0b, mu, nesterov, mp + idx, xf + idx, xb + idx, acc);
-      if (two) momentum8(g1, m1a, m1b, mu, nesterov, mp + j, xf + j, xb + j, acc);
+      momentum8(g0, m0a, m0b, mu, nesterov, mp + idx, xl + idx, xb + idx, acc);
+      if (two) momentum8(g1, m1a, m1b, mu, nesterov, mp + j, xl + j, xb + j, acc);
     }
   } else {
     for (long long idx = e0 + threadIdx.x; idx < e1; idx += MOM_THREADS) {
@@ -144,8 +152,9 @@ __global__ void __launch_bounds__(MOM_THREADS) momentum_kernel(const MomEntry* _
       const float u = nesterov ? fmaf(mu, m, g) : m;
       acc += static_cast<double>(u) * static_cast<double>(u);
       const long long row = idx / cols, col = idx - row * cols;
-      xf[row * ld + col] = u;
-      xb[row * ld + col] = __float2bfloat16_rn(u);
+      const __nv_bfloat16 h = __float2bfloat16_rn(u);
+      xb[row * ld + col] = h;
+      xl[row * ld + col] = __float2bfloat16_rn(u - __bfloat162float(h));
     }
   }
   // Fixed-order block reduction (deterministic).

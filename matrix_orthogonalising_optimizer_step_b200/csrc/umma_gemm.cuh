@@ -7,14 +7,17 @@
 //   EPI_GRAM        A_k   = s^2 * X X^T            (symmetric: upper tiles only,
 //                                                  each element stored twice)
 //   EPI_POLY        B_k   = b*A + c*(A A) [+ a*I]  (symmetric, mirrored store)
-//   EPI_APPLY       X_k+1 = s * (a*X + B X)        (fp32 iterate read/written in
-//                           or  P X, P = aI+bA+cA^2  place when flagged + bf16 copy)
+//   EPI_APPLY       X_k+1 = s * (a*X + B X)        (a*X from the hi + lo copy of
+//                           or  P X, P = aI+bA+cA^2  the iterate; stores the bf16
+//                                                  iterate, its lo half when flagged)
 //   EPI_APPLY_FINAL W     = (1 - lr*wd) W - lr * rms * X_N   (last iteration; X_N
 //                                                  never touches memory)
 //
 // Precision: operands are bf16, accumulation fp32.  While singular values are
-// still small (the first two iterations) the a*X term is taken from an fp32
-// copy of the iterate, so only B X sees a rounded X; afterwards a*I is folded
+// still small (the first two iterations) the a*X term is taken from a
+// two-part copy of the iterate, hi = bf16(X) (the MMA operand itself) plus
+// lo = bf16(X - hi), about 16 significant bits, so only B X sees a rounded X
+// (emulated against an fp32 copy: the same error to within 1 %); afterwards a*I is folded
 // into B, because once the singular values sit in the polynomial's band
 // |a + b s^2 + c s^4| (the factor on a rounded X in P X) is smaller than
 // |b s^2 + c s^4| (the factor in B X).
@@ -128,9 +131,15 @@ struct GemmGroup {
   long long d_ld, d_bs;
   const void* src;         // bf16 epilogue source (EPI_POLY)
   long long src_ld, src_bs;
-  float* xf;               // fp32 iterate (EPI_APPLY*)
+  const __nv_bfloat16* xh; // EPI_APPLY*: hi half of the iterate (its bf16 copy)
+  long long xh_ld, xh_bs;
+  __nv_bfloat16* xl;       // EPI_APPLY*: lo half of the iterate, bf16(X - hi)
+  long long xl_ld, xl_bs;
+  float* xf;               // EPI_APPLY: fp32 copy of the new iterate (when xf_write)
   long long xf_ld, xf_bs;
-  int xf_read, xf_write;   // EPI_APPLY*: take a*X from xf; store the new iterate to xf
+  int xf_read;             // EPI_APPLY*: take a*X from hi + lo
+  int xl_write;            // EPI_APPLY: store the new iterate's lo half to xl
+  int xf_write;            // EPI_APPLY: store the new iterate in fp32 to xf
   void* const* w_ptrs;     // per-problem weight (EPI_APPLY_FINAL), row-major M x N
   float* const* u_ptrs;    // per-problem update output, entries may be null
   const float* scale;      // per-problem s, or null for 1
@@ -173,6 +182,15 @@ __host__ __device__ inline long long sched_tiles_per_prob(int sched, int tiles_m
 struct TileInfo {
   int g, prob, tm, tn, num_kb;
 };
+
+// A symmetric-output tile of 256 rows x 512 columns whose first 256 columns
+// lie wholly below the diagonal (odd tile rows, first kept tile): only its
+// second N block holds kept entries, so the first block is neither loaded,
+// multiplied nor drained.
+template <int NB>
+__host__ __device__ inline bool sym_skip_first_block(const GemmGroup& G, const TileInfo& ti) {
+  return NB == 2 && G.sched == SCHED_SYM && 2 * ti.tn + 1 <= ti.tm;
+}
 
 __host__ __device__ inline void decode_tile(const GemmGroup* groups, int num_groups, long long t,
                                             TileInfo& ti) {
@@ -280,8 +298,9 @@ __device__ __forceinline__ void store_sym_chunk(__nv_bfloat16* D, long long ld, 
 // latencies overlap, then the chunk is finished (epi_finish).
 
 // Global operands of one chunk, kept as raw 128-bit words until used:
-// x = the b*A source (EPI_POLY, bf16) or the fp32 iterate (EPI_APPLY* with
-// xf_read); w = the weight (EPI_APPLY_FINAL, bf16 or fp32).
+// x = the b*A source (EPI_POLY, bf16: x[0..1]) or the iterate's hi and lo
+// halves (EPI_APPLY* with xf_read: x[0..1] and x[2..3]); w = the weight
+// (EPI_APPLY_FINAL, bf16 or fp32).
 struct EpiPre {
   uint4 x[4];
   uint4 w[4];
@@ -289,11 +308,12 @@ struct EpiPre {
 
 // `valid` columns are in range; `vec`: the 16 elements may be read as two
 // 16-byte words (aligned row and full chunk), else element by element.
-__device__ __forceinline__ void raw_load_bf16x16(const __nv_bfloat16* p, int valid, bool vec, uint4 (&q)[4]) {
+__device__ __forceinline__ void raw_load_bf16x16(const __nv_bfloat16* p, int valid, bool vec, uint4& q0,
+                                                 uint4& q1) {
   if (vec && valid >= 16) {
     const uint4* s = reinterpret_cast<const uint4*>(p);
-    q[0] = s[0];
-    q[1] = s[1];
+    q0 = s[0];
+    q1 = s[1];
   } else {
     uint32_t w[8];
 #pragma unroll
@@ -303,9 +323,12 @@ __device__ __forceinline__ void raw_load_bf16x16(const __nv_bfloat16* p, int val
           (2 * i + 1 < valid) ? static_cast<uint32_t>(*reinterpret_cast<const uint16_t*>(p + 2 * i + 1)) : 0u;
       w[i] = lo | (hi << 16);
     }
-    q[0] = make_uint4(w[0], w[1], w[2], w[3]);
-    q[1] = make_uint4(w[4], w[5], w[6], w[7]);
+    q0 = make_uint4(w[0], w[1], w[2], w[3]);
+    q1 = make_uint4(w[4], w[5], w[6], w[7]);
   }
+}
+__device__ __forceinline__ void raw_load_bf16x16(const __nv_bfloat16* p, int valid, bool vec, uint4 (&q)[4]) {
+  raw_load_bf16x16(p, valid, vec, q[0], q[1]);
 }
 __device__ __forceinline__ void raw_load_f32x16(const float* p, int valid, bool vec, uint4 (&q)[4]) {
   if (vec && valid >= 16) {
@@ -326,6 +349,16 @@ __device__ __forceinline__ void raw_to_bf16x16(const uint4 (&q)[4], float (&x)[1
   for (int i = 0; i < 8; ++i) {
     x[2 * i] = __uint_as_float(w[i] << 16);
     x[2 * i + 1] = __uint_as_float(w[i] & 0xFFFF0000u);
+  }
+}
+// hi + lo halves (x[0..1] and x[2..3], bf16 each) back to fp32; the sum is exact.
+__device__ __forceinline__ void raw_hilo_to_f32x16(const uint4 (&q)[4], float (&x)[16]) {
+  const uint32_t h[8] = {q[0].x, q[0].y, q[0].z, q[0].w, q[1].x, q[1].y, q[1].z, q[1].w};
+  const uint32_t l[8] = {q[2].x, q[2].y, q[2].z, q[2].w, q[3].x, q[3].y, q[3].z, q[3].w};
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    x[2 * i] = __uint_as_float(h[i] << 16) + __uint_as_float(l[i] << 16);
+    x[2 * i + 1] = __uint_as_float(h[i] & 0xFFFF0000u) + __uint_as_float(l[i] & 0xFFFF0000u);
   }
 }
 __device__ __forceinline__ void raw_to_f32x16(const uint4 (&q)[4], float (&x)[16]) {
@@ -349,8 +382,10 @@ __device__ __forceinline__ void epi_prefetch(const GemmGroup& G, int prob, int r
     raw_load_bf16x16(S + c0, valid, true, pre.x);
   } else if constexpr (EPI == EPI_APPLY || EPI == EPI_APPLY_FINAL) {
     if (G.xf_read) {
-      const float* X = G.xf + (long long)prob * G.xf_bs + (long long)r * G.xf_ld;
-      raw_load_f32x16(X + c0, valid, true, pre.x);
+      const __nv_bfloat16* Xh = G.xh + (long long)prob * G.xh_bs + (long long)r * G.xh_ld;
+      const __nv_bfloat16* Xl = G.xl + (long long)prob * G.xl_bs + (long long)r * G.xl_ld;
+      raw_load_bf16x16(Xh + c0, valid, true, pre.x[0], pre.x[1]);
+      raw_load_bf16x16(Xl + c0, valid, true, pre.x[2], pre.x[3]);
     }
     if constexpr (EPI == EPI_APPLY_FINAL) {
       const long long row = (long long)r * G.N;
@@ -394,7 +429,7 @@ __device__ __forceinline__ void epi_finish(const GemmGroup& G, int prob, int r, 
     float o[16];
     if (G.xf_read) {
       float x[16];
-      raw_to_f32x16(pre.x, x);
+      raw_hilo_to_f32x16(pre.x, x);
 #pragma unroll
       for (int j = 0; j < 16; ++j) o[j] = s * fmaf(G.coef_src, x[j], v[j]);
     } else {
@@ -402,17 +437,25 @@ __device__ __forceinline__ void epi_finish(const GemmGroup& G, int prob, int r, 
       for (int j = 0; j < 16; ++j) o[j] = s * v[j];
     }
     if constexpr (EPI == EPI_APPLY) {
-      float* X = G.xf ? G.xf + (long long)prob * G.xf_bs + (long long)r * G.xf_ld : nullptr;
+      float* X = G.xf_write ? G.xf + (long long)prob * G.xf_bs + (long long)r * G.xf_ld : nullptr;
+      __nv_bfloat16* XL = G.xl_write ? G.xl + (long long)prob * G.xl_bs + (long long)r * G.xl_ld : nullptr;
       __nv_bfloat16* D =
           static_cast<__nv_bfloat16*>(G.d) + (long long)prob * G.d_bs + (long long)r * G.d_ld;
+      float lo[16];
+      if (G.xl_write) {
+#pragma unroll
+        for (int j = 0; j < 16; ++j) lo[j] = o[j] - __bfloat162float(__float2bfloat16_rn(o[j]));
+      }
       if (full) {
         if (G.xf_write) store_f32x16(X + c0, o);
+        if (G.xl_write) store_bf16x16(XL + c0, lo);
         store_bf16x16(D + c0, o);
       } else {
 #pragma unroll
         for (int j = 0; j < 16; ++j)
           if (c0 + j < G.N) {
             if (G.xf_write) X[c0 + j] = o[j];
+            if (G.xl_write) XL[c0 + j] = __float2bfloat16_rn(lo[j]);
             D[c0 + j] = __float2bfloat16_rn(o[j]);
           }
       }
@@ -580,8 +623,10 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1) umma_gemm_kernel(const __grid
             break;
           }
           const uint32_t fb_local = smem_u32(&full_bar[stage]);
+          const bool skip0 = sym_skip_first_block<T::NB>(G, ti);
           if (leader) {
-            mbar_arrive_expect_tx(fb_local, T::PAIR_STAGE_BYTES);
+            // both CTAs of the pair skip the same block (it depends on the tile only)
+            mbar_arrive_expect_tx(fb_local, skip0 ? T::PAIR_STAGE_BYTES - 2 * B_STAGE_BYTES : T::PAIR_STAGE_BYTES);
             filled |= 1u << stage;
             fill_parity = (fill_parity & ~(1u << stage)) | (phase << stage);
           }
@@ -611,6 +656,7 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1) umma_gemm_kernel(const __grid
             }
 #pragma unroll
             for (int h = 0; h < T::NB; ++h) {
+              if (h == 0 && skip0) continue;
               const uint32_t sb = sa + A_STAGE_BYTES + h * B_STAGE_BYTES;
               const int nh = n0 + h * MMA_N;
               if (!G.b_mn) {
@@ -665,6 +711,7 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1) umma_gemm_kernel(const __grid
         // carry out of it since shared memory ends below 2^18).
         const uint64_t ad0 = smem_desc_sw128(s0, a_lbo, 1024);
         const uint64_t bd0 = smem_desc_sw128(s0 + A_STAGE_BYTES, b_lbo, 1024);
+        const bool skip0 = sym_skip_first_block<T::NB>(G, ti);
         for (int kb = 0; kb < ti.num_kb; ++kb) {
           // The TMA writes are made visible by the barrier's complete_tx; the
           // MMAs read them through the same async proxy.
@@ -678,6 +725,7 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1) umma_gemm_kernel(const __grid
             const uint64_t ad = ad0 + soff + ((kk * a_kstep) >> 4);
 #pragma unroll
             for (int h = 0; h < T::NB; ++h) {
+              if (h == 0 && skip0) continue;
               const uint64_t bd = bd0 + soff + ((h * B_STAGE_BYTES + kk * b_kstep) >> 4);
               umma_bf16_pair(d_tmem + h * MMA_N, ad, bd, idesc, (kb | kk) != 0);
             }
@@ -724,12 +772,15 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1) umma_gemm_kernel(const __grid
       const uint32_t t_row = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + acc * T::N + half * WCOLS;
       float run_max = -INFINITY;
       constexpr int CH = EpiBatch<EPI>::CH;
+      // With two column groups, group 0 is exactly the first N block.
+      static_assert(T::NB == 1 || EPI_COL_GROUPS == T::NB, "column groups match the N blocks");
+      const bool idle = half == 0 && sym_skip_first_block<T::NB>(G, ti);
       const int cbase = ti.tn * T::N + half * WCOLS;
       // Last row of this warp: a chunk that starts beyond it lies above the
       // diagonal for every lane, as do all later chunks (causal max only).
       const int r_warp_last = ti.tm * BM + HALF * static_cast<int>(rank) + q * 32 + 31;
 #pragma unroll 1
-      for (int cb = 0; cb < WCOLS / 16; cb += CH) {
+      for (int cb = 0; cb < (idle ? 0 : WCOLS / 16); cb += CH) {
         if constexpr (EPI == EPI_CAUSALMAX) {
           if (G.mask_causal && cbase + cb * 16 > r_warp_last) break;
         }

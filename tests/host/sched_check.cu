@@ -27,6 +27,8 @@ static void check_groups(std::vector<GemmGroup> gs) {
   long long total = 0;
   for (auto& g : gs) { g.tile_start = total; total += g.tiles_per_prob * g.count; }
   std::vector<std::set<std::tuple<int, int, int>>> seen(gs.size());
+  // (prob, tm, tn) of wide symmetric tiles whose first 256-column block is skipped
+  std::vector<std::set<std::tuple<int, int, int>>> skipped(gs.size());
   for (long long t = 0; t < total; ++t) {
     TileInfo ti;
     decode_tile(gs.data(), (int)gs.size(), t, ti);
@@ -39,6 +41,11 @@ static void check_groups(std::vector<GemmGroup> gs) {
     CHECK(!seen[ti.g].count(key), "duplicate tile");
     seen[ti.g].insert(key);
     const long long BNt = MMA_N << G.nshift;
+    if (G.nshift == 1 && sym_skip_first_block<2>(G, ti)) {
+      skipped[ti.g].insert(key);
+      // the skipped block must hold no element on or above the diagonal
+      CHECK((long long)ti.tn * BNt + MMA_N - 1 < (long long)ti.tm * BM, "skipped block reaches the diagonal");
+    }
     if (G.sched == SCHED_SYM) {
       CHECK(ti.tn >= (ti.tm >> G.nshift), "sym tile below diagonal");
       CHECK((long long)ti.tn * BNt + BNt - 1 >= (long long)ti.tm * BM, "sym tile with no upper element");
@@ -57,9 +64,15 @@ static void check_groups(std::vector<GemmGroup> gs) {
           for (int j = 0; j < G.tiles_n; ++j) CHECK(seen[gi].count({p, i, j}), "dense tile missing");
       } else if (G.sched == SCHED_SYM) {
         // every element (r, c) with c >= r must lie in a computed tile
+        // (and not in a skipped first block)
+        auto kept = [&](int r, int c) {
+          const auto key = std::make_tuple(p, r / BM, c / BN);
+          if (!seen[gi].count(key)) return false;
+          return !(skipped[gi].count(key) && (c % BN) < MMA_N);
+        };
         for (int r = 0; r < G.M; r += 7)
-          for (int c = r; c < G.N; c += 5) CHECK(seen[gi].count({p, r / BM, c / BN}), "sym element (%d,%d) uncovered", r, c);
-        for (int r = 0; r < G.M; ++r) CHECK(seen[gi].count({p, r / BM, r / BN}), "sym diagonal uncovered");
+          for (int c = r; c < G.N; c += 5) CHECK(kept(r, c), "sym element (%d,%d) uncovered", r, c);
+        for (int r = 0; r < G.M; ++r) CHECK(kept(r, r), "sym diagonal uncovered");
       } else {
         for (int r = 0; r < G.M; r += 3)
           for (int c = 0; c <= r; c += 11) CHECK(seen[gi].count({p, r / BM, c / BN}), "causal element (%d,%d) uncovered", r, c);
