@@ -34,3 +34,44 @@ def test_host_grads_match_the_device_step(hp, chunks):
         assert torch.equal(a.cpu(), b.cpu())
     for g, (_, G, _) in zip(g_dev, mats):
         assert torch.equal(g.cpu(), G)
+
+
+def test_engine_owned_workspace_matches(hp):
+    """NULL workspace (the library sizes and keeps its own) for mc_muon_step,
+    mc_normuon_step and mc_muon_step_host_grads gives the results of the
+    caller-workspace calls bit for bit."""
+    import ctypes
+    lib = mc.load_library()
+    mats = [wl.generic_matrix(r, c, seed=90 + i) for i, (r, c) in enumerate(SHAPES[:6])]
+    stream = torch.cuda.current_stream().cuda_stream
+
+    def fresh():
+        return ([W.to(DEV) for W, _, _ in mats], [G.to(DEV) for _, G, _ in mats], [M.to(DEV) for _, _, M in mats])
+
+    # muon: binding (caller workspace) vs raw ABI call with NULL workspace
+    Wa, Ga, Ma = fresh()
+    mc.muon_step(Wa, Ga, Ma, **hp)
+    Wb, Gb, Mb = fresh()
+    arr, n = mc.make_params(Wb, Gb, Mb)
+    h = mc.make_hparams(**hp)
+    assert lib.mc_muon_step(arr, n, ctypes.byref(h), None, 0, None, stream) == mc.MC_OK, mc.last_error()
+    # normuon, both ways
+    Wc, Gc, Mc_ = fresh()
+    Vc = [torch.zeros(W.shape[0], device=DEV) for W in Wc]
+    mc.normuon_step(Wc, Gc, Mc_, Vc, **hp)
+    Wd, Gd, Md = fresh()
+    Vd = [torch.zeros(W.shape[0], device=DEV) for W in Wd]
+    arr_d, _ = mc.make_params(Wd, Gd, Md)
+    nm = mc.make_normuon(Vd)
+    assert lib.mc_normuon_step(arr_d, n, ctypes.byref(h), ctypes.byref(nm), None, 0, None, stream) == mc.MC_OK
+    # host grads with NULL workspace
+    We, Ge, Me = fresh()
+    keep = [G.pin_memory() for _, G, _ in mats]
+    hptr = (ctypes.c_void_p * n)(*[k.data_ptr() for k in keep])
+    arr_e, _ = mc.make_params(We, Ge, Me)
+    assert lib.mc_muon_step_host_grads(arr_e, hptr, n, ctypes.byref(h), 3, None, 0, None, stream) == mc.MC_OK
+    assert mc.device_status() == mc.MC_OK, mc.last_error()
+    for a, b, e in zip(Wa + Ma, Wb + Mb, We + Me):
+        assert torch.equal(a.cpu(), b.cpu()) and torch.equal(a.cpu(), e.cpu())
+    for a, b in zip(Wc + Mc_ + Vc, Wd + Md + Vd):
+        assert torch.equal(a.cpu(), b.cpu())
