@@ -111,7 +111,16 @@ class ClockSampler:
         names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
         reasons = sorted({names[i] for r in rows for i in range(4) if r[5 + i].strip() == "Active"})
         return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(smax) if smax else None,
-                "reasons": reasons, "samples": len(rows)}
+                "reasons": reasons, "samples": len(rows), "persistence_mode": self.persistence()}
+
+    def persistence(self):
+        """The GPU's persistence mode, read (never set)."""
+        try:
+            out = subprocess.run(["nvidia-smi", f"--id={self.gpu}", "--query-gpu=persistence_mode",
+                                  "--format=csv,noheader"], capture_output=True, text=True, timeout=10)
+            return out.stdout.strip() or None
+        except (OSError, subprocess.TimeoutExpired):
+            return None
 
 
 # --------------------------------------------------------------- workload
@@ -160,19 +169,46 @@ def make_muon_inputs(device, layers, seed):
 
 
 # ---------------------------------------------------------------- oracle
-def oracle_sample_seconds(repeats=1):
-    """Time the fp64 oracle on one 4096 x 4096 matrix of the 7B-shaped set."""
+# One matrix of each shape class of the 7B-shaped set (index in cfg2_shapes, count in the set).
+ORACLE_SAMPLE = ((0, 128), (4, 64), (6, 32))   # 4096 x 4096, 14336 x 4096 (tall), 4096 x 14336 (wide)
+
+
+def oracle_sample_seconds(repeats=1, rotate=False):
+    """Time the fp64 oracle on the 7B-shaped set's shape classes.  Each repeat
+    runs one matrix of every class (about 20 s of CPU work), or, with
+    ``rotate``, one matrix of class (repeat mod 3) only.  Returns (seconds per
+    repeat, FLOPs per repeat, extrapolated seconds for the whole set from the
+    last time of each class)."""
     import oracle
     from matrix_orthogonalising_optimizer_step_b200 import workloads as wl
-    W, G, M = wl.cfg2_matrix(0)
-    W, G, M = (t.double().numpy() for t in (W, G, M))
     hp = dict(wl.HPARAMS)
-    ts = []
-    for _ in range(repeats):
-        t0 = time.perf_counter()
-        oracle.muon_step(W, G, M, **hp)
-        ts.append(time.perf_counter() - t0)
-    return ts, ns_dense_flops([(4096, 4096)])
+    shapes = wl.cfg2_shapes()
+    mats = [(i, count, [t.double().numpy() for t in wl.cfg2_matrix(i)]) for i, count in ORACLE_SAMPLE]
+    ts, fl, last = [], [], {}
+    for r in range(repeats):
+        picked = [mats[r % len(mats)]] if rotate else mats
+        total = 0.0
+        for i, count, (W, G, M) in picked:
+            t0 = time.perf_counter()
+            oracle.muon_step(W, G, M, **hp)
+            dt = time.perf_counter() - t0
+            total += dt
+            last[i] = (dt, count)
+        ts.append(total)
+        fl.append(ns_dense_flops([shapes[i] for i, _, _ in picked]))
+    full = sum(dt * count for dt, count in last.values()) if len(last) == len(mats) else None
+    return ts, fl, full
+
+
+def cpu_model():
+    try:
+        with open("/proc/cpuinfo") as f:
+            for line in f:
+                if line.startswith("model name"):
+                    return line.split(":", 1)[1].strip()
+    except OSError:
+        pass
+    return None
 
 
 def blas_threads():
@@ -189,17 +225,19 @@ def run_reference(args, rank, world):
     if rank != 0:
         return 0
     for _ in range(args.warmup):
-        oracle_sample_seconds(1)
-    ts, flops = oracle_sample_seconds(args.steps)
+        oracle_sample_seconds(1, rotate=True)
+    ts, fl, full = oracle_sample_seconds(args.steps, rotate=True)
     mean_s = sum(ts) / len(ts)
-    value = flops / mean_s / 1e12
-    sample = "one 4096x4096 matrix of the 7B-shaped set per step (fp64 oracle, full Muon step, 5 NS iterations)"
+    value = sum(fl) / sum(ts) / 1e12
+    sample = ("per step one matrix of the 7B-shaped set, the shape classes 4096x4096, 14336x4096 and "
+              "4096x14336 in turn (fp64 oracle, full Muon step, 5 NS iterations)")
     out = {"impl": "reference", "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": args.gpus,
            "steps": args.steps, "warmup": args.warmup, "ms_per_step": mean_s * 1e3, "higher_is_better": True,
            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
            "config": {"workload": WORKLOAD, "sample": sample},
            "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": blas_threads(), "kind": "oracle",
-                            "sample": sample},
+                            "sample": sample, "cpu_model": cpu_model(), "nproc": os.cpu_count(),
+                            "extrapolated_full_set_s": full},
            "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(out), flush=True)
     return 0
@@ -397,6 +435,8 @@ def main(argv=None):
     ns_ms = sum(kernels[k]["total_ms"] for k in ns_kinds if k in kernels) / K
     muon_ms = sum(kernels[k]["total_ms"] for k in muon_kinds if k in kernels) / K
     ns_tflops = ns_flops / (ns_ms / 1e3) / 1e12 if ns_ms > 0 else None
+    ns_exec = sum(kernels[k]["flops_executed"] for k in ns_kinds if k in kernels) / K
+    ns_tflops_exec = ns_exec / (ns_ms / 1e3) / 1e12 if ns_ms > 0 else None
     mom = kernels.get("momentum")
     elem_gbs = mom["bytes"] / (mom["total_ms"] / 1e3) / 1e9 if mom else None
     qk_ms = sum(kernels[k]["total_ms"] for k in ("qk_proj", "qk_causal_max", "qk_keys") if k in kernels) / K
@@ -475,10 +515,12 @@ def main(argv=None):
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        ts, f = oracle_sample_seconds(1)
-        cpu = {"value": f / ts[0] / 1e12, "unit": "TFLOP/s", "cores": blas_threads(), "kind": "oracle",
-               "sample": "one 4096x4096 matrix of the 7B-shaped set, full fp64 Muon step (5 NS iterations), "
-                         f"{ts[0]:.1f} s"}
+        ts, fl, full = oracle_sample_seconds(1)
+        cpu = {"value": fl[0] / ts[0] / 1e12, "unit": "TFLOP/s", "cores": blas_threads(), "kind": "oracle",
+               "sample": "one matrix of each shape class of the 7B-shaped set (4096x4096, 14336x4096, "
+                         f"4096x14336), full fp64 Muon step (5 NS iterations), {ts[0]:.1f} s",
+               "cpu_model": cpu_model(), "nproc": os.cpu_count(),
+               "extrapolated_full_set_s": full}
 
     if rank == 0:
         out = {
@@ -494,6 +536,9 @@ def main(argv=None):
             "components": {
                 "muon_step_ms": muon_ms, "ns_tflops_dense_equiv": ns_tflops,
                 "ns_pct_bf16_peak": (100.0 * ns_tflops / peaks["bf16_tflops_sustained"]) if ns_tflops else None,
+                "ns_tflops_executed": ns_tflops_exec,
+                "ns_pct_bf16_peak_executed": (100.0 * ns_tflops_exec / peaks["bf16_tflops_sustained"])
+                if ns_tflops_exec else None,
                 "elementwise_gbs": elem_gbs,
                 "elementwise_pct_hbm": (100.0 * elem_gbs / peaks["hbm_gbs"]) if elem_gbs else None,
                 "qk_max_tokens_per_s": qk_tokens},
