@@ -18,8 +18,15 @@
  *     device; they must be 16-byte aligned.  The library never frees or
  *     retains caller memory beyond the call (the call is asynchronous, so the
  *     buffers must stay valid until the stream reaches that point).
- *   - `stream` is a cudaStream_t (NULL = legacy default stream).  Calls only
- *     enqueue work; none synchronises the host.
+ *   - `stream` is a cudaStream_t (NULL = legacy default stream).  Calls
+ *     enqueue work and return.  A call may wait on the host for the upload of
+ *     a parameter table it issued four calls earlier (the tables go through a
+ *     4-slot page-locked staging ring), and for the device to go idle when the
+ *     engine-owned workspace has to grow; mc_device_status synchronises.
+ *   - Host-side state is guarded by one mutex, so calls may come from several
+ *     threads.  GPU work of calls that share the engine-owned workspace (NULL
+ *     workspace) or, for mc_muon_step_host_grads, the library's copy stream on
+ *     one device must be ordered by the caller (one stream, or events).
  *   - Matrices are row-major and contiguous.  A weight of shape rows x cols
  *     uses the nn.Linear layout: rows = out-features.
  *   - Return value: MC_OK (0) or a negative MC_ERR_* code.  On an argument
