@@ -188,3 +188,61 @@ def test_cfg4_full_size_sampled(hp):
         Ms = [torch.zeros(s, device=DEV, dtype=torch.float32) for s in shapes]
         return Ws, Gs, Ms
     _full_size_sampled(hp, shapes, [0, 2, 191], wl.cfg4_matrix, gen)
+
+
+def test_matrix_past_2_31_elements(hp):
+    """One 32768 x 65600 weight (2.15e9 elements, past 2^31): 64-bit indexing
+    in the momentum kernel, the GEMM epilogues and the apply.  The oracle
+    cannot run at this size, so the checks are elementwise on sampled flat
+    indices (momentum; the apply against the update it reports) and, for the
+    Newton-Schulz output O, properties that hold at any size: O X0^T is
+    symmetric (O = q(X0 X0^T) X0 for the composed polynomial q), and the
+    singular values sit near the polynomial's band, so ||O||_F / sqrt(m) does."""
+    r, c = 32768, 65600
+    g = torch.Generator(device=DEV)
+    g.manual_seed(123)
+    W = (torch.randn((r, c), device=DEV, generator=g) * 0.02).to(torch.bfloat16)
+    G = (torch.randn((r, c), device=DEV, generator=g) * 1e-3).to(torch.bfloat16)
+    M = torch.randn((r, c), device=DEV, generator=g) * 1e-3
+    idx = torch.cat([torch.randint(0, r * c, (4000,), device=DEV, generator=g),
+                     torch.tensor([0, 2**31 - 1, 2**31, 2**31 + 12345, r * c - 1], device=DEV)])
+    w0, g0, m0 = W.view(-1)[idx].double().cpu(), G.view(-1)[idx].double().cpu(), M.view(-1)[idx].double().cpu()
+    mu = float(np.float32(hp["mu"]))
+    # the NS input, kept for the property check (fp32, the kernels' own arithmetic)
+    m_new = torch.addcmul(G.float(), M, torch.tensor(mu, device=DEV))
+    X0 = G.float() + mu * m_new if hp["nesterov"] else m_new.clone()
+    del m_new
+    X0 /= torch.linalg.vector_norm(X0)
+    U = torch.empty((r, c), dtype=torch.float32, device=DEV)
+    mc.muon_step([W], [G], [M], update_outs=[U], **hp)
+    assert mc.device_status() == mc.MC_OK, mc.last_error()
+    # momentum, elementwise
+    m1 = M.view(-1)[idx].double().cpu()
+    want = mu * m0 + g0
+    assert torch.all(torch.abs(m1 - want) <= 1e-6 * torch.abs(want) + 1e-12)
+    # the apply: W1 = (1 - lr wd) W0 - lr U, to one bf16 ulp
+    w1, u = W.view(-1)[idx].double().cpu(), U.view(-1)[idx].double().cpu()
+    w_exp = (1 - hp["lr"] * hp["wd"]) * w0 - hp["lr"] * u
+    ulp = torch.from_numpy(np.spacing(np.abs(w_exp.numpy()).astype(np.float32)).astype(np.float64)) * 65536
+    assert torch.all(torch.abs(w1 - w_exp) <= ulp)
+    # Newton-Schulz output O = U / (rms * sqrt(max(r, c)))
+    O = U / (hp["rms_scale"] * np.sqrt(max(r, c)))
+    del U
+    # A Gaussian X0 of this shape has its singular values in [1.6e-3, 9.4e-3]
+    # (Marchenko-Pastur edges over ||X0||_F); five tuned quintic steps map them
+    # into [0.68, 1.20], and weighting by the Marchenko-Pastur density gives
+    # ||O||_F / sqrt(m) = 1.020 in exact arithmetic.
+    scale = float(torch.linalg.vector_norm(O)) / np.sqrt(min(r, c))
+    assert abs(scale - 1.020) <= 0.04, scale
+    prev = torch.backends.cuda.matmul.allow_tf32
+    torch.backends.cuda.matmul.allow_tf32 = False
+    try:
+        P = O @ X0.T
+    finally:
+        torch.backends.cuda.matmul.allow_tf32 = prev
+    asym = float(torch.linalg.matrix_norm(P - P.T) / torch.linalg.matrix_norm(P))
+    assert asym <= 2e-2, asym
+    print(f"2^31+ matrix: ||O||_F/sqrt(m) = {scale:.3f}, asymmetry of O X0^T = {asym:.2e}")
+    del W, G, M, X0, O, P
+    mc.release_workspaces()
+    torch.cuda.empty_cache()

@@ -126,3 +126,14 @@ def test_cfg3_smax_and_clip(cfg3):
     for h in range(H):
         if not mask[h]:
             assert after[h] == got[h]
+
+
+@pytest.mark.parametrize("H", [4096, 4100])
+def test_many_heads_both_sides_of_the_shared_head_table(H):
+    """The causal max keeps per-head maxima in shared memory for up to 4096
+    heads and uses global atomics beyond: both sides against the oracle."""
+    B, S, D, dh = 1, 40, 16, 8
+    X, Wq, Wk = wl.qk_inputs(B, S, D, H, dh, seed=19, w_std=0.3)
+    got = gpu_smax(X, Wq, Wk, H, dh)
+    refb = oracle.qk_max_logit(to64(X), to64(Wq), to64(Wk), H, dh, causal=True, qk_bf16=True)
+    assert np.all(rel(got, refb) <= 2e-3), np.max(rel(got, refb))
