@@ -190,15 +190,16 @@ def test_cfg4_full_size_sampled(hp):
     _full_size_sampled(hp, shapes, [0, 2, 191], wl.cfg4_matrix, gen)
 
 
-def test_matrix_past_2_31_elements(hp):
-    """One 32768 x 65600 weight (2.15e9 elements, past 2^31): 64-bit indexing
+@pytest.mark.parametrize("r,c", [(32768, 65600), (65600, 32768)])
+def test_matrix_past_2_31_elements(hp, r, c):
+    """One 2.15e9-element weight (past 2^31), wide and tall: 64-bit indexing
     in the momentum kernel, the GEMM epilogues and the apply.  The oracle
     cannot run at this size, so the checks are elementwise on sampled flat
     indices (momentum; the apply against the update it reports) and, for the
-    Newton-Schulz output O, properties that hold at any size: O X0^T is
-    symmetric (O = q(X0 X0^T) X0 for the composed polynomial q), and the
-    singular values sit near the polynomial's band, so ||O||_F / sqrt(m) does."""
-    r, c = 32768, 65600
+    Newton-Schulz output O, properties that hold at any size: O X0^T (tall:
+    X0^T O) is symmetric (O = q(X0 X0^T) X0 for the composed polynomial q),
+    and the singular values sit near the polynomial's band, so
+    ||O||_F / sqrt(min(r, c)) does."""
     g = torch.Generator(device=DEV)
     g.manual_seed(123)
     W = (torch.randn((r, c), device=DEV, generator=g) * 0.02).to(torch.bfloat16)
@@ -237,12 +238,12 @@ def test_matrix_past_2_31_elements(hp):
     prev = torch.backends.cuda.matmul.allow_tf32
     torch.backends.cuda.matmul.allow_tf32 = False
     try:
-        P = O @ X0.T
+        P = X0.T @ O if r > c else O @ X0.T
     finally:
         torch.backends.cuda.matmul.allow_tf32 = prev
     asym = float(torch.linalg.matrix_norm(P - P.T) / torch.linalg.matrix_norm(P))
     assert asym <= 2e-2, asym
-    print(f"2^31+ matrix: ||O||_F/sqrt(m) = {scale:.3f}, asymmetry of O X0^T = {asym:.2e}")
+    print(f"2^31+ matrix {r}x{c}: ||O||_F/sqrt(m) = {scale:.3f}, asymmetry = {asym:.2e}")
     del W, G, M, X0, O, P
     mc.release_workspaces()
     torch.cuda.empty_cache()
