@@ -132,9 +132,11 @@ int mc_muon_step(const mc_param* params, int n, const mc_hparams* hp, void* work
  * host memory.  g_host[i] (HOST, page-locked for the copies to overlap,
  * rows*cols elements of params[i].g_dtype) is copied into params[i].g
  * (device) on the library's own copy stream.  The list is split in order into
- * `chunks` pieces of about equal bytes; the step of piece k runs on `stream`
- * once piece k has landed, so the transfer of later pieces runs under the
- * Newton-Schulz GEMMs of earlier ones.  Every result is bit-for-bit that of
+ * pieces: the first ones grow geometrically (from 1/256 of the gradient bytes,
+ * x1.75 each) up to 1/chunks of the bytes, the size the rest keep (chunks = 1:
+ * one piece).  The step of piece k runs on `stream` once piece k has landed,
+ * so the transfer of later pieces runs under the Newton-Schulz GEMMs of
+ * earlier ones and only the small first upload is exposed.  Every result is bit-for-bit that of
  * mc_muon_step (a matrix's update does not depend on the other matrices of a
  * call).  The copies start after the work already queued on `stream`, and
  * everything this call enqueues is ordered before later work on `stream`.

@@ -584,18 +584,29 @@ int check_out_align(const float* norms_out, const void* workspace) {
   return MC_OK;
 }
 
-// Split params[0, n) in order into at most `chunks` pieces of about equal
-// gradient bytes; returns the piece boundaries (first entry 0, last n).
+// Pieces of the host-gradient step, in order: the first ones ramp up
+// geometrically, from total/256 of the gradient bytes by x1.75 each, to
+// total/chunks, the size the rest keep.  The step takes about 1.9x longer
+// per byte than the upload, so a piece 1.75x the size of the one before
+// still lands before that one's step ends: only the small first upload is
+// exposed.  Returns the piece boundaries (first entry 0, last n).
 std::vector<int> split_chunks(const mc_param* params, int n, int chunks) {
+  auto bytes = [&](int i) {
+    return double(params[i].rows) * double(params[i].cols) * (params[i].g_dtype == MC_F32 ? 4 : 2);
+  };
   double total = 0;
-  for (int i = 0; i < n; ++i)
-    total += double(params[i].rows) * double(params[i].cols) * (params[i].g_dtype == MC_F32 ? 4 : 2);
+  for (int i = 0; i < n; ++i) total += bytes(i);
+  const double even = total / chunks;
+  double target = chunks > 1 ? std::min(even, total / 256.0) : total;
   std::vector<int> b{0};
   double acc = 0;
   for (int i = 0; i < n; ++i) {
-    acc += double(params[i].rows) * double(params[i].cols) * (params[i].g_dtype == MC_F32 ? 4 : 2);
-    const int k = static_cast<int>(b.size());
-    if (i + 1 < n && k < chunks && acc >= total * k / chunks) b.push_back(i + 1);
+    acc += bytes(i);
+    if (i + 1 < n && acc >= target) {
+      b.push_back(i + 1);
+      acc = 0;
+      target = std::min(even, target * 1.75);
+    }
   }
   b.push_back(n);
   return b;

@@ -239,7 +239,8 @@ def test_host_grads_entry_arguments_and_workspace(lib):
     full = lib.mc_muon_workspace_size(arr, 6, P(hp))
     one = lib.mc_muon_host_grads_workspace_size(arr, 6, P(hp), 1)
     assert full < one <= full + 64 * 1024
+    # six equal matrices: the ramp starts below one matrix, so every piece holds one
     three = lib.mc_muon_host_grads_workspace_size(arr, 6, P(hp), 3)
-    two = lib.mc_muon_workspace_size(arr, 2, P(hp))                  # six equal matrices in pieces of two
-    assert two < three <= two + 64 * 1024 and three < one
+    single = lib.mc_muon_workspace_size(arr, 1, P(hp))
+    assert single < three <= single + 64 * 1024 and three < one
     assert lib.mc_muon_host_grads_workspace_size(arr, 6, P(hp), 0) == 0
