@@ -107,7 +107,7 @@ typedef struct {
  * (X <- (aI + B) X), which amplifies the bf16 rounding of X less once the
  * singular values have entered the polynomial's band.  The last iteration
  * applies the update to W straight from the fp32 accumulator.
- * The list is processed in consecutive pieces of at most 2^30 elements (at
+ * The list is processed in consecutive pieces of at most 2^29 elements (at
  * least one matrix each), all reusing one workspace; inside a piece, matrices
  * of equal shape and weight dtype are batched into one problem group.  A
  * matrix's result does not depend on the other matrices of the call.

