@@ -517,13 +517,11 @@ __device__ __forceinline__ void epi_finish(const GemmGroup& G, int prob, int r, 
   } else if constexpr (EPI == EPI_CAUSALMAX) {
     if (r >= G.M) return;
     if (c0 + 16 <= G.N && (!G.mask_causal || c0 + 15 <= r)) {
-      // Whole chunk inside the mask and the bounds: a max tree, no compares.
-      float m[8];
-#pragma unroll
-      for (int j = 0; j < 8; ++j) m[j] = fmaxf(v[2 * j], v[2 * j + 1]);
-#pragma unroll
-      for (int j = 0; j < 4; ++j) m[j] = fmaxf(m[2 * j], m[2 * j + 1]);
-      run_max = fmaxf(run_max, fmaxf(fmaxf(m[0], m[1]), fmaxf(m[2], m[3])));
+      // Whole chunk inside the mask and the bounds: a tree of three-input
+      // maxima (8 instructions for 16 scores), no compares.
+      const float a0 = fmax3(v[0], v[1], v[2]), a1 = fmax3(v[3], v[4], v[5]), a2 = fmax3(v[6], v[7], v[8]);
+      const float a3 = fmax3(v[9], v[10], v[11]), a4 = fmax3(v[12], v[13], v[14]);
+      run_max = fmax3(run_max, fmax3(a0, a1, a2), fmax3(a3, a4, v[15]));
     } else {
 #pragma unroll
       for (int j = 0; j < 16; ++j) {
@@ -537,11 +535,12 @@ __device__ __forceinline__ void epi_finish(const GemmGroup& G, int prob, int r, 
 
 // Chunks per batch.  One for the NS phases: measured against batches of four
 // chunks (one 64-column TMEM load, all global loads issued first) on the same
-// GPU, the single-chunk drain was as fast or faster.  Four for the causal max,
-// whose epilogue has no global operands and is bound by the TMEM load latency.
+// GPU, the single-chunk drain was as fast or faster.  Eight for the causal
+// max (a warp's whole 128 columns: two TMEM loads in flight, one wait), whose
+// epilogue has no global operands and is bound by the TMEM load latency.
 template <int EPI>
 struct EpiBatch {
-  static constexpr int CH = (EPI == EPI_CAUSALMAX) ? 4 : 1;
+  static constexpr int CH = (EPI == EPI_CAUSALMAX) ? 8 : 1;
 };
 
 // ------------------------------------------------------------------ kernel
@@ -788,10 +787,12 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1) umma_gemm_kernel(const __grid
 #pragma unroll
         for (int b = 0; b < CH; ++b) epi_prefetch<EPI>(G, ti.prob, r, cbase + (cb + b) * 16, pre[b]);
         float v[CH * 16];
-        if constexpr (CH == 4) {
+        if constexpr (CH == 8) {
+          tmem_ld128(t_row + cb * 16, v);
+        } else if constexpr (CH == 4) {
           tmem_ld64(t_row + cb * 16, v);
         } else {
-          static_assert(CH == 1, "one 16- or 64-column TMEM load per batch");
+          static_assert(CH == 1, "one 16-, 64- or 128-column TMEM drain per batch");
           tmem_ld16(t_row + cb * 16, *reinterpret_cast<float(*)[16]>(v));
         }
 #pragma unroll
