@@ -1,17 +1,22 @@
 /*
  * muonclip.h -- C ABI of the B200 (sm_100a) MuonClip step library.
  *
- * Three operations, as the MuonClip training step composes them
- * ("MuonClip: speed, then stability", §07 "One complete training step"):
+ * The three operations of the MuonClip training step ("MuonClip: speed, then
+ * stability", §07 "One complete training step"):
  *
  *   mc_muon_step     the Muon update of a list of hidden 2D weights
- *   mc_muon_step_host_grads  the same, with the gradient upload overlapped
  *   mc_qk_max_logit  per-head causal max of the pre-softmax logit (S_max)
  *   mc_qk_clip       QK-Clip: rescale the W_q / W_k rows of heads with S_max > tau
- *   mc_normuon_step  the Muon update with NorMuon's per-row normalisation
- *   mc_qk_clip_slices   QK-Clip over an explicit slice map (multi-head latent
- *                       attention, fused projection layouts)
- *   mc_mla_max_logit    S_max of multi-head latent attention (content + rotary parts)
+ *
+ * and their widenings:
+ *
+ *   mc_muon_step_host_grads  mc_muon_step with the gradient upload overlapped
+ *   mc_normuon_step          the Muon update with NorMuon's per-row normalisation
+ *   mc_mla_max_logit         S_max of multi-head latent attention (content + rotary)
+ *   mc_qk_clip_slices        QK-Clip over an explicit slice map (MLA, fused layouts)
+ *   mc_qk_max_logit_static   mc_qk_max_logit without a workspace or any allocation
+ *   mc_polar_express_coeffs  host: a Polar Express coefficient table for mc_hparams
+ *   mc_shard_plan            host: whole-matrix ownership for a sharded step
  *
  * Conventions for every call
  *   - All pointers named "device" are CUDA device pointers on the current
@@ -60,7 +65,8 @@ enum { MC_F32 = 0, MC_BF16 = 1 };
 /* One hidden 2D weight, its gradient and its momentum buffer. */
 typedef struct {
   void* w;            /* device, rows x cols, dtype w_dtype; updated in place      */
-  const void* g;      /* device, rows x cols, dtype g_dtype; read only              */
+  const void* g;      /* device, rows x cols, dtype g_dtype; read only (only
+                         mc_muon_step_host_grads writes it, from host memory)    */
   float* m;           /* device, rows x cols fp32 momentum; updated in place        */
   int64_t rows;       /* >= 1 */
   int64_t cols;       /* >= 1 */
