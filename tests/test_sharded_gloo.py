@@ -94,7 +94,7 @@ def _reference(world, steps):
     return Ws, Ms
 
 
-@pytest.mark.parametrize("world,steps", [(2, 2), (3, 1)])
+@pytest.mark.parametrize("world,steps", [(2, 2), (3, 1), (4, 1)])
 def test_sharded_step_equals_single_process_step(tmp_path, world, steps):
     mp.start_processes(_worker, args=(world, _free_port(), str(tmp_path), steps), nprocs=world,
                        start_method="spawn", join=True)
