@@ -1,15 +1,17 @@
 // Grouped, persistent tcgen05 GEMM for sm_100a with the MuonClip epilogues.
 //
-// One kernel computes D = A * B^T tile by tile (128 x 256 fp32 accumulator in
-// TMEM) for up to MAX_GROUPS groups of equally shaped problems, and hands each
-// finished tile to a fused epilogue:
+// One kernel computes D = A * B^T tile by tile (a CTA pair's 256 x 256 or
+// 256 x 512 fp32 accumulator in TMEM) for up to MAX_GROUPS groups of equally
+// shaped problems, and hands each finished tile to a fused epilogue:
 //
 //   EPI_GRAM        A_k   = s^2 * X X^T            (symmetric: upper tiles only,
-//                                                  each element stored twice)
+//                                                  each element stored twice;
+//                                                  dead diagonal blocks skipped)
 //   EPI_POLY        B_k   = b*A + c*(A A) [+ a*I]  (symmetric, mirrored store)
 //   EPI_APPLY       X_k+1 = s * (a*X + B X)        (a*X from the hi + lo copy of
 //                           or  P X, P = aI+bA+cA^2  the iterate; stores the bf16
-//                                                  iterate, its lo half when flagged)
+//                                                  iterate, its lo half when flagged,
+//                                                  and the fp32 NS output for NorMuon)
 //   EPI_APPLY_FINAL W     = (1 - lr*wd) W - lr * rms * X_N   (last iteration; X_N
 //                                                  never touches memory)
 //
