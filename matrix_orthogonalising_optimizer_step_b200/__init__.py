@@ -6,6 +6,10 @@ device memory and the current stream.  There is no fallback: if the library is
 missing or the device is not a B200 the calls raise.
 
     from matrix_orthogonalising_optimizer_step_b200 import muon_step, qk_max_logit, qk_clip
+
+Also: muon_step_host_grads, normuon_step, mla_max_logit, qk_clip_slices (with
+mla_slices), polar_express_coeffs, shard_plan, qk_max_logit_static, and the
+data-parallel step in ``sharded``.
 """
 from __future__ import annotations
 

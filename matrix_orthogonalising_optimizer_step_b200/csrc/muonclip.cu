@@ -1,12 +1,14 @@
 // Host engine and C ABI of the MuonClip step library (see include/muonclip.h).
 //
-// mc_muon_step enqueues, on the caller's stream:
-//   1. momentum_kernel       one launch over every matrix (momentum, Nesterov,
-//                            fp32 + bf16 iterate, ||U||^2 partials)
+// mc_muon_step splits the list into pieces of at most 2^29 elements and
+// enqueues, per piece, on the caller's stream:
+//   1. momentum_kernel       one launch over every matrix of the piece
+//                            (momentum, Nesterov, the iterate's bf16 hi and lo
+//                            halves, ||U||^2 partials)
 //   2. norm_finalize_kernel  s = 1 / max(||U||_F, eps) per matrix
 //   3. ns_steps x { GRAM, POLY, APPLY } grouped tcgen05 GEMM launches; the last
 //      APPLY writes W directly (decay + scaled update), so the final iterate
-//      never goes to memory.
+//      never goes to memory (NorMuon: it goes out in fp32 for the row pass).
 // Matrices with equal (rows, cols, weight dtype) form one problem group; their
 // iterates sit back to back in the workspace so that one 3-D TMA descriptor
 // covers the whole group.  Tall matrices (rows > cols) are never transposed in
