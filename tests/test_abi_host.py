@@ -244,3 +244,28 @@ def test_host_grads_entry_arguments_and_workspace(lib):
     single = lib.mc_muon_workspace_size(arr, 1, P(hp))
     assert single < three <= single + 64 * 1024 and three < one
     assert lib.mc_muon_host_grads_workspace_size(arr, 6, P(hp), 0) == 0
+
+
+def test_product_never_imports_the_oracle():
+    """The library package (binding, sharded step, workloads, build) has no
+    path to oracle/: the oracle is test infrastructure only."""
+    pkg = os.path.join(ROOT, "matrix_orthogonalising_optimizer_step_b200")
+    for dirpath, _, files in os.walk(pkg):
+        for f in files:
+            if f.endswith((".py", ".cu", ".cuh", ".h")):
+                text = open(os.path.join(dirpath, f)).read()
+                assert not re.search(r"^\s*(import|from)\s+oracle\b", text, flags=re.M), f
+                assert "oracle." not in re.sub(r"#.*|\"\"\".*?\"\"\"", "", text, flags=re.S), f
+
+
+def test_binding_rejects_cpu_tensors_without_computing():
+    """No CPU fallback: host tensors are refused before anything runs."""
+    import torch
+    W = torch.zeros(8, 16, dtype=torch.bfloat16)
+    G = torch.zeros(8, 16, dtype=torch.bfloat16)
+    M = torch.zeros(8, 16)
+    with pytest.raises(ValueError, match="CUDA"):
+        mc.muon_step([W], [G], [M])
+    X = torch.zeros(1, 4, 16, dtype=torch.bfloat16)
+    with pytest.raises(ValueError, match="CUDA"):
+        mc.qk_max_logit(X, torch.zeros(16, 16, dtype=torch.bfloat16), torch.zeros(16, 16, dtype=torch.bfloat16), 2, 8)
