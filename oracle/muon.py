@@ -17,7 +17,7 @@ Sources (page title, then section):
   row, each row of the orthogonalised update divided by the square root of it,
   then the whole matrix rescaled to the Frobenius norm it had before).
 
-Readings where the pages are silent (each also listed in the design doc):
+Readings where the pages are silent:
 
 * Nesterov lookahead: [MC] §02 only says one "may be applied".  Read as the
   recurrence applied once more with the current gradient, U = G + mu*M_t, in

@@ -17,7 +17,7 @@ Sources (page title, then section):
   the head-specific rotary query q^R by gamma_h, the shared rotary key k^R is
   left untouched; [MC] §12 asks implementers to name the physical slices).
 
-Readings (also in DESIGN.md):
+Readings where the pages are silent:
 
 * The 1/sqrt(d_head) factor is inside S_max ([MV]).
 * Causal attention: a query i sees keys j <= i (the diagonal counts).
