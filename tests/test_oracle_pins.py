@@ -481,6 +481,50 @@ def test_normuon_fresh_state_is_independent_of_beta2():
         assert np.allclose(o[2], outs[0][2], rtol=1e-10, atol=1e-13)
 
 
+def test_normuon_worked_example_by_hand():
+    """A 2 x 2 example worked out by hand, with a prior state.  O = [[3, -3],
+    [1, 1]] has row mean squares (9, 1).  From v0 = (1, 4) with beta2 = 3/4:
+    v1 = 3/4 (1, 4) + 1/4 (9, 1) = (3, 13/4).  Dividing the rows by sqrt(v1)
+    gives (sqrt3, -sqrt3) and (1, 1)/sqrt(13/4), of squared norm 6 + 8/13 =
+    86/13; ||O||_F^2 = 20, so both rows are then scaled by sqrt(20 * 13/86) =
+    sqrt(130/43): O_hat = [[r0, -r0], [r1, r1]] with r0 = sqrt(390/43) and
+    r1 = sqrt(40/43).  The weights swapped (1/4 on the state, 3/4 on the new
+    mean square) would give v1 = (7, 7/4) instead."""
+    O = np.array([[3.0, -3.0], [1.0, 1.0]])
+    O_hat, v1 = oracle.normuon_rows(O, np.array([1.0, 4.0]), beta2=0.75, eps_v=0.0)
+    assert np.allclose(v1, [3.0, 3.25], rtol=0, atol=1e-15)
+    r0, r1 = np.sqrt(390.0 / 43.0), np.sqrt(40.0 / 43.0)
+    assert np.allclose(O_hat, [[r0, -r0], [r1, r1]], rtol=1e-14, atol=0)
+
+
+def test_normuon_second_moment_is_an_exponential_average():
+    """Fed the same rows k times, an exponential average with factor beta2
+    closes to the geometric series v_k = q + beta2^k (v0 - q), q being the
+    row's mean square (here each row has entries of one magnitude c_i, so
+    q = c_i^2 exactly).  A row whose prior state is far above q is therefore
+    damped more, step after step, the larger beta2 is."""
+    rng = np.random.default_rng(43)
+    r, c = 6, 10
+    mag = rng.uniform(0.5, 2.0, r)
+    O = mag[:, None] * rng.choice([-1.0, 1.0], (r, c))
+    v0 = rng.uniform(0.0, 20.0, r)
+    for beta2 in (0.3, 0.9):
+        v = v0.copy()
+        for k in range(1, 6):
+            _, v = oracle.normuon_rows(O, v, beta2=beta2, eps_v=1e-8)
+            want = mag ** 2 + beta2 ** k * (v0 - mag ** 2)
+            assert np.allclose(v, want, rtol=1e-13, atol=0), (beta2, k)
+    # one step from a large prior state on row 0 only: row 0's share of the
+    # (norm-preserving) update falls as beta2 grows
+    v_big = np.full(r, 1.0)
+    v_big[0] = 1e4
+    share = []
+    for beta2 in (0.1, 0.5, 0.9):
+        O_hat, _ = oracle.normuon_rows(O, v_big, beta2=beta2, eps_v=0.0)
+        share.append(np.linalg.norm(O_hat[0]) / np.linalg.norm(O_hat))
+    assert share[0] > share[1] > share[2]
+
+
 # ------------------------------------------------------------ Polar Express
 def test_polar_express_ten_steps_printed_value():
     g = GOLD["polar_express_10"]
