@@ -6,10 +6,17 @@ dh 128), all through the C ABI.  Prints one JSON line.
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
 
 --impl reference times the fp64 oracle on the host cores instead (a bounded
-sample of the same workload: one 4096 x 4096 matrix of the 7B-shaped set per
-step).  Multi-GPU (torchrun): every rank updates its own 7B-shaped parameter
-set (weak scaling, no collective on the data path); the time is the max over
-ranks.
+sample of the same workload: one matrix of the 7B-shaped set per step).
+
+Multi-GPU (torchrun, --mode sharded, the default there): the data-parallel
+step of one 7B-shaped set, each matrix owned whole by one rank (reduce-scatter
+of the gradients, the owner's Muon step, all-gather of the weights), with each
+rank's own QK batch and an all-reduce (max) of S_max before the clip; strong
+scaling, the time is the max over ranks.  --mode replicas gives every rank its
+own set instead (weak scaling, no collective).
+
+--config {0,1,3,4} times one other workload of the pages' configurations
+alone (see CONFIG_WORKLOADS), with the oracle beside it.
 """
 from __future__ import annotations
 
@@ -34,8 +41,8 @@ WORKLOAD = ("7B-shaped Muon step (224 matrices, 7.78e9 params, bf16 W/G, fp32 M,
 
 
 # DRAM bytes (dram__bytes_read.sum + dram__bytes_write.sum) of one launch of a
-# kernel kind over ONE layer of the 7B-shaped set, from the ncu capture in
-# profiles/ns_gemm_1layer_full.md (third NS iteration).  A launch at full size
+# kernel kind over ONE layer of the 7B-shaped set, from an ncu capture of the
+# one-layer step (third NS iteration).  A launch at full size
 # covers several layers (the engine runs the list in pieces), and traffic is
 # proportional to the matrices processed, so the per-launch figure is this
 # times the layers one launch covers.  Kinds without a capture of the kernel
@@ -57,6 +64,13 @@ def parse_args(argv=None):
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--no-extras", action="store_true",
                    help="skip the separately timed MLA QK-Clip layer and coefficient-table step")
+    p.add_argument("--mode", choices=["plain", "sharded", "replicas"], default=None,
+                   help="plain: one GPU's MuonClip step (default at 1 GPU); sharded: the ownership-sharded "
+                        "data-parallel step over one 7B-shaped set (default under torchrun); replicas: every "
+                        "rank its own set, no collective")
+    p.add_argument("--config", type=int, choices=[0, 1, 3, 4], default=None,
+                   help="time one other workload alone instead of the MuonClip step: 0 = one fp32 256x512 "
+                        "matrix, 1 = 64 x 1024^2, 3 = the causal MHA S_max + QK-Clip layer, 4 = 64 MoE experts")
     return p.parse_args(argv)
 
 
@@ -344,6 +358,314 @@ def time_extras(mc, wl, dev, stream, hp, steps, peaks, barrier, max_over_ranks, 
     return out
 
 
+# --------------------------------------------------------- other configs
+CONFIG_WORKLOADS = {
+    0: "one fp32 256x512 Muon step (rank-8 spike gradient, zero momentum)",
+    1: "64 x 1024^2 bf16 Muon step (power-law spectrum gradients, fp32 momentum N(0, 1e-3))",
+    3: "causal MHA S_max and QK-Clip, B4 S4096 D4096 H32 dh128 (heads 3, 17, 29 hot)",
+    4: "64 MoE experts: 128 x 2048x7168 + 64 x 7168x2048 bf16 Muon step (spectrum i^-0.5)",
+}
+
+
+def _timed_alone(mc, fn, reps, stream):
+    """Device time per call of ``fn`` (CUDA events on ``stream``) and the
+    per-kernel rows over those calls."""
+    import torch
+    for _ in range(3):
+        fn()
+    torch.cuda.synchronize()
+    mc.profile_begin()
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record(stream)
+    for _ in range(reps):
+        fn()
+    b.record(stream)
+    torch.cuda.synchronize()
+    k = mc.profile_end()
+    assert mc.device_status() == mc.MC_OK, mc.last_error()
+    return a.elapsed_time(b) / reps, k
+
+
+def _roofline_row(kernels, peaks, reps):
+    """Roofline of the dominant kernel kind of a config timed alone: burst
+    peak (the kernels are not inside a seconds-long step)."""
+    dom = max(((k, v) for k, v in kernels.items() if k != "table_upload"), key=lambda kv: kv[1]["total_ms"])[0]
+    d = kernels[dom]
+    if d["flops"] > 0:
+        ach = d["flops"] / (d["total_ms"] / 1e3) / 1e12
+        return {"kernel": dom, "bound": "tensor", "achieved": ach, "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
+                "frac": ach / peaks["bf16_tflops"], "traffic": None,
+                "achieved_executed": d["flops_executed"] / (d["total_ms"] / 1e3) / 1e12 if d["flops_executed"] else None,
+                "peak_source": f"{peaks['source']} bf16_tflops (burst: a short workload timed alone)"}
+    ach = d["bytes"] / (d["total_ms"] / 1e3) / 1e9 if d["total_ms"] > 0 else 0.0
+    return {"kernel": dom, "bound": "hbm", "achieved": ach, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+            "frac": ach / peaks["hbm_gbs"], "traffic": None, "peak_source": f"{peaks['source']} hbm_gbs"}
+
+
+def run_config(args, cfg):
+    """One other workload of the pages' configurations, timed alone on one GPU
+    at full size, with the fp64 oracle timed on the host cores beside it."""
+    import numpy as np
+    import torch
+    import matrix_orthogonalising_optimizer_step_b200 as mc
+    from matrix_orthogonalising_optimizer_step_b200 import build as mcbuild
+    from matrix_orthogonalising_optimizer_step_b200 import workloads as wl
+    import oracle
+
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    mcbuild.build()
+    mc.load_library()
+    peaks = measured_peaks()
+    hp = dict(wl.HPARAMS)
+    stream = torch.cuda.current_stream()
+    steps = max(args.steps, 5)
+    out = {"metric": METRIC, "n_gpus": 1, "steps": steps, "warmup": max(args.warmup, 3),
+           "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "data": "synthetic",
+           "config": {"workload": CONFIG_WORKLOADS[cfg], "config_index": cfg}, "e2e": None}
+    if cfg in (0, 1, 4):
+        if cfg == 0:
+            mats = [wl.cfg0_matrix()]
+            reps = max(steps, 200)
+        elif cfg == 1:
+            mats = [wl.cfg1_matrix(i) for i in range(64)]
+            reps = max(steps, 50)
+        else:
+            mats = None
+            reps = max(steps, 10)
+        if mats is not None:
+            shapes = [tuple(W.shape) for W, _, _ in mats]
+            Ws = [W.to(dev) for W, _, _ in mats]
+            Gs = [G.to(dev) for _, G, _ in mats]
+            Ms = [M.to(dev) for _, _, M in mats]
+        else:
+            shapes = wl.cfg4_shapes()
+            g = torch.Generator(device=dev)
+            g.manual_seed(4004)
+            Ws = [(torch.randn(sh, device=dev, generator=g) * 0.02).to(torch.bfloat16) for sh in shapes]
+            Gs = [(torch.randn(sh, device=dev, generator=g) * 1e-3).to(torch.bfloat16) for sh in shapes]
+            Ms = [torch.zeros(sh, device=dev, dtype=torch.float32) for sh in shapes]
+        ms, k = _timed_alone(mc, lambda: mc.muon_step(Ws, Gs, Ms, stream=stream, **hp), reps, stream)
+        dense = ns_dense_flops(shapes, hp["ns_steps"])
+        ns_kinds = ("ns_gram", "ns_poly", "ns_apply_mixed", "ns_apply", "ns_apply_final", "ns_thin")
+        ns_ms = sum(k[n]["total_ms"] for n in ns_kinds if n in k) / reps
+        ns_exec = sum(k[n]["flops_executed"] for n in ns_kinds if n in k) / reps
+        mom = k.get("momentum")
+        out.update(value=dense / (ms / 1e3) / 1e12, unit="TFLOP/s", ms_per_step=ms, dtype="bf16" if cfg else "f32",
+                   components={"muon_step_ms": ms, "ns_ms": ns_ms,
+                               "ns_tflops_dense_equiv": dense / (ns_ms / 1e3) / 1e12,
+                               "ns_tflops_executed": ns_exec / (ns_ms / 1e3) / 1e12,
+                               "ns_frac_burst_dense_equiv": dense / (ns_ms / 1e3) / 1e12 / peaks["bf16_tflops"],
+                               "ns_frac_burst_executed": ns_exec / (ns_ms / 1e3) / 1e12 / peaks["bf16_tflops"],
+                               "momentum_gbs": mom["bytes"] / (mom["total_ms"] / 1e3) / 1e9 if mom else None})
+        out["config"].update(matrices=len(shapes), params=int(sum(r * c for r, c in shapes)),
+                             flops_per_step=dense, flops_convention="dense-equivalent 5*(4 m^2 n + 2 m^3)",
+                             l2="inputs larger than L2" if cfg == 4 else "inputs fit in L2 (no flush)")
+        # the oracle on the host cores: the whole config (0, 1), or one matrix
+        # per shape class scaled by the class counts (4)
+        if cfg in (0, 1):
+            host = mats
+            t0 = time.perf_counter()
+            for W, G, M in host:
+                oracle.muon_step(W.double().numpy(), G.double().numpy(), M.double().numpy(), **hp)
+            cpu_s = time.perf_counter() - t0
+            sample, extrap = f"the whole config, {cpu_s:.1f} s", None
+        else:
+            cpu_s = 0.0
+            for idx, count in ((0, 128), (2, 64)):
+                W, G, M = wl.cfg4_matrix(idx)
+                t0 = time.perf_counter()
+                oracle.muon_step(W.double().numpy(), G.double().numpy(), M.double().numpy(), **hp)
+                cpu_s += (time.perf_counter() - t0) * count
+            sample, extrap = "one 2048x7168 and one 7168x2048 matrix, scaled by the class counts (128, 64)", True
+        out["cpu_baseline"] = {"value": dense / cpu_s / 1e12, "unit": "TFLOP/s", "cores": blas_threads(),
+                               "kind": "oracle", "sample": sample, "ms_per_step": cpu_s * 1e3,
+                               "extrapolated": bool(extrap), "cpu_model": cpu_model(), "nproc": os.cpu_count()}
+    else:
+        c3 = wl.CFG3
+        B, S, D, H, dh = c3["B"], c3["S"], c3["D"], c3["H"], c3["dh"]
+        X, Wq, Wk = wl.cfg3_inputs()
+        x, wq, wk = X.to(dev), Wq.to(dev), Wk.to(dev)
+        smax = torch.empty(H, dtype=torch.float32, device=dev)
+        gamma = torch.empty(H, dtype=torch.float32, device=dev)
+        mask = torch.empty(H, dtype=torch.int32, device=dev)
+        wq0, wk0 = wq.clone(), wk.clone()
+
+        def layer():
+            # the clip rescales W_q/W_k in place: start every layer from the
+            # same weights so each one clips the same three heads
+            wq.copy_(wq0)
+            wk.copy_(wk0)
+            mc.qk_max_logit(x, wq, wk, H, dh, causal=True, smax_out=smax, stream=stream)
+            mc.qk_clip(wq, wk, smax, H, dh, tau=wl.QK_TAU, alpha=wl.QK_ALPHA, gamma_out=gamma, mask_out=mask,
+                       stream=stream)
+        reps = max(steps, 20)
+        ms, k = _timed_alone(mc, layer, reps, stream)
+        qk_ms = sum(k[n]["total_ms"] for n in ("qk_proj", "qk_causal_max", "qk_keys", "qk_clip") if n in k) / reps
+        qf = qk_flops(B, S, D, H, dh)
+        out.update(value=B * S / (qk_ms / 1e3), unit="tokens/s", ms_per_step=qk_ms, dtype="bf16",
+                   components={"qk_ms": qk_ms, "layer_ms_with_weight_reset": ms,
+                               "qk_tflops": qf / (qk_ms / 1e3) / 1e12,
+                               "qk_proj_tflops": k["qk_proj"]["flops"] / (k["qk_proj"]["total_ms"] / 1e3) / 1e12,
+                               "qk_causal_max_tflops": k["qk_causal_max"]["flops"] /
+                               (k["qk_causal_max"]["total_ms"] / 1e3) / 1e12,
+                               "clipped_heads": [int(h) for h in np.nonzero(mask.cpu().numpy())[0]]})
+        out["config"].update(tokens=B * S, flops_per_layer=qf, l2="inputs larger than L2 (X 134 MB, Q/K 268 MB)")
+        t0 = time.perf_counter()
+        oracle.qk_max_logit(X.double().numpy(), Wq.double().numpy(), Wk.double().numpy(), H, dh, causal=True)
+        cpu_s = time.perf_counter() - t0
+        out["cpu_baseline"] = {"value": B * S / cpu_s, "unit": "tokens/s", "cores": blas_threads(), "kind": "oracle",
+                               "sample": f"the whole layer's S_max in fp64, {cpu_s:.1f} s",
+                               "ms_per_step": cpu_s * 1e3, "extrapolated": False, "cpu_model": cpu_model(),
+                               "nproc": os.cpu_count()}
+    out["kernels"] = {n: dict(v, ms_per_launch=v["total_ms"] / max(v["launches"], 1)) for n, v in k.items()}
+    out["roofline"] = _roofline_row(k, peaks, reps)
+    out["gpu_launches"] = sum(v["launches"] for n, v in k.items() if n != "table_upload")
+    out["peaks"] = peaks
+    print(json.dumps(out), flush=True)
+    return 0
+
+
+# ------------------------------------------------------ sharded (N GPUs)
+class GpuCtx:
+    """What the sharded bench loop needs from one rank's GPU: the C-ABI calls
+    on the rank's stream, CUDA-event timing and the per-kernel rows."""
+
+    def __init__(self, mc, dev, stream, rank, world):
+        self.mc, self.device, self.stream, self.rank, self.world = mc, dev, stream, rank, world
+
+    def local_step(self, Ws, Gs, Ms, **hp):
+        self.mc.muon_step(Ws, Gs, Ms, stream=self.stream, **hp)
+
+    def qk_max_logit(self, x, wq, wk, H, dh, smax):
+        self.mc.qk_max_logit(x, wq, wk, H, dh, causal=True, smax_out=smax, stream=self.stream)
+
+    def qk_clip(self, wq, wk, smax, H, dh, tau, alpha, gamma, mask):
+        self.mc.qk_clip(wq, wk, smax, H, dh, tau=tau, alpha=alpha, gamma_out=gamma, mask_out=mask,
+                        stream=self.stream)
+
+    def sync(self):
+        import torch
+        torch.cuda.synchronize()
+
+    def start(self):
+        import torch
+        e = torch.cuda.Event(enable_timing=True)
+        e.record(self.stream)
+        return e
+
+    def stop(self, e0):
+        import torch
+        e1 = torch.cuda.Event(enable_timing=True)
+        e1.record(self.stream)
+        torch.cuda.synchronize()
+        return e0.elapsed_time(e1)
+
+    def profile_begin(self):
+        self.mc.profile_begin()
+
+    def profile_end(self):
+        k = self.mc.profile_end()
+        assert self.mc.device_status() == self.mc.MC_OK, self.mc.last_error()
+        return k
+
+
+def run_sharded(args, ctx, shapes, qk_cfg, hp, barrier, max_over_ranks, make_e2e=None):
+    """The data-parallel MuonClip step of "MuonClip: speed, then stability" §08
+    over ``ctx.world`` ranks: one parameter set whose matrices are owned whole
+    by one rank each (reduce-scatter of the gradients, the owner's Muon step,
+    all-gather of the weights), and per-rank QK batches whose S_max is made
+    global by an all-reduce (max) before the clip.  Strong scaling: the
+    parameter set is fixed, so the Muon work per rank falls as 1/world; each
+    rank's QK batch is its own.  Returns the JSON dict on rank 0."""
+    import torch
+    from matrix_orthogonalising_optimizer_step_b200.sharded import ShardedMuon, global_smax
+    from matrix_orthogonalising_optimizer_step_b200 import workloads as wl
+
+    dev = ctx.device
+    shard = ShardedMuon(shapes, w_dtype=torch.bfloat16, g_dtype=torch.bfloat16, device=dev,
+                        ns_steps=hp["ns_steps"], local_step=ctx.local_step)
+    gen = torch.Generator(device=dev)
+    gen.manual_seed(2024)                   # the same weights on every replica
+    for W in shard.weights:
+        W.copy_(torch.randn(W.shape, device=dev, generator=gen) * 0.02)
+    gen.manual_seed(3000 + ctx.rank)        # each rank's own gradients
+    for G in shard.grads:
+        z = torch.randn((G.shape[0], 1), device=dev, generator=gen)
+        G.copy_(torch.randn(G.shape, device=dev, generator=gen) * 1e-3 * torch.exp(z))
+    B, S, D, H, dh = (qk_cfg[k] for k in ("B", "S", "D", "H", "dh"))
+    X, Wq, Wk = wl.qk_inputs(B, S, D, H, dh, seed=3 + 100 * ctx.rank, hot_heads=qk_cfg["hot_heads"],
+                             hot_scale=qk_cfg["hot_scale"])
+    _, Wq, Wk = wl.qk_inputs(B, S, D, H, dh, seed=3, hot_heads=qk_cfg["hot_heads"], hot_scale=qk_cfg["hot_scale"])
+    x, wq, wk = X.to(dev), Wq.to(dev), Wk.to(dev)
+    smax = torch.empty(H, dtype=torch.float32, device=dev)
+    gamma = torch.empty(H, dtype=torch.float32, device=dev)
+    mask = torch.empty(H, dtype=torch.int32, device=dev)
+
+    def step():
+        shard.step(**hp)
+        ctx.qk_max_logit(x, wq, wk, H, dh, smax)
+        global_smax(smax)
+        ctx.qk_clip(wq, wk, smax, H, dh, wl.QK_TAU, wl.QK_ALPHA, gamma, mask)
+
+    warmup = max(args.warmup, 3)
+    for _ in range(warmup):
+        step()
+    ctx.sync()
+    barrier()
+    sampler = ClockSampler(getattr(ctx, "gpu_index", 0)) if ctx.rank == 0 and hasattr(ctx, "gpu_index") else None
+    if sampler:
+        sampler.start()
+        time.sleep(0.3)
+    ctx.profile_begin()
+    t = ctx.start()
+    for _ in range(args.steps):
+        step()
+    ms = max_over_ranks(ctx.stop(t)) / args.steps
+    kernels = ctx.profile_end()
+    barrier()
+    clocks = sampler.stop() if sampler else None
+
+    ns_flops = ns_dense_flops(shapes, hp["ns_steps"])
+    qkf = qk_flops(B, S, D, H, dh)
+    step_flops = ns_flops + ctx.world * qkf
+    value = step_flops / (ms / 1e3) / 1e12
+    e2e = make_e2e(shard, step, step_flops, (smax, gamma, mask)) if make_e2e else None
+    if ctx.rank != 0:
+        return None
+    launches = sum(v["launches"] for k, v in kernels.items() if k != "table_upload")
+    roof = None
+    ks = {k: v for k, v in kernels.items() if k != "table_upload" and v["total_ms"] > 0}
+    if ks:
+        dom = max(ks.items(), key=lambda kv: kv[1]["total_ms"])[0]
+        d = ks[dom]
+        peaks = measured_peaks()
+        if d["flops"] > 0:
+            ach = d["flops"] / (d["total_ms"] / 1e3) / 1e12
+            roof = {"kernel": dom, "bound": "tensor", "achieved": ach, "peak": peaks["bf16_tflops_sustained"],
+                    "unit": "TFLOP/s", "frac": ach / peaks["bf16_tflops_sustained"], "traffic": None,
+                    "peak_source": f"{peaks['source']} bf16_tflops_sustained (rank 0's kernels inside the step)"}
+        else:
+            ach = d["bytes"] / (d["total_ms"] / 1e3) / 1e9
+            roof = {"kernel": dom, "bound": "hbm", "achieved": ach, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                    "frac": ach / peaks["hbm_gbs"], "traffic": None, "peak_source": f"{peaks['source']} hbm_gbs"}
+    return {
+        "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": ctx.world, "steps": args.steps,
+        "warmup": warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "strong", "vs_baseline": None,
+        "dtype": "bf16", "data": "synthetic",
+        "config": {"workload": WORKLOAD, "mode": "sharded", "matrices": len(shapes),
+                   "params": int(sum(r * c for r, c in shapes)), "flops_per_step": step_flops,
+                   "flops_convention": "dense-equivalent NS FLOPs of the one parameter set + every rank's QK "
+                                       "projection and causal scores",
+                   "l2": "inputs larger than L2",
+                   "parallelism": f"dp{ctx.world}: whole-matrix ownership, reduce-scatter of gradients, owner "
+                                  "Muon step, all-gather of weights; all-reduce(max) of S_max",
+                   "owned_matrices_rank0": len(shard.owned),
+                   "owner_load_balance": max(shard.load) / (sum(shard.load) / len(shard.load))},
+        "kernels": {k: dict(v, ms_per_launch=v["total_ms"] / max(v["launches"], 1)) for k, v in kernels.items()},
+        "roofline": roof, "cpu_baseline": None, "e2e": e2e, "gpu_launches": launches, "clocks": clocks}
+
+
 def main(argv=None):
     args = parse_args(argv)
     world = int(os.environ.get("WORLD_SIZE", "1"))
@@ -351,6 +673,8 @@ def main(argv=None):
     local_rank = int(os.environ.get("LOCAL_RANK", "0"))
     if args.impl == "reference":
         return run_reference(args, rank, world)
+    if args.config is not None:
+        return run_config(args, args.config)
 
     import torch
     import torch.distributed as dist
@@ -366,6 +690,58 @@ def main(argv=None):
     mc.load_library()
     peaks = measured_peaks()
     hp = dict(wl.HPARAMS)
+    mode = args.mode or ("sharded" if world > 1 else "plain")
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+
+    def max_over_ranks(v):
+        if world == 1:
+            return v
+        t = torch.tensor([v], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        return float(t.item())
+
+    if mode == "sharded":
+        ctx = GpuCtx(mc, dev, torch.cuda.current_stream(), rank, world)
+        ctx.gpu_index = local_rank
+
+        def e2e(shard, step, step_flops, outs):
+            # the rank's local gradients come up from pinned host memory, the
+            # sharded step runs, the statistics (S_max, gamma, mask) go back down
+            g_bytes = shard.g_flat.numel() * shard.g_flat.element_size()
+            g_host = torch.empty(shard.g_flat.shape, dtype=shard.g_flat.dtype, pin_memory=True)
+            g_host.copy_(shard.g_flat)
+            outs_host = [torch.empty(t.shape, dtype=t.dtype).pin_memory() for t in outs]
+            d2h = sum(t.numel() * t.element_size() for t in outs_host)
+
+            def e2e_step():
+                shard.g_flat.copy_(g_host, non_blocking=True)
+                step()
+                for dst, src in zip(outs_host, outs):
+                    dst.copy_(src, non_blocking=True)
+
+            e2e_step()
+            barrier()
+            t = ctx.start()
+            for _ in range(args.steps):
+                e2e_step()
+            ms_e = max_over_ranks(ctx.stop(t)) / args.steps
+            barrier()
+            del g_host, outs_host
+            return {"value": step_flops / (ms_e / 1e3) / 1e12, "unit": "TFLOP/s", "ms_per_step": ms_e,
+                    "h2d_bytes_per_step": int(g_bytes), "d2h_bytes_per_step": int(d2h),
+                    "api": "ShardedMuon.step (reduce-scatter, muon_step, all-gather), qk_max_logit, global_smax, "
+                           "qk_clip; each rank's gradients uploaded from pinned host memory first"}
+
+        out = run_sharded(args, ctx, wl.cfg2_shapes(layers=args.layers), wl.CFG3, hp, barrier, max_over_ranks,
+                          make_e2e=None if args.no_e2e else e2e)
+        if rank == 0:
+            print(json.dumps(out), flush=True)
+        if world > 1:
+            dist.destroy_process_group()
+        return 0
 
     # --- inputs (each rank its own 7B-shaped set: weak scaling)
     shapes, (Wf, Ws), (Gf, Gs), (Mf, Ms) = make_muon_inputs(dev, args.layers, seed=2 + 1000 * rank)
@@ -385,17 +761,6 @@ def main(argv=None):
         mc.qk_max_logit(x, wq, wk, H, dh, causal=True, smax_out=smax, stream=stream)
         mc.qk_clip(wq, wk, smax, H, dh, tau=wl.QK_TAU, alpha=wl.QK_ALPHA, gamma_out=gamma, mask_out=mask,
                    stream=stream)
-
-    def barrier():
-        if world > 1:
-            dist.barrier()
-
-    def max_over_ranks(v):
-        if world == 1:
-            return v
-        t = torch.tensor([v], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        return float(t.item())
 
     for _ in range(max(args.warmup, 3)):
         step()
@@ -441,10 +806,11 @@ def main(argv=None):
     elem_gbs = mom["bytes"] / (mom["total_ms"] / 1e3) / 1e9 if mom else None
     qk_ms = sum(kernels[k]["total_ms"] for k in ("qk_proj", "qk_causal_max", "qk_keys") if k in kernels) / K
     qk_tokens = B * S / (qk_ms / 1e3) if qk_ms > 0 else None
-    gpu_launches = sum(v["launches"] for v in kernels.values())
+    # kernels only: the parameter-table copy is profiled but is not a launch
+    gpu_launches = sum(v["launches"] for k, v in kernels.items() if k != "table_upload")
 
     # dominant kernel: the kernel kind with the largest device time
-    dom = max(kernels.items(), key=lambda kv: kv[1]["total_ms"])[0]
+    dom = max(((k, v) for k, v in kernels.items() if k != "table_upload"), key=lambda kv: kv[1]["total_ms"])[0]
     d = kernels[dom]
     if d["flops"] > 0:
         ach = d["flops"] / (d["total_ms"] / 1e3) / 1e12
