@@ -20,8 +20,8 @@ from typing import Optional, Sequence
 _PKG = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_PKG, "libmuonclip.so")
 
-MC_OK, MC_ERR_INVAL, MC_ERR_ALIGN, MC_ERR_NOSPC, MC_ERR_CUDA, MC_ERR_UNSUPPORTED, MC_ERR_DEVICE = (
-    0, -1, -2, -3, -4, -5, -6)
+MC_OK, MC_ERR_INVAL, MC_ERR_ALIGN, MC_ERR_NOSPC, MC_ERR_CUDA, MC_ERR_UNSUPPORTED, MC_ERR_DEVICE, MC_ERR_NONFINITE = (
+    0, -1, -2, -3, -4, -5, -6, -7)
 MC_F32, MC_BF16 = 0, 1
 
 # Names the C ABI exports (include/muonclip.h).
@@ -29,7 +29,7 @@ EXPORTS = ("mc_muon_workspace_size", "mc_muon_step", "mc_qk_workspace_size", "mc
            "mc_qk_clip", "mc_last_error", "mc_device_status", "mc_profile_begin", "mc_profile_end",
            "mc_qk_max_logit_static", "mc_qk_clip_slices", "mc_mla_workspace_size", "mc_mla_max_logit",
            "mc_shard_plan", "mc_normuon_workspace_size", "mc_normuon_step", "mc_polar_express_coeffs",
-           "mc_muon_host_grads_workspace_size", "mc_muon_step_host_grads")
+           "mc_muon_host_grads_workspace_size", "mc_muon_step_host_grads", "mc_selftest_bounded_wait")
 MC_QK_STATIC_MAX_ELEMS = 1 << 24
 MC_QK_STATIC_MAX_HEADS = 4096
 
@@ -119,6 +119,8 @@ def load_library():
     lib.mc_shard_plan.argtypes = [P(ctypes.c_int64), P(ctypes.c_int64), i32, i32, i32, P(ctypes.c_int32),
                                   P(ctypes.c_double)]
     lib.mc_shard_plan.restype = i32
+    lib.mc_selftest_bounded_wait.argtypes = [ctypes.c_longlong, vp]
+    lib.mc_selftest_bounded_wait.restype = i32
     lib.mc_profile_begin.argtypes = []
     lib.mc_profile_begin.restype = i32
     lib.mc_profile_end.argtypes = [P(McKernelStat), i32, P(ctypes.c_int)]
@@ -138,7 +140,8 @@ def last_error() -> str:
 
 def device_status() -> int:
     """Synchronise the current device and return (and clear) the library's
-    device error word: MC_OK or MC_ERR_DEVICE."""
+    device error word: MC_OK, MC_ERR_DEVICE (a bounded wait ran out) or
+    MC_ERR_NONFINITE (a Muon step met a NaN/Inf gradient or momentum)."""
     return load_library().mc_device_status()
 
 
@@ -193,6 +196,43 @@ def _need_cuda_contig(t, name):
         raise ValueError(f"{name} must be a CUDA tensor")
     if not t.is_contiguous():
         raise ValueError(f"{name} must be contiguous")
+
+
+def _one_device(tensors):
+    """The device every (non-None) tensor lives on; raises if they differ.
+    Each C call runs with that device current, so the library's per-device
+    state, the stream and the pointers all belong to it."""
+    devs = {t.device for t in tensors if t is not None}
+    if len(devs) != 1:
+        raise ValueError(f"all tensors must be on one CUDA device, got {sorted(str(d) for d in devs)}")
+    return devs.pop()
+
+
+def _check_qk_args(x, wq, wk, H, dh, smax_out, names=("x", "wq", "wk")):
+    """Shapes of the MHA S_max call: x [B, S, D] and wq, wk [H*dh, D], bf16,
+    contiguous; smax_out (if given) fp32, contiguous, at least H entries."""
+    torch = _torch()
+    for t, nm in zip((x, wq, wk), names):
+        _need_cuda_contig(t, nm)
+        if t.dtype != torch.bfloat16:
+            raise TypeError(f"{nm} must be bfloat16")
+    if x.dim() != 3:
+        raise ValueError(f"x must be 3-D [B, S, D], got shape {tuple(x.shape)}")
+    want = (int(H) * int(dh), int(x.shape[2]))
+    for t, nm in ((wq, names[1]), (wk, names[2])):
+        if tuple(t.shape) != want:
+            raise ValueError(f"{nm} must have shape (H*dh, D) = {want}, got {tuple(t.shape)}")
+    _check_out(smax_out, "smax_out", torch.float32, H)
+
+
+def _check_out(t, name, dtype, n):
+    if t is None:
+        return
+    _need_cuda_contig(t, name)
+    if t.dtype != dtype:
+        raise TypeError(f"{name} must be {dtype}")
+    if t.numel() < int(n):
+        raise ValueError(f"{name} must hold at least {int(n)} entries, got {t.numel()}")
 
 
 def make_hparams(mu=0.95, nesterov=True, lr=0.02, wd=0.1, ns_steps=5, a=3.4445, b=-4.7750,
@@ -275,14 +315,15 @@ def muon_step(weights: Sequence, grads: Sequence, moms: Sequence, *, norms_out=N
     h = hparams if hparams is not None else make_hparams(**hp)
     if n == 0:
         return
-    if norms_out is not None:
-        _need_cuda_contig(norms_out, "norms_out")
+    _check_out(norms_out, "norms_out", _torch().float32, n)
+    dev = _one_device(list(weights) + list(grads) + list(moms) + list(update_outs or []) + [norms_out, workspace])
     need = int(lib.mc_muon_workspace_size(arr, n, ctypes.byref(h)))
     if need == 0:
         _check(lib.mc_muon_step(arr, n, ctypes.byref(h), None, 0, None, None))
-    ws = workspace if workspace is not None else _workspace("muon", weights[0].device, need)
-    _check(lib.mc_muon_step(arr, n, ctypes.byref(h), _ptr(ws), int(ws.numel() * ws.element_size()),
-                            _ptr(norms_out), _stream_handle(stream)))
+    with _torch().cuda.device(dev):
+        ws = workspace if workspace is not None else _workspace("muon", dev, need)
+        _check(lib.mc_muon_step(arr, n, ctypes.byref(h), _ptr(ws), int(ws.numel() * ws.element_size()),
+                                _ptr(norms_out), _stream_handle(stream)))
 
 
 def muon_step_host_grads(weights: Sequence, grads: Sequence, grads_host: Sequence, moms: Sequence, *,
@@ -304,15 +345,16 @@ def muon_step_host_grads(weights: Sequence, grads: Sequence, grads_host: Sequenc
     h = hparams if hparams is not None else make_hparams(**hp)
     if n == 0:
         return
-    if norms_out is not None:
-        _need_cuda_contig(norms_out, "norms_out")
+    _check_out(norms_out, "norms_out", _torch().float32, n)
+    dev = _one_device(list(weights) + list(grads) + list(moms) + list(update_outs or []) + [norms_out, workspace])
     need = int(lib.mc_muon_host_grads_workspace_size(arr, n, ctypes.byref(h), int(chunks)))
     if need == 0:
         _check(lib.mc_muon_step_host_grads(arr, hptr, n, ctypes.byref(h), int(chunks), None, 0, None, None))
-    ws = workspace if workspace is not None else _workspace("muon", weights[0].device, need)
-    _check(lib.mc_muon_step_host_grads(arr, hptr, n, ctypes.byref(h), int(chunks), _ptr(ws),
-                                       int(ws.numel() * ws.element_size()), _ptr(norms_out),
-                                       _stream_handle(stream)))
+    with _torch().cuda.device(dev):
+        ws = workspace if workspace is not None else _workspace("muon", dev, need)
+        _check(lib.mc_muon_step_host_grads(arr, hptr, n, ctypes.byref(h), int(chunks), _ptr(ws),
+                                           int(ws.numel() * ws.element_size()), _ptr(norms_out),
+                                           _stream_handle(stream)))
 
 
 def make_normuon(vs, beta2: float = 0.95, eps: float = 1e-8) -> McNormuon:
@@ -348,14 +390,16 @@ def normuon_step(weights: Sequence, grads: Sequence, moms: Sequence, vs: Sequenc
     nm = make_normuon(vs, beta2, eps_v)
     if n == 0:
         return
-    if norms_out is not None:
-        _need_cuda_contig(norms_out, "norms_out")
+    _check_out(norms_out, "norms_out", _torch().float32, n)
+    dev = _one_device(list(weights) + list(grads) + list(moms) + list(vs) + list(update_outs or []) +
+                      [norms_out, workspace])
     need = int(lib.mc_normuon_workspace_size(arr, n, ctypes.byref(h)))
     if need == 0:
         _check(lib.mc_normuon_step(arr, n, ctypes.byref(h), ctypes.byref(nm), None, 0, None, None))
-    ws = workspace if workspace is not None else _workspace("muon", weights[0].device, need)
-    _check(lib.mc_normuon_step(arr, n, ctypes.byref(h), ctypes.byref(nm), _ptr(ws),
-                               int(ws.numel() * ws.element_size()), _ptr(norms_out), _stream_handle(stream)))
+    with _torch().cuda.device(dev):
+        ws = workspace if workspace is not None else _workspace("muon", dev, need)
+        _check(lib.mc_normuon_step(arr, n, ctypes.byref(h), ctypes.byref(nm), _ptr(ws),
+                                   int(ws.numel() * ws.element_size()), _ptr(norms_out), _stream_handle(stream)))
 
 
 def qk_workspace_size(B, S, D, H, dh) -> int:
@@ -367,20 +411,19 @@ def qk_max_logit(x, wq, wk, H: int, dh: int, *, causal: bool = True, smax_out=No
     """Per-head S_max (fp32 [H]) of causal attention with Q = x Wq^T, K = x Wk^T."""
     torch = _torch()
     lib = load_library()
-    for t, nm in ((x, "x"), (wq, "wq"), (wk, "wk")):
-        _need_cuda_contig(t, nm)
-        if t.dtype != torch.bfloat16:
-            raise TypeError(f"{nm} must be bfloat16")
+    _check_qk_args(x, wq, wk, H, dh, smax_out)
+    dev = _one_device([x, wq, wk, smax_out, workspace])
     B, S, D = x.shape
     if smax_out is None:
-        smax_out = torch.empty(H, dtype=torch.float32, device=x.device)
+        smax_out = torch.empty(H, dtype=torch.float32, device=dev)
     need = int(lib.mc_qk_workspace_size(B, S, D, H, dh))
     if need == 0:
         _check(lib.mc_qk_max_logit(None, None, None, B, S, D, H, dh, int(causal), None, None, 0, None))
-    ws = workspace if workspace is not None else _workspace("qk", x.device, need)
-    _check(lib.mc_qk_max_logit(_ptr(x), _ptr(wq), _ptr(wk), B, S, D, H, dh, int(causal),
-                               _ptr(smax_out), _ptr(ws), int(ws.numel() * ws.element_size()),
-                               _stream_handle(stream)))
+    with torch.cuda.device(dev):
+        ws = workspace if workspace is not None else _workspace("qk", dev, need)
+        _check(lib.mc_qk_max_logit(_ptr(x), _ptr(wq), _ptr(wk), B, S, D, H, dh, int(causal),
+                                   _ptr(smax_out), _ptr(ws), int(ws.numel() * ws.element_size()),
+                                   _stream_handle(stream)))
     return smax_out
 
 
@@ -394,14 +437,22 @@ def qk_clip(wq, wk, smax, H: int, dh: int, *, tau: float = 100.0, alpha: float =
         _need_cuda_contig(t, nm)
         if t.dtype != torch.bfloat16:
             raise TypeError(f"{nm} must be bfloat16")
-    _need_cuda_contig(smax, "smax")
+        if t.dim() != 2 or int(t.shape[0]) != int(H) * int(dh):
+            raise ValueError(f"{nm} must have shape (H*dh, D) with H*dh = {int(H) * int(dh)}, got {tuple(t.shape)}")
+    if wk.shape != wq.shape:
+        raise ValueError("wq and wk must have the same shape")
+    _check_out(smax, "smax", torch.float32, H)
+    _check_out(gamma_out, "gamma_out", torch.float32, H)
+    _check_out(mask_out, "mask_out", torch.int32, H)
+    dev = _one_device([wq, wk, smax, gamma_out, mask_out])
     D = int(wq.shape[1])
     if gamma_out is None:
-        gamma_out = torch.empty(H, dtype=torch.float32, device=wq.device)
+        gamma_out = torch.empty(H, dtype=torch.float32, device=dev)
     if mask_out is None:
-        mask_out = torch.empty(H, dtype=torch.int32, device=wq.device)
-    _check(lib.mc_qk_clip(_ptr(wq), _ptr(wk), H, dh, D, _ptr(smax), float(tau), float(alpha),
-                          _ptr(gamma_out), _ptr(mask_out), _stream_handle(stream)))
+        mask_out = torch.empty(H, dtype=torch.int32, device=dev)
+    with torch.cuda.device(dev):
+        _check(lib.mc_qk_clip(_ptr(wq), _ptr(wk), H, dh, D, _ptr(smax), float(tau), float(alpha),
+                              _ptr(gamma_out), _ptr(mask_out), _stream_handle(stream)))
     return gamma_out, mask_out
 
 
@@ -433,14 +484,18 @@ def qk_clip_slices(slices, smax, H: int, *, tau: float = 100.0, gamma_out=None, 
     Returns (gamma [H] fp32, mask [H] int32)."""
     torch = _torch()
     lib = load_library()
-    _need_cuda_contig(smax, "smax")
+    _check_out(smax, "smax", torch.float32, H)
+    _check_out(gamma_out, "gamma_out", torch.float32, H)
+    _check_out(mask_out, "mask_out", torch.int32, H)
     arr, n = make_clip_slices(slices)
+    dev = _one_device([smax, gamma_out, mask_out] + [sl[0] for sl in slices])
     if gamma_out is None:
-        gamma_out = torch.empty(H, dtype=torch.float32, device=smax.device)
+        gamma_out = torch.empty(H, dtype=torch.float32, device=dev)
     if mask_out is None:
-        mask_out = torch.empty(H, dtype=torch.int32, device=smax.device)
-    _check(lib.mc_qk_clip_slices(arr, n, _ptr(smax), H, float(tau), _ptr(gamma_out), _ptr(mask_out),
-                                 _stream_handle(stream)))
+        mask_out = torch.empty(H, dtype=torch.int32, device=dev)
+    with torch.cuda.device(dev):
+        _check(lib.mc_qk_clip_slices(arr, n, _ptr(smax), H, float(tau), _ptr(gamma_out), _ptr(mask_out),
+                                     _stream_handle(stream)))
     return gamma_out, mask_out
 
 
@@ -459,17 +514,26 @@ def mla_max_logit(x, wqc, wkc, wqr, wkr, H: int, dc: int, dr: int, *, causal: bo
         _need_cuda_contig(t, nm)
         if t.dtype != torch.bfloat16:
             raise TypeError(f"{nm} must be bfloat16")
+    if x.dim() != 3:
+        raise ValueError(f"x must be 3-D [B, S, D], got shape {tuple(x.shape)}")
+    D = int(x.shape[2])
+    for t, nm, rows in ((wqc, "wqc", H * dc), (wkc, "wkc", H * dc), (wqr, "wqr", H * dr), (wkr, "wkr", dr)):
+        if tuple(t.shape) != (int(rows), D):
+            raise ValueError(f"{nm} must have shape {(int(rows), D)}, got {tuple(t.shape)}")
+    _check_out(smax_out, "smax_out", torch.float32, H)
+    dev = _one_device([x, wqc, wkc, wqr, wkr, smax_out, workspace])
     B, S, D = x.shape
     if smax_out is None:
-        smax_out = torch.empty(H, dtype=torch.float32, device=x.device)
+        smax_out = torch.empty(H, dtype=torch.float32, device=dev)
     need = int(lib.mc_mla_workspace_size(B, S, D, H, dc, dr))
     if need == 0:
         _check(lib.mc_mla_max_logit(None, None, None, None, None, B, S, D, H, dc, dr, int(causal), None, None, 0,
                                     None))
-    ws = workspace if workspace is not None else _workspace("mla", x.device, need)
-    _check(lib.mc_mla_max_logit(_ptr(x), _ptr(wqc), _ptr(wkc), _ptr(wqr), _ptr(wkr), B, S, D, H, dc, dr,
-                                int(causal), _ptr(smax_out), _ptr(ws), int(ws.numel() * ws.element_size()),
-                                _stream_handle(stream)))
+    with torch.cuda.device(dev):
+        ws = workspace if workspace is not None else _workspace("mla", dev, need)
+        _check(lib.mc_mla_max_logit(_ptr(x), _ptr(wqc), _ptr(wkc), _ptr(wqr), _ptr(wkr), B, S, D, H, dc, dr,
+                                    int(causal), _ptr(smax_out), _ptr(ws), int(ws.numel() * ws.element_size()),
+                                    _stream_handle(stream)))
     return smax_out
 
 
@@ -505,13 +569,12 @@ def qk_max_logit_static(x, wq, wk, H: int, dh: int, *, causal: bool = True, smax
     pass it in to keep the whole call allocation-free.)"""
     torch = _torch()
     lib = load_library()
-    for t, nm in ((x, "x"), (wq, "wq"), (wk, "wk")):
-        _need_cuda_contig(t, nm)
-        if t.dtype != torch.bfloat16:
-            raise TypeError(f"{nm} must be bfloat16")
+    _check_qk_args(x, wq, wk, H, dh, smax_out)
+    dev = _one_device([x, wq, wk, smax_out])
     B, S, D = x.shape
     if smax_out is None:
-        smax_out = torch.empty(H, dtype=torch.float32, device=x.device)
-    _check(lib.mc_qk_max_logit_static(_ptr(x), _ptr(wq), _ptr(wk), B, S, D, H, dh, int(causal),
-                                      _ptr(smax_out), _stream_handle(stream)))
+        smax_out = torch.empty(H, dtype=torch.float32, device=dev)
+    with torch.cuda.device(dev):
+        _check(lib.mc_qk_max_logit_static(_ptr(x), _ptr(wq), _ptr(wk), B, S, D, H, dh, int(causal),
+                                          _ptr(smax_out), _stream_handle(stream)))
     return smax_out

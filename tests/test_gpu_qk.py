@@ -24,8 +24,11 @@ def rel(a, b):
     return np.abs(a - b) / np.maximum(np.abs(b), 1e-30)
 
 
+# dh up to 256 takes the row-owned kernel (Q resident); dh = 320 (five 64-column
+# k-blocks) the tile GEMM with the max epilogue
 @pytest.mark.parametrize("B,S,D,H,dh", [(2, 300, 64, 3, 64), (1, 129, 40, 2, 72), (3, 700, 96, 4, 32),
-                                        (1, 1, 16, 1, 8), (2, 520, 256, 2, 128)])
+                                        (1, 1, 16, 1, 8), (2, 520, 256, 2, 128), (1, 770, 64, 3, 256),
+                                        (2, 333, 64, 2, 320), (1, 1300, 128, 5, 192)])
 @pytest.mark.parametrize("causal", [True, False])
 def test_smax_small(B, S, D, H, dh, causal):
     X, Wq, Wk = wl.qk_inputs(B, S, D, H, dh, seed=11, w_std=0.2)
@@ -137,3 +140,26 @@ def test_many_heads_both_sides_of_the_shared_head_table(H):
     got = gpu_smax(X, Wq, Wk, H, dh)
     refb = oracle.qk_max_logit(to64(X), to64(Wq), to64(Wk), H, dh, causal=True, qk_bf16=True)
     assert np.all(rel(got, refb) <= 2e-3), np.max(rel(got, refb))
+
+
+def test_binding_rejects_mismatched_shapes_before_the_call():
+    """The C side builds its tensor maps from H*dh and D, so a W_q or W_k with
+    too few rows, or a too-short output, must be refused before any launch."""
+    B, S, D, H, dh = 1, 64, 64, 2, 64
+    X, Wq, Wk = wl.qk_inputs(B, S, D, H, dh, seed=5)
+    x, wq, wk = X.to("cuda"), Wq.to("cuda"), Wk.to("cuda")
+    short = wq[: H * dh - 8].contiguous()
+    for fn in (mc.qk_max_logit, mc.qk_max_logit_static):
+        with pytest.raises(ValueError):
+            fn(x, short, wk, H, dh)
+        with pytest.raises(ValueError):
+            fn(x, wq, short, H, dh)
+        with pytest.raises(ValueError):
+            fn(x[0], wq, wk, H, dh)
+        with pytest.raises(ValueError):
+            fn(x, wq, wk, H, dh, smax_out=torch.zeros(H - 1, dtype=torch.float32, device="cuda"))
+        with pytest.raises(TypeError):
+            fn(x, wq, wk, H, dh, smax_out=torch.zeros(H, dtype=torch.float64, device="cuda"))
+    with pytest.raises(ValueError):
+        mc.qk_clip(short, short.clone(), torch.zeros(H, device="cuda"), H, dh)
+    assert mc.device_status() == mc.MC_OK

@@ -20,6 +20,7 @@ import pytest
 import torch
 
 import matrix_orthogonalising_optimizer_step_b200 as mc
+import oracle
 from matrix_orthogonalising_optimizer_step_b200 import workloads as wl
 from gpu_util import SMAX_TOL
 
@@ -46,15 +47,29 @@ def test_static_entry_matches_workspace_entry_twice(B, S, D, H, dh, causal):
     x, wq, wk = X.to(DEV), Wq.to(DEV), Wk.to(DEV)
     want = mc.qk_max_logit(x, wq, wk, H, dh, causal=causal)
     outs = [torch.full((H,), float("nan"), dtype=torch.float32, device=DEV) for _ in range(2)]
+    # a first call settles any one-time set-up (the scratch address lookup);
+    # after it the two calls checked below must leave device memory as it is
+    assert call_static(lib, x, wq, wk, H, dh, causal, outs[0]) == mc.MC_OK, mc.last_error()
+    for out in outs:
+        out.fill_(float("nan"))
+    torch.cuda.synchronize()
+    free0, reserved0 = torch.cuda.mem_get_info()[0], torch.cuda.memory_reserved()
     for out in outs:
         rc = call_static(lib, x, wq, wk, H, dh, causal, out)
         assert rc == mc.MC_OK, mc.last_error()
     assert mc.device_status() == mc.MC_OK, mc.last_error()
+    assert torch.cuda.mem_get_info()[0] == free0
+    assert torch.cuda.memory_reserved() == reserved0
     w = want.cpu().double().numpy()
+    # the small cases also against the fp64 oracle (Q, K in fp64, as defined)
+    ref = (oracle.qk_max_logit(X.double().numpy(), Wq.double().numpy(), Wk.double().numpy(), H, dh, causal=causal)
+           if B * S * D <= 2 ** 20 else None)
     for out in outs:
         got = out.cpu().double().numpy()
         assert np.all(np.isfinite(got))
         assert np.all(np.abs(got - w) <= SMAX_TOL * np.abs(w)), (got, w)
+        if ref is not None:
+            assert np.all(np.abs(got - ref) <= SMAX_TOL * np.abs(ref)), (got, ref)
 
 
 def test_static_entry_rejects_sizes_beyond_its_scratch():
@@ -67,3 +82,13 @@ def test_static_entry_rejects_sizes_beyond_its_scratch():
     assert rc == mc.MC_ERR_NOSPC
     assert "static scratch" in mc.last_error()
     assert torch.all(out == 7.0)  # nothing was enqueued
+    # more heads than the scratch's head table, with few elements
+    B, S, D, H, dh = 1, 1, 8, 4104, 8
+    x = torch.zeros((B, S, D), dtype=torch.bfloat16, device=DEV)
+    wq = torch.zeros((H * dh, D), dtype=torch.bfloat16, device=DEV)
+    out = torch.full((H,), 7.0, dtype=torch.float32, device=DEV)
+    rc = call_static(lib, x, wq, wq.clone(), H, dh, True, out)
+    assert rc == mc.MC_ERR_NOSPC
+    assert "heads" in mc.last_error()
+    torch.cuda.synchronize()
+    assert torch.all(out == 7.0)
