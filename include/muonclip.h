@@ -24,10 +24,12 @@
  *     retains caller memory beyond the call (the call is asynchronous, so the
  *     buffers must stay valid until the stream reaches that point).
  *   - `stream` is a cudaStream_t (NULL = legacy default stream).  Calls
- *     enqueue work and return.  A call may wait on the host for the upload of
- *     a parameter table it issued four calls earlier (the tables go through a
- *     4-slot page-locked staging ring), and for the device to go idle when the
- *     engine-owned workspace has to grow; mc_device_status synchronises.
+ *     enqueue work and return without waiting for the device.  The two
+ *     exceptions: a call waits for the oldest of the library's parameter-table
+ *     uploads on the device when 32 of them are still queued (each Muon-type
+ *     call makes one upload, through its own page-locked staging buffer), and,
+ *     with a NULL workspace, for the device to go idle when the engine-owned
+ *     workspace has to grow.  mc_device_status synchronises.
  *   - Host-side state is guarded by one mutex, so calls may come from several
  *     threads.  GPU work of calls that share the engine-owned workspace (NULL
  *     workspace) or, for mc_muon_step_host_grads, the library's copy stream on
@@ -57,7 +59,8 @@ enum {
   MC_ERR_NOSPC = -3,       /* workspace smaller than the *_workspace_size query */
   MC_ERR_CUDA = -4,        /* a CUDA runtime call failed (message in mc_last_error) */
   MC_ERR_UNSUPPORTED = -5, /* not a compute capability 10.0 device */
-  MC_ERR_DEVICE = -6       /* mc_device_status: a kernel gave up on a bounded wait */
+  MC_ERR_DEVICE = -6,      /* mc_device_status: a kernel gave up on a bounded wait */
+  MC_ERR_NONFINITE = -7    /* mc_device_status: a Muon step met a NaN/Inf NS input */
 };
 
 enum { MC_F32 = 0, MC_BF16 = 1 };
@@ -112,22 +115,35 @@ typedef struct {
  * significant bits); from the third on, a*I is folded into B
  * (X <- (aI + B) X), which amplifies the bf16 rounding of X less once the
  * singular values have entered the polynomial's band.  The last iteration
- * applies the update to W straight from the fp32 accumulator.
+ * applies the update to W straight from the fp32 accumulator.  Matrices whose
+ * short side is at most 32 are no tensor-core contraction (A is at most
+ * 32 x 32): they run the same iteration in fp32 on CUDA cores, streaming the
+ * long side.
  * The list is processed in consecutive pieces of at most 2^29 elements (at
  * least one matrix each), all reusing one workspace; inside a piece, matrices
- * of equal shape and weight dtype are batched into one problem group.  A
- * matrix's result does not depend on the other matrices of the call.
+ * of equal shape and weight dtype are batched into one problem group.  The
+ * parameter tables of every piece go to the device in one copy at the start
+ * of the call.  A matrix's result does not depend on the other matrices of
+ * the call.
  *
  * params/n      host array of n >= 0 entries (n == 0 is a no-op).  W, G, M of
  *               one entry must not alias; G is left unchanged.
  * hp            host pointer.
  * workspace     device scratch of at least mc_muon_workspace_size(...) bytes
- *               (what the largest piece needs), or NULL to let the library
- *               allocate (and keep) its own.
+ *               (what the largest piece needs, plus every piece's tables), or
+ *               NULL to let the library allocate (and keep) its own.
  *               Must not be used by anything else until the step completes.
- * norms_out     optional device fp32 [n]: ||U||_F of each matrix (NULL = skip).
+ * norms_out     optional device fp32 [n]: ||U||_F of each matrix (NULL = skip);
+ *               NaN or Inf exactly when that matrix's U has a non-finite element.
  * Errors        MC_ERR_INVAL, MC_ERR_ALIGN, MC_ERR_NOSPC, MC_ERR_CUDA,
  *               MC_ERR_UNSUPPORTED.
+ * Non-finite input ("MuonClip: speed, then stability" §12 lists overflow
+ * events among what a run should watch): a matrix whose U holds a NaN or Inf
+ * (from its gradient or momentum) gets a zero orthogonalised update, so its
+ * W only decays; its momentum keeps the non-finite values (reset it before
+ * the next step); its norms_out entry is not finite, and the next
+ * mc_device_status returns MC_ERR_NONFINITE.  The other matrices of the call
+ * are not affected.
  */
 size_t mc_muon_workspace_size(const mc_param* params, int n, const mc_hparams* hp);
 int mc_muon_step(const mc_param* params, int n, const mc_hparams* hp, void* workspace,
@@ -313,7 +329,9 @@ int mc_mla_max_logit(const void* x, const void* wqc, const void* wkc, const void
  * array and it keeps the last call's contents (each call resets what must
  * start fresh), so calls that can overlap on the GPU -- on different streams,
  * or from different threads -- race and must be ordered by the caller.
- * Arguments, layouts and the other errors are as for mc_qk_max_logit.
+ * Arguments, layouts and the other errors are as for mc_qk_max_logit.  The
+ * measurement support below does not record this call's launches (it would
+ * have to create CUDA events).
  */
 #define MC_QK_STATIC_MAX_ELEMS (1u << 24)
 #define MC_QK_STATIC_MAX_HEADS 4096
@@ -369,10 +387,24 @@ const char* mc_last_error(void);
 
 /*
  * mc_device_status -- synchronises the current device, then reads and clears
- * the library's device error word.  Returns MC_OK, MC_ERR_DEVICE when a kernel
- * abandoned a bounded wait (its outputs are then invalid), or MC_ERR_CUDA.
+ * the library's device error word.  Returns MC_OK; MC_ERR_DEVICE when a kernel
+ * abandoned a bounded wait (its outputs are then invalid); MC_ERR_NONFINITE
+ * when a Muon step since the last call met a non-finite Newton-Schulz input
+ * (see mc_muon_step); or MC_ERR_CUDA.
  */
 int mc_device_status(void);
+
+/*
+ * mc_selftest_bounded_wait -- test support with no counterpart on the pages:
+ * launches one small kernel whose single wait (on an mbarrier that expects an
+ * arrival nothing makes) runs out after limit_cycles SM cycles, the way every
+ * wait in the library's kernels gives up instead of hanging.  The kernel then
+ * returns normally, and the next mc_device_status returns MC_ERR_DEVICE (and
+ * clears the word).  Lets a test check the timeout path and that the context
+ * stays usable, without breaking a real kernel.
+ * limit_cycles in [1000, 2^32]; MC_ERR_INVAL otherwise.
+ */
+int mc_selftest_bounded_wait(long long limit_cycles, void* stream);
 
 /*
  * Measurement support.  Between mc_profile_begin() and mc_profile_end(), every
@@ -398,6 +430,9 @@ int mc_device_status(void);
  *   qk_proj         flops = 2 * B*S * H*dh * D * 2 (Q and K)
  *   qk_causal_max   flops = 2 * dh * (score pairs inside the causal mask)
  *   norm_finalize, qk_keys, qk_clip   (small kernels; counted, no work figure)
+ *   table_upload    not a kernel: the host-to-device copy of a call's
+ *                   parameter tables (bytes = the table bytes); one per
+ *                   mc_muon_step, mc_normuon_step or mc_muon_step_host_grads
  *
  * The rows are written to `out` (up to `max_rows`), `*rows` receives the count.
  * Recording events adds no synchronisation; the durations are device time.

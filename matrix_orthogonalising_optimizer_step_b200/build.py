@@ -19,7 +19,7 @@ CSRC = os.path.join(PKG, "csrc")
 INCLUDE = os.path.join(ROOT, "include")
 LIB = os.path.join(PKG, "libmuonclip.so")
 SOURCES = ["muonclip.cu"]
-HEADERS = ["ptx.cuh", "umma_gemm.cuh", "stream_kernels.cuh"]
+HEADERS = ["ptx.cuh", "umma_gemm.cuh", "stream_kernels.cuh", "thin_ns.cuh", "qk_rowmax.cuh"]
 
 NVCC_FLAGS = [
     "-O3", "-std=c++17", "-lineinfo",

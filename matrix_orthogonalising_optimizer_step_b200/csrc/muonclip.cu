@@ -27,7 +27,9 @@
 
 #include "muonclip.h"
 #include "ptx.cuh"
+#include "qk_rowmax.cuh"
 #include "stream_kernels.cuh"
+#include "thin_ns.cuh"
 #include "umma_gemm.cuh"
 
 #define MC_API extern "C" __attribute__((visibility("default")))
@@ -57,9 +59,22 @@ using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t
                                    const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
                                    CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
 
-constexpr int kRing = 4;
+// Page-locked staging buffers for the parameter-table uploads: a call takes a
+// buffer whose last copy has finished, or adds one, and only when this many
+// are still in flight does it wait (for the oldest).
+constexpr int kMaxStaging = 32;
+// Largest dynamic shared memory a CTA may opt into on sm_100.
+constexpr int kSmemOptIn = 232448;
+constexpr size_t kStagingMin = 64 << 10;
 // Newton-Schulz iterations that take a*X from the iterate's hi + lo halves.
 constexpr int kMixedIters = 2;
+
+struct StagingBuf {
+  void* host = nullptr;
+  size_t bytes = 0;
+  cudaEvent_t done = nullptr;  // recorded after the buffer's latest copy
+  unsigned long long seq = 0;  // order of use (the oldest is waited for first)
+};
 
 struct DeviceState {
   bool init = false;
@@ -69,10 +84,8 @@ struct DeviceState {
   int* err_ptr = nullptr;
   void* own_ws = nullptr;
   size_t own_ws_bytes = 0;
-  void* pinned[kRing] = {};
-  size_t pinned_bytes[kRing] = {};
-  cudaEvent_t ev[kRing] = {};
-  int next = 0;
+  std::vector<StagingBuf> staging;
+  unsigned long long staging_seq = 0;
   // mc_muon_step_host_grads: a non-blocking stream for the gradient copies and
   // events that order each chunk's compute after its copies
   cudaStream_t copy_stream = nullptr;
@@ -111,8 +124,13 @@ int device_state(DeviceState** out) {
     MC_CUDA((set_gemm_attr<EPI_POLY, 1>()));
     MC_CUDA((set_gemm_attr<EPI_APPLY, 1>()));
     MC_CUDA((set_gemm_attr<EPI_APPLY_FINAL, 1>()));
+    MC_CUDA((set_gemm_attr<EPI_GRAM, 0>()));
+    MC_CUDA((set_gemm_attr<EPI_POLY, 0>()));
+    MC_CUDA((set_gemm_attr<EPI_APPLY, 0>()));
+    MC_CUDA((set_gemm_attr<EPI_APPLY_FINAL, 0>()));
     MC_CUDA((set_gemm_attr<EPI_STORE, 1>()));
     MC_CUDA((set_gemm_attr<EPI_CAUSALMAX, 0>()));
+    MC_CUDA(cudaFuncSetAttribute(qk_rowmax_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemOptIn));
     {
       cudaLaunchConfig_t cfg = {};
       cudaLaunchAttribute attr[1];
@@ -144,27 +162,103 @@ int device_state(DeviceState** out) {
   return MC_OK;
 }
 
-// Copy a small host table into device memory through a pinned staging ring
-// (so the copy is asynchronous and the host buffer can be reused at once).
+// ----------------------------------------------------------- profiling
+enum Kind : int { K_MOMENTUM, K_FINALIZE, K_GRAM, K_POLY, K_APPLY_MIXED, K_APPLY, K_APPLY_FINAL, K_QK_PROJ,
+                  K_QK_CMAX, K_QK_KEYS, K_QK_CLIP, K_MLA_PROJ, K_MLA_CMAX, K_QK_CLIP_SLICES, K_NORM_ROWS,
+                  K_NORM_APPLY, K_TABLE_UPLOAD, K_NS_THIN, K_COUNT };
+const char* const kKindNames[K_COUNT] = {"momentum",  "norm_finalize",  "ns_gram", "ns_poly",
+                                         "ns_apply_mixed", "ns_apply", "ns_apply_final", "qk_proj",
+                                         "qk_causal_max", "qk_keys", "qk_clip", "mla_proj",
+                                         "mla_causal_max", "qk_clip_slices", "normuon_rows",
+                                         "normuon_apply", "table_upload", "ns_thin"};
+struct ProfRec {
+  int kind;
+  cudaEvent_t b, e;
+  double flops, flops_exec, flops_dense, bytes;
+};
+thread_local bool t_prof = false;
+thread_local std::vector<ProfRec> t_recs;
+
+// Brackets one launch with CUDA events on its stream while profiling is on.
+struct ProfScope {
+  bool on = false;
+  ProfRec r{};
+  cudaStream_t s;
+  ProfScope(int kind, cudaStream_t st, double flops = 0, double flops_exec = 0, double bytes = 0,
+            double flops_dense = -1) : s(st) {
+    if (!t_prof || kind < 0) return;
+    r.kind = kind;
+    r.flops = flops;
+    r.flops_exec = flops_exec;
+    r.flops_dense = flops_dense < 0 ? flops : flops_dense;
+    r.bytes = bytes;
+    if (cudaEventCreate(&r.b) != cudaSuccess) return;
+    if (cudaEventCreate(&r.e) != cudaSuccess) {
+      cudaEventDestroy(r.b);
+      return;
+    }
+    on = cudaEventRecord(r.b, s) == cudaSuccess;
+  }
+  ~ProfScope() {
+    if (!on) return;
+    cudaEventRecord(r.e, s);
+    t_recs.push_back(r);
+  }
+};
+
+// Copy a small host table into device memory through a page-locked staging
+// buffer, so that the copy is asynchronous and the caller's host memory can be
+// reused at once.  Never waits on the host unless kMaxStaging earlier copies
+// are all still queued on the device.
 int upload(DeviceState& st, const void* host, size_t bytes, void* dst, cudaStream_t s) {
   if (bytes == 0) return MC_OK;
-  const int i = st.next;
-  st.next = (st.next + 1) % kRing;
-  if (st.ev[i]) {
-    MC_CUDA(cudaEventSynchronize(st.ev[i]));
-  } else {
-    MC_CUDA(cudaEventCreateWithFlags(&st.ev[i], cudaEventDisableTiming));
+  StagingBuf* pick = nullptr;
+  for (auto& b : st.staging) {
+    if (b.bytes < bytes) continue;
+    const cudaError_t q = cudaEventQuery(b.done);
+    if (q == cudaSuccess) {
+      pick = &b;
+      break;
+    }
+    if (q != cudaErrorNotReady) return fail(MC_ERR_CUDA, std::string("cudaEventQuery: ") + cudaGetErrorString(q));
+    // "not ready" is also left as the thread's last error; clear it so that
+    // the launch checks that follow do not take it for a launch failure
+    (void)cudaGetLastError();
   }
-  if (st.pinned_bytes[i] < bytes) {
-    if (st.pinned[i]) MC_CUDA(cudaFreeHost(st.pinned[i]));
-    st.pinned[i] = nullptr;
-    st.pinned_bytes[i] = 0;
-    MC_CUDA(cudaMallocHost(&st.pinned[i], bytes));
-    st.pinned_bytes[i] = bytes;
+  if (!pick && static_cast<int>(st.staging.size()) < kMaxStaging) {
+    StagingBuf b;
+    b.bytes = std::max(bytes, kStagingMin);
+    MC_CUDA(cudaMallocHost(&b.host, b.bytes));
+    const cudaError_t e = cudaEventCreateWithFlags(&b.done, cudaEventDisableTiming);
+    if (e != cudaSuccess) {
+      cudaFreeHost(b.host);
+      return fail(MC_ERR_CUDA, std::string("cudaEventCreateWithFlags: ") + cudaGetErrorString(e));
+    }
+    st.staging.push_back(b);
+    pick = &st.staging.back();
   }
-  std::memcpy(st.pinned[i], host, bytes);
-  MC_CUDA(cudaMemcpyAsync(dst, st.pinned[i], bytes, cudaMemcpyHostToDevice, s));
-  MC_CUDA(cudaEventRecord(st.ev[i], s));
+  if (!pick) {
+    // every buffer is in flight: wait for the oldest, then reuse (and if
+    // need be enlarge) it
+    pick = &st.staging.front();
+    for (auto& b : st.staging)
+      if (b.seq < pick->seq) pick = &b;
+    MC_CUDA(cudaEventSynchronize(pick->done));
+    if (pick->bytes < bytes) {
+      MC_CUDA(cudaFreeHost(pick->host));
+      pick->host = nullptr;
+      pick->bytes = 0;
+      MC_CUDA(cudaMallocHost(&pick->host, bytes));
+      pick->bytes = bytes;
+    }
+  }
+  pick->seq = ++st.staging_seq;
+  std::memcpy(pick->host, host, bytes);
+  {
+    ProfScope prof(K_TABLE_UPLOAD, s, 0, 0, static_cast<double>(bytes));
+    MC_CUDA(cudaMemcpyAsync(dst, pick->host, bytes, cudaMemcpyHostToDevice, s));
+  }
+  MC_CUDA(cudaEventRecord(pick->done, s));
   return MC_OK;
 }
 
@@ -209,50 +303,6 @@ int map_batched(CUtensorMap* map, const void* base, int64_t count, int64_t rows,
   const uint32_t box[3] = {64, box_rows, 1};
   return make_map(map, base, 3, dims, strides, box);
 }
-
-// ----------------------------------------------------------- profiling
-enum Kind : int { K_MOMENTUM, K_FINALIZE, K_GRAM, K_POLY, K_APPLY_MIXED, K_APPLY, K_APPLY_FINAL, K_QK_PROJ,
-                  K_QK_CMAX, K_QK_KEYS, K_QK_CLIP, K_MLA_PROJ, K_MLA_CMAX, K_QK_CLIP_SLICES, K_NORM_ROWS,
-                  K_NORM_APPLY, K_COUNT };
-const char* const kKindNames[K_COUNT] = {"momentum",  "norm_finalize",  "ns_gram", "ns_poly",
-                                         "ns_apply_mixed", "ns_apply", "ns_apply_final", "qk_proj",
-                                         "qk_causal_max", "qk_keys", "qk_clip", "mla_proj",
-                                         "mla_causal_max", "qk_clip_slices", "normuon_rows",
-                                         "normuon_apply"};
-struct ProfRec {
-  int kind;
-  cudaEvent_t b, e;
-  double flops, flops_exec, flops_dense, bytes;
-};
-thread_local bool t_prof = false;
-thread_local std::vector<ProfRec> t_recs;
-
-// Brackets one launch with CUDA events on its stream while profiling is on.
-struct ProfScope {
-  bool on = false;
-  ProfRec r{};
-  cudaStream_t s;
-  ProfScope(int kind, cudaStream_t st, double flops = 0, double flops_exec = 0, double bytes = 0,
-            double flops_dense = -1) : s(st) {
-    if (!t_prof) return;
-    r.kind = kind;
-    r.flops = flops;
-    r.flops_exec = flops_exec;
-    r.flops_dense = flops_dense < 0 ? flops : flops_dense;
-    r.bytes = bytes;
-    if (cudaEventCreate(&r.b) != cudaSuccess) return;
-    if (cudaEventCreate(&r.e) != cudaSuccess) {
-      cudaEventDestroy(r.b);
-      return;
-    }
-    on = cudaEventRecord(r.b, s) == cudaSuccess;
-  }
-  ~ProfScope() {
-    if (!on) return;
-    cudaEventRecord(r.e, s);
-    t_recs.push_back(r);
-  }
-};
 
 double gemm_exec_flops(const GemmParams& p) {
   double f = 0;
@@ -307,6 +357,102 @@ void finish_group(GemmParams& p, int gi, GemmGroup& G, int wide) {
   p.num_groups = gi + 1;
 }
 
+// Key-ring depth of qk_rowmax_kernel for a contraction of nkb k-blocks: as
+// many stages as fit beside the Q double buffer, at most RM_STAGES_MAX.
+int rowmax_stages(int nkb) {
+  const long long room = kSmemOptIn - 1024 - GEMM_BARRIER_BYTES - 4LL * SMEM_HEADS - 2LL * nkb * RM_KB_BYTES;
+  return static_cast<int>(std::min<long long>(RM_STAGES_MAX, room / RM_KB_BYTES));
+}
+
+// Per-head max of the score tiles, scores never stored.  `cm` holds the Q and
+// K maps (slot 1: the rotary part of a split contraction) and the group as
+// the tile GEMM takes them.  A contraction of at most RM_KB_MAX k-blocks runs
+// the row-owned kernel (Q resident, only key blocks stream); a longer one the
+// tile GEMM with the max epilogue.
+int launch_causal_max(const GemmParams& cm, const DeviceState& st, cudaStream_t s, int kind, double flops,
+                      bool profiled) {
+  const GemmGroup& G = cm.g[0];
+  const int nkb = (G.K + BK - 1) / BK;
+  const int stages = rowmax_stages(nkb);
+  if (nkb > RM_KB_MAX || stages < nkb) {
+    if (!profiled) {
+      if (cm.total_tiles > 0) MC_CUDA((launch_pairs<EPI_CAUSALMAX, 0>(cm, st.pair_clusters, s)));
+      return MC_OK;
+    }
+    return launch_gemm<EPI_CAUSALMAX, 0>(cm, st, s, kind, flops);
+  }
+  RowMaxParams R;
+  std::memset(&R, 0, sizeof(R));
+  R.map_q[0] = cm.map_a[0];
+  R.map_k[0] = cm.map_b[0];
+  R.map_q[1] = cm.map_a[1];
+  R.map_k[1] = cm.map_b[1];
+  R.S = G.M;
+  R.H = G.heads;
+  R.B = G.count / G.heads;
+  R.nkb = nkb;
+  R.k_split = G.k_split;
+  R.stages = stages;
+  R.causal = G.mask_causal;
+  R.nblk = (G.M + BM - 1) / BM;
+  R.tasks = static_cast<long long>(G.count) * R.nblk;
+  R.out_scale = G.out_scale;
+  R.keys = G.keys;
+  R.err = cm.err;
+  if (R.tasks <= 0) return MC_OK;
+  const double nb = R.nblk;
+  const double tiles = double(G.count) * (R.causal ? nb * (nb + 1) / 2 : nb * nb);
+  ProfScope prof(profiled ? kind : -1, s, flops, tiles * 2.0 * BM * MMA_N * nkb * BK);
+  const long long pairs = std::min<long long>(st.pair_clusters, R.tasks);
+  cudaLaunchConfig_t cfg = {};
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = 2;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.gridDim = dim3(static_cast<unsigned>(2 * pairs));
+  cfg.blockDim = dim3(GEMM_THREADS);
+  cfg.dynamicSmemBytes = rowmax_smem_bytes(nkb, stages);
+  cfg.stream = s;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  MC_CUDA(cudaLaunchKernelEx(&cfg, qk_rowmax_kernel, R));
+  return MC_OK;
+}
+
+// Newton-Schulz phases whose contraction is at most this long use the
+// 256 x 256 tile with two accumulators (WIDE = 0), so one tile's epilogue
+// overlaps the next tile's MMAs; longer ones the 256 x 512 tile with one
+// accumulator (WIDE = 1), which shares each A tile between two MMAs and so
+// stays under the per-SM operand feed limit, but exposes its epilogue.  With a
+// short contraction the main loop of a tile is short and the exposed epilogue
+// (its global reads and writes) would cost more than the narrower tile loses.
+constexpr int kNarrowMaxK = 2048;
+
+// Up to MAX_GROUPS problem groups of one launch, with their work figures.
+struct GemmBatch {
+  GemmParams p;
+  double f = 0, fd = 0;
+  int n = 0;
+};
+
+void add_to_batch(std::vector<GemmBatch>& v, const DeviceState& st, const CUtensorMap& ma, const CUtensorMap& mb,
+                  const GemmGroup& G, int wide, double flops, double flops_dense) {
+  if (v.empty() || v.back().n == MAX_GROUPS) {
+    v.emplace_back();
+    std::memset(&v.back().p, 0, sizeof(GemmParams));
+    v.back().p.err = st.err_ptr;
+  }
+  GemmBatch& b = v.back();
+  b.p.map_a[b.n] = ma;
+  b.p.map_b[b.n] = mb;
+  GemmGroup g = G;
+  finish_group(b.p, b.n, g, wide);
+  b.f += flops;
+  b.fd += flops_dense;
+  ++b.n;
+}
+
 // ------------------------------------------------------------------ muon plan
 struct NsGroup {
   int64_t rows = 0, cols = 0;
@@ -315,6 +461,7 @@ struct NsGroup {
   int64_t m = 0, n = 0;   // min, max
   int64_t ld = 0;         // row stride of the iterate
   int64_t ldm = 0;        // row stride of A and B
+  bool thin = false;       // m <= THIN_M (32): the fp32 CUDA-core iteration of thin_ns.cuh
   std::vector<int> members;
   int prob_base = 0;
   size_t off_xb[2] = {0, 0}, off_xl = 0, off_xf = 0, off_a = 0, off_b = 0, off_wptr = 0, off_uptr = 0;
@@ -330,6 +477,11 @@ struct MuonLayout {
   bool normuon = false;
   size_t off_ntab = 0, off_rowsq = 0, off_rowf = 0;
   long long total_rows = 0;
+  // thin matrices: ThinEntry[n_thin] inside the table block, the chunk
+  // partial sums of A and the P matrices
+  int n_thin = 0;
+  long long thin_ctas = 0;
+  size_t off_ttab = 0, off_tpart = 0, off_pmat = 0;
 };
 
 int validate_muon(const mc_param* params, int n, const mc_hparams* hp) {
@@ -378,6 +530,7 @@ void plan_muon(const mc_param* params, int n, MuonLayout& L, bool normuon = fals
       g.n = std::max(g.rows, g.cols);
       g.ld = round8(g.cols);
       g.ldm = round8(g.m);
+      g.thin = g.m <= THIN_M;
       index[key] = static_cast<int>(L.groups.size());
       L.groups.push_back(g);
       it = index.find(key);
@@ -414,6 +567,17 @@ void plan_muon(const mc_param* params, int n, MuonLayout& L, bool normuon = fals
     L.off_ntab = off;
     off += sizeof(NormEntry) * n;
   }
+  for (const auto& g : L.groups) {
+    if (!g.thin) continue;
+    for (size_t j = 0; j < g.members.size(); ++j)
+      L.thin_ctas += (g.n + THIN_COLS - 1) / THIN_COLS;
+    L.n_thin += static_cast<int>(g.members.size());
+  }
+  if (L.n_thin) {
+    off = align_up(off, 256);
+    L.off_ttab = off;
+    off += sizeof(ThinEntry) * size_t(L.n_thin);
+  }
   L.tab_bytes = off;
   off = align_up(off, 1024);
   L.off_partials = off;
@@ -424,14 +588,24 @@ void plan_muon(const mc_param* params, int n, MuonLayout& L, bool normuon = fals
     const size_t cnt = g.members.size();
     const size_t xe = cnt * size_t(g.rows) * size_t(g.ld);
     const size_t ae = cnt * size_t(g.m) * size_t(g.ldm);
-    g.off_xb[0] = off; off = align_up(off + 2 * xe, 1024);
+    g.off_xb[0] = off; off = align_up(off + 2 * xe, 1024);   // U's hi half (momentum kernel)
+    g.off_xl = off;    off = align_up(off + 2 * xe, 1024);   // U's lo half
+    if (g.thin) {        // fp32 iterate; no GEMM operands
+      g.off_xf = off;    off = align_up(off + 4 * xe, 1024);
+      continue;
+    }
     g.off_xb[1] = off; off = align_up(off + 2 * xe, 1024);
-    g.off_xl = off;    off = align_up(off + 2 * xe, 1024);
     if (normuon) {       // NorMuon's row pass reads the NS output in fp32
       g.off_xf = off;    off = align_up(off + 4 * xe, 1024);
     }
     g.off_a = off;     off = align_up(off + 2 * ae, 1024);
     g.off_b = off;     off = align_up(off + 2 * ae, 1024);
+  }
+  if (L.n_thin) {
+    L.off_tpart = off;
+    off = align_up(off + sizeof(float) * THIN_PAIRS * size_t(L.thin_ctas), 1024);
+    L.off_pmat = off;
+    off = align_up(off + sizeof(float) * THIN_PMAT * size_t(L.n_thin), 1024);
   }
   if (normuon) {
     for (int i = 0; i < n; ++i) L.total_rows += params[i].rows;
@@ -508,7 +682,7 @@ int validate_normuon(const mc_param* params, int n, const mc_normuon* nm) {
 }
 
 int run_muon(const mc_param* params, int n, const mc_hparams* hp, const mc_normuon* nm, void* workspace,
-             size_t workspace_bytes, float* norms_out, cudaStream_t s, uint8_t* tab_dev = nullptr);
+             size_t workspace_bytes, float* norms_out, cudaStream_t s, uint8_t* tab_dev);
 void build_muon_table(const mc_param* params, int n, const mc_hparams* hp, const mc_normuon* nm, uint8_t* ws,
                       const MuonLayout& L, uint8_t* tab);
 }  // namespace
@@ -536,40 +710,90 @@ std::vector<int> split_pieces(const mc_param* params, int n) {
   return b;
 }
 
-size_t pieces_workspace(const mc_param* params, int n, bool normuon) {
-  const std::vector<int> b = split_pieces(params, n);
-  size_t need = 0;
-  for (size_t k = 0; k + 1 < b.size(); ++k) {
-    MuonLayout L;
-    plan_muon(params + b[k], b[k + 1] - b[k], L, normuon);
-    need = std::max(need, L.total);
+// Workspace of a call that runs the list in pieces: one compute region that
+// every piece reuses in turn, then every piece's device tables, all built on
+// the host and uploaded in one copy at the start of the call (so the call
+// never waits on the host for an earlier piece).
+struct PiecesPlan {
+  std::vector<int> bounds;
+  std::vector<MuonLayout> layouts;
+  std::vector<size_t> tab_off;
+  size_t compute = 0, total = 0;
+};
+
+void plan_pieces(const mc_param* params, std::vector<int> bounds, bool normuon, PiecesPlan& P) {
+  P.bounds = std::move(bounds);
+  const int np = static_cast<int>(P.bounds.size()) - 1;
+  P.layouts.resize(static_cast<size_t>(np));
+  for (int k = 0; k < np; ++k) {
+    plan_muon(params + P.bounds[k], P.bounds[k + 1] - P.bounds[k], P.layouts[size_t(k)], normuon);
+    P.compute = std::max(P.compute, P.layouts[size_t(k)].total);
   }
-  return need;
+  size_t off = align_up(P.compute, 1024);
+  for (int k = 0; k < np; ++k) {
+    P.tab_off.push_back(off);
+    off = align_up(off + P.layouts[size_t(k)].tab_bytes, 256);
+  }
+  P.total = align_up(off, 1024);
 }
 
-// mc_muon_step / mc_normuon_step body: one run_muon per piece.
+size_t pieces_workspace(const mc_param* params, int n, bool normuon) {
+  PiecesPlan P;
+  plan_pieces(params, split_pieces(params, n), normuon, P);
+  return P.total;
+}
+
+// Every piece's tables, built on the host, in one upload (caller holds g_mu).
+int upload_piece_tables(DeviceState& st, const mc_param* params, const mc_hparams* hp, const mc_normuon* nm,
+                        const PiecesPlan& P, uint8_t* ws, cudaStream_t s) {
+  const size_t t0 = P.tab_off.front();
+  std::vector<uint8_t> tabs(P.total - t0, 0);
+  mc_normuon sub{};
+  for (size_t k = 0; k + 1 < P.bounds.size(); ++k) {
+    const mc_normuon* pn = nullptr;
+    if (nm) {
+      sub = *nm;
+      sub.v = nm->v + P.bounds[k];
+      pn = &sub;
+    }
+    build_muon_table(params + P.bounds[k], P.bounds[k + 1] - P.bounds[k], hp, pn, ws, P.layouts[k],
+                     tabs.data() + (P.tab_off[k] - t0));
+  }
+  return upload(st, tabs.data(), tabs.size(), ws + t0, s);
+}
+
+// mc_muon_step / mc_normuon_step body: the tables of every piece in one
+// upload, then one run_muon per piece.
 int run_pieces(const mc_param* params, int n, const mc_hparams* hp, const mc_normuon* nm, void* workspace,
                size_t workspace_bytes, float* norms_out, cudaStream_t s) {
-  const std::vector<int> b = split_pieces(params, n);
-  if (!workspace) {
-    // size the engine-owned buffer for the largest piece up front
+  PiecesPlan P;
+  plan_pieces(params, split_pieces(params, n), nm != nullptr, P);
+  uint8_t* ws = nullptr;
+  {
     std::lock_guard<std::mutex> lock(g_mu);
     DeviceState* st = nullptr;
     int rc = device_state(&st);
     if (rc != MC_OK) return rc;
-    workspace_bytes = pieces_workspace(params, n, nm != nullptr);
-    if ((rc = own_workspace(*st, workspace_bytes, &workspace)) != MC_OK) return rc;
+    if (workspace) {
+      if (workspace_bytes < P.total)
+        return fail(MC_ERR_NOSPC, "workspace has " + std::to_string(workspace_bytes) + " bytes, needs " +
+                                      std::to_string(P.total));
+    } else if ((rc = own_workspace(*st, P.total, &workspace)) != MC_OK) {
+      return rc;
+    }
+    ws = static_cast<uint8_t*>(workspace);
+    if ((rc = upload_piece_tables(*st, params, hp, nm, P, ws, s)) != MC_OK) return rc;
   }
   mc_normuon sub{};
-  for (size_t k = 0; k + 1 < b.size(); ++k) {
+  for (size_t k = 0; k + 1 < P.bounds.size(); ++k) {
     const mc_normuon* pn = nullptr;
     if (nm) {
       sub = *nm;
-      sub.v = nm->v + b[k];
+      sub.v = nm->v + P.bounds[k];
       pn = &sub;
     }
-    const int rc = run_muon(params + b[k], b[k + 1] - b[k], hp, pn, workspace, workspace_bytes,
-                            norms_out ? norms_out + b[k] : nullptr, s);
+    const int rc = run_muon(params + P.bounds[k], P.bounds[k + 1] - P.bounds[k], hp, pn, ws, P.compute,
+                            norms_out ? norms_out + P.bounds[k] : nullptr, s, ws + P.tab_off[k]);
     if (rc != MC_OK) return rc;
   }
   return MC_OK;
@@ -635,36 +859,17 @@ MC_API int mc_muon_step(const mc_param* params, int n, const mc_hparams* hp, voi
                     static_cast<cudaStream_t>(stream));
 }
 
-// Workspace of mc_muon_step_host_grads: one compute region that every piece
-// reuses in turn, then every piece's tables, all uploaded before the first
-// gradient copy.  (A table upload queued behind the gradient copies would
-// wait for all of them in the copy engine, and so would the first piece.)
-struct HostGradsPlan {
-  std::vector<int> bounds;
-  std::vector<MuonLayout> layouts;
-  std::vector<size_t> tab_off;
-  size_t compute = 0, total = 0;
-};
-
-void plan_host_grads(const mc_param* params, int n, int chunks, HostGradsPlan& P) {
-  P.bounds = split_chunks(params, n, chunks);
-  const int nch = static_cast<int>(P.bounds.size()) - 1;
-  P.layouts.resize(static_cast<size_t>(nch));
-  for (int k = 0; k < nch; ++k) {
-    plan_muon(params + P.bounds[k], P.bounds[k + 1] - P.bounds[k], P.layouts[size_t(k)]);
-    P.compute = std::max(P.compute, P.layouts[size_t(k)].total);
-  }
-  size_t off = align_up(P.compute, 1024);
-  for (int k = 0; k < nch; ++k) {
-    P.tab_off.push_back(off);
-    off = align_up(off + P.layouts[size_t(k)].tab_bytes, 256);
-  }
-  P.total = align_up(off, 1024);
+// Workspace of mc_muon_step_host_grads: as for mc_muon_step, with the pieces
+// of split_chunks.  Every piece's tables go up before the first gradient copy
+// (a table upload queued behind the gradient copies would wait for all of
+// them in the copy engine, and so would the first piece).
+void plan_host_grads(const mc_param* params, int n, int chunks, PiecesPlan& P) {
+  plan_pieces(params, split_chunks(params, n, chunks), false, P);
 }
 
 MC_API size_t mc_muon_host_grads_workspace_size(const mc_param* params, int n, const mc_hparams* hp, int chunks) {
   if (validate_muon(params, n, hp) != MC_OK || n == 0 || chunks < 1) return 0;
-  HostGradsPlan P;
+  PiecesPlan P;
   plan_host_grads(params, n, chunks, P);
   return P.total;
 }
@@ -680,7 +885,7 @@ MC_API int mc_muon_step_host_grads(const mc_param* params, const void* const* g_
   for (int i = 0; i < n; ++i)
     if (!g_host[i]) return fail(MC_ERR_INVAL, "g_host[" + std::to_string(i) + "] is NULL");
   if (n == 0) return MC_OK;
-  HostGradsPlan P;
+  PiecesPlan P;
   plan_host_grads(params, n, chunks, P);
   const std::vector<int>& b = P.bounds;
   const int nch = static_cast<int>(b.size()) - 1;
@@ -700,12 +905,7 @@ MC_API int mc_muon_step_host_grads(const mc_param* params, const void* const* g_
     }
     ws = static_cast<uint8_t*>(workspace);
     // every piece's tables, in one upload, ahead of the gradient copies
-    const size_t t0 = P.tab_off.front();
-    std::vector<uint8_t> tabs(P.total - t0, 0);
-    for (int k = 0; k < nch; ++k)
-      build_muon_table(params + b[k], b[k + 1] - b[k], hp, nullptr, ws, P.layouts[size_t(k)],
-                       tabs.data() + (P.tab_off[size_t(k)] - t0));
-    if ((rc = upload(*st, tabs.data(), tabs.size(), ws + t0, s)) != MC_OK) return rc;
+    if ((rc = upload_piece_tables(*st, params, hp, nullptr, P, ws, s)) != MC_OK) return rc;
     if (!st->copy_stream) MC_CUDA(cudaStreamCreateWithFlags(&st->copy_stream, cudaStreamNonBlocking));
     while (static_cast<int>(st->chunk_ev.size()) < nch + 1) {
       cudaEvent_t e;
@@ -772,6 +972,36 @@ void build_muon_table(const mc_param* params, int n, const mc_hparams* hp, const
       up[j] = q.update_out;
     }
   }
+  if (L.n_thin) {
+    ThinEntry* te = reinterpret_cast<ThinEntry*>(tab + L.off_ttab);
+    int t = 0, kk = 0;
+    long long ctas = 0;
+    for (const auto& g : L.groups) {
+      const size_t xe = size_t(g.rows) * size_t(g.ld);
+      for (size_t j = 0; j < g.members.size(); ++j, ++kk) {
+        if (!g.thin) continue;
+        const mc_param& q = params[g.members[j]];
+        ThinEntry& e = te[t];
+        e.xh = reinterpret_cast<const __nv_bfloat16*>(ws + g.off_xb[0]) + j * xe;
+        e.xl = reinterpret_cast<const __nv_bfloat16*>(ws + g.off_xl) + j * xe;
+        e.xf = reinterpret_cast<float*>(ws + g.off_xf) + j * xe;
+        e.w = nm ? nullptr : q.w;  // NorMuon keeps O in xf for its row pass
+        e.u = nm ? nullptr : q.update_out;
+        e.pmat = reinterpret_cast<float*>(ws + L.off_pmat) + size_t(t) * THIN_PMAT;
+        e.ld = g.ld;
+        e.cols = q.cols;
+        e.n = g.n;
+        e.cta_begin = ctas;
+        e.m = static_cast<int>(g.m);
+        e.tall = g.tall ? 1 : 0;
+        e.w_f32 = q.w_dtype == MC_F32;
+        e.prob = g.prob_base + static_cast<int>(j);
+        e.rms = hp->rms_scale * std::sqrt(static_cast<float>(std::max(q.rows, q.cols)));
+        ctas += (g.n + THIN_COLS - 1) / THIN_COLS;
+        ++t;
+      }
+    }
+  }
   if (nm) {
     NormEntry* ne = reinterpret_cast<NormEntry*>(tab + L.off_ntab);
     long long rb = 0;
@@ -795,8 +1025,7 @@ void build_muon_table(const mc_param* params, int n, const mc_hparams* hp, const
   }
 }
 
-// `tab_dev`: where the tables already are (uploaded by the caller), or NULL to
-// upload them to the start of the workspace here.
+// One piece of the list; `tab_dev`: where the caller uploaded its tables.
 int run_muon(const mc_param* params, int n, const mc_hparams* hp, const mc_normuon* nm, void* workspace,
              size_t workspace_bytes, float* norms_out, cudaStream_t s, uint8_t* tab_dev) {
   int rc = MC_OK;
@@ -815,15 +1044,8 @@ int run_muon(const mc_param* params, int n, const mc_hparams* hp, const mc_normu
   }
   uint8_t* ws = static_cast<uint8_t*>(workspace);
 
-  // ---- device tables
+  // ---- device tables (uploaded by the caller, ahead of every piece)
   uint8_t* tb = tab_dev;
-  if (!tb) {
-    tb = ws + L.off_tab;
-    std::vector<uint8_t> tab(L.tab_bytes, 0);
-    build_muon_table(params, n, hp, nm, ws, L, tab.data());
-    if ((rc = upload(*st, tab.data(), tab.size(), tb, s)) != MC_OK) return rc;
-  }
-
 
   // ---- momentum, Nesterov, fp32/bf16 iterate, norm partials
   const MomEntry* dtab = reinterpret_cast<const MomEntry*>(tb);
@@ -841,19 +1063,30 @@ int run_muon(const mc_param* params, int n, const mc_hparams* hp, const mc_normu
   {
     ProfScope prof(K_FINALIZE, s);
     norm_finalize_kernel<<<(n * 32 + 255) / 256, 256, 0, s>>>(dtab, n, partials, L.total_ctas, hp->eps, scale,
-                                                              norms_out);
+                                                              norms_out, st->err_ptr);
     MC_CUDA(cudaGetLastError());
   }
 
   // ---- tensor maps
   std::vector<GroupMaps> maps(L.groups.size());
-  for (size_t gi = 0; gi < L.groups.size(); ++gi)
+  std::vector<int> tc;  // groups on the tensor cores (the others take the thin path)
+  for (size_t gi = 0; gi < L.groups.size(); ++gi) {
+    if (L.groups[gi].thin) continue;
+    tc.push_back(static_cast<int>(gi));
     if ((rc = build_group_maps(L.groups[gi], ws, maps[gi])) != MC_OK) return rc;
+  }
+  const ThinEntry* ttab = reinterpret_cast<const ThinEntry*>(tb + L.off_ttab);
+  float* tpart = reinterpret_cast<float*>(ws + L.off_tpart);
+  double thin_flops = 0;
+  for (const auto& g : L.groups)
+    if (g.thin)
+      thin_flops += double(g.members.size()) * (4.0 * double(g.m) * double(g.m) * double(g.n) +
+                                                2.0 * double(g.m) * double(g.m) * double(g.m));
 
   // ---- Newton-Schulz iterations, MAX_GROUPS problem groups per launch.
   // Iterations it < kMixedIters take a*X from the hi + lo iterate; later ones
   // fold a*I into B (see the precision note in umma_gemm.cuh).
-  const int ng = static_cast<int>(L.groups.size());
+  const int ng = static_cast<int>(tc.size());
   for (int it = 0; it < hp->ns_steps; ++it) {
     const int par = it & 1;
     const bool first = it == 0, last = it + 1 == hp->ns_steps;
@@ -861,113 +1094,119 @@ int run_muon(const mc_param* params, int n, const mc_hparams* hp, const mc_normu
     const float ca = hp->coeffs ? hp->coeffs[3 * it] : hp->a;
     const float cb = hp->coeffs ? hp->coeffs[3 * it + 1] : hp->b;
     const float cc = hp->coeffs ? hp->coeffs[3 * it + 2] : hp->c;
-    for (int g0 = 0; g0 < ng; g0 += MAX_GROUPS) {
-      const int g1 = std::min(ng, g0 + MAX_GROUPS);
-      GemmParams gram, poly, apply;
-      double f_gram = 0, f_poly = 0, f_apply = 0, fd_gram = 0, fd_poly = 0;
-      std::memset(&gram, 0, sizeof(gram));
-      std::memset(&poly, 0, sizeof(poly));
-      std::memset(&apply, 0, sizeof(apply));
-      gram.err = poly.err = apply.err = st->err_ptr;
-      for (int gi = g0; gi < g1; ++gi) {
-        const int slot = gi - g0;
-        const NsGroup& g = L.groups[gi];
-        const GroupMaps& Mp = maps[gi];
-        const double cnt = double(g.members.size()), dm = double(g.m), dn = double(g.n);
-        f_gram += dm * (dm + 1) * dn * cnt;  // symmetric: entries on and above the diagonal
-        fd_gram += 2.0 * dm * dm * dn * cnt;
-        f_poly += dm * dm * (dm + 1) * cnt;
-        fd_poly += 2.0 * dm * dm * dm * cnt;
-        f_apply += 2.0 * dm * dm * dn * cnt;
-        // A = s^2 X X^T  (oriented; tall matrices read MN-major: X^T X)
-        GemmGroup G = base_group(g);
-        G.M = G.N = static_cast<int>(g.m);
-        G.K = static_cast<int>(g.n);
-        G.sched = SCHED_SYM;
-        G.a_mn = G.b_mn = g.tall ? 1 : 0;
-        G.d = ws + g.off_a;
-        G.d_ld = g.ldm;
-        G.d_bs = g.m * g.ldm;
-        G.scale = first ? scale : nullptr;
-        gram.map_a[slot] = g.tall ? Mp.x_mn[par] : Mp.x_k[par];
-        gram.map_b[slot] = g.tall ? Mp.x_mn[par] : Mp.x_k[par];
-        finish_group(gram, slot, G, 1);
-        // B = b A + c A A
-        G = base_group(g);
-        G.M = G.N = G.K = static_cast<int>(g.m);
-        G.sched = SCHED_SYM;
-        G.src = ws + g.off_a;
-        G.src_ld = g.ldm;
-        G.src_bs = g.m * g.ldm;
-        G.d = ws + g.off_b;
-        G.d_ld = g.ldm;
-        G.d_bs = g.m * g.ldm;
-        G.coef_acc = cc;
-        G.coef_src = cb;
-        G.diag = mixed ? 0.f : ca;
-        poly.map_a[slot] = Mp.a_k;
-        poly.map_b[slot] = Mp.a_k;
-        finish_group(poly, slot, G, 1);
-        // X' = s (a X + B X)   (tall: s (a X + X B), in the stored layout)
-        G = base_group(g);
-        G.M = static_cast<int>(g.rows);
-        G.N = static_cast<int>(g.cols);
-        G.K = static_cast<int>(g.m);
-        G.sched = SCHED_DENSE;
-        if (g.tall) {
-          G.a_mn = 0;
-          G.b_mn = 0;
-          apply.map_a[slot] = Mp.x_k[par];
-          apply.map_b[slot] = Mp.b_k;
-        } else {
-          G.a_mn = 0;
-          G.b_mn = 1;
-          apply.map_a[slot] = Mp.b_k;
-          apply.map_b[slot] = Mp.x_mn[par];
-        }
-        G.xh = reinterpret_cast<const __nv_bfloat16*>(ws + g.off_xb[par]);
-        G.xh_ld = g.ld;
-        G.xh_bs = g.rows * g.ld;
-        G.xl = reinterpret_cast<__nv_bfloat16*>(ws + g.off_xl);
-        G.xl_ld = g.ld;
-        G.xl_bs = g.rows * g.ld;
-        G.xf = nm ? reinterpret_cast<float*>(ws + g.off_xf) : nullptr;
-        G.xf_ld = g.ld;
-        G.xf_bs = g.rows * g.ld;
-        G.xf_read = mixed ? 1 : 0;
-        G.xl_write = (!last && it + 1 < kMixedIters) ? 1 : 0;
-        // NorMuon keeps the last iterate (the NS output O) in fp32 for the row pass.
-        G.xf_write = (last && nm) ? 1 : 0;
-        G.d = ws + g.off_xb[par ^ 1];
-        G.d_ld = g.ld;
-        G.d_bs = g.rows * g.ld;
-        G.scale = first ? scale : nullptr;
-        G.coef_src = ca;
-        if (last && !nm) {
-          G.w_ptrs = reinterpret_cast<void* const*>(tb + g.off_wptr);
-          bool any_u = false;
-          for (int i : g.members) any_u |= params[i].update_out != nullptr;
-          G.u_ptrs = any_u ? reinterpret_cast<float* const*>(tb + g.off_uptr) : nullptr;
-          G.w_f32 = g.w_f32;
-          G.w_vec = g.w_f32 ? (g.cols % 4 == 0) : (g.cols % 8 == 0);
-          G.rms = hp->rms_scale * std::sqrt(static_cast<float>(std::max(g.rows, g.cols)));
-          G.decay = 1.f - hp->lr * hp->wd;
-          G.step = -hp->lr * G.rms;
-        }
-        finish_group(apply, slot, G, 1);
-      }
-      // All NS phases use the 256 x 512 tile.  For the apply iterations that
-      // read (and write) the lo half of the iterate the exposed epilogue costs about what
-      // the narrower tile loses to the operand feed, and measured on one GPU
-      // the whole step was 2-3 % faster this way (the power cap).
-      if ((rc = launch_gemm<EPI_GRAM, 1>(gram, *st, s, K_GRAM, f_gram, fd_gram)) != MC_OK) return rc;
-      if ((rc = launch_gemm<EPI_POLY, 1>(poly, *st, s, K_POLY, f_poly, fd_poly)) != MC_OK) return rc;
+    // Batches of up to MAX_GROUPS problem groups per launch, one list per
+    // phase and tile shape (see kNarrowMaxK); every Gram launch of the
+    // iteration is enqueued before any polynomial launch, and those before
+    // any apply launch, so each group's three phases stay in order.
+    std::vector<GemmBatch> grams[2], polys[2], applies[2];
+    for (int ti = 0; ti < ng; ++ti) {
+      const int gi = tc[static_cast<size_t>(ti)];
+      const NsGroup& g = L.groups[gi];
+      const GroupMaps& Mp = maps[gi];
+      const double cnt = double(g.members.size()), dm = double(g.m), dn = double(g.n);
+      const int wide_gram = g.n > kNarrowMaxK ? 1 : 0;   // contraction n
+      const int wide_m = g.m > kNarrowMaxK ? 1 : 0;      // contraction m (polynomial, apply)
+      // A = s^2 X X^T  (oriented; tall matrices read MN-major: X^T X)
+      GemmGroup G = base_group(g);
+      G.M = G.N = static_cast<int>(g.m);
+      G.K = static_cast<int>(g.n);
+      G.sched = SCHED_SYM;
+      G.a_mn = G.b_mn = g.tall ? 1 : 0;
+      G.d = ws + g.off_a;
+      G.d_ld = g.ldm;
+      G.d_bs = g.m * g.ldm;
+      G.scale = first ? scale : nullptr;
+      // symmetric: the entries on and above the diagonal, 2n flops each
+      add_to_batch(grams[wide_gram], *st, g.tall ? Mp.x_mn[par] : Mp.x_k[par], g.tall ? Mp.x_mn[par] : Mp.x_k[par], G,
+                   wide_gram, dm * (dm + 1) * dn * cnt, 2.0 * dm * dm * dn * cnt);
+      // B = b A + c A A
+      G = base_group(g);
+      G.M = G.N = G.K = static_cast<int>(g.m);
+      G.sched = SCHED_SYM;
+      G.src = ws + g.off_a;
+      G.src_ld = g.ldm;
+      G.src_bs = g.m * g.ldm;
+      G.d = ws + g.off_b;
+      G.d_ld = g.ldm;
+      G.d_bs = g.m * g.ldm;
+      G.coef_acc = cc;
+      G.coef_src = cb;
+      G.diag = mixed ? 0.f : ca;
+      add_to_batch(polys[wide_m], *st, Mp.a_k, Mp.a_k, G, wide_m, dm * dm * (dm + 1) * cnt, 2.0 * dm * dm * dm * cnt);
+      // X' = s (a X + B X)   (tall: s (a X + X B), in the stored layout)
+      G = base_group(g);
+      G.M = static_cast<int>(g.rows);
+      G.N = static_cast<int>(g.cols);
+      G.K = static_cast<int>(g.m);
+      G.sched = SCHED_DENSE;
+      G.a_mn = 0;
+      G.b_mn = g.tall ? 0 : 1;
+      G.xh = reinterpret_cast<const __nv_bfloat16*>(ws + g.off_xb[par]);
+      G.xh_ld = g.ld;
+      G.xh_bs = g.rows * g.ld;
+      G.xl = reinterpret_cast<__nv_bfloat16*>(ws + g.off_xl);
+      G.xl_ld = g.ld;
+      G.xl_bs = g.rows * g.ld;
+      G.xf = nm ? reinterpret_cast<float*>(ws + g.off_xf) : nullptr;
+      G.xf_ld = g.ld;
+      G.xf_bs = g.rows * g.ld;
+      G.xf_read = mixed ? 1 : 0;
+      G.xl_write = (!last && it + 1 < kMixedIters) ? 1 : 0;
+      // NorMuon keeps the last iterate (the NS output O) in fp32 for the row pass.
+      G.xf_write = (last && nm) ? 1 : 0;
+      G.d = ws + g.off_xb[par ^ 1];
+      G.d_ld = g.ld;
+      G.d_bs = g.rows * g.ld;
+      G.scale = first ? scale : nullptr;
+      G.coef_src = ca;
       if (last && !nm) {
-        rc = launch_gemm<EPI_APPLY_FINAL, 1>(apply, *st, s, K_APPLY_FINAL, f_apply);
-      } else {
-        rc = launch_gemm<EPI_APPLY, 1>(apply, *st, s, mixed ? K_APPLY_MIXED : K_APPLY, f_apply);
+        G.w_ptrs = reinterpret_cast<void* const*>(tb + g.off_wptr);
+        bool any_u = false;
+        for (int i : g.members) any_u |= params[i].update_out != nullptr;
+        G.u_ptrs = any_u ? reinterpret_cast<float* const*>(tb + g.off_uptr) : nullptr;
+        G.w_f32 = g.w_f32;
+        G.w_vec = g.w_f32 ? (g.cols % 4 == 0) : (g.cols % 8 == 0);
+        G.rms = hp->rms_scale * std::sqrt(static_cast<float>(std::max(g.rows, g.cols)));
+        G.decay = 1.f - hp->lr * hp->wd;
+        G.step = -hp->lr * G.rms;
       }
+      const double fa = 2.0 * dm * dm * dn * cnt;
+      add_to_batch(applies[wide_m], *st, g.tall ? Mp.x_k[par] : Mp.b_k, g.tall ? Mp.b_k : Mp.x_mn[par], G, wide_m,
+                   fa, fa);
+    }
+    for (int w = 0; w < 2; ++w)
+      for (const auto& b : grams[w])
+        if ((rc = w ? launch_gemm<EPI_GRAM, 1>(b.p, *st, s, K_GRAM, b.f, b.fd)
+                    : launch_gemm<EPI_GRAM, 0>(b.p, *st, s, K_GRAM, b.f, b.fd)) != MC_OK)
+          return rc;
+    for (int w = 0; w < 2; ++w)
+      for (const auto& b : polys[w])
+        if ((rc = w ? launch_gemm<EPI_POLY, 1>(b.p, *st, s, K_POLY, b.f, b.fd)
+                    : launch_gemm<EPI_POLY, 0>(b.p, *st, s, K_POLY, b.f, b.fd)) != MC_OK)
+          return rc;
+    for (int w = 0; w < 2; ++w)
+      for (const auto& b : applies[w]) {
+        if (last && !nm) {
+          rc = w ? launch_gemm<EPI_APPLY_FINAL, 1>(b.p, *st, s, K_APPLY_FINAL, b.f)
+                 : launch_gemm<EPI_APPLY_FINAL, 0>(b.p, *st, s, K_APPLY_FINAL, b.f);
+        } else {
+          const int kind = mixed ? K_APPLY_MIXED : K_APPLY;
+          rc = w ? launch_gemm<EPI_APPLY, 1>(b.p, *st, s, kind, b.f) : launch_gemm<EPI_APPLY, 0>(b.p, *st, s, kind, b.f);
+        }
       if (rc != MC_OK) return rc;
+    }
+    if (L.n_thin) {
+      // thin matrices: fp32 Gram chunks, P = aI + bA + cA^2, X <- P X (the
+      // last iteration writes W, or keeps O for NorMuon)
+      ProfScope prof(K_NS_THIN, s, thin_flops, thin_flops);
+      thin_gram_kernel<<<static_cast<unsigned>(L.thin_ctas), THIN_THREADS, 0, s>>>(ttab, L.n_thin, tpart, scale,
+                                                                                  first ? 1 : 0);
+      MC_CUDA(cudaGetLastError());
+      thin_poly_kernel<<<static_cast<unsigned>(L.n_thin), THIN_THREADS, 0, s>>>(ttab, tpart, ca, cb, cc);
+      MC_CUDA(cudaGetLastError());
+      thin_apply_kernel<<<static_cast<unsigned>(L.thin_ctas), THIN_THREADS, 0, s>>>(
+          ttab, L.n_thin, last ? 1 : 0, 1.f - hp->lr * hp->wd, -hp->lr);
+      MC_CUDA(cudaGetLastError());
     }
   }
   if (nm) {
@@ -1111,7 +1350,7 @@ MC_API int mc_qk_max_logit(const void* x, const void* wq, const void* wk, int B,
     finish_group(cm, 0, G, 0);
   }
   const double pairs = causal ? double(S) * (double(S) + 1) / 2 : double(S) * S;
-  if ((rc = launch_gemm<EPI_CAUSALMAX, 0>(cm, *st, s, K_QK_CMAX, 2.0 * dh * pairs * B * H)) != MC_OK) return rc;
+  if ((rc = launch_causal_max(cm, *st, s, K_QK_CMAX, 2.0 * dh * pairs * B * H, true)) != MC_OK) return rc;
   {
     ProfScope prof(K_QK_KEYS, s);
     qk_keys_decode_kernel<<<(H + 255) / 256, 256, 0, s>>>(keys, smax_out, H);
@@ -1358,7 +1597,7 @@ MC_API int mc_mla_max_logit(const void* x, const void* wqc, const void* wkc, con
     finish_group(cm, 0, G, 0);
   }
   const double pairs = causal ? double(S) * (double(S) + 1) / 2 : double(S) * S;
-  if ((rc = launch_gemm<EPI_CAUSALMAX, 0>(cm, *st, s, K_MLA_CMAX, 2.0 * (dc + dr) * pairs * B * H)) != MC_OK)
+  if ((rc = launch_causal_max(cm, *st, s, K_MLA_CMAX, 2.0 * (dc + dr) * pairs * B * H, true)) != MC_OK)
     return rc;
   {
     ProfScope prof(K_QK_KEYS, s);
@@ -1368,16 +1607,48 @@ MC_API int mc_mla_max_logit(const void* x, const void* wqc, const void* wkc, con
   return MC_OK;
 }
 
+// Self-test of the bounded wait: one thread waits on an mbarrier that
+// expects an arrival nobody makes, so the wait runs out after `limit` cycles,
+// raises the abort flag and sets the device error word, and the kernel
+// returns normally.
+namespace mc {
+__global__ void bounded_wait_selftest_kernel(int* err, long long limit) {
+  __shared__ uint64_t bar;
+  __shared__ int abort_flag;
+  if (threadIdx.x == 0) {
+    mbar_init(smem_u32(&bar), 1);
+    abort_flag = 0;
+    fence_mbar_init();
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) wait_bounded(smem_u32(&bar), 0, &abort_flag, err, limit);
+}
+}  // namespace mc
+
+MC_API int mc_selftest_bounded_wait(long long limit_cycles, void* stream) {
+  if (limit_cycles < 1000 || limit_cycles > kWaitLimitCycles)
+    return fail(MC_ERR_INVAL, "limit_cycles must be in [1000, 2^32]");
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  std::lock_guard<std::mutex> lock(g_mu);
+  DeviceState* st = nullptr;
+  const int rc = device_state(&st);
+  if (rc != MC_OK) return rc;
+  bounded_wait_selftest_kernel<<<1, 32, 0, s>>>(st->err_ptr, limit_cycles);
+  MC_CUDA(cudaGetLastError());
+  return MC_OK;
+}
+
 MC_API int mc_device_status(void) {
   MC_CUDA(cudaDeviceSynchronize());
   int v = 0;
   MC_CUDA(cudaMemcpyFromSymbol(&v, g_device_error, sizeof(int)));
-  if (v != 0) {
-    const int zero = 0;
-    MC_CUDA(cudaMemcpyToSymbol(g_device_error, &zero, sizeof(int)));
-    return fail(MC_ERR_DEVICE, "a kernel abandoned a bounded wait (device error " + std::to_string(v) + ")");
-  }
-  return MC_OK;
+  if (v == 0) return MC_OK;
+  const int zero = 0;
+  MC_CUDA(cudaMemcpyToSymbol(g_device_error, &zero, sizeof(int)));
+  if (v & MC_DEV_ERR_TIMEOUT)
+    return fail(MC_ERR_DEVICE, "a kernel abandoned a bounded wait (device error word " + std::to_string(v) + ")");
+  return fail(MC_ERR_NONFINITE, "a Muon step met a non-finite Newton-Schulz input (a NaN or Inf gradient or "
+                                "momentum); that matrix's norms_out entry is not finite and its W only decayed");
 }
 
 // =========================================================================
@@ -1661,7 +1932,7 @@ MC_API int mc_qk_max_logit_static(const void* x, const void* wq, const void* wk,
   G.keys = keys;
   G.out_scale = 1.f / std::sqrt(static_cast<float>(dh));
   finish_group(cm, 0, G, 0);
-  if ((rc = launch_gemm_unprofiled<EPI_CAUSALMAX, 0>(cm, *st, s)) != MC_OK) return rc;
+  if ((rc = launch_causal_max(cm, *st, s, -1, 0, false)) != MC_OK) return rc;
 
   qk_keys_decode_kernel<<<(H + 255) / 256, 256, 0, s>>>(keys, smax_out, H);
   MC_CUDA(cudaGetLastError());

@@ -18,7 +18,9 @@ constexpr long long kWaitLimitCycles = 1ll << 32;
 // Bound used while draining in-flight copies on the way out.
 constexpr long long kDrainLimitCycles = 1ll << 27;
 
-enum DeviceError : int { MC_DEV_OK = 0, MC_DEV_ERR_TIMEOUT = 1 };
+// Bits of the device error word (set with atomicOr, read and cleared by
+// mc_device_status).
+enum DeviceError : int { MC_DEV_OK = 0, MC_DEV_ERR_TIMEOUT = 1, MC_DEV_ERR_NONFINITE = 2 };
 
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));
@@ -62,7 +64,7 @@ __device__ __forceinline__ bool wait_bounded(uint32_t bar, uint32_t parity, vola
     if (*abort) return false;
     if (clock64() - t0 > limit) {
       *abort = 1;
-      if (err) atomicExch(err, MC_DEV_ERR_TIMEOUT);
+      if (err) atomicOr(err, MC_DEV_ERR_TIMEOUT);
       return false;
     }
   }

@@ -8,7 +8,10 @@
 //                    MuonClip: orthogonalised updates for LLM training", §2
 //                    Frobenius normalisation.)
 //  norm_finalize     sums each matrix's partials in a fixed order (bitwise
-//                    deterministic) and stores s = 1 / max(||U||_F, eps).
+//                    deterministic) and stores s = 1 / max(||U||_F, eps); a
+//                    non-finite ||U||_F (U holds a NaN or Inf) gives s = 0,
+//                    which the first Newton-Schulz products turn into a zero
+//                    iterate, and raises MC_DEV_ERR_NONFINITE.
 //  qk_keys_*         order-preserving int encoding of the per-head S_max.
 //  qk_clip_kernel    gamma_h = tau / S_max_h when S_max_h > tau; rows of head h
 //                    in W_q scaled by gamma^alpha, in W_k by gamma^(1-alpha)
@@ -170,10 +173,12 @@ __global__ void __launch_bounds__(MOM_THREADS) momentum_kernel(const MomEntry* _
   }
 }
 
-// One warp per matrix.
+// One warp per matrix.  The fp64 sum of squares of finite fp32 values cannot
+// overflow (at most 2^36 terms below 2^256 each), so the norm is finite
+// exactly when every element of U is.
 __global__ void norm_finalize_kernel(const MomEntry* __restrict__ tab, int n, const double* __restrict__ partials,
                                      long long total_ctas, float eps, float* __restrict__ scale,
-                                     float* __restrict__ norms_out) {
+                                     float* __restrict__ norms_out, int* __restrict__ err) {
   const int i = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
   const int lane = threadIdx.x & 31;
   if (i >= n) return;
@@ -186,7 +191,9 @@ __global__ void norm_finalize_kernel(const MomEntry* __restrict__ tab, int n, co
   if (lane == 0) {
     const double nrm = sqrt(s);
     const double den = nrm > static_cast<double>(eps) ? nrm : static_cast<double>(eps);
-    scale[i] = static_cast<float>(1.0 / den);
+    const bool finite = isfinite(nrm);
+    scale[i] = finite ? static_cast<float>(1.0 / den) : 0.f;
+    if (!finite && err) atomicOr(err, MC_DEV_ERR_NONFINITE);
     if (norms_out) norms_out[tab[i].orig] = static_cast<float>(nrm);
   }
 }

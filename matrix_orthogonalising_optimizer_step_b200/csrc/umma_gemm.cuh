@@ -411,9 +411,10 @@ __device__ __forceinline__ void epi_finish(const GemmGroup& G, int prob, int r, 
       const float s = G.scale[G.prob_base + prob];
       s2 = s * s;
     }
+    // s = 0 marks a non-finite NS input: its Gram is zero, not NaN
     float o[16];
 #pragma unroll
-    for (int j = 0; j < 16; ++j) o[j] = v[j] * s2;
+    for (int j = 0; j < 16; ++j) o[j] = s2 == 0.f ? 0.f : v[j] * s2;
     __nv_bfloat16* D = static_cast<__nv_bfloat16*>(G.d) + (long long)prob * G.d_bs;
     store_sym_chunk(D, G.d_ld, G.M, r, c0, o);
   } else if constexpr (EPI == EPI_POLY) {
@@ -437,6 +438,10 @@ __device__ __forceinline__ void epi_finish(const GemmGroup& G, int prob, int r, 
     } else {
 #pragma unroll
       for (int j = 0; j < 16; ++j) o[j] = s * v[j];
+    }
+    if (s == 0.f) {  // a non-finite NS input: the first iterate is zero, not NaN
+#pragma unroll
+      for (int j = 0; j < 16; ++j) o[j] = 0.f;
     }
     if constexpr (EPI == EPI_APPLY) {
       float* X = G.xf_write ? G.xf + (long long)prob * G.xf_bs + (long long)r * G.xf_ld : nullptr;

@@ -35,7 +35,7 @@ def w64(w):
 
 @pytest.mark.parametrize("B,S,D,H,dc,dr", [(2, 300, 64, 3, 64, 32), (1, 129, 40, 2, 128, 64),
                                            (3, 700, 96, 4, 64, 8), (1, 1, 16, 1, 64, 16),
-                                           (2, 520, 256, 2, 128, 72)])
+                                           (2, 520, 256, 2, 128, 72), (1, 300, 64, 2, 256, 64)])
 @pytest.mark.parametrize("causal", [True, False])
 def test_mla_smax_small(B, S, D, H, dc, dr, causal):
     X, w = wl.mla_inputs(B, S, D, H, dc, dr, seed=13, w_std=0.2)

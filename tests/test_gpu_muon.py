@@ -95,6 +95,24 @@ def test_ragged_and_tall_wide_shapes(hp):
     check_all(mats, hp, run_step(mats, hp), "ragged")
 
 
+THIN = [(2, 70000), (70000, 2), (32, 1024), (1024, 32), (12, 1025), (1025, 12), (16, 16), (32, 32),
+        (31, 33), (33, 31)]
+
+
+def test_thin_matrices_and_the_tensor_core_boundary(hp):
+    """Short side <= 32: the fp32 thin path (several 256-column chunks, a
+    chunk boundary, both orientations), in one call beside matrices just past
+    the boundary that take the tensor-core GEMMs."""
+    shapes = THIN + [(33, 90), (90, 33), (48, 48)]
+    mats = [wl.generic_matrix(r, c, seed=500 + i) for i, (r, c) in enumerate(shapes)]
+    mats.append(wl.generic_matrix(24, 700, seed=600, w_dtype=torch.float32, g_dtype=torch.float32))
+    errs = check_all(mats, hp, run_step(mats, hp), "thin")
+    # the thin path is fp32 throughout: far inside the bound
+    for (r, c), e in zip(shapes, errs):
+        if min(r, c) <= 32:
+            assert e[0] < 1e-4, ((r, c), e[0])
+
+
 def test_mixed_dtypes_and_repeated_shapes(hp):
     f32, bf = torch.float32, torch.bfloat16
     mats = []
