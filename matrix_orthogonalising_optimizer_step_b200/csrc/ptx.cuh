@@ -85,9 +85,14 @@ __device__ __forceinline__ uint32_t mapa_shared(uint32_t addr, uint32_t rank) {
 __device__ __forceinline__ void cluster_sync() {
   asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
 }
-// Arrive once on an mbarrier given by its shared::cluster address (may be a peer CTA's).
+// Arrive once on an mbarrier given by its shared::cluster address (may be a
+// peer CTA's), with release semantics at CTA scope.  The epilogues use it to
+// hand an accumulator back after tcgen05.wait::ld and
+// tcgen05.fence::before_thread_sync, which already order their TMEM reads; a
+// cluster-scope release would also make every arrive wait until the warp's
+// earlier global stores are performed at cluster scope.
 __device__ __forceinline__ void mbar_arrive_cluster(uint32_t cluster_addr) {
-  asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr) : "memory");
+  asm volatile("mbarrier.arrive.release.cta.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr) : "memory");
 }
 
 // ------------------------------------------------------------------- TMA

@@ -13,8 +13,9 @@
 // that reloads both operands moves), and the per-head running max stays in
 // registers for the whole task.  The score matrix is never stored.
 //
-// Tasks are taken longest first (query block nblk-1 first under the causal
-// mask), task t by pair t mod npairs.  The contraction may be split in two
+// Tasks go head by head (all query blocks of one (b, h) in a row, the longest
+// first under the causal mask), task t to pair t mod npairs, so the pairs that
+// work on one head at the same time share its key blocks in L2.  The contraction may be split in two
 // (multi-head latent attention: content columns [0, k_split) from operand
 // slot 0, rotary columns from slot 1, whose key has one head shared by all).
 //
@@ -62,10 +63,16 @@ struct RmTask {
   int b, h, i, jn;  // jn: key blocks of this task
 };
 
+// Task order: head-major takes all query blocks of one (b, h) in a row, so
+// that the pairs working on one head at the same time share its key blocks in
+// L2; level-major (false) takes every (b, h) at one query-block level before
+// the next.  Measured on the B4 S4096 H32 dh128 layer: 0.272 against 0.273 ms.
+constexpr bool kRowmaxHeadMajor = true;
+
 __device__ __forceinline__ RmTask rowmax_task(const RowMaxParams& P, long long t) {
   const long long bh_count = (long long)P.B * P.H;
-  const int level = static_cast<int>(t / bh_count);
-  const long long bh = t - (long long)level * bh_count;
+  const int level = kRowmaxHeadMajor ? static_cast<int>(t % P.nblk) : static_cast<int>(t / bh_count);
+  const long long bh = kRowmaxHeadMajor ? t / P.nblk : t - (long long)level * bh_count;
   RmTask k;
   k.i = P.causal ? P.nblk - 1 - level : level;
   k.b = static_cast<int>(bh / P.H);

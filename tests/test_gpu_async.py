@@ -67,3 +67,26 @@ def test_many_calls_queue_without_waiting(hp):
     assert mc.device_status() == mc.MC_OK, mc.last_error()
     assert busy
     assert host_s < 0.5, host_s
+
+
+def test_thirty_third_queued_copy_waits_for_the_oldest(hp):
+    """The staging pool holds 32 buffers: behind a stream that stays busy for
+    a second, 32 calls queue at once and the 33rd waits (on the host) until
+    the first call's table copy has run, i.e. until the busy kernel ends."""
+    Ws = [torch.randn((128, 192), device=DEV).to(torch.bfloat16) * 0.02]
+    Gs = [torch.randn((128, 192), device=DEV).to(torch.bfloat16) * 1e-3]
+    Ms = [torch.zeros((128, 192), device=DEV)]
+    for _ in range(40):   # the pool reaches its 32 buffers
+        mc.muon_step(Ws, Gs, Ms, **hp)
+    torch.cuda.synchronize()
+    _busy_stream(1.0)
+    t0 = time.perf_counter()
+    for _ in range(32):
+        mc.muon_step(Ws, Gs, Ms, **hp)
+    queued_s = time.perf_counter() - t0
+    mc.muon_step(Ws, Gs, Ms, **hp)
+    waited_s = time.perf_counter() - t0 - queued_s
+    torch.cuda.synchronize()
+    assert mc.device_status() == mc.MC_OK, mc.last_error()
+    assert queued_s < 0.5, queued_s
+    assert waited_s > 0.2, waited_s
