@@ -47,7 +47,7 @@ WORKLOAD = ("7B-shaped Muon step (224 matrices, 7.78e9 params, bf16 W/G, fp32 M,
 # proportional to the matrices processed, so the per-launch figure is this
 # times the layers one launch covers.  Kinds without a capture of the kernel
 # as it stands are absent (reported as null).
-KERNEL_TRAFFIC_PER_LAYER = {"ns_gram": 1.103e9, "ns_apply": 1.700e9}
+KERNEL_TRAFFIC_PER_LAYER = {"ns_gram": 1.087e9, "ns_apply": 1.711e9}
 
 # Pieces the end-to-end step splits the gradient upload into.
 E2E_CHUNKS = 16
@@ -463,7 +463,9 @@ def run_config(args, cfg):
                              l2="inputs larger than L2" if cfg == 4 else "inputs fit in L2 (no flush)")
         # the oracle on the host cores: the whole config (0, 1), or one matrix
         # per shape class scaled by the class counts (4)
-        if cfg in (0, 1):
+        if args.no_cpu_baseline:
+            out["cpu_baseline"] = None
+        elif cfg in (0, 1):
             host = mats
             t0 = time.perf_counter()
             for W, G, M in host:
@@ -478,9 +480,10 @@ def run_config(args, cfg):
                 oracle.muon_step(W.double().numpy(), G.double().numpy(), M.double().numpy(), **hp)
                 cpu_s += (time.perf_counter() - t0) * count
             sample, extrap = "one 2048x7168 and one 7168x2048 matrix, scaled by the class counts (128, 64)", True
-        out["cpu_baseline"] = {"value": dense / cpu_s / 1e12, "unit": "TFLOP/s", "cores": blas_threads(),
-                               "kind": "oracle", "sample": sample, "ms_per_step": cpu_s * 1e3,
-                               "extrapolated": bool(extrap), "cpu_model": cpu_model(), "nproc": os.cpu_count()}
+        if not args.no_cpu_baseline:
+            out["cpu_baseline"] = {"value": dense / cpu_s / 1e12, "unit": "TFLOP/s", "cores": blas_threads(),
+                                   "kind": "oracle", "sample": sample, "ms_per_step": cpu_s * 1e3,
+                                   "extrapolated": bool(extrap), "cpu_model": cpu_model(), "nproc": os.cpu_count()}
     else:
         c3 = wl.CFG3
         B, S, D, H, dh = c3["B"], c3["S"], c3["D"], c3["H"], c3["dh"]
@@ -511,13 +514,15 @@ def run_config(args, cfg):
                                (k["qk_causal_max"]["total_ms"] / 1e3) / 1e12,
                                "clipped_heads": [int(h) for h in np.nonzero(mask.cpu().numpy())[0]]})
         out["config"].update(tokens=B * S, flops_per_layer=qf, l2="inputs larger than L2 (X 134 MB, Q/K 268 MB)")
-        t0 = time.perf_counter()
-        oracle.qk_max_logit(X.double().numpy(), Wq.double().numpy(), Wk.double().numpy(), H, dh, causal=True)
-        cpu_s = time.perf_counter() - t0
-        out["cpu_baseline"] = {"value": B * S / cpu_s, "unit": "tokens/s", "cores": blas_threads(), "kind": "oracle",
-                               "sample": f"the whole layer's S_max in fp64, {cpu_s:.1f} s",
-                               "ms_per_step": cpu_s * 1e3, "extrapolated": False, "cpu_model": cpu_model(),
-                               "nproc": os.cpu_count()}
+        out["cpu_baseline"] = None
+        if not args.no_cpu_baseline:
+            t0 = time.perf_counter()
+            oracle.qk_max_logit(X.double().numpy(), Wq.double().numpy(), Wk.double().numpy(), H, dh, causal=True)
+            cpu_s = time.perf_counter() - t0
+            out["cpu_baseline"] = {"value": B * S / cpu_s, "unit": "tokens/s", "cores": blas_threads(),
+                                   "kind": "oracle", "sample": f"the whole layer's S_max in fp64, {cpu_s:.1f} s",
+                                   "ms_per_step": cpu_s * 1e3, "extrapolated": False, "cpu_model": cpu_model(),
+                                   "nproc": os.cpu_count()}
     out["kernels"] = {n: dict(v, ms_per_launch=v["total_ms"] / max(v["launches"], 1)) for n, v in k.items()}
     out["roofline"] = _roofline_row(k, peaks, reps)
     out["gpu_launches"] = sum(v["launches"] for n, v in k.items() if n != "table_upload")
