@@ -128,6 +128,8 @@ int device_state(DeviceState** out) {
     MC_CUDA((set_gemm_attr<EPI_POLY, 0>()));
     MC_CUDA((set_gemm_attr<EPI_APPLY, 0>()));
     MC_CUDA((set_gemm_attr<EPI_APPLY_FINAL, 0>()));
+    MC_CUDA((set_gemm_attr<EPI_APPLY_MIXED, 1>()));
+    MC_CUDA((set_gemm_attr<EPI_APPLY_MIXED, 0>()));
     MC_CUDA((set_gemm_attr<EPI_STORE, 1>()));
     MC_CUDA((set_gemm_attr<EPI_CAUSALMAX, 0>()));
     MC_CUDA(cudaFuncSetAttribute(qk_rowmax_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemOptIn));
@@ -1189,9 +1191,11 @@ int run_muon(const mc_param* params, int n, const mc_hparams* hp, const mc_normu
         if (last && !nm) {
           rc = w ? launch_gemm<EPI_APPLY_FINAL, 1>(b.p, *st, s, K_APPLY_FINAL, b.f)
                  : launch_gemm<EPI_APPLY_FINAL, 0>(b.p, *st, s, K_APPLY_FINAL, b.f);
+        } else if (mixed) {
+          rc = w ? launch_gemm<EPI_APPLY_MIXED, 1>(b.p, *st, s, K_APPLY_MIXED, b.f)
+                 : launch_gemm<EPI_APPLY_MIXED, 0>(b.p, *st, s, K_APPLY_MIXED, b.f);
         } else {
-          const int kind = mixed ? K_APPLY_MIXED : K_APPLY;
-          rc = w ? launch_gemm<EPI_APPLY, 1>(b.p, *st, s, kind, b.f) : launch_gemm<EPI_APPLY, 0>(b.p, *st, s, kind, b.f);
+          rc = w ? launch_gemm<EPI_APPLY, 1>(b.p, *st, s, K_APPLY, b.f) : launch_gemm<EPI_APPLY, 0>(b.p, *st, s, K_APPLY, b.f);
         }
       if (rc != MC_OK) return rc;
     }

@@ -8,10 +8,11 @@
 //                                                  each element stored twice;
 //                                                  dead diagonal blocks skipped)
 //   EPI_POLY        B_k   = b*A + c*(A A) [+ a*I]  (symmetric, mirrored store)
-//   EPI_APPLY       X_k+1 = s * (a*X + B X)        (a*X from the hi + lo copy of
-//                           or  P X, P = aI+bA+cA^2  the iterate; stores the bf16
-//                                                  iterate, its lo half when flagged,
-//                                                  and the fp32 NS output for NorMuon)
+//   EPI_APPLY_MIXED X_k+1 = s * (a*X + B X)        (a*X from the hi + lo copy of the
+//                                                  iterate; stores the bf16 iterate
+//                                                  and, when flagged, its lo half)
+//   EPI_APPLY       X_k+1 = P X, P = aI+bA+cA^2    (stores the bf16 iterate, and the
+//                                                  fp32 NS output for NorMuon)
 //   EPI_APPLY_FINAL W     = (1 - lr*wd) W - lr * rms * X_N   (last iteration; X_N
 //                                                  never touches memory)
 //
@@ -107,13 +108,36 @@ enum Epi : int {
   EPI_APPLY = 2,
   EPI_APPLY_FINAL = 3,
   EPI_STORE = 4,
-  EPI_CAUSALMAX = 5
+  EPI_CAUSALMAX = 5,
+  EPI_APPLY_MIXED = 6   // EPI_APPLY whose a*X term comes from the iterate's hi + lo halves
 };
+
+// The apply epilogues: X' = s(aX + BX) (EPI_APPLY_MIXED, a*X from hi + lo),
+// X' = P X (EPI_APPLY) and the last iteration's weight update (EPI_APPLY_FINAL,
+// either form, chosen at run time by xf_read).
+template <int EPI>
+__host__ __device__ constexpr bool is_apply_epi() {
+  return EPI == EPI_APPLY || EPI == EPI_APPLY_MIXED || EPI == EPI_APPLY_FINAL;
+}
+
+
+// Epilogues that move bf16 row blocks to or from global memory stage them
+// through one 4 KiB shared-memory buffer per epilogue warp (32 rows x 64
+// columns); see warp_rows_from_frags / warp_store_rows64.
+constexpr int EPI_BUF_BYTES = 32 * 64 * 2;
+template <int EPI>
+__host__ __device__ constexpr bool epi_uses_row_buffers() {
+  return EPI == EPI_GRAM || EPI == EPI_POLY || is_apply_epi<EPI>() || EPI == EPI_STORE;
+}
 
 template <int EPI, int WIDE>
 constexpr size_t gemm_smem_bytes() {
-  return EPI == EPI_CAUSALMAX ? TileCfg<WIDE>::SMEM_BYTES_HEADS : TileCfg<WIDE>::SMEM_BYTES;
+  return EPI == EPI_CAUSALMAX ? TileCfg<WIDE>::SMEM_BYTES_HEADS
+                              : TileCfg<WIDE>::SMEM_BYTES +
+                                    (epi_uses_row_buffers<EPI>() ? size_t(NUM_EPI_WARPS) * EPI_BUF_BYTES : 0);
 }
+static_assert(TileCfg<1>::SMEM_BYTES + size_t(NUM_EPI_WARPS) * EPI_BUF_BYTES <= 232448, "shared memory per CTA");
+static_assert(TileCfg<0>::SMEM_BYTES + size_t(NUM_EPI_WARPS) * EPI_BUF_BYTES <= 232448, "shared memory per CTA");
 
 struct GemmGroup {
   int M, N, K;             // D is M x N, contraction K
@@ -154,6 +178,13 @@ struct GemmGroup {
   float decay, step, rms;  // EPI_APPLY_FINAL
   float out_scale;         // EPI_CAUSALMAX: 1/sqrt(d_head)
 };
+
+template <int EPI>
+__device__ __forceinline__ bool apply_reads_x(const GemmGroup& G) {
+  if constexpr (EPI == EPI_APPLY_MIXED) return true;
+  else if constexpr (EPI == EPI_APPLY) return false;
+  else return G.xf_read != 0;
+}
 
 struct GemmParams {
   CUtensorMap map_a[MAX_GROUPS];
@@ -382,8 +413,8 @@ __device__ __forceinline__ void epi_prefetch(const GemmGroup& G, int prob, int r
     const __nv_bfloat16* S =
         static_cast<const __nv_bfloat16*>(G.src) + (long long)prob * G.src_bs + (long long)r * G.src_ld;
     raw_load_bf16x16(S + c0, valid, true, pre.x);
-  } else if constexpr (EPI == EPI_APPLY || EPI == EPI_APPLY_FINAL) {
-    if (G.xf_read) {
+  } else if constexpr (is_apply_epi<EPI>()) {
+    if (apply_reads_x<EPI>(G)) {
       const __nv_bfloat16* Xh = G.xh + (long long)prob * G.xh_bs + (long long)r * G.xh_ld;
       const __nv_bfloat16* Xl = G.xl + (long long)prob * G.xl_bs + (long long)r * G.xl_ld;
       raw_load_bf16x16(Xh + c0, valid, true, pre.x[0], pre.x[1]);
@@ -426,11 +457,11 @@ __device__ __forceinline__ void epi_finish(const GemmGroup& G, int prob, int r, 
     for (int j = 0; j < 16; ++j) o[j] = fmaf(G.coef_acc, v[j], G.coef_src * x[j]) + (c0 + j == r ? G.diag : 0.f);
     __nv_bfloat16* D = static_cast<__nv_bfloat16*>(G.d) + (long long)prob * G.d_bs;
     store_sym_chunk(D, G.d_ld, G.M, r, c0, o);
-  } else if constexpr (EPI == EPI_APPLY || EPI == EPI_APPLY_FINAL) {
+  } else if constexpr (is_apply_epi<EPI>()) {
     if (r >= G.M) return;
     const float s = G.scale ? G.scale[G.prob_base + prob] : 1.f;
     float o[16];
-    if (G.xf_read) {
+    if (apply_reads_x<EPI>(G)) {
       float x[16];
       raw_hilo_to_f32x16(pre.x, x);
 #pragma unroll
@@ -443,7 +474,7 @@ __device__ __forceinline__ void epi_finish(const GemmGroup& G, int prob, int r, 
 #pragma unroll
       for (int j = 0; j < 16; ++j) o[j] = 0.f;
     }
-    if constexpr (EPI == EPI_APPLY) {
+    if constexpr (EPI == EPI_APPLY || EPI == EPI_APPLY_MIXED) {
       float* X = G.xf_write ? G.xf + (long long)prob * G.xf_bs + (long long)r * G.xf_ld : nullptr;
       __nv_bfloat16* XL = G.xl_write ? G.xl + (long long)prob * G.xl_bs + (long long)r * G.xl_ld : nullptr;
       __nv_bfloat16* D =
@@ -538,6 +569,256 @@ __device__ __forceinline__ void epi_finish(const GemmGroup& G, int prob, int r, 
       }
     }
   }
+}
+
+// ---------------------------------------------------- coalesced row blocks
+// The accumulator gives each epilogue thread one row of the tile, so a warp's
+// 16-byte accesses to global memory would each touch 32 rows (32 L1
+// wavefronts).  Whole blocks of 32 rows x 64 bf16 columns go through the
+// warp's shared-memory buffer instead: global memory is read and written four
+// 128-byte row segments per warp instruction, and each thread reads or writes
+// its own row in shared memory.  The buffer's 16-byte chunks are XOR-swizzled
+// by row, so neither side has bank conflicts.
+__device__ __forceinline__ uint32_t epi_swz(int row, int chunk) {
+  return static_cast<uint32_t>(row * 128 + ((chunk ^ (row & 7)) << 4));
+}
+
+// Fragments of rows 0..31, columns 0..63 of the block at `base` (row stride
+// ld elements): fragment k of lane l is row 4k + l/8, columns 8(l%8)..+7.
+__device__ __forceinline__ void warp_issue_rows64(const __nv_bfloat16* base, long long ld, int lane, uint4 (&g)[8]) {
+#pragma unroll
+  for (int k = 0; k < 8; ++k)
+    g[k] = *reinterpret_cast<const uint4*>(base + (long long)(4 * k + (lane >> 3)) * ld + (lane & 7) * 8);
+}
+
+// The fragments, regrouped so that lane l holds row l: out[i] = columns 2i, 2i+1.
+__device__ __forceinline__ void warp_rows_from_frags(const uint4 (&g)[8], int lane, uint8_t* buf, uint32_t (&out)[32]) {
+#pragma unroll
+  for (int k = 0; k < 8; ++k) *reinterpret_cast<uint4*>(buf + epi_swz(4 * k + (lane >> 3), lane & 7)) = g[k];
+  __syncwarp();
+#pragma unroll
+  for (int c = 0; c < 8; ++c) {
+    const uint4 v = *reinterpret_cast<const uint4*>(buf + epi_swz(lane, c));
+    out[4 * c] = v.x;
+    out[4 * c + 1] = v.y;
+    out[4 * c + 2] = v.z;
+    out[4 * c + 3] = v.w;
+  }
+  __syncwarp();
+}
+
+// Lane l's row `in` (bf16 pairs) to row l of the block at `base`.
+__device__ __forceinline__ void warp_store_rows64(__nv_bfloat16* base, long long ld, int lane, uint8_t* buf,
+                                                  const uint32_t (&in)[32]) {
+#pragma unroll
+  for (int c = 0; c < 8; ++c)
+    *reinterpret_cast<uint4*>(buf + epi_swz(lane, c)) = make_uint4(in[4 * c], in[4 * c + 1], in[4 * c + 2], in[4 * c + 3]);
+  __syncwarp();
+#pragma unroll
+  for (int k0 = 0; k0 < 8; k0 += 4) {  // four fragments at a time (registers)
+    uint4 g[4];
+#pragma unroll
+    for (int k = 0; k < 4; ++k)
+      g[k] = *reinterpret_cast<const uint4*>(buf + epi_swz(4 * (k0 + k) + (lane >> 3), lane & 7));
+#pragma unroll
+    for (int k = 0; k < 4; ++k)
+      *reinterpret_cast<uint4*>(base + (long long)(4 * (k0 + k) + (lane >> 3)) * ld + (lane & 7) * 8) = g[k];
+  }
+  __syncwarp();
+}
+
+// The same for blocks of 32 rows x 32 columns (64-byte rows; 2 KiB of the
+// buffer), for the epilogue that holds two operands: fragment k of lane l is
+// row 8k + l/4, columns 8(l%4)..+7; chunks are swizzled by (row / 2) % 4.
+__device__ __forceinline__ uint32_t epi_swz32(int row, int chunk) {
+  return static_cast<uint32_t>(row * 64 + ((chunk ^ ((row >> 1) & 3)) << 4));
+}
+__device__ __forceinline__ void warp_issue_rows32(const __nv_bfloat16* base, long long ld, int lane, uint4 (&g)[4]) {
+#pragma unroll
+  for (int k = 0; k < 4; ++k)
+    g[k] = *reinterpret_cast<const uint4*>(base + (long long)(8 * k + (lane >> 2)) * ld + (lane & 3) * 8);
+}
+__device__ __forceinline__ void warp_rows_from_frags32(const uint4 (&g)[4], int lane, uint8_t* buf, uint32_t (&out)[16]) {
+#pragma unroll
+  for (int k = 0; k < 4; ++k) *reinterpret_cast<uint4*>(buf + epi_swz32(8 * k + (lane >> 2), lane & 3)) = g[k];
+  __syncwarp();
+#pragma unroll
+  for (int c = 0; c < 4; ++c) {
+    const uint4 v = *reinterpret_cast<const uint4*>(buf + epi_swz32(lane, c));
+    out[4 * c] = v.x;
+    out[4 * c + 1] = v.y;
+    out[4 * c + 2] = v.z;
+    out[4 * c + 3] = v.w;
+  }
+  __syncwarp();
+}
+__device__ __forceinline__ void warp_store_rows32(__nv_bfloat16* base, long long ld, int lane, uint8_t* buf,
+                                                  const uint32_t (&in)[16]) {
+#pragma unroll
+  for (int c = 0; c < 4; ++c)
+    *reinterpret_cast<uint4*>(buf + epi_swz32(lane, c)) = make_uint4(in[4 * c], in[4 * c + 1], in[4 * c + 2], in[4 * c + 3]);
+  __syncwarp();
+  uint4 g[4];
+#pragma unroll
+  for (int k = 0; k < 4; ++k) g[k] = *reinterpret_cast<const uint4*>(buf + epi_swz32(8 * k + (lane >> 2), lane & 3));
+#pragma unroll
+  for (int k = 0; k < 4; ++k)
+    *reinterpret_cast<uint4*>(base + (long long)(8 * k + (lane >> 2)) * ld + (lane & 3) * 8) = g[k];
+  __syncwarp();
+}
+
+__device__ __forceinline__ void pack_row64(const float (&o)[64], uint32_t (&out)[32]) {
+#pragma unroll
+  for (int i = 0; i < 32; ++i) out[i] = pack_bf16x2(o[2 * i], o[2 * i + 1]);
+}
+__device__ __forceinline__ float bf16_lo(uint32_t w) { return __uint_as_float(w << 16); }
+__device__ __forceinline__ float bf16_hi(uint32_t w) { return __uint_as_float(w & 0xFFFF0000u); }
+
+// Whether a warp's 32 x 64 block (rows r0.., columns c0..) takes the
+// coalesced path: every row and column in range, rows 16-byte aligned, no
+// fp32 operand, and for the symmetric outputs every column strictly above
+// every row (the block's elements are all stored directly and mirrored).
+// Columns of the blocks that take the coalesced path: 32 for the epilogue that
+// holds two operands (EPI_APPLY_MIXED), 64 for the others.
+template <int EPI>
+__host__ __device__ constexpr int epi_fast_cols() {
+  return EPI == EPI_APPLY_MIXED ? 32 : 64;
+}
+
+template <int EPI>
+__device__ __forceinline__ bool epi_fast_ok(const GemmGroup& G, int prob, int r0, int c0) {
+  if (r0 + 32 > G.M || c0 + epi_fast_cols<EPI>() > G.N) return false;
+  if constexpr (EPI == EPI_GRAM || EPI == EPI_POLY) {
+    if (c0 <= r0 + 31 || (G.d_ld & 7) != 0) return false;
+    if constexpr (EPI == EPI_POLY) {
+      if ((G.src_ld & 7) != 0) return false;
+    }
+    return true;
+  } else if constexpr (EPI == EPI_APPLY || EPI == EPI_APPLY_MIXED) {
+    if (G.xf_write || (G.d_ld & 7) != 0 || (G.xl_write && (G.xl_ld & 7) != 0)) return false;
+    if (EPI == EPI_APPLY_MIXED && ((G.xh_ld | G.xl_ld) & 7) != 0) return false;
+    return true;
+  } else if constexpr (EPI == EPI_APPLY_FINAL) {
+    return !G.xf_read && !G.w_f32 && G.w_vec && !(G.u_ptrs && G.u_ptrs[prob]);
+  } else if constexpr (EPI == EPI_STORE) {
+    return (G.d_ld & 7) == 0;
+  } else {
+    return false;
+  }
+}
+
+// The epilogue of one warp's 32 x 64 block through the coalesced path (see
+// epi_finish for what each epilogue computes; EPI_APPLY_MIXED has its own,
+// epi_fast32_mixed).  The block's global operand is requested first, then its
+// accumulator columns are read from TMEM.
+template <int EPI>
+__device__ __forceinline__ void epi_fast64(const GemmGroup& G, int prob, int r0, int c0, int lane, uint32_t taddr,
+                                           uint8_t* buf) {
+  static_assert(EPI != EPI_APPLY_MIXED, "the mixed apply uses epi_fast32_mixed");
+  uint4 ga[8];
+  if constexpr (EPI == EPI_POLY) {
+    warp_issue_rows64(static_cast<const __nv_bfloat16*>(G.src) + (long long)prob * G.src_bs + (long long)r0 * G.src_ld + c0,
+                      G.src_ld, lane, ga);
+  } else if constexpr (EPI == EPI_APPLY_FINAL) {
+    warp_issue_rows64(static_cast<const __nv_bfloat16*>(G.w_ptrs[prob]) + (long long)r0 * G.N + c0, G.N, lane, ga);
+  }
+  float v[64];  // the accumulator columns, turned into the block's outputs in place
+  tmem_ld64(taddr, v);
+  uint32_t pk[32];
+  if constexpr (EPI == EPI_GRAM) {
+    float s2 = 1.f;
+    if (G.scale) {
+      const float sc = G.scale[G.prob_base + prob];
+      s2 = sc * sc;
+    }
+#pragma unroll
+    for (int j = 0; j < 64; ++j) v[j] = s2 == 0.f ? 0.f : v[j] * s2;
+  } else if constexpr (EPI == EPI_POLY) {
+    uint32_t x[32];
+    warp_rows_from_frags(ga, lane, buf, x);
+#pragma unroll
+    for (int i = 0; i < 32; ++i) {
+      v[2 * i] = fmaf(G.coef_acc, v[2 * i], G.coef_src * bf16_lo(x[i]));
+      v[2 * i + 1] = fmaf(G.coef_acc, v[2 * i + 1], G.coef_src * bf16_hi(x[i]));
+    }
+  } else if constexpr (is_apply_epi<EPI>()) {
+    const float sc = G.scale ? G.scale[G.prob_base + prob] : 1.f;
+    {
+#pragma unroll
+      for (int j = 0; j < 64; ++j) v[j] = sc * v[j];
+    }
+    if (sc == 0.f) {  // a non-finite NS input: the first iterate is zero, not NaN
+#pragma unroll
+      for (int j = 0; j < 64; ++j) v[j] = 0.f;
+    }
+  }
+
+  if constexpr (EPI == EPI_GRAM || EPI == EPI_POLY) {
+    __nv_bfloat16* D = static_cast<__nv_bfloat16*>(G.d) + (long long)prob * G.d_bs;
+    pack_row64(v, pk);
+    warp_store_rows64(D + (long long)r0 * G.d_ld + c0, G.d_ld, lane, buf, pk);
+    // the mirror image: column c0+j of rows r0..r0+31 is one 64-byte segment
+    // of row c0+j, written by the warp in one store
+    unsigned short* pm = reinterpret_cast<unsigned short*>(D + (long long)c0 * G.d_ld + r0 + lane);
+    const long long ld = G.d_ld;
+#pragma unroll
+    for (int i = 0; i < 32; ++i) {
+      pm[0] = static_cast<unsigned short>(pk[i] & 0xFFFFu);
+      pm[ld] = static_cast<unsigned short>(pk[i] >> 16);
+      pm += 2 * ld;
+    }
+  } else if constexpr (EPI == EPI_APPLY) {
+    __nv_bfloat16* D = static_cast<__nv_bfloat16*>(G.d) + (long long)prob * G.d_bs + (long long)r0 * G.d_ld + c0;
+    pack_row64(v, pk);
+    warp_store_rows64(D, G.d_ld, lane, buf, pk);
+  } else if constexpr (EPI == EPI_APPLY_FINAL) {
+    warp_rows_from_frags(ga, lane, buf, pk);
+#pragma unroll
+    for (int i = 0; i < 32; ++i)
+      pk[i] = pack_bf16x2(fmaf(G.step, v[2 * i], G.decay * bf16_lo(pk[i])),
+                          fmaf(G.step, v[2 * i + 1], G.decay * bf16_hi(pk[i])));
+    warp_store_rows64(static_cast<__nv_bfloat16*>(G.w_ptrs[prob]) + (long long)r0 * G.N + c0, G.N, lane, buf, pk);
+  } else if constexpr (EPI == EPI_STORE) {
+    pack_row64(v, pk);
+    warp_store_rows64(static_cast<__nv_bfloat16*>(G.d) + (long long)prob * G.d_bs + (long long)r0 * G.d_ld + c0,
+                      G.d_ld, lane, buf, pk);
+  }
+}
+
+// EPI_APPLY_MIXED through the coalesced path, a 32 x 32 block: X' = s(aX + BX)
+// with aX from the iterate's hi and lo halves, stored as bf16 (and its lo
+// half when flagged).
+__device__ __forceinline__ void epi_fast32_mixed(const GemmGroup& G, int prob, int r0, int c0, int lane,
+                                                 uint32_t taddr, uint8_t* buf) {
+  uint4 gh[4], gl[4];
+  warp_issue_rows32(G.xh + (long long)prob * G.xh_bs + (long long)r0 * G.xh_ld + c0, G.xh_ld, lane, gh);
+  warp_issue_rows32(G.xl + (long long)prob * G.xl_bs + (long long)r0 * G.xl_ld + c0, G.xl_ld, lane, gl);
+  float v[32];
+  tmem_ld16(taddr, *reinterpret_cast<float(*)[16]>(v));
+  tmem_ld16(taddr + 16, *reinterpret_cast<float(*)[16]>(v + 16));
+  uint32_t xh[16], xl[16];
+  warp_rows_from_frags32(gh, lane, buf, xh);
+  warp_rows_from_frags32(gl, lane, buf, xl);
+  const float sc = G.scale ? G.scale[G.prob_base + prob] : 1.f;
+#pragma unroll
+  for (int i = 0; i < 16; ++i) {
+    v[2 * i] = sc * fmaf(G.coef_src, bf16_lo(xh[i]) + bf16_lo(xl[i]), v[2 * i]);
+    v[2 * i + 1] = sc * fmaf(G.coef_src, bf16_hi(xh[i]) + bf16_hi(xl[i]), v[2 * i + 1]);
+  }
+  if (sc == 0.f) {  // a non-finite NS input: the first iterate is zero, not NaN
+#pragma unroll
+    for (int j = 0; j < 32; ++j) v[j] = 0.f;
+  }
+  // hi = bf16(o) and lo = bf16(o - hi)
+#pragma unroll
+  for (int i = 0; i < 16; ++i) {
+    xh[i] = pack_bf16x2(v[2 * i], v[2 * i + 1]);
+    xl[i] = pack_bf16x2(v[2 * i] - bf16_lo(xh[i]), v[2 * i + 1] - bf16_hi(xh[i]));
+  }
+  warp_store_rows32(static_cast<__nv_bfloat16*>(G.d) + (long long)prob * G.d_bs + (long long)r0 * G.d_ld + c0, G.d_ld,
+                    lane, buf, xh);
+  if (G.xl_write)
+    warp_store_rows32(G.xl + (long long)prob * G.xl_bs + (long long)r0 * G.xl_ld + c0, G.xl_ld, lane, buf, xl);
 }
 
 // Chunks per batch.  One for the NS phases: measured against batches of four
@@ -759,6 +1040,7 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1) umma_gemm_kernel(const __grid
     constexpr int WCOLS = T::N / EPI_COL_GROUPS;  // columns per epilogue warp
     const int q = warp & 3;                       // TMEM lane quarter this warp may read
     const int half = (warp - 2) >> 2;             // which column group of the tile
+    uint8_t* epi_buf = smem + STAGES * STAGE_BYTES + GEMM_BARRIER_BYTES + (warp - 2) * EPI_BUF_BYTES;
     uint32_t tempty_leader[NACC];
 #pragma unroll
     for (int b = 0; b < NACC; ++b) tempty_leader[b] = mapa_shared(smem_u32(&tempty_bar[b]), 0);
@@ -785,10 +1067,24 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1) umma_gemm_kernel(const __grid
       // Last row of this warp: a chunk that starts beyond it lies above the
       // diagonal for every lane, as do all later chunks (causal max only).
       const int r_warp_last = ti.tm * BM + HALF * static_cast<int>(rank) + q * 32 + 31;
+      const int r0w = r_warp_last - 31;             // first row of this warp
 #pragma unroll 1
       for (int cb = 0; cb < (idle ? 0 : WCOLS / 16); cb += CH) {
         if constexpr (EPI == EPI_CAUSALMAX) {
           if (G.mask_causal && cbase + cb * 16 > r_warp_last) break;
+        }
+        if constexpr (epi_uses_row_buffers<EPI>()) {
+          // a whole 32-row block through the coalesced path when it can
+          constexpr int FB = epi_fast_cols<EPI>() / 16;
+          if (cb % FB == 0 && epi_fast_ok<EPI>(G, ti.prob, r0w, cbase + cb * 16)) {
+            if constexpr (EPI == EPI_APPLY_MIXED) {
+              epi_fast32_mixed(G, ti.prob, r0w, cbase + cb * 16, lane, t_row + cb * 16, epi_buf);
+            } else {
+              epi_fast64<EPI>(G, ti.prob, r0w, cbase + cb * 16, lane, t_row + cb * 16, epi_buf);
+            }
+            cb += FB - 1;
+            continue;
+          }
         }
         EpiPre pre[CH];
 #pragma unroll
