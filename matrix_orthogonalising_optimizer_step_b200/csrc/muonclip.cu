@@ -279,9 +279,9 @@ int own_workspace(DeviceState& st, size_t bytes, void** ws) {
   return MC_OK;
 }
 
-// bf16 tensor map, 128-byte swizzle, zero fill out of bounds.
+// bf16 tensor map (128-byte swizzle unless given), zero fill out of bounds.
 int make_map(CUtensorMap* map, const void* base, int rank, const uint64_t* dims, const uint64_t* strides,
-             const uint32_t* box) {
+             const uint32_t* box, CUtensorMapSwizzle swizzle = CU_TENSOR_MAP_SWIZZLE_128B) {
   cuuint64_t gd[5], gs[4];
   cuuint32_t bx[5], es[5];
   for (int i = 0; i < rank; ++i) {
@@ -291,19 +291,32 @@ int make_map(CUtensorMap* map, const void* base, int rank, const uint64_t* dims,
   }
   for (int i = 0; i + 1 < rank; ++i) gs[i] = strides[i];
   const CUresult r = g_encode(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, rank, const_cast<void*>(base), gd, gs, bx, es,
-                              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                              CU_TENSOR_MAP_INTERLEAVE_NONE, swizzle,
                               CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   if (r != CUDA_SUCCESS) return fail(MC_ERR_CUDA, "cuTensorMapEncodeTiled failed with code " + std::to_string(r));
   return MC_OK;
 }
 
-// [count][rows][ld] bf16, box {64, box_rows, 1}
+// [count][rows][ld] bf16, box {box_cols, box_rows, 1}
 int map_batched(CUtensorMap* map, const void* base, int64_t count, int64_t rows, int64_t cols, int64_t ld,
-                uint32_t box_rows) {
+                uint32_t box_rows, uint32_t box_cols = 64, CUtensorMapSwizzle swizzle = CU_TENSOR_MAP_SWIZZLE_128B) {
   const uint64_t dims[3] = {uint64_t(cols), uint64_t(rows), uint64_t(count)};
   const uint64_t strides[2] = {uint64_t(ld) * 2, uint64_t(rows) * uint64_t(ld) * 2};
-  const uint32_t box[3] = {64, box_rows, 1};
-  return make_map(map, base, 3, dims, strides, box);
+  const uint32_t box[3] = {box_cols, box_rows, 1};
+  return make_map(map, base, 3, dims, strides, box, swizzle);
+}
+
+// Epilogue map of a [count][rows][ld] bf16 matrix for the coalesced tensor
+// path: boxes of 32 rows x 64 columns (128-byte swizzle) or, when `narrow`,
+// 32 x 32 (64-byte swizzle).  `*ok` is false (and nothing is encoded) when the
+// matrix is smaller than one box; the epilogue then keeps its other paths.
+int map_epilogue(CUtensorMap* map, bool* ok, const void* base, int64_t count, int64_t rows, int64_t cols, int64_t ld,
+                 bool narrow) {
+  const uint32_t bc = narrow ? 32 : 64;
+  *ok = rows >= 32 && cols >= bc && ld % 8 == 0;
+  if (!*ok) return MC_OK;
+  return map_batched(map, base, count, rows, cols, ld, 32, bc,
+                     narrow ? CU_TENSOR_MAP_SWIZZLE_64B : CU_TENSOR_MAP_SWIZZLE_128B);
 }
 
 double gemm_exec_flops(const GemmParams& p) {
@@ -413,7 +426,7 @@ int launch_causal_max(const GemmParams& cm, const DeviceState& st, cudaStream_t 
   attr[0].val.clusterDim.y = 1;
   attr[0].val.clusterDim.z = 1;
   cfg.gridDim = dim3(static_cast<unsigned>(2 * pairs));
-  cfg.blockDim = dim3(GEMM_THREADS);
+  cfg.blockDim = dim3(RM_THREADS);
   cfg.dynamicSmemBytes = rowmax_smem_bytes(nkb, stages);
   cfg.stream = s;
   cfg.attrs = attr;
@@ -438,8 +451,11 @@ struct GemmBatch {
   int n = 0;
 };
 
+// eo / ei / ei2: the group's epilogue maps (output, inputs), or NULL: when eo
+// is given the group's full blocks move by tensor copies (GemmGroup::tma_epi).
 void add_to_batch(std::vector<GemmBatch>& v, const DeviceState& st, const CUtensorMap& ma, const CUtensorMap& mb,
-                  const GemmGroup& G, int wide, double flops, double flops_dense) {
+                  const GemmGroup& G, int wide, double flops, double flops_dense, const CUtensorMap* eo = nullptr,
+                  const CUtensorMap* ei = nullptr, const CUtensorMap* ei2 = nullptr) {
   if (v.empty() || v.back().n == MAX_GROUPS) {
     v.emplace_back();
     std::memset(&v.back().p, 0, sizeof(GemmParams));
@@ -449,6 +465,10 @@ void add_to_batch(std::vector<GemmBatch>& v, const DeviceState& st, const CUtens
   b.p.map_a[b.n] = ma;
   b.p.map_b[b.n] = mb;
   GemmGroup g = G;
+  g.tma_epi = eo != nullptr ? 1 : 0;
+  if (eo) b.p.map_eo[b.n] = *eo;
+  if (ei) b.p.map_ei[b.n] = *ei;
+  if (ei2) b.p.map_ei2[b.n] = *ei2;
   finish_group(b.p, b.n, g, wide);
   b.f += flops;
   b.fd += flops_dense;
@@ -623,6 +643,10 @@ void plan_muon(const mc_param* params, int n, MuonLayout& L, bool normuon = fals
 // operand); MN-major maps use {64, 64} boxes.
 struct GroupMaps {
   CUtensorMap x_k[2], x_mn[2], a_k, b_k;
+  // epilogue maps (see map_epilogue): A and B, the iterate by 64 and by 32
+  // columns, its lo half by 32 columns
+  CUtensorMap a_e, b_e, x_e64[2], x_e32[2], xl_e32;
+  bool ok_ab = false, ok_x64 = false, ok_x32 = false;
 };
 
 int build_group_maps(const NsGroup& g, uint8_t* ws, GroupMaps& M) {
@@ -636,6 +660,15 @@ int build_group_maps(const NsGroup& g, uint8_t* ws, GroupMaps& M) {
   int rc;
   if ((rc = map_batched(&M.a_k, ws + g.off_a, cnt, g.m, g.m, g.ldm, HALF)) != MC_OK) return rc;
   if ((rc = map_batched(&M.b_k, ws + g.off_b, cnt, g.m, g.m, g.ldm, HALF)) != MC_OK) return rc;
+  bool ok = true;
+  if ((rc = map_epilogue(&M.a_e, &M.ok_ab, ws + g.off_a, cnt, g.m, g.m, g.ldm, false)) != MC_OK) return rc;
+  if ((rc = map_epilogue(&M.b_e, &ok, ws + g.off_b, cnt, g.m, g.m, g.ldm, false)) != MC_OK) return rc;
+  for (int par = 0; par < 2; ++par) {
+    const void* xb = ws + g.off_xb[par];
+    if ((rc = map_epilogue(&M.x_e64[par], &M.ok_x64, xb, cnt, g.rows, g.cols, g.ld, false)) != MC_OK) return rc;
+    if ((rc = map_epilogue(&M.x_e32[par], &M.ok_x32, xb, cnt, g.rows, g.cols, g.ld, true)) != MC_OK) return rc;
+  }
+  if ((rc = map_epilogue(&M.xl_e32, &ok, ws + g.off_xl, cnt, g.rows, g.cols, g.ld, true)) != MC_OK) return rc;
   return MC_OK;
 }
 
@@ -1120,7 +1153,7 @@ int run_muon(const mc_param* params, int n, const mc_hparams* hp, const mc_normu
       G.scale = first ? scale : nullptr;
       // symmetric: the entries on and above the diagonal, 2n flops each
       add_to_batch(grams[wide_gram], *st, g.tall ? Mp.x_mn[par] : Mp.x_k[par], g.tall ? Mp.x_mn[par] : Mp.x_k[par], G,
-                   wide_gram, dm * (dm + 1) * dn * cnt, 2.0 * dm * dm * dn * cnt);
+                   wide_gram, dm * (dm + 1) * dn * cnt, 2.0 * dm * dm * dn * cnt, Mp.ok_ab ? &Mp.a_e : nullptr);
       // B = b A + c A A
       G = base_group(g);
       G.M = G.N = G.K = static_cast<int>(g.m);
@@ -1134,7 +1167,8 @@ int run_muon(const mc_param* params, int n, const mc_hparams* hp, const mc_normu
       G.coef_acc = cc;
       G.coef_src = cb;
       G.diag = mixed ? 0.f : ca;
-      add_to_batch(polys[wide_m], *st, Mp.a_k, Mp.a_k, G, wide_m, dm * dm * (dm + 1) * cnt, 2.0 * dm * dm * dm * cnt);
+      add_to_batch(polys[wide_m], *st, Mp.a_k, Mp.a_k, G, wide_m, dm * dm * (dm + 1) * cnt, 2.0 * dm * dm * dm * cnt,
+                   Mp.ok_ab ? &Mp.b_e : nullptr, &Mp.a_e);
       // X' = s (a X + B X)   (tall: s (a X + X B), in the stored layout)
       G = base_group(g);
       G.M = static_cast<int>(g.rows);
@@ -1173,8 +1207,22 @@ int run_muon(const mc_param* params, int n, const mc_hparams* hp, const mc_normu
         G.step = -hp->lr * G.rms;
       }
       const double fa = 2.0 * dm * dm * dn * cnt;
+      // epilogue maps: none for the last apply (each weight has its own
+      // pointer); the iterate by 32 columns with its lo half for the mixed
+      // apply, by 64 columns for the plain one
+      const bool final_apply = last && !nm;
+      const CUtensorMap* eo = nullptr;
+      const CUtensorMap* ei = nullptr;
+      const CUtensorMap* ei2 = nullptr;
+      if (!final_apply && mixed && Mp.ok_x32) {
+        eo = &Mp.x_e32[par ^ 1];
+        ei = &Mp.x_e32[par];
+        ei2 = &Mp.xl_e32;
+      } else if (!final_apply && !mixed && Mp.ok_x64) {
+        eo = &Mp.x_e64[par ^ 1];
+      }
       add_to_batch(applies[wide_m], *st, g.tall ? Mp.x_k[par] : Mp.b_k, g.tall ? Mp.b_k : Mp.x_mn[par], G, wide_m,
-                   fa, fa);
+                   fa, fa, eo, ei, ei2);
     }
     for (int w = 0; w < 2; ++w)
       for (const auto& b : grams[w])
@@ -1323,6 +1371,10 @@ MC_API int mc_qk_max_logit(const void* x, const void* wq, const void* wk, int B,
     G.band = 8;
     G.d = ws + (which == 0 ? L.off_q : L.off_k);
     G.d_ld = HD;
+    // the projection's full 32 x 64 output blocks leave by tensor stores
+    bool e_ok = false;
+    if ((rc = map_epilogue(&proj.map_eo[which], &e_ok, G.d, 1, BS, HD, HD, false)) != MC_OK) return rc;
+    G.tma_epi = e_ok ? 1 : 0;
     finish_group(proj, which, G, 1);
   }
   if ((rc = launch_gemm<EPI_STORE, 1>(proj, *st, s, K_QK_PROJ, 2.0 * 2.0 * double(BS) * HD * D)) != MC_OK)
@@ -1562,6 +1614,10 @@ MC_API int mc_mla_max_logit(const void* x, const void* wqc, const void* wkc, con
     G.band = 8;
     G.d = ws + offs[which];
     G.d_ld = outs[which];
+    bool e_ok = false;
+    if ((rc = map_epilogue(&proj.map_eo[which], &e_ok, G.d, 1, BS, outs[which], outs[which], false)) != MC_OK)
+      return rc;
+    G.tma_epi = e_ok ? 1 : 0;
     finish_group(proj, which, G, 1);
     proj_flops += 2.0 * double(BS) * outs[which] * D;
   }
@@ -1910,6 +1966,10 @@ MC_API int mc_qk_max_logit_static(const void* x, const void* wq, const void* wk,
     G.band = 8;
     G.d = which == 0 ? q : k;
     G.d_ld = HD;
+    // the projection's full 32 x 64 output blocks leave by tensor stores
+    bool e_ok = false;
+    if ((rc = map_epilogue(&proj.map_eo[which], &e_ok, G.d, 1, BS, HD, HD, false)) != MC_OK) return rc;
+    G.tma_epi = e_ok ? 1 : 0;
     finish_group(proj, which, G, 1);
   }
   if ((rc = launch_gemm_unprofiled<EPI_STORE, 1>(proj, *st, s)) != MC_OK) return rc;

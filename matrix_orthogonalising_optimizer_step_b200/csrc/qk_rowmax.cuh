@@ -19,11 +19,11 @@
 // (multi-head latent attention: content columns [0, k_split) from operand
 // slot 0, rotary columns from slot 1, whose key has one head shared by all).
 //
-// Warp roles (320 threads per CTA), as in umma_gemm.cuh:
+// Warp roles (RM_THREADS per CTA), as in umma_gemm.cuh:
 //   warp 0      TMA producer: the task's Q block, then the key k-blocks
 //   warp 1      TMEM allocation; in the leader CTA one thread issues the MMAs
-//   warps 2-9   epilogue: warp w reads TMEM lanes 32*(w%4).. and the column
-//               half (w-2)/4 of the 256-column tile
+//   warps 2..   epilogue (RM_EPI_WARPS): warp w reads TMEM lanes 32*(w%4)..
+//               and column group (w-2)/4 of the 256-column tile
 // Every wait is bounded (wait_bounded); on a timeout the roles drain their
 // in-flight copies and MMAs before TMEM is freed.
 #pragma once
@@ -36,6 +36,12 @@
 namespace mc {
 
 constexpr int RM_STAGES_MAX = 8;
+// Epilogue warps: four per TMEM lane quarter would give each 64 of a tile's
+// 256 columns, two give each 128.
+constexpr int RM_EPI_WARPS = 8;
+constexpr int RM_THREADS = 64 + 32 * RM_EPI_WARPS;
+constexpr int RM_COLS = MMA_N / (RM_EPI_WARPS / 4);  // columns per epilogue warp
+static_assert(RM_EPI_WARPS % 4 == 0 && (RM_COLS == 64 || RM_COLS == 128), "epilogue split");
 constexpr int RM_KB_MAX = 4;                 // contraction up to 256 columns
 constexpr uint32_t RM_KB_BYTES = HALF * BK * 2;  // one CTA's 128 rows x 64 columns: 16 KiB
 
@@ -81,7 +87,7 @@ __device__ __forceinline__ RmTask rowmax_task(const RowMaxParams& P, long long t
   return k;
 }
 
-__global__ void __launch_bounds__(GEMM_THREADS, 1) qk_rowmax_kernel(const __grid_constant__ RowMaxParams P) {
+__global__ void __launch_bounds__(RM_THREADS, 1) qk_rowmax_kernel(const __grid_constant__ RowMaxParams P) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const int nkb = P.nkb, STG = P.stages;
@@ -114,7 +120,7 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1) qk_rowmax_kernel(const __grid
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(smem_u32(&tfull_bar[b]), 1);
-      mbar_init(smem_u32(&tempty_bar[b]), 2 * NUM_EPI_WARPS);
+      mbar_init(smem_u32(&tempty_bar[b]), 2 * RM_EPI_WARPS);
       mbar_init(smem_u32(&qfull_bar[b]), 1);
       mbar_init(smem_u32(&qempty_bar[b]), 1);
     }
@@ -268,7 +274,7 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1) qk_rowmax_kernel(const __grid
   } else {
     // ------------------------------------------------------- epilogue
     const int q = warp & 3;                 // TMEM lane quarter
-    const int half = (warp - 2) >> 2;       // column half of the 256-column tile
+    const int cg = (warp - 2) >> 2;         // column group of the 256-column tile
     uint32_t tempty_leader[2];
     for (int b = 0; b < 2; ++b) tempty_leader[b] = mapa_shared(smem_u32(&tempty_bar[b]), 0);
     int acc = 0;
@@ -286,23 +292,28 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1) qk_rowmax_kernel(const __grid
           break;
         }
         tc_fence_after();
-        const int c0 = j * BM + half * 128;
-        // a warp whose 128 columns all lie above its last row has nothing to read
+        const int c0 = j * BM + cg * RM_COLS;
+        // a warp whose columns all lie above its last row has nothing to read
         const bool dead = P.causal && c0 > r_warp_last;
         if (!dead) {
-          float v[128];
-          tmem_ld128(tmem_base + (static_cast<uint32_t>(q * 32) << 16) + acc * MMA_N + half * 128, v);
+          float v[RM_COLS];
+          const uint32_t ta = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + acc * MMA_N + cg * RM_COLS;
+          if constexpr (RM_COLS == 128) {
+            tmem_ld128(ta, v);
+          } else {
+            tmem_ld64(ta, v);
+          }
           if (r < P.S) {
-            if (c0 + 128 <= P.S && (!P.causal || c0 + 127 <= r)) {
+            if (c0 + RM_COLS <= P.S && (!P.causal || c0 + RM_COLS - 1 <= r)) {
               float m = run_max;
 #pragma unroll
-              for (int x = 0; x < 128; x += 8)
+              for (int x = 0; x < RM_COLS; x += 8)
                 m = fmax3(m, fmax3(v[x], v[x + 1], v[x + 2]),
                           fmax3(fmax3(v[x + 3], v[x + 4], v[x + 5]), v[x + 6], v[x + 7]));
               run_max = m;
             } else {
 #pragma unroll
-              for (int x = 0; x < 128; ++x) {
+              for (int x = 0; x < RM_COLS; ++x) {
                 const int c = c0 + x;
                 if (c < P.S && (!P.causal || c <= r)) run_max = fmaxf(run_max, v[x]);
               }

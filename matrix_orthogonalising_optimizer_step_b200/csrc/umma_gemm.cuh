@@ -49,7 +49,9 @@
 //               "empty" and "accumulator full" barriers.
 //   warps 2..   epilogue: warp w reads TMEM lanes 32*(w%4)..+31 and column
 //               group (w-2)/4 of the tile; the leader's "accumulator empty"
-//               barrier counts both CTAs' epilogue warps.
+//               barrier counts both CTAs' epilogue warps.  Whole 32-row
+//               blocks move to and from global memory through a per-warp
+//               shared-memory buffer (coalesced rows; see epi_fast64).
 #pragma once
 
 #include <climits>
@@ -177,6 +179,7 @@ struct GemmGroup {
   float diag;              // EPI_POLY: added on the diagonal (a for P = aI + B)
   float decay, step, rms;  // EPI_APPLY_FINAL
   float out_scale;         // EPI_CAUSALMAX: 1/sqrt(d_head)
+  int tma_epi;             // the group's epilogue tensor maps are set (map_eo, map_ei, map_ei2)
 };
 
 template <int EPI>
@@ -189,6 +192,13 @@ __device__ __forceinline__ bool apply_reads_x(const GemmGroup& G) {
 struct GemmParams {
   CUtensorMap map_a[MAX_GROUPS];
   CUtensorMap map_b[MAX_GROUPS];
+  // Epilogue tensor maps per group, boxes of 32 rows x 64 columns (128-byte
+  // swizzle) or 32 x 32 (64-byte swizzle, EPI_APPLY_MIXED): the output, and
+  // the one or two inputs (EPI_POLY: the b*A source; EPI_APPLY_MIXED: the
+  // iterate's hi half, and its lo half, which is also written).
+  CUtensorMap map_eo[MAX_GROUPS];
+  CUtensorMap map_ei[MAX_GROUPS];
+  CUtensorMap map_ei2[MAX_GROUPS];
   GemmGroup g[MAX_GROUPS];
   int num_groups;
   long long total_tiles;
@@ -715,6 +725,8 @@ template <int EPI>
 __device__ __forceinline__ void epi_fast64(const GemmGroup& G, int prob, int r0, int c0, int lane, uint32_t taddr,
                                            uint8_t* buf) {
   static_assert(EPI != EPI_APPLY_MIXED, "the mixed apply uses epi_fast32_mixed");
+  if (lane == 0) bulk_wait_read_all();  // no tensor store of the warp still reads the buffer
+  __syncwarp();
   uint4 ga[8];
   if constexpr (EPI == EPI_POLY) {
     warp_issue_rows64(static_cast<const __nv_bfloat16*>(G.src) + (long long)prob * G.src_bs + (long long)r0 * G.src_ld + c0,
@@ -790,6 +802,8 @@ __device__ __forceinline__ void epi_fast64(const GemmGroup& G, int prob, int r0,
 // half when flagged).
 __device__ __forceinline__ void epi_fast32_mixed(const GemmGroup& G, int prob, int r0, int c0, int lane,
                                                  uint32_t taddr, uint8_t* buf) {
+  if (lane == 0) bulk_wait_read_all();  // no tensor store of the warp still reads the buffer
+  __syncwarp();
   uint4 gh[4], gl[4];
   warp_issue_rows32(G.xh + (long long)prob * G.xh_bs + (long long)r0 * G.xh_ld + c0, G.xh_ld, lane, gh);
   warp_issue_rows32(G.xl + (long long)prob * G.xl_bs + (long long)r0 * G.xl_ld + c0, G.xl_ld, lane, gl);
@@ -821,6 +835,141 @@ __device__ __forceinline__ void epi_fast32_mixed(const GemmGroup& G, int prob, i
     warp_store_rows32(G.xl + (long long)prob * G.xl_bs + (long long)r0 * G.xl_ld + c0, G.xl_ld, lane, buf, xl);
 }
 
+// The coalesced path with tensor copies, for groups that carry epilogue maps:
+// the block's inputs arrive by TMA loads into the warp's buffer (completing on
+// the warp's barrier `ebar`) and its outputs leave by a TMA store from it, so
+// the global side takes no load or store instructions; each thread only reads
+// and writes its own row of the buffer (the buffer's swizzle is the maps'
+// 128- or 64-byte swizzle).  Returns false if the loads' wait timed out.
+template <int EPI>
+__device__ __forceinline__ bool epi_tma_block(const GemmParams& P, int gi, const GemmGroup& G, int prob, int r0, int c0,
+                                              int lane, uint32_t taddr, uint8_t* buf, uint32_t ebar, uint32_t& ephase,
+                                              bool& load_pending, volatile int* abort_flag) {
+  constexpr int COLS = epi_fast_cols<EPI>();
+  constexpr int NLOAD = EPI == EPI_APPLY_MIXED ? 2 : (EPI == EPI_POLY ? 1 : 0);
+  const uint32_t sbuf = smem_u32(buf);
+  if (lane == 0) {
+    bulk_wait_read_all();  // the previous block's store has read the buffer
+    if constexpr (NLOAD > 0) {
+      fence_proxy_async_smem();
+      mbar_arrive_expect_tx(ebar, uint32_t(NLOAD) * 32u * COLS * 2u);
+      tma_load_3d(sbuf, &P.map_ei[gi], ebar, c0, r0, prob);
+      if constexpr (NLOAD == 2) tma_load_3d(sbuf + 2048, &P.map_ei2[gi], ebar, c0, r0, prob);
+    }
+  }
+  if constexpr (NLOAD > 0) load_pending = true;
+  __syncwarp();
+  float v[COLS];
+  if constexpr (COLS == 64) {
+    tmem_ld64(taddr, v);
+  } else {
+    tmem_ld16(taddr, *reinterpret_cast<float(*)[16]>(v));
+    tmem_ld16(taddr + 16, *reinterpret_cast<float(*)[16]>(v + 16));
+  }
+  if constexpr (NLOAD > 0) {
+    const bool got = wait_bounded(ebar, ephase, abort_flag, P.err);
+    if (!__all_sync(0xffffffffu, got)) return false;
+    ephase ^= 1;
+    load_pending = false;
+  }
+  uint32_t pk[COLS / 2];
+  if constexpr (EPI == EPI_GRAM) {
+    float s2 = 1.f;
+    if (G.scale) {
+      const float sc = G.scale[G.prob_base + prob];
+      s2 = sc * sc;
+    }
+#pragma unroll
+    for (int i = 0; i < 32; ++i) pk[i] = pack_bf16x2(s2 == 0.f ? 0.f : v[2 * i] * s2, s2 == 0.f ? 0.f : v[2 * i + 1] * s2);
+  } else if constexpr (EPI == EPI_POLY) {
+#pragma unroll
+    for (int c = 0; c < 8; ++c) {
+      const uint4 x = *reinterpret_cast<const uint4*>(buf + epi_swz(lane, c));
+      const uint32_t xs[4] = {x.x, x.y, x.z, x.w};
+#pragma unroll
+      for (int t = 0; t < 4; ++t) {
+        const int i = 4 * c + t;
+        pk[i] = pack_bf16x2(fmaf(G.coef_acc, v[2 * i], G.coef_src * bf16_lo(xs[t])),
+                            fmaf(G.coef_acc, v[2 * i + 1], G.coef_src * bf16_hi(xs[t])));
+      }
+    }
+  } else if constexpr (EPI == EPI_APPLY) {
+    const float sc = G.scale ? G.scale[G.prob_base + prob] : 1.f;
+#pragma unroll
+    for (int i = 0; i < 32; ++i)
+      pk[i] = sc == 0.f ? 0u : pack_bf16x2(sc * v[2 * i], sc * v[2 * i + 1]);
+  } else if constexpr (EPI == EPI_APPLY_MIXED) {
+    const float sc = G.scale ? G.scale[G.prob_base + prob] : 1.f;
+#pragma unroll
+    for (int c = 0; c < 4; ++c) {
+      const uint4 h = *reinterpret_cast<const uint4*>(buf + epi_swz32(lane, c));
+      const uint4 l = *reinterpret_cast<const uint4*>(buf + 2048 + epi_swz32(lane, c));
+      const uint32_t hs[4] = {h.x, h.y, h.z, h.w}, ls[4] = {l.x, l.y, l.z, l.w};
+#pragma unroll
+      for (int t = 0; t < 4; ++t) {
+        const int i = 4 * c + t;
+        v[2 * i] = sc * fmaf(G.coef_src, bf16_lo(hs[t]) + bf16_lo(ls[t]), v[2 * i]);
+        v[2 * i + 1] = sc * fmaf(G.coef_src, bf16_hi(hs[t]) + bf16_hi(ls[t]), v[2 * i + 1]);
+      }
+    }
+    if (sc == 0.f) {  // a non-finite NS input: the first iterate is zero, not NaN
+#pragma unroll
+      for (int j = 0; j < 32; ++j) v[j] = 0.f;
+    }
+#pragma unroll
+    for (int i = 0; i < 16; ++i) pk[i] = pack_bf16x2(v[2 * i], v[2 * i + 1]);
+  } else {  // EPI_STORE
+#pragma unroll
+    for (int i = 0; i < 32; ++i) pk[i] = pack_bf16x2(v[2 * i], v[2 * i + 1]);
+  }
+  // own row of the outputs into the buffer, then one tensor store per output
+  if constexpr (COLS == 64) {
+#pragma unroll
+    for (int c = 0; c < 8; ++c)
+      *reinterpret_cast<uint4*>(buf + epi_swz(lane, c)) = make_uint4(pk[4 * c], pk[4 * c + 1], pk[4 * c + 2], pk[4 * c + 3]);
+  } else {
+#pragma unroll
+    for (int c = 0; c < 4; ++c)
+      *reinterpret_cast<uint4*>(buf + epi_swz32(lane, c)) = make_uint4(pk[4 * c], pk[4 * c + 1], pk[4 * c + 2], pk[4 * c + 3]);
+    if constexpr (EPI == EPI_APPLY_MIXED) {
+      if (G.xl_write) {
+        uint32_t lo[4];
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+#pragma unroll
+          for (int t = 0; t < 4; ++t) {
+            const int i = 4 * c + t;
+            lo[t] = pack_bf16x2(v[2 * i] - bf16_lo(pk[i]), v[2 * i + 1] - bf16_hi(pk[i]));
+          }
+          *reinterpret_cast<uint4*>(buf + 2048 + epi_swz32(lane, c)) = make_uint4(lo[0], lo[1], lo[2], lo[3]);
+        }
+      }
+    }
+  }
+  fence_proxy_async_smem();
+  __syncwarp();
+  if (lane == 0) {
+    tma_store_3d(&P.map_eo[gi], sbuf, c0, r0, prob);
+    if constexpr (EPI == EPI_APPLY_MIXED) {
+      if (G.xl_write) tma_store_3d(&P.map_ei2[gi], sbuf + 2048, c0, r0, prob);
+    }
+    bulk_commit_group();
+  }
+  if constexpr (EPI == EPI_GRAM || EPI == EPI_POLY) {
+    // the mirror image, as in epi_fast64
+    __nv_bfloat16* D = static_cast<__nv_bfloat16*>(G.d) + (long long)prob * G.d_bs;
+    unsigned short* pm = reinterpret_cast<unsigned short*>(D + (long long)c0 * G.d_ld + r0 + lane);
+    const long long ld = G.d_ld;
+#pragma unroll
+    for (int i = 0; i < 32; ++i) {
+      pm[0] = static_cast<unsigned short>(pk[i] & 0xFFFFu);
+      pm[ld] = static_cast<unsigned short>(pk[i] >> 16);
+      pm += 2 * ld;
+    }
+  }
+  return true;
+}
+
 // Chunks per batch.  One for the NS phases: measured against batches of four
 // chunks (one 64-column TMEM load, all global loads issued first) on the same
 // GPU, the single-chunk drain was as fast or faster.  Eight for the causal
@@ -840,15 +989,19 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1) umma_gemm_kernel(const __grid
   constexpr uint32_t STAGE_BYTES = T::STAGE_BYTES;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + STAGES * STAGE_BYTES);
+  // [stages][epilogue row buffers (1 KiB-aligned, 4 KiB per warp)][barriers][head maxima]
+  constexpr size_t BUF_BYTES = epi_uses_row_buffers<EPI>() ? size_t(NUM_EPI_WARPS) * EPI_BUF_BYTES : 0;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + STAGES * STAGE_BYTES + BUF_BYTES);
   uint64_t* full_bar = bars;                          // [STAGES]  used in the leader only
   uint64_t* empty_bar = bars + STAGES;                // [STAGES]  every CTA
   uint64_t* tfull_bar = bars + 2 * STAGES;            // [NACC]    every CTA
   uint64_t* tempty_bar = bars + 2 * STAGES + NACC;    // [NACC]    used in the leader only
   uint64_t* drain_bar = bars + 2 * STAGES + 2 * NACC; // [1]       leader
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain_bar + 1);
+  uint64_t* epi_bar = drain_bar + 1;                  // [NUM_EPI_WARPS] epilogue tensor loads
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(epi_bar + NUM_EPI_WARPS);
+  static_assert((2 * 6 + 2 * 2 + 1 + NUM_EPI_WARPS) * 8 + 8 <= GEMM_BARRIER_BYTES, "barrier block");
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
-  int* head_max = reinterpret_cast<int*>(smem + STAGES * STAGE_BYTES + GEMM_BARRIER_BYTES);  // EPI_CAUSALMAX
+  int* head_max = reinterpret_cast<int*>(smem + STAGES * STAGE_BYTES + BUF_BYTES + GEMM_BARRIER_BYTES);  // EPI_CAUSALMAX
   const int nheads_smem = (EPI == EPI_CAUSALMAX && P.g[0].heads <= SMEM_HEADS) ? P.g[0].heads : 0;
   for (int i = threadIdx.x; i < nheads_smem; i += blockDim.x) head_max[i] = INT_MIN;
 
@@ -867,6 +1020,7 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1) umma_gemm_kernel(const __grid
       mbar_init(smem_u32(&tempty_bar[b]), 2 * NUM_EPI_WARPS);
     }
     mbar_init(smem_u32(drain_bar), 1);
+    for (int w = 0; w < NUM_EPI_WARPS; ++w) mbar_init(smem_u32(&epi_bar[w]), 1);
     *abort_flag = 0;
     fence_mbar_init();
   }
@@ -1040,7 +1194,10 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1) umma_gemm_kernel(const __grid
     constexpr int WCOLS = T::N / EPI_COL_GROUPS;  // columns per epilogue warp
     const int q = warp & 3;                       // TMEM lane quarter this warp may read
     const int half = (warp - 2) >> 2;             // which column group of the tile
-    uint8_t* epi_buf = smem + STAGES * STAGE_BYTES + GEMM_BARRIER_BYTES + (warp - 2) * EPI_BUF_BYTES;
+    uint8_t* epi_buf = smem + STAGES * STAGE_BYTES + (warp - 2) * EPI_BUF_BYTES;
+    const uint32_t ebar = smem_u32(&epi_bar[warp - 2]);
+    uint32_t ephase = 0;
+    bool load_pending = false;
     uint32_t tempty_leader[NACC];
 #pragma unroll
     for (int b = 0; b < NACC; ++b) tempty_leader[b] = mapa_shared(smem_u32(&tempty_bar[b]), 0);
@@ -1068,6 +1225,7 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1) umma_gemm_kernel(const __grid
       // diagonal for every lane, as do all later chunks (causal max only).
       const int r_warp_last = ti.tm * BM + HALF * static_cast<int>(rank) + q * 32 + 31;
       const int r0w = r_warp_last - 31;             // first row of this warp
+      bool tile_ok = true;                          // false: an epilogue load's wait timed out
 #pragma unroll 1
       for (int cb = 0; cb < (idle ? 0 : WCOLS / 16); cb += CH) {
         if constexpr (EPI == EPI_CAUSALMAX) {
@@ -1077,6 +1235,17 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1) umma_gemm_kernel(const __grid
           // a whole 32-row block through the coalesced path when it can
           constexpr int FB = epi_fast_cols<EPI>() / 16;
           if (cb % FB == 0 && epi_fast_ok<EPI>(G, ti.prob, r0w, cbase + cb * 16)) {
+            if constexpr (EPI != EPI_APPLY_FINAL) {
+              if (G.tma_epi) {
+                if (!epi_tma_block<EPI>(P, ti.g, G, ti.prob, r0w, cbase + cb * 16, lane, t_row + cb * 16, epi_buf, ebar,
+                                        ephase, load_pending, abort_flag)) {
+                  tile_ok = false;
+                  break;
+                }
+                cb += FB - 1;
+                continue;
+              }
+            }
             if constexpr (EPI == EPI_APPLY_MIXED) {
               epi_fast32_mixed(G, ti.prob, r0w, cbase + cb * 16, lane, t_row + cb * 16, epi_buf);
             } else {
@@ -1102,6 +1271,7 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1) umma_gemm_kernel(const __grid
         for (int b = 0; b < CH; ++b)
           epi_finish<EPI>(G, ti.prob, r, cbase + (cb + b) * 16, v + b * 16, pre[b], run_max);
       }
+      if (!tile_ok) break;
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive_cluster(tempty_leader[acc]);
@@ -1122,6 +1292,18 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1) umma_gemm_kernel(const __grid
         acc = 0;
         acc_phase ^= 1;
       }
+    }
+    if constexpr (epi_uses_row_buffers<EPI>()) {
+      // the warp's tensor stores complete, and a load abandoned on a timeout
+      // lands, before the CTA's shared memory is released
+      if (lane == 0) {
+        bulk_wait_all();
+        if (load_pending) {
+          volatile int no_abort = 0;
+          wait_bounded(ebar, ephase, &no_abort, nullptr, kDrainLimitCycles);
+        }
+      }
+      __syncwarp();
     }
   }
 
