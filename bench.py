@@ -367,14 +367,28 @@ CONFIG_WORKLOADS = {
 }
 
 
-def _timed_alone(mc, fn, reps, stream):
+def _timed_alone(mc, fn, reps, stream, flush_l2=False):
     """Device time per call of ``fn`` (CUDA events on ``stream``) and the
-    per-kernel rows over those calls."""
+    per-kernel rows over those calls.  With ``flush_l2`` (inputs that fit in
+    L2) a 256 MB buffer is written between calls, outside the timed events."""
     import torch
     for _ in range(3):
         fn()
     torch.cuda.synchronize()
     mc.profile_begin()
+    if flush_l2:
+        scrub = torch.empty(256 << 20, dtype=torch.uint8, device=torch.cuda.current_device())
+        evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(reps)]
+        with torch.cuda.stream(stream):
+            for a, b in evs:
+                scrub.fill_(1)
+                a.record(stream)
+                fn()
+                b.record(stream)
+        torch.cuda.synchronize()
+        k = mc.profile_end()
+        assert mc.device_status() == mc.MC_OK, mc.last_error()
+        return sum(a.elapsed_time(b) for a, b in evs) / reps, k
     a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     a.record(stream)
     for _ in range(reps):
@@ -445,7 +459,8 @@ def run_config(args, cfg):
             Ws = [(torch.randn(sh, device=dev, generator=g) * 0.02).to(torch.bfloat16) for sh in shapes]
             Gs = [(torch.randn(sh, device=dev, generator=g) * 1e-3).to(torch.bfloat16) for sh in shapes]
             Ms = [torch.zeros(sh, device=dev, dtype=torch.float32) for sh in shapes]
-        ms, k = _timed_alone(mc, lambda: mc.muon_step(Ws, Gs, Ms, stream=stream, **hp), reps, stream)
+        ms, k = _timed_alone(mc, lambda: mc.muon_step(Ws, Gs, Ms, stream=stream, **hp), reps, stream,
+                             flush_l2=cfg == 0)
         dense = ns_dense_flops(shapes, hp["ns_steps"])
         ns_kinds = ("ns_gram", "ns_poly", "ns_apply_mixed", "ns_apply", "ns_apply_final", "ns_thin")
         ns_ms = sum(k[n]["total_ms"] for n in ns_kinds if n in k) / reps
@@ -460,7 +475,8 @@ def run_config(args, cfg):
                                "momentum_gbs": mom["bytes"] / (mom["total_ms"] / 1e3) / 1e9 if mom else None})
         out["config"].update(matrices=len(shapes), params=int(sum(r * c for r, c in shapes)),
                              flops_per_step=dense, flops_convention="dense-equivalent 5*(4 m^2 n + 2 m^3)",
-                             l2="inputs larger than L2" if cfg == 4 else "inputs fit in L2 (no flush)")
+                             l2=("inputs fit in L2: 256 MB written between timed calls" if cfg == 0 else
+                                 f"inputs larger than L2 (W, G, M {sum(r * c for r, c in shapes) * 8 / 1e6:.0f} MB)"))
         # the oracle on the host cores: the whole config (0, 1), or one matrix
         # per shape class scaled by the class counts (4)
         if args.no_cpu_baseline:
