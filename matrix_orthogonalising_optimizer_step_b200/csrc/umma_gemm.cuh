@@ -76,7 +76,9 @@ constexpr int GEMM_BARRIER_BYTES = 256;
 
 // Two tile shapes per CTA pair:
 //   WIDE = 0: 256 x 256, two 256-column accumulators (the next tile's MMAs
-//             overlap this tile's epilogue), 6 stages of 32 KB per CTA;
+//             overlap this tile's epilogue), 3 stages of 64 KB per CTA, each
+//             two k-blocks under one pair of barriers (eight MMAs per round
+//             trip, as WIDE = 1 has);
 //   WIDE = 1: 256 x 512, one 512-column accumulator, 4 stages of 48 KB per
 //             CTA.  Sharing each A tile between two N=256 MMAs cuts the
 //             operand bytes per MMA cycle from 64 to 48 per SM, below the
@@ -90,10 +92,12 @@ template <int WIDE>
 struct TileCfg {
   static constexpr int N = MMA_N << WIDE;               // tile columns per pair
   static constexpr int NB = 1 << WIDE;                  // B blocks (MMAs per k-step)
-  static constexpr int STAGES = WIDE ? 4 : 6;
+  static constexpr int KPS = WIDE ? 1 : 2;              // k-blocks per stage
+  static constexpr int STAGES = WIDE ? 4 : 3;
   static constexpr int NACC = WIDE ? 1 : 2;             // accumulator buffers
-  static constexpr uint32_t STAGE_BYTES = A_STAGE_BYTES + NB * B_STAGE_BYTES;
-  static constexpr uint32_t PAIR_STAGE_BYTES = 2 * STAGE_BYTES;
+  static constexpr uint32_t KB_BYTES = A_STAGE_BYTES + NB * B_STAGE_BYTES;  // one k-block, one CTA
+  static constexpr uint32_t PAIR_KB_BYTES = 2 * KB_BYTES;
+  static constexpr uint32_t STAGE_BYTES = KPS * KB_BYTES;
   static constexpr size_t SMEM_BYTES = 1024 + size_t(STAGES) * STAGE_BYTES + GEMM_BARRIER_BYTES;
   static constexpr size_t SMEM_BYTES_HEADS = SMEM_BYTES + 4 * size_t(SMEM_HEADS);
   static_assert(NACC * N <= int(TMEM_COLS), "accumulators exceed TMEM");
@@ -1058,7 +1062,8 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1) umma_gemm_kernel(const __grid
         const CUtensorMap* mb = &P.map_b[ti.g];
         const int m0 = ti.tm * BM + HALF * static_cast<int>(rank);
         const int n0 = ti.tn * T::N + HALF * static_cast<int>(rank);
-        for (int kb = 0; kb < ti.num_kb; ++kb) {
+        for (int kb0 = 0; kb0 < ti.num_kb; kb0 += T::KPS) {
+          const int nk = ti.num_kb - kb0 < T::KPS ? ti.num_kb - kb0 : T::KPS;
           if (!wait_bounded(smem_u32(&empty_bar[stage]), phase ^ 1, abort_flag, P.err)) {
             ok = false;
             break;
@@ -1067,44 +1072,47 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1) umma_gemm_kernel(const __grid
           const bool skip0 = sym_skip_first_block<T::NB>(G, ti);
           if (leader) {
             // both CTAs of the pair skip the same block (it depends on the tile only)
-            mbar_arrive_expect_tx(fb_local, skip0 ? T::PAIR_STAGE_BYTES - 2 * B_STAGE_BYTES : T::PAIR_STAGE_BYTES);
+            mbar_arrive_expect_tx(fb_local, uint32_t(nk) * (skip0 ? T::PAIR_KB_BYTES - 2 * B_STAGE_BYTES
+                                                                   : T::PAIR_KB_BYTES));
             filled |= 1u << stage;
             fill_parity = (fill_parity & ~(1u << stage)) | (phase << stage);
           }
           const uint32_t fb = mapa_shared(fb_local, 0);
-          const uint32_t sa = smem_u32(smem + stage * STAGE_BYTES);
-          const int k0 = kb * BK;
-          if (G.layout == LAYOUT_HEADS) {
-            const int bb = ti.prob / G.heads, hh = ti.prob % G.heads;
-            // A split contraction concatenates two per-head operand pairs along K
-            // (MLA's content and rotary parts); the second key operand has one
-            // head shared by all query heads.
-            const bool second = G.k_split > 0 && k0 >= G.k_split;
-            const CUtensorMap* qa = second ? &P.map_a[1] : ma;
-            const CUtensorMap* kb_map = second ? &P.map_b[1] : mb;
-            const int kk = second ? k0 - G.k_split : k0;
-            const int hk = second ? 0 : hh;
-            tma_load_4d_pair(sa, qa, fb, kk, hh, m0, bb);
+          for (int j = 0; j < nk; ++j) {
+            const uint32_t sa = smem_u32(smem + stage * STAGE_BYTES + j * T::KB_BYTES);
+            const int k0 = (kb0 + j) * BK;
+            if (G.layout == LAYOUT_HEADS) {
+              const int bb = ti.prob / G.heads, hh = ti.prob % G.heads;
+              // A split contraction concatenates two per-head operand pairs along K
+              // (MLA's content and rotary parts); the second key operand has one
+              // head shared by all query heads.
+              const bool second = G.k_split > 0 && k0 >= G.k_split;
+              const CUtensorMap* qa = second ? &P.map_a[1] : ma;
+              const CUtensorMap* kb_map = second ? &P.map_b[1] : mb;
+              const int kk = second ? k0 - G.k_split : k0;
+              const int hk = second ? 0 : hh;
+              tma_load_4d_pair(sa, qa, fb, kk, hh, m0, bb);
 #pragma unroll
-            for (int h = 0; h < T::NB; ++h)
-              tma_load_4d_pair(sa + A_STAGE_BYTES + h * B_STAGE_BYTES, kb_map, fb, kk, hk, n0 + h * MMA_N, bb);
-          } else {
-            if (!G.a_mn) {
-              tma_load_3d_pair(sa, ma, fb, k0, m0, ti.prob);
+              for (int h = 0; h < T::NB; ++h)
+                tma_load_4d_pair(sa + A_STAGE_BYTES + h * B_STAGE_BYTES, kb_map, fb, kk, hk, n0 + h * MMA_N, bb);
             } else {
-              tma_load_3d_pair(sa, ma, fb, m0, k0, ti.prob);
-              tma_load_3d_pair(sa + MN_BOX_BYTES, ma, fb, m0 + 64, k0, ti.prob);
-            }
-#pragma unroll
-            for (int h = 0; h < T::NB; ++h) {
-              if (h == 0 && skip0) continue;
-              const uint32_t sb = sa + A_STAGE_BYTES + h * B_STAGE_BYTES;
-              const int nh = n0 + h * MMA_N;
-              if (!G.b_mn) {
-                tma_load_3d_pair(sb, mb, fb, k0, nh, ti.prob);
+              if (!G.a_mn) {
+                tma_load_3d_pair(sa, ma, fb, k0, m0, ti.prob);
               } else {
-                tma_load_3d_pair(sb, mb, fb, nh, k0, ti.prob);
-                tma_load_3d_pair(sb + MN_BOX_BYTES, mb, fb, nh + 64, k0, ti.prob);
+                tma_load_3d_pair(sa, ma, fb, m0, k0, ti.prob);
+                tma_load_3d_pair(sa + MN_BOX_BYTES, ma, fb, m0 + 64, k0, ti.prob);
+              }
+#pragma unroll
+              for (int h = 0; h < T::NB; ++h) {
+                if (h == 0 && skip0) continue;
+                const uint32_t sb = sa + A_STAGE_BYTES + h * B_STAGE_BYTES;
+                const int nh = n0 + h * MMA_N;
+                if (!G.b_mn) {
+                  tma_load_3d_pair(sb, mb, fb, k0, nh, ti.prob);
+                } else {
+                  tma_load_3d_pair(sb, mb, fb, nh, k0, ti.prob);
+                  tma_load_3d_pair(sb + MN_BOX_BYTES, mb, fb, nh + 64, k0, ti.prob);
+                }
               }
             }
           }
@@ -1153,22 +1161,27 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1) umma_gemm_kernel(const __grid
         const uint64_t ad0 = smem_desc_sw128(s0, a_lbo, 1024);
         const uint64_t bd0 = smem_desc_sw128(s0 + A_STAGE_BYTES, b_lbo, 1024);
         const bool skip0 = sym_skip_first_block<T::NB>(G, ti);
-        for (int kb = 0; kb < ti.num_kb; ++kb) {
+        for (int kb0 = 0; kb0 < ti.num_kb; kb0 += T::KPS) {
+          const int nk = ti.num_kb - kb0 < T::KPS ? ti.num_kb - kb0 : T::KPS;
           // The TMA writes are made visible by the barrier's complete_tx; the
           // MMAs read them through the same async proxy.
           if (!wait_bounded(smem_u32(&full_bar[stage]), phase, abort_flag, P.err)) {
             ok = false;
             break;
           }
-          const uint64_t soff = static_cast<uint64_t>((stage * STAGE_BYTES) >> 4);
 #pragma unroll
-          for (int kk = 0; kk < BK / 16; ++kk) {
-            const uint64_t ad = ad0 + soff + ((kk * a_kstep) >> 4);
+          for (int j = 0; j < T::KPS; ++j) {
+            if (j >= nk) break;
+            const uint64_t soff = static_cast<uint64_t>((stage * STAGE_BYTES + j * T::KB_BYTES) >> 4);
 #pragma unroll
-            for (int h = 0; h < T::NB; ++h) {
-              if (h == 0 && skip0) continue;
-              const uint64_t bd = bd0 + soff + ((h * B_STAGE_BYTES + kk * b_kstep) >> 4);
-              umma_bf16_pair(d_tmem + h * MMA_N, ad, bd, idesc, (kb | kk) != 0);
+            for (int kk = 0; kk < BK / 16; ++kk) {
+              const uint64_t ad = ad0 + soff + ((kk * a_kstep) >> 4);
+#pragma unroll
+              for (int h = 0; h < T::NB; ++h) {
+                if (h == 0 && skip0) continue;
+                const uint64_t bd = bd0 + soff + ((h * B_STAGE_BYTES + kk * b_kstep) >> 4);
+                umma_bf16_pair(d_tmem + h * MMA_N, ad, bd, idesc, ((kb0 + j) | kk) != 0);
+              }
             }
           }
           umma_commit_pair_mc(smem_u32(&empty_bar[stage]), 0x3);
