@@ -376,7 +376,7 @@ void finish_group(GemmParams& p, int gi, GemmGroup& G, int wide) {
 // many stages as fit beside the Q double buffer, at most RM_STAGES_MAX.
 int rowmax_stages(int nkb) {
   const long long room = kSmemOptIn - 1024 - GEMM_BARRIER_BYTES - 4LL * SMEM_HEADS - 2LL * nkb * RM_KB_BYTES;
-  return static_cast<int>(std::min<long long>(RM_STAGES_MAX, room / RM_KB_BYTES));
+  return static_cast<int>(std::min<long long>(RM_STAGES_MAX, room / (nkb * (long long)RM_KB_BYTES)));
 }
 
 // Per-head max of the score tiles, scores never stored.  `cm` holds the Q and
@@ -389,7 +389,7 @@ int launch_causal_max(const GemmParams& cm, const DeviceState& st, cudaStream_t 
   const GemmGroup& G = cm.g[0];
   const int nkb = (G.K + BK - 1) / BK;
   const int stages = rowmax_stages(nkb);
-  if (nkb > RM_KB_MAX || stages < nkb) {
+  if (nkb > RM_KB_MAX || stages < 1) {
     if (!profiled) {
       if (cm.total_tiles > 0) MC_CUDA((launch_pairs<EPI_CAUSALMAX, 0>(cm, st.pair_clusters, s)));
       return MC_OK;

@@ -6,7 +6,8 @@
 // A CTA pair owns one task (b, h, query block i of 256 rows: 128 per CTA) at
 // a time, loads that block's Q once and keeps it in shared memory, then
 // streams the key blocks j = 0 .. i (all blocks without the causal mask)
-// through a ring of k-block stages.  Per key block the pair runs a
+// through a ring of stages, one key block (all its k-blocks) per stage, so
+// that one barrier round trip feeds a whole tile's MMAs.  Per key block the pair runs a
 // 256 x 256 x d tile on the tensor cores (tcgen05, cta_group::2) into one of
 // two TMEM accumulators, so the epilogue's max over one tile overlaps the
 // next tile's MMAs.  Only the key blocks move per tile (half of what a tile
@@ -51,7 +52,7 @@ struct RowMaxParams {
   int S, B, H;
   int nkb;               // k-blocks of 64 columns in the contraction
   int k_split;           // 0, or the first column taken from slot 1 (a multiple of 64)
-  int stages;            // key ring depth in k-blocks, nkb <= stages <= RM_STAGES_MAX
+  int stages;            // key ring depth in key blocks of nkb k-blocks, 1 <= stages <= RM_STAGES_MAX
   int causal;
   int nblk;              // ceil(S / 256)
   long long tasks;       // B * H * nblk
@@ -62,7 +63,7 @@ struct RowMaxParams {
 
 // Shared memory: Q double buffer, key ring, barriers, per-head maxima.
 __host__ __device__ constexpr size_t rowmax_smem_bytes(int nkb, int stages) {
-  return 1024 + size_t(2 * nkb + stages) * RM_KB_BYTES + GEMM_BARRIER_BYTES + 4 * size_t(SMEM_HEADS);
+  return 1024 + size_t(2 + stages) * nkb * RM_KB_BYTES + GEMM_BARRIER_BYTES + 4 * size_t(SMEM_HEADS);
 }
 
 struct RmTask {
@@ -92,8 +93,8 @@ __global__ void __launch_bounds__(RM_THREADS, 1) qk_rowmax_kernel(const __grid_c
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const int nkb = P.nkb, STG = P.stages;
   uint8_t* q_smem = smem;                                  // [2][nkb] x 16 KiB
-  uint8_t* k_smem = smem + size_t(2 * nkb) * RM_KB_BYTES;  // [STG] x 16 KiB
-  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + size_t(2 * nkb + STG) * RM_KB_BYTES);
+  uint8_t* k_smem = smem + size_t(2 * nkb) * RM_KB_BYTES;  // [STG][nkb] x 16 KiB
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + size_t(2 + STG) * nkb * RM_KB_BYTES);
   uint64_t* full_bar = bars;                               // [RM_STAGES_MAX] leader
   uint64_t* empty_bar = bars + RM_STAGES_MAX;              // [RM_STAGES_MAX] every CTA
   uint64_t* tfull_bar = bars + 2 * RM_STAGES_MAX;          // [2] every CTA
@@ -104,7 +105,7 @@ __global__ void __launch_bounds__(RM_THREADS, 1) qk_rowmax_kernel(const __grid_c
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain_bar + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
   static_assert((2 * RM_STAGES_MAX + 9) * 8 + 8 <= GEMM_BARRIER_BYTES, "barrier block");
-  int* head_max = reinterpret_cast<int*>(smem + size_t(2 * nkb + STG) * RM_KB_BYTES + GEMM_BARRIER_BYTES);
+  int* head_max = reinterpret_cast<int*>(smem + size_t(2 + STG) * nkb * RM_KB_BYTES + GEMM_BARRIER_BYTES);
   const int nheads_smem = P.H <= SMEM_HEADS ? P.H : 0;
   for (int i = threadIdx.x; i < nheads_smem; i += blockDim.x) head_max[i] = INT_MIN;
 
@@ -180,25 +181,27 @@ __global__ void __launch_bounds__(RM_THREADS, 1) qk_rowmax_kernel(const __grid_c
         }
         for (int j = 0; ok && j < T.jn; ++j) {
           const int n0 = j * BM + HALF * static_cast<int>(rank);
+          if (!wait_bounded(smem_u32(&empty_bar[stage]), phase ^ 1, abort_flag, P.err)) {
+            ok = false;
+            break;
+          }
+          const uint32_t fb_local = smem_u32(&full_bar[stage]);
+          if (leader) {
+            mbar_arrive_expect_tx(fb_local, 2u * nkb * RM_KB_BYTES);
+            filled |= 1u << stage;
+            fill_parity = (fill_parity & ~(1u << stage)) | (phase << stage);
+          }
+          const uint32_t fb = mapa_shared(fb_local, 0);
           for (int kb = 0; kb < nkb; ++kb) {
-            if (!wait_bounded(smem_u32(&empty_bar[stage]), phase ^ 1, abort_flag, P.err)) {
-              ok = false;
-              break;
-            }
-            const uint32_t fb_local = smem_u32(&full_bar[stage]);
-            if (leader) {
-              mbar_arrive_expect_tx(fb_local, 2u * RM_KB_BYTES);
-              filled |= 1u << stage;
-              fill_parity = (fill_parity & ~(1u << stage)) | (phase << stage);
-            }
             const int k0 = kb * BK;
             const bool second = P.k_split > 0 && k0 >= P.k_split;
-            tma_load_4d_pair(smem_u32(k_smem + size_t(stage) * RM_KB_BYTES), second ? &P.map_k[1] : &P.map_k[0],
-                             mapa_shared(fb_local, 0), second ? k0 - P.k_split : k0, second ? 0 : T.h, n0, T.b);
-            if (++stage == STG) {
-              stage = 0;
-              phase ^= 1;
-            }
+            tma_load_4d_pair(smem_u32(k_smem + size_t(stage * nkb + kb) * RM_KB_BYTES),
+                             second ? &P.map_k[1] : &P.map_k[0], fb, second ? k0 - P.k_split : k0, second ? 0 : T.h,
+                             n0, T.b);
+          }
+          if (++stage == STG) {
+            stage = 0;
+            phase ^= 1;
           }
         }
       }
@@ -241,24 +244,23 @@ __global__ void __launch_bounds__(RM_THREADS, 1) qk_rowmax_kernel(const __grid_c
           }
           tc_fence_after();
           const uint32_t d_tmem = tmem_base + acc * MMA_N;
+          if (!wait_bounded(smem_u32(&full_bar[stage]), phase, abort_flag, P.err)) {
+            ok = false;
+            break;
+          }
           for (int kb = 0; kb < nkb; ++kb) {
-            if (!wait_bounded(smem_u32(&full_bar[stage]), phase, abort_flag, P.err)) {
-              ok = false;
-              break;
-            }
             const uint64_t qoff = static_cast<uint64_t>((size_t(qb * nkb + kb) * RM_KB_BYTES) >> 4);
-            const uint64_t koff = static_cast<uint64_t>((size_t(stage) * RM_KB_BYTES) >> 4);
+            const uint64_t koff = static_cast<uint64_t>((size_t(stage * nkb + kb) * RM_KB_BYTES) >> 4);
 #pragma unroll
             for (int kk = 0; kk < BK / 16; ++kk)
               umma_bf16_pair(d_tmem, qd0 + qoff + ((kk * 32u) >> 4), kd0 + koff + ((kk * 32u) >> 4), idesc,
                              (kb | kk) != 0);
-            umma_commit_pair_mc(smem_u32(&empty_bar[stage]), 0x3);
-            if (++stage == STG) {
-              stage = 0;
-              phase ^= 1;
-            }
           }
-          if (!ok) break;
+          umma_commit_pair_mc(smem_u32(&empty_bar[stage]), 0x3);
+          if (++stage == STG) {
+            stage = 0;
+            phase ^= 1;
+          }
           umma_commit_pair_mc(smem_u32(&tfull_bar[acc]), 0x3);
           acc ^= 1;
           if (acc == 0) acc_phase ^= 1;
