@@ -442,6 +442,8 @@ int launch_causal_max(const GemmParams& cm, const DeviceState& st, cudaStream_t 
 // stays under the per-SM operand feed limit, but exposes its epilogue.  With a
 // short contraction the main loop of a tile is short and the exposed epilogue
 // (its global reads and writes) would cost more than the narrower tile loses.
+// The plain apply (X' = (aI + B) X, bf16 out, nothing read) has the lightest
+// epilogue and takes the wide tile at every length.
 constexpr int kNarrowMaxK = 2048;
 
 // Up to MAX_GROUPS problem groups of one launch, with their work figures.
@@ -1141,6 +1143,7 @@ int run_muon(const mc_param* params, int n, const mc_hparams* hp, const mc_normu
       const double cnt = double(g.members.size()), dm = double(g.m), dn = double(g.n);
       const int wide_gram = g.n > kNarrowMaxK ? 1 : 0;   // contraction n
       const int wide_m = g.m > kNarrowMaxK ? 1 : 0;      // contraction m (polynomial, apply)
+      const int wide_apply = (wide_m || (!mixed && !last)) ? 1 : 0;
       // A = s^2 X X^T  (oriented; tall matrices read MN-major: X^T X)
       GemmGroup G = base_group(g);
       G.M = G.N = static_cast<int>(g.m);
@@ -1221,8 +1224,8 @@ int run_muon(const mc_param* params, int n, const mc_hparams* hp, const mc_normu
       } else if (!final_apply && !mixed && Mp.ok_x64) {
         eo = &Mp.x_e64[par ^ 1];
       }
-      add_to_batch(applies[wide_m], *st, g.tall ? Mp.x_k[par] : Mp.b_k, g.tall ? Mp.b_k : Mp.x_mn[par], G, wide_m,
-                   fa, fa, eo, ei, ei2);
+      add_to_batch(applies[wide_apply], *st, g.tall ? Mp.x_k[par] : Mp.b_k, g.tall ? Mp.b_k : Mp.x_mn[par], G,
+                   wide_apply, fa, fa, eo, ei, ei2);
     }
     for (int w = 0; w < 2; ++w)
       for (const auto& b : grams[w])
