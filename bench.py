@@ -47,7 +47,7 @@ WORKLOAD = ("7B-shaped Muon step (224 matrices, 7.78e9 params, bf16 W/G, fp32 M,
 # proportional to the matrices processed, so the per-launch figure is this
 # times the layers one launch covers.  Kinds without a capture of the kernel
 # as it stands are absent (reported as null).
-KERNEL_TRAFFIC_PER_LAYER = {"ns_gram": 1.087e9, "ns_apply": 1.711e9}
+KERNEL_TRAFFIC_PER_LAYER = {"ns_gram": 1.033e9, "ns_poly": 0.538e9, "ns_apply": 1.861e9}
 
 # Pieces the end-to-end step splits the gradient upload into.
 E2E_CHUNKS = 16
@@ -487,7 +487,7 @@ def run_config(args, cfg):
             for W, G, M in host:
                 oracle.muon_step(W.double().numpy(), G.double().numpy(), M.double().numpy(), **hp)
             cpu_s = time.perf_counter() - t0
-            sample, extrap = f"the whole config, {cpu_s:.1f} s", None
+            sample, extrap = f"the whole config, {cpu_s:.3g} s", None
         else:
             cpu_s = 0.0
             for idx, count in ((0, 128), (2, 64)):
