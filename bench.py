@@ -368,36 +368,47 @@ CONFIG_WORKLOADS = {
 
 
 def _timed_alone(mc, fn, reps, stream, flush_l2=False):
-    """Device time per call of ``fn`` (CUDA events on ``stream``) and the
-    per-kernel rows over those calls.  With ``flush_l2`` (inputs that fit in
-    L2) a 256 MB buffer is written between calls, outside the timed events."""
+    """Device time per call of ``fn`` (CUDA events on ``stream``), then the
+    per-kernel rows from a second pass of as many calls with the library's
+    per-kernel events on.  The timed pass has no events between kernels, so a
+    tensor-core kernel may start its prologue while the previous kernel of the
+    stream drains (programmatic dependent launch), as in unprofiled use; the
+    per-kernel events of the second pass serialise the launches.  With
+    ``flush_l2`` (inputs that fit in L2) a 256 MB buffer is written between
+    calls, outside the timed events."""
     import torch
     for _ in range(3):
         fn()
     torch.cuda.synchronize()
-    mc.profile_begin()
-    if flush_l2:
-        scrub = torch.empty(256 << 20, dtype=torch.uint8, device=torch.cuda.current_device())
-        evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(reps)]
-        with torch.cuda.stream(stream):
+    scrub = torch.empty(256 << 20, dtype=torch.uint8, device=torch.cuda.current_device()) if flush_l2 else None
+
+    def run(profiled):
+        if profiled:
+            mc.profile_begin()
+        if flush_l2:
+            evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(reps)]
             for a, b in evs:
                 scrub.fill_(1)
                 a.record(stream)
                 fn()
                 b.record(stream)
-        torch.cuda.synchronize()
-        k = mc.profile_end()
+            torch.cuda.synchronize()
+            ms = sum(a.elapsed_time(b) for a, b in evs) / reps
+        else:
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record(stream)
+            for _ in range(reps):
+                fn()
+            b.record(stream)
+            torch.cuda.synchronize()
+            ms = a.elapsed_time(b) / reps
+        k = mc.profile_end() if profiled else None
         assert mc.device_status() == mc.MC_OK, mc.last_error()
-        return sum(a.elapsed_time(b) for a, b in evs) / reps, k
-    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    a.record(stream)
-    for _ in range(reps):
-        fn()
-    b.record(stream)
-    torch.cuda.synchronize()
-    k = mc.profile_end()
-    assert mc.device_status() == mc.MC_OK, mc.last_error()
-    return a.elapsed_time(b) / reps, k
+        return ms, k
+
+    ms, _ = run(False)
+    ms_profiled, k = run(True)
+    return ms, k, ms_profiled
 
 
 def _roofline_row(kernels, peaks, reps):
@@ -459,15 +470,15 @@ def run_config(args, cfg):
             Ws = [(torch.randn(sh, device=dev, generator=g) * 0.02).to(torch.bfloat16) for sh in shapes]
             Gs = [(torch.randn(sh, device=dev, generator=g) * 1e-3).to(torch.bfloat16) for sh in shapes]
             Ms = [torch.zeros(sh, device=dev, dtype=torch.float32) for sh in shapes]
-        ms, k = _timed_alone(mc, lambda: mc.muon_step(Ws, Gs, Ms, stream=stream, **hp), reps, stream,
-                             flush_l2=cfg == 0)
+        ms, k, ms_prof = _timed_alone(mc, lambda: mc.muon_step(Ws, Gs, Ms, stream=stream, **hp), reps, stream,
+                                      flush_l2=cfg == 0)
         dense = ns_dense_flops(shapes, hp["ns_steps"])
         ns_kinds = ("ns_gram", "ns_poly", "ns_apply_mixed", "ns_apply", "ns_apply_final", "ns_thin")
         ns_ms = sum(k[n]["total_ms"] for n in ns_kinds if n in k) / reps
         ns_exec = sum(k[n]["flops_executed"] for n in ns_kinds if n in k) / reps
         mom = k.get("momentum")
         out.update(value=dense / (ms / 1e3) / 1e12, unit="TFLOP/s", ms_per_step=ms, dtype="bf16" if cfg else "f32",
-                   components={"muon_step_ms": ms, "ns_ms": ns_ms,
+                   components={"muon_step_ms": ms, "muon_step_ms_profiled": ms_prof, "ns_ms": ns_ms,
                                "ns_tflops_dense_equiv": dense / (ns_ms / 1e3) / 1e12,
                                "ns_tflops_executed": ns_exec / (ns_ms / 1e3) / 1e12,
                                "ns_frac_burst_dense_equiv": dense / (ns_ms / 1e3) / 1e12 / peaks["bf16_tflops"],
@@ -519,11 +530,12 @@ def run_config(args, cfg):
             mc.qk_clip(wq, wk, smax, H, dh, tau=wl.QK_TAU, alpha=wl.QK_ALPHA, gamma_out=gamma, mask_out=mask,
                        stream=stream)
         reps = max(steps, 20)
-        ms, k = _timed_alone(mc, layer, reps, stream)
+        ms, k, ms_prof = _timed_alone(mc, layer, reps, stream)
         qk_ms = sum(k[n]["total_ms"] for n in ("qk_proj", "qk_causal_max", "qk_keys", "qk_clip") if n in k) / reps
         qf = qk_flops(B, S, D, H, dh)
         out.update(value=B * S / (qk_ms / 1e3), unit="tokens/s", ms_per_step=qk_ms, dtype="bf16",
                    components={"qk_ms": qk_ms, "layer_ms_with_weight_reset": ms,
+                               "layer_ms_with_weight_reset_profiled": ms_prof,
                                "qk_tflops": qf / (qk_ms / 1e3) / 1e12,
                                "qk_proj_tflops": k["qk_proj"]["flops"] / (k["qk_proj"]["total_ms"] / 1e3) / 1e12,
                                "qk_causal_max_tflops": k["qk_causal_max"]["flops"] /
@@ -540,6 +552,8 @@ def run_config(args, cfg):
                                    "ms_per_step": cpu_s * 1e3, "extrapolated": False, "cpu_model": cpu_model(),
                                    "nproc": os.cpu_count()}
     out["kernels"] = {n: dict(v, ms_per_launch=v["total_ms"] / max(v["launches"], 1)) for n, v in k.items()}
+    out["timing"] = ("the step time from CUDA events around the calls with no events between kernels; kernel "
+                     "rows, NS rates and the roofline from a second pass of as many calls with per-kernel events")
     out["roofline"] = _roofline_row(k, peaks, reps)
     out["gpu_launches"] = sum(v["launches"] for n, v in k.items() if n != "table_upload")
     out["peaks"] = peaks

@@ -331,21 +331,35 @@ double gemm_exec_flops(const GemmParams& p) {
 
 // Persistent launch in clusters of two CTAs (one 2-SM MMA pair each), as
 // many pairs as fit on the device at once, at most one per tile.
+// Programmatic stream serialisation for the Newton-Schulz GEMMs: a kernel so
+// launched may begin (its prologue: barriers, TMEM, tensor-map prefetch) while
+// the previous kernel of the stream finishes its last tiles; it touches global
+// memory only after griddepcontrol.wait, i.e. once that kernel has completed
+// and its writes are visible, so stream order is kept for all memory effects.
+// Measured A/B on one box: one fp32 256 x 512 step 0.269 -> 0.239 ms, the MoE
+// set 98.1 -> 97.2 ms, 64 x 1024^2 1.943 -> 1.933 ms; the QK layer (projection
+// and causal max) gained nothing, so its launches keep plain stream order.
+void set_pdl(cudaLaunchAttribute& a, bool on) {
+  a.id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  a.val.programmaticStreamSerializationAllowed = on ? 1 : 0;
+}
+
 template <int EPI, int WIDE>
 cudaError_t launch_pairs(const GemmParams& p, int pair_clusters, cudaStream_t s) {
   const long long pairs = std::min<long long>(pair_clusters, p.total_tiles);
   cudaLaunchConfig_t cfg = {};
-  cudaLaunchAttribute attr[1];
+  cudaLaunchAttribute attr[2];
   attr[0].id = cudaLaunchAttributeClusterDimension;
   attr[0].val.clusterDim.x = 2;
   attr[0].val.clusterDim.y = 1;
   attr[0].val.clusterDim.z = 1;
+  set_pdl(attr[1], EPI != EPI_STORE && EPI != EPI_CAUSALMAX);
   cfg.gridDim = dim3(static_cast<unsigned>(2 * pairs));
   cfg.blockDim = dim3(GEMM_THREADS);
   cfg.dynamicSmemBytes = gemm_smem_bytes<EPI, WIDE>();
   cfg.stream = s;
   cfg.attrs = attr;
-  cfg.numAttrs = 1;
+  cfg.numAttrs = 2;
   return cudaLaunchKernelEx(&cfg, umma_gemm_kernel<EPI, WIDE>, p);
 }
 

@@ -1042,6 +1042,11 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1) umma_gemm_kernel(const __grid
   cluster_sync();   // barriers initialised and TMEM allocated in both CTAs
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
+  // Everything above touches only the parameters, shared memory and TMEM, so
+  // it may overlap the previous kernel's last tiles; no global memory is read
+  // or written before that kernel has completed.
+  griddep_launch_dependents();
+  griddep_wait();
   const long long total = P.total_tiles;
   const long long first_tile = blockIdx.x >> 1;
   const long long tile_step = gridDim.x >> 1;
