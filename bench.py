@@ -368,14 +368,13 @@ CONFIG_WORKLOADS = {
 
 
 def _timed_alone(mc, fn, reps, stream, flush_l2=False):
-    """Device time per call of ``fn`` (CUDA events on ``stream``), then the
-    per-kernel rows from a second pass of as many calls with the library's
-    per-kernel events on.  The timed pass has no events between kernels, so a
-    tensor-core kernel may start its prologue while the previous kernel of the
-    stream drains (programmatic dependent launch), as in unprofiled use; the
-    per-kernel events of the second pass serialise the launches.  With
-    ``flush_l2`` (inputs that fit in L2) a 256 MB buffer is written between
-    calls, outside the timed events."""
+    """Per-kernel rows of ``reps`` calls of ``fn`` with the library's
+    per-kernel CUDA events on, then the device time per call of another
+    ``reps`` calls with events around the calls only (so the NS launches may
+    overlap their prologues, as in unprofiled use; the per-kernel events
+    serialise them).  Clocks are sampled during each pass.  With ``flush_l2``
+    (inputs that fit in L2) a 256 MB buffer is written between calls, outside
+    the timed events."""
     import torch
     for _ in range(3):
         fn()
@@ -383,6 +382,9 @@ def _timed_alone(mc, fn, reps, stream, flush_l2=False):
     scrub = torch.empty(256 << 20, dtype=torch.uint8, device=torch.cuda.current_device()) if flush_l2 else None
 
     def run(profiled):
+        sampler = ClockSampler(torch.cuda.current_device())
+        sampler.start()
+        time.sleep(0.2)
         if profiled:
             mc.profile_begin()
         if flush_l2:
@@ -403,12 +405,13 @@ def _timed_alone(mc, fn, reps, stream, flush_l2=False):
             torch.cuda.synchronize()
             ms = a.elapsed_time(b) / reps
         k = mc.profile_end() if profiled else None
+        clocks = sampler.stop()
         assert mc.device_status() == mc.MC_OK, mc.last_error()
-        return ms, k
+        return ms, k, clocks
 
-    ms, _ = run(False)
-    ms_profiled, k = run(True)
-    return ms, k, ms_profiled
+    ms_prof, k, clocks_prof = run(True)
+    ms, _, clocks = run(False)
+    return ms, k, ms_prof, {"timed_pass": clocks, "profiled_pass": clocks_prof}
 
 
 def _roofline_row(kernels, peaks, reps):
@@ -451,10 +454,10 @@ def run_config(args, cfg):
     if cfg in (0, 1, 4):
         if cfg == 0:
             mats = [wl.cfg0_matrix()]
-            reps = max(steps, 200)
+            reps = max(steps, 1000)
         elif cfg == 1:
             mats = [wl.cfg1_matrix(i) for i in range(64)]
-            reps = max(steps, 50)
+            reps = max(steps, 200)
         else:
             mats = None
             reps = max(steps, 10)
@@ -470,8 +473,8 @@ def run_config(args, cfg):
             Ws = [(torch.randn(sh, device=dev, generator=g) * 0.02).to(torch.bfloat16) for sh in shapes]
             Gs = [(torch.randn(sh, device=dev, generator=g) * 1e-3).to(torch.bfloat16) for sh in shapes]
             Ms = [torch.zeros(sh, device=dev, dtype=torch.float32) for sh in shapes]
-        ms, k, ms_prof = _timed_alone(mc, lambda: mc.muon_step(Ws, Gs, Ms, stream=stream, **hp), reps, stream,
-                                      flush_l2=cfg == 0)
+        ms, k, ms_prof, clocks = _timed_alone(mc, lambda: mc.muon_step(Ws, Gs, Ms, stream=stream, **hp), reps,
+                                              stream, flush_l2=cfg == 0)
         dense = ns_dense_flops(shapes, hp["ns_steps"])
         ns_kinds = ("ns_gram", "ns_poly", "ns_apply_mixed", "ns_apply", "ns_apply_final", "ns_thin")
         ns_ms = sum(k[n]["total_ms"] for n in ns_kinds if n in k) / reps
@@ -529,8 +532,8 @@ def run_config(args, cfg):
             mc.qk_max_logit(x, wq, wk, H, dh, causal=True, smax_out=smax, stream=stream)
             mc.qk_clip(wq, wk, smax, H, dh, tau=wl.QK_TAU, alpha=wl.QK_ALPHA, gamma_out=gamma, mask_out=mask,
                        stream=stream)
-        reps = max(steps, 20)
-        ms, k, ms_prof = _timed_alone(mc, layer, reps, stream)
+        reps = max(steps, 100)
+        ms, k, ms_prof, clocks = _timed_alone(mc, layer, reps, stream)
         qk_ms = sum(k[n]["total_ms"] for n in ("qk_proj", "qk_causal_max", "qk_keys", "qk_clip") if n in k) / reps
         qf = qk_flops(B, S, D, H, dh)
         out.update(value=B * S / (qk_ms / 1e3), unit="tokens/s", ms_per_step=qk_ms, dtype="bf16",
@@ -553,9 +556,10 @@ def run_config(args, cfg):
                                    "nproc": os.cpu_count()}
     out["kernels"] = {n: dict(v, ms_per_launch=v["total_ms"] / max(v["launches"], 1)) for n, v in k.items()}
     out["timing"] = ("the step time from CUDA events around the calls with no events between kernels; kernel "
-                     "rows, NS rates and the roofline from a second pass of as many calls with per-kernel events")
+                     "rows, NS rates and the roofline from a first pass of as many calls with per-kernel events")
+    out["clocks"] = clocks
     out["roofline"] = _roofline_row(k, peaks, reps)
-    out["gpu_launches"] = sum(v["launches"] for n, v in k.items() if n != "table_upload")
+    out["gpu_launches"] = sum(v["launches"] for n, v in k.items())
     out["peaks"] = peaks
     print(json.dumps(out), flush=True)
     return 0
@@ -668,7 +672,7 @@ def run_sharded(args, ctx, shapes, qk_cfg, hp, barrier, max_over_ranks, make_e2e
     e2e = make_e2e(shard, step, step_flops, (smax, gamma, mask)) if make_e2e else None
     if ctx.rank != 0:
         return None
-    launches = sum(v["launches"] for k, v in kernels.items() if k != "table_upload")
+    launches = sum(v["launches"] for k, v in kernels.items())
     roof = None
     ks = {k: v for k, v in kernels.items() if k != "table_upload" and v["total_ms"] > 0}
     if ks:
@@ -842,7 +846,7 @@ def main(argv=None):
     qk_ms = sum(kernels[k]["total_ms"] for k in ("qk_proj", "qk_causal_max", "qk_keys") if k in kernels) / K
     qk_tokens = B * S / (qk_ms / 1e3) if qk_ms > 0 else None
     # kernels only: the parameter-table copy is profiled but is not a launch
-    gpu_launches = sum(v["launches"] for k, v in kernels.items() if k != "table_upload")
+    gpu_launches = sum(v["launches"] for k, v in kernels.items())
 
     # dominant kernel: the kernel kind with the largest device time
     dom = max(((k, v) for k, v in kernels.items() if k != "table_upload"), key=lambda kv: kv[1]["total_ms"])[0]

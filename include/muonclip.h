@@ -24,12 +24,16 @@
  *     retains caller memory beyond the call (the call is asynchronous, so the
  *     buffers must stay valid until the stream reaches that point).
  *   - `stream` is a cudaStream_t (NULL = legacy default stream).  Calls
- *     enqueue work and return without waiting for the device.  The two
- *     exceptions: a call waits for the oldest of the library's parameter-table
- *     uploads on the device when 32 of them are still queued (each Muon-type
- *     call makes one upload, through its own page-locked staging buffer), and,
- *     with a NULL workspace, for the device to go idle when the engine-owned
- *     workspace has to grow.  mc_device_status synchronises.
+ *     enqueue work and return without waiting for the device.  A Muon-type
+ *     call's parameter tables travel inside the parameters of its first
+ *     launches, so no host buffer outlives the call.  The one exception: with
+ *     a NULL workspace a call waits for the device to go idle when the
+ *     engine-owned workspace has to grow.  mc_device_status synchronises.
+ *   - CUDA graphs: a call with a workspace of its own may be captured into a
+ *     graph once an earlier, uncaptured call has set the library up on the
+ *     device; each replay repeats the captured call (same buffers,
+ *     hyper-parameters and workspace).  mc_muon_step_host_grads, calls with a
+ *     NULL workspace and calls made while profiling is on are not capturable.
  *   - Host-side state is guarded by one mutex, so calls may come from several
  *     threads.  GPU work of calls that share the engine-owned workspace (NULL
  *     workspace) or, for mc_muon_step_host_grads, the library's copy stream on
@@ -430,8 +434,9 @@ int mc_selftest_bounded_wait(long long limit_cycles, void* stream);
  *   qk_proj         flops = 2 * B*S * H*dh * D * 2 (Q and K)
  *   qk_causal_max   flops = 2 * dh * (score pairs inside the causal mask)
  *   norm_finalize, qk_keys, qk_clip   (small kernels; counted, no work figure)
- *   table_upload    not a kernel: the host-to-device copy of a call's
- *                   parameter tables (bytes = the table bytes); one per
+ *   table_upload    the launches that carry a call's parameter tables in
+ *                   their parameters to device memory (bytes = the table
+ *                   bytes); one launch per 32704 bytes of tables, per
  *                   mc_muon_step, mc_normuon_step or mc_muon_step_host_grads
  *
  * The rows are written to `out` (up to `max_rows`), `*rows` receives the count.

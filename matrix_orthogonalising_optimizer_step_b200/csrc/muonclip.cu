@@ -59,22 +59,10 @@ using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t
                                    const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
                                    CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
 
-// Page-locked staging buffers for the parameter-table uploads: a call takes a
-// buffer whose last copy has finished, or adds one, and only when this many
-// are still in flight does it wait (for the oldest).
-constexpr int kMaxStaging = 32;
 // Largest dynamic shared memory a CTA may opt into on sm_100.
 constexpr int kSmemOptIn = 232448;
-constexpr size_t kStagingMin = 64 << 10;
 // Newton-Schulz iterations that take a*X from the iterate's hi + lo halves.
 constexpr int kMixedIters = 2;
-
-struct StagingBuf {
-  void* host = nullptr;
-  size_t bytes = 0;
-  cudaEvent_t done = nullptr;  // recorded after the buffer's latest copy
-  unsigned long long seq = 0;  // order of use (the oldest is waited for first)
-};
 
 struct DeviceState {
   bool init = false;
@@ -84,8 +72,6 @@ struct DeviceState {
   int* err_ptr = nullptr;
   void* own_ws = nullptr;
   size_t own_ws_bytes = 0;
-  std::vector<StagingBuf> staging;
-  unsigned long long staging_seq = 0;
   // mc_muon_step_host_grads: a non-blocking stream for the gradient copies and
   // events that order each chunk's compute after its copies
   cudaStream_t copy_stream = nullptr;
@@ -208,59 +194,35 @@ struct ProfScope {
   }
 };
 
-// Copy a small host table into device memory through a page-locked staging
-// buffer, so that the copy is asynchronous and the caller's host memory can be
-// reused at once.  Never waits on the host unless kMaxStaging earlier copies
-// are all still queued on the device.
-int upload(DeviceState& st, const void* host, size_t bytes, void* dst, cudaStream_t s) {
-  if (bytes == 0) return MC_OK;
-  StagingBuf* pick = nullptr;
-  for (auto& b : st.staging) {
-    if (b.bytes < bytes) continue;
-    const cudaError_t q = cudaEventQuery(b.done);
-    if (q == cudaSuccess) {
-      pick = &b;
-      break;
-    }
-    if (q != cudaErrorNotReady) return fail(MC_ERR_CUDA, std::string("cudaEventQuery: ") + cudaGetErrorString(q));
-    // "not ready" is also left as the thread's last error; clear it so that
-    // the launch checks that follow do not take it for a launch failure
-    (void)cudaGetLastError();
+// One launch of table_fill_kernel<BYTES> with `n` bytes (n <= BYTES).
+template <unsigned BYTES>
+int fill_launch(const uint8_t* host, size_t n, uint8_t* dst, cudaStream_t s) {
+  static thread_local TableBlob<BYTES> blob;  // off the stack
+  blob.dst = reinterpret_cast<uint4*>(dst);
+  blob.n16 = static_cast<unsigned>(n / 16);
+  std::memcpy(blob.data, host, n);
+  ProfScope prof(K_TABLE_UPLOAD, s, 0, 0, static_cast<double>(n));
+  table_fill_kernel<BYTES><<<1, 256, 0, s>>>(blob);
+  MC_CUDA(cudaGetLastError());
+  return MC_OK;
+}
+
+// Copy a host table (a multiple of 16 bytes) to 16-byte aligned device
+// memory, in launches of table_fill_kernel that carry it in their parameters.
+// Stream-ordered like any launch, it never waits on the host, the host buffer
+// may be reused at once, and a captured graph keeps its own copy of the bytes.
+int upload(const void* host, size_t bytes, void* dst, cudaStream_t s) {
+  if (bytes % 16 != 0 || !aligned16(dst)) return fail(MC_ERR_INVAL, "internal: table upload not 16-byte aligned");
+  const uint8_t* h = static_cast<const uint8_t*>(host);
+  uint8_t* d = static_cast<uint8_t*>(dst);
+  for (size_t off = 0; off < bytes;) {
+    const size_t n = std::min<size_t>(TABLE_BLOB_MAX, bytes - off);
+    int rc = n <= 1024   ? fill_launch<1024>(h + off, n, d + off, s)
+             : n <= 4096 ? fill_launch<4096>(h + off, n, d + off, s)
+                         : fill_launch<TABLE_BLOB_MAX>(h + off, n, d + off, s);
+    if (rc != MC_OK) return rc;
+    off += n;
   }
-  if (!pick && static_cast<int>(st.staging.size()) < kMaxStaging) {
-    StagingBuf b;
-    b.bytes = std::max(bytes, kStagingMin);
-    MC_CUDA(cudaMallocHost(&b.host, b.bytes));
-    const cudaError_t e = cudaEventCreateWithFlags(&b.done, cudaEventDisableTiming);
-    if (e != cudaSuccess) {
-      cudaFreeHost(b.host);
-      return fail(MC_ERR_CUDA, std::string("cudaEventCreateWithFlags: ") + cudaGetErrorString(e));
-    }
-    st.staging.push_back(b);
-    pick = &st.staging.back();
-  }
-  if (!pick) {
-    // every buffer is in flight: wait for the oldest, then reuse (and if
-    // need be enlarge) it
-    pick = &st.staging.front();
-    for (auto& b : st.staging)
-      if (b.seq < pick->seq) pick = &b;
-    MC_CUDA(cudaEventSynchronize(pick->done));
-    if (pick->bytes < bytes) {
-      MC_CUDA(cudaFreeHost(pick->host));
-      pick->host = nullptr;
-      pick->bytes = 0;
-      MC_CUDA(cudaMallocHost(&pick->host, bytes));
-      pick->bytes = bytes;
-    }
-  }
-  pick->seq = ++st.staging_seq;
-  std::memcpy(pick->host, host, bytes);
-  {
-    ProfScope prof(K_TABLE_UPLOAD, s, 0, 0, static_cast<double>(bytes));
-    MC_CUDA(cudaMemcpyAsync(dst, pick->host, bytes, cudaMemcpyHostToDevice, s));
-  }
-  MC_CUDA(cudaEventRecord(pick->done, s));
   return MC_OK;
 }
 
@@ -810,7 +772,8 @@ int upload_piece_tables(DeviceState& st, const mc_param* params, const mc_hparam
     build_muon_table(params + P.bounds[k], P.bounds[k + 1] - P.bounds[k], hp, pn, ws, P.layouts[k],
                      tabs.data() + (P.tab_off[k] - t0));
   }
-  return upload(st, tabs.data(), tabs.size(), ws + t0, s);
+  (void)st;
+  return upload(tabs.data(), tabs.size(), ws + t0, s);
 }
 
 // mc_muon_step / mc_normuon_step body: the tables of every piece in one

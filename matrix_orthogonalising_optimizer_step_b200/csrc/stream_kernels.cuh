@@ -198,6 +198,27 @@ __global__ void norm_finalize_kernel(const MomEntry* __restrict__ tab, int n, co
   }
 }
 
+// A parameter table of up to BYTES carried in the launch's own parameters:
+// the launch copies them, so the caller's host buffer is free as soon as the
+// launch returns, no host memory is read later, and the upload stays valid
+// when the launch is captured into a CUDA graph.  The launch queue holds the
+// whole parameter block, so a table takes the smallest size that fits; the
+// largest (32720 bytes of parameters) stays under the 32764-byte limit.
+constexpr unsigned TABLE_BLOB_MAX = 32704;
+template <unsigned BYTES>
+struct TableBlob {
+  uint4* dst;     // 16-byte aligned
+  unsigned n16;   // 16-byte words to copy, <= BYTES / 16
+  unsigned pad_;
+  uint4 data[BYTES / 16];
+};
+static_assert(sizeof(TableBlob<TABLE_BLOB_MAX>) <= 32764, "kernel parameters");
+
+template <unsigned BYTES>
+__global__ void table_fill_kernel(const __grid_constant__ TableBlob<BYTES> b) {
+  for (unsigned i = threadIdx.x; i < b.n16; i += blockDim.x) b.dst[i] = b.data[i];
+}
+
 __global__ void qk_keys_init_kernel(int* keys, int H) {
   const int h = blockIdx.x * blockDim.x + threadIdx.x;
   if (h < H) keys[h] = INT_MIN;

@@ -1,8 +1,10 @@
 """A Muon-type call enqueues its work and returns without waiting for the
-device: every piece's parameter tables go up in one copy at the start of the
-call, through a page-locked staging buffer of its own ("MuonClip: speed, then
-stability", §07: the optimizer step is one stage of a training step, so the
-host must be free to queue the next stage behind it)."""
+device: every piece's parameter tables go up at the start of the call inside
+the parameters of a small copy kernel, so no host buffer has to outlive the
+call ("MuonClip: speed, then stability", §07: the optimizer step is one stage
+of a training step, so the host must be free to queue the next stage behind
+it).  For the same reason a call can be captured into a CUDA graph and
+replayed."""
 import time
 
 import pytest
@@ -50,8 +52,8 @@ def test_eight_piece_call_returns_while_the_device_is_busy(hp):
 
 
 def test_many_calls_queue_without_waiting(hp):
-    """Twenty calls behind a busy stream: each takes a staging buffer of its
-    own, so none waits for an earlier call's table copy."""
+    """Twenty calls behind a stream that stays busy for a second: none of them
+    waits on the host for an earlier call's table copy."""
     Ws = [torch.randn((256, 384), device=DEV).to(torch.bfloat16) * 0.02 for _ in range(3)]
     Gs = [torch.randn((256, 384), device=DEV).to(torch.bfloat16) * 1e-3 for _ in range(3)]
     Ms = [torch.zeros((256, 384), device=DEV) for _ in range(3)]
@@ -69,24 +71,44 @@ def test_many_calls_queue_without_waiting(hp):
     assert host_s < 0.5, host_s
 
 
-def test_thirty_third_queued_copy_waits_for_the_oldest(hp):
-    """The staging pool holds 32 buffers: behind a stream that stays busy for
-    a second, 32 calls queue at once and the 33rd waits (on the host) until
-    the first call's table copy has run, i.e. until the busy kernel ends."""
-    Ws = [torch.randn((128, 192), device=DEV).to(torch.bfloat16) * 0.02]
-    Gs = [torch.randn((128, 192), device=DEV).to(torch.bfloat16) * 1e-3]
-    Ms = [torch.zeros((128, 192), device=DEV)]
-    for _ in range(40):   # the pool reaches its 32 buffers
-        mc.muon_step(Ws, Gs, Ms, **hp)
+def _workspace_for(Ws, Gs, Ms, hp):
+    import ctypes
+    lib = mc.load_library()
+    arr, n = mc.make_params(Ws, Gs, Ms, None)
+    need = int(lib.mc_muon_workspace_size(arr, n, ctypes.byref(mc.make_hparams(**hp))))
+    return torch.empty(need, dtype=torch.uint8, device=DEV)
+
+
+def test_captured_step_replays_like_direct_calls(hp):
+    """A step captured into a CUDA graph (with a workspace of its own) and
+    replayed twice gives, bit for bit, what two direct calls give: the tables
+    travel inside the captured launches, so a replay re-reads nothing from the
+    host."""
+    g = torch.Generator(device=DEV)
+    g.manual_seed(11)
+    shapes = [(256, 768), (768, 256), (512, 512), (300, 520)]
+    W0 = [(torch.randn(sh, device=DEV, generator=g) * 0.02).to(torch.bfloat16) for sh in shapes]
+    Gs = [(torch.randn(sh, device=DEV, generator=g) * 1e-3).to(torch.bfloat16) for sh in shapes]
+    M0 = [torch.randn(sh, device=DEV, generator=g) * 1e-4 for sh in shapes]
+    WE, ME = [w.clone() for w in W0], [m.clone() for m in M0]
+    WC, MC = [w.clone() for w in W0], [m.clone() for m in M0]
+    wsE, wsC = _workspace_for(WE, Gs, ME, hp), _workspace_for(WC, Gs, MC, hp)
+    for _ in range(2):
+        mc.muon_step(WE, Gs, ME, workspace=wsE, **hp)
     torch.cuda.synchronize()
-    _busy_stream(1.0)
-    t0 = time.perf_counter()
-    for _ in range(32):
-        mc.muon_step(Ws, Gs, Ms, **hp)
-    queued_s = time.perf_counter() - t0
-    mc.muon_step(Ws, Gs, Ms, **hp)
-    waited_s = time.perf_counter() - t0 - queued_s
+    side = torch.cuda.Stream()
+    side.wait_stream(torch.cuda.current_stream())
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph, stream=side):
+        mc.muon_step(WC, Gs, MC, workspace=wsC, **hp)
+    torch.cuda.synchronize()
+    # capturing ran nothing
+    for w, w0 in zip(WC, W0):
+        assert torch.equal(w, w0)
+    graph.replay()
+    graph.replay()
     torch.cuda.synchronize()
     assert mc.device_status() == mc.MC_OK, mc.last_error()
-    assert queued_s < 0.5, queued_s
-    assert waited_s > 0.2, waited_s
+    for a, b in zip(WC + MC, WE + ME):
+        assert torch.equal(a, b)
+    del graph
