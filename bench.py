@@ -47,7 +47,7 @@ WORKLOAD = ("7B-shaped Muon step (224 matrices, 7.78e9 params, bf16 W/G, fp32 M,
 # proportional to the matrices processed, so the per-launch figure is this
 # times the layers one launch covers.  Kinds without a capture of the kernel
 # as it stands are absent (reported as null).
-KERNEL_TRAFFIC_PER_LAYER = {"ns_gram": 1.033e9, "ns_poly": 0.538e9, "ns_apply": 1.861e9}
+KERNEL_TRAFFIC_PER_LAYER = {"ns_gram": 0.990e9, "ns_poly": 0.534e9, "ns_apply": 1.797e9}
 
 # Pieces the end-to-end step splits the gradient upload into.
 E2E_CHUNKS = 16
