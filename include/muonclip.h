@@ -99,6 +99,12 @@ typedef struct {
                           the simple quintic (2, -1.5, 0.5) of "Muon and MuonClip:
                           orthogonalised updates for LLM training" §2, or a
                           per-step schedule; NULL = (a, b, c) in every iteration */
+  const float* lr_wd; /* optional device fp32 [2]: (lr, wd) read by the kernels when
+                         they run, in place of lr and wd above (which are then not
+                         used), so that a step captured into a CUDA graph can follow
+                         a learning-rate schedule: write the next values before each
+                         replay.  Finite values are the caller's responsibility.
+                         NULL = lr and wd above */
 } mc_hparams;
 
 /*

@@ -45,7 +45,7 @@ class McHparams(ctypes.Structure):
     _fields_ = [("mu", ctypes.c_float), ("nesterov", ctypes.c_int32), ("lr", ctypes.c_float),
                 ("wd", ctypes.c_float), ("ns_steps", ctypes.c_int32), ("a", ctypes.c_float),
                 ("b", ctypes.c_float), ("c", ctypes.c_float), ("eps", ctypes.c_float),
-                ("rms_scale", ctypes.c_float), ("coeffs", ctypes.c_void_p)]
+                ("rms_scale", ctypes.c_float), ("coeffs", ctypes.c_void_p), ("lr_wd", ctypes.c_void_p)]
 
 
 class McNormuon(ctypes.Structure):
@@ -236,12 +236,20 @@ def _check_out(t, name, dtype, n):
 
 
 def make_hparams(mu=0.95, nesterov=True, lr=0.02, wd=0.1, ns_steps=5, a=3.4445, b=-4.7750,
-                 c=2.0315, eps=1e-7, rms_scale=0.2, coeffs=None) -> McHparams:
+                 c=2.0315, eps=1e-7, rms_scale=0.2, coeffs=None, lr_wd=None) -> McHparams:
     """``coeffs``: optional list of ns_steps (a_k, b_k, c_k) triples, one per
     Newton-Schulz iteration.  The returned struct keeps the coefficient array
-    alive (as ``_coeff_buf``)."""
+    alive (as ``_coeff_buf``).  ``lr_wd``: optional CUDA float32 tensor of two
+    elements (lr, wd) that the kernels read when they run, in place of ``lr``
+    and ``wd`` (for a learning-rate schedule under a captured CUDA graph)."""
     h = McHparams(float(mu), int(bool(nesterov)), float(lr), float(wd), int(ns_steps),
-                  float(a), float(b), float(c), float(eps), float(rms_scale), None)
+                  float(a), float(b), float(c), float(eps), float(rms_scale), None, None)
+    if lr_wd is not None:
+        torch = _torch()
+        if not (lr_wd.is_cuda and lr_wd.dtype == torch.float32 and lr_wd.is_contiguous() and lr_wd.numel() == 2):
+            raise ValueError("lr_wd must be a contiguous CUDA float32 tensor of two elements (lr, wd)")
+        h._lr_wd = lr_wd
+        h.lr_wd = lr_wd.data_ptr()
     if coeffs is not None:
         flat = [float(v) for t in coeffs for v in t]
         if len(flat) != 3 * int(ns_steps):

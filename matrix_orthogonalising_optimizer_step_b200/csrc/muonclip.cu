@@ -484,6 +484,13 @@ struct MuonLayout {
   size_t off_ttab = 0, off_tpart = 0, off_pmat = 0;
 };
 
+// 1 - lr*wd as two rounded fp32 operations (the kernels that read a device
+// (lr, wd) pair do the same, so both routes give the same bits).
+float host_decay(const mc_hparams* hp) {
+  volatile float t = hp->lr * hp->wd;
+  return 1.f - t;
+}
+
 int validate_muon(const mc_param* params, int n, const mc_hparams* hp) {
   if (n < 0) return fail(MC_ERR_INVAL, "n must be >= 0");
   if (n > 0 && !params) return fail(MC_ERR_INVAL, "params is NULL");
@@ -496,6 +503,8 @@ int validate_muon(const mc_param* params, int n, const mc_hparams* hp) {
     for (int i = 0; i < 3 * hp->ns_steps; ++i)
       if (!std::isfinite(hp->coeffs[i])) return fail(MC_ERR_INVAL, "non-finite coefficient in hp->coeffs");
   if (!(hp->eps > 0.f)) return fail(MC_ERR_INVAL, "eps must be > 0");
+  if (hp->lr_wd && (reinterpret_cast<uintptr_t>(hp->lr_wd) & 3u) != 0)
+    return fail(MC_ERR_ALIGN, "hp->lr_wd must be 4-byte aligned");
   for (int i = 0; i < n; ++i) {
     const mc_param& q = params[i];
     const std::string at = "params[" + std::to_string(i) + "]: ";
@@ -1183,8 +1192,9 @@ int run_muon(const mc_param* params, int n, const mc_hparams* hp, const mc_normu
         G.w_f32 = g.w_f32;
         G.w_vec = g.w_f32 ? (g.cols % 4 == 0) : (g.cols % 8 == 0);
         G.rms = hp->rms_scale * std::sqrt(static_cast<float>(std::max(g.rows, g.cols)));
-        G.decay = 1.f - hp->lr * hp->wd;
+        G.decay = host_decay(hp);
         G.step = -hp->lr * G.rms;
+        G.lr_wd = hp->lr_wd;
       }
       const double fa = 2.0 * dm * dm * dn * cnt;
       // epilogue maps: none for the last apply (each weight has its own
@@ -1237,7 +1247,7 @@ int run_muon(const mc_param* params, int n, const mc_hparams* hp, const mc_normu
       thin_poly_kernel<<<static_cast<unsigned>(L.n_thin), THIN_THREADS, 0, s>>>(ttab, tpart, ca, cb, cc);
       MC_CUDA(cudaGetLastError());
       thin_apply_kernel<<<static_cast<unsigned>(L.thin_ctas), THIN_THREADS, 0, s>>>(
-          ttab, L.n_thin, last ? 1 : 0, 1.f - hp->lr * hp->wd, -hp->lr);
+          ttab, L.n_thin, last ? 1 : 0, host_decay(hp), -hp->lr, hp->lr_wd);
       MC_CUDA(cudaGetLastError());
     }
   }
@@ -1265,7 +1275,7 @@ int run_muon(const mc_param* params, int n, const mc_hparams* hp, const mc_normu
     {
       ProfScope prof(K_NORM_APPLY, s, 0, 0, w_bytes);
       normuon_apply_kernel<<<static_cast<unsigned>(L.total_ctas), NORM_THREADS, 0, s>>>(
-          ntab, n, rowf, 1.f - hp->lr * hp->wd, -hp->lr);
+          ntab, n, rowf, host_decay(hp), -hp->lr, hp->lr_wd);
       MC_CUDA(cudaGetLastError());
     }
   }

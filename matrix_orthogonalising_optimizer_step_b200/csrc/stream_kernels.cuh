@@ -356,8 +356,13 @@ __global__ void normuon_finalize_kernel(const NormEntry* __restrict__ tab, const
 // W <- decay W + step * (rowf_i O_ij), update_out = rms * rowf_i O_ij;
 // MOM_ELEMS_PER_CTA elements of one matrix per CTA, 8 at a time when rows are
 // 16-byte multiples.
+// lr_wd: optional device (lr, wd) replacing decay = 1 - lr*wd and neg_lr = -lr.
 __global__ void normuon_apply_kernel(const NormEntry* __restrict__ tab, int n, const float* __restrict__ rowf,
-                                     float decay, float neg_lr) {
+                                     float decay, float neg_lr, const float* __restrict__ lr_wd) {
+  if (lr_wd) {
+    decay = __fsub_rn(1.f, __fmul_rn(lr_wd[0], lr_wd[1]));
+    neg_lr = -lr_wd[0];
+  }
   const int k = find_entry(n, blockIdx.x, [&](int i) { return tab[i].cta_begin; });
   const NormEntry& E = tab[k];
   const long long total = E.rows * E.cols;

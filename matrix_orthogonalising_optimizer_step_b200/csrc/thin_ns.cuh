@@ -147,8 +147,14 @@ __global__ void __launch_bounds__(THIN_THREADS) thin_poly_kernel(const ThinEntry
 
 // X <- P X, one thread per column of the oriented X; on the last iteration
 // (when the entry has a weight) W = decay W + step * X_new instead.
+// lr_wd: optional device (lr, wd) replacing decay = 1 - lr*wd and neg_lr = -lr.
 __global__ void __launch_bounds__(THIN_THREADS) thin_apply_kernel(const ThinEntry* __restrict__ tab, int n,
-                                                                  int last, float decay, float neg_lr) {
+                                                                  int last, float decay, float neg_lr,
+                                                                  const float* __restrict__ lr_wd) {
+  if (lr_wd) {
+    decay = __fsub_rn(1.f, __fmul_rn(lr_wd[0], lr_wd[1]));
+    neg_lr = -lr_wd[0];
+  }
   const ThinEntry& E = tab[thin_find(tab, n, blockIdx.x)];
   const long long j0 = ((long long)blockIdx.x - E.cta_begin) * THIN_COLS;
   const int cols = static_cast<int>(E.n - j0 < THIN_COLS ? E.n - j0 : THIN_COLS);

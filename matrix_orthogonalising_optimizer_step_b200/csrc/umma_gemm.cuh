@@ -182,9 +182,24 @@ struct GemmGroup {
   float coef_acc, coef_src;
   float diag;              // EPI_POLY: added on the diagonal (a for P = aI + B)
   float decay, step, rms;  // EPI_APPLY_FINAL
+  const float* lr_wd;      // EPI_APPLY_FINAL: device (lr, wd) replacing decay and step, or null
   float out_scale;         // EPI_CAUSALMAX: 1/sqrt(d_head)
   int tma_epi;             // the group's epilogue tensor maps are set (map_eo, map_ei, map_ei2)
 };
+
+// The last apply's W <- decay W + step O coefficients: the group's own, or
+// computed when the kernel runs from a device (lr, wd) pair, with the same
+// fp32 operations (and roundings) as the host's 1 - lr*wd and -lr*rms.
+__device__ __forceinline__ void final_coefs(const GemmGroup& G, float& decay, float& step) {
+  if (G.lr_wd) {
+    const float lr = G.lr_wd[0], wd = G.lr_wd[1];
+    decay = __fsub_rn(1.f, __fmul_rn(lr, wd));
+    step = __fmul_rn(-lr, G.rms);
+  } else {
+    decay = G.decay;
+    step = G.step;
+  }
+}
 
 template <int EPI>
 __device__ __forceinline__ bool apply_reads_x(const GemmGroup& G) {
@@ -532,9 +547,10 @@ __device__ __forceinline__ void epi_finish(const GemmGroup& G, int prob, int r, 
       } else {
         raw_to_bf16x16(pre.w, w);
       }
-      float nw[16];
+      float nw[16], decay, step;
+      final_coefs(G, decay, step);
 #pragma unroll
-      for (int j = 0; j < 16; ++j) nw[j] = fmaf(G.step, o[j], G.decay * w[j]);
+      for (int j = 0; j < 16; ++j) nw[j] = fmaf(step, o[j], decay * w[j]);
       if (G.w_f32) {
         float* W = static_cast<float*>(G.w_ptrs[prob]) + row;
         if (full && G.w_vec) {
@@ -789,10 +805,12 @@ __device__ __forceinline__ void epi_fast64(const GemmGroup& G, int prob, int r0,
     warp_store_rows64(D, G.d_ld, lane, buf, pk);
   } else if constexpr (EPI == EPI_APPLY_FINAL) {
     warp_rows_from_frags(ga, lane, buf, pk);
+    float decay, step;
+    final_coefs(G, decay, step);
 #pragma unroll
     for (int i = 0; i < 32; ++i)
-      pk[i] = pack_bf16x2(fmaf(G.step, v[2 * i], G.decay * bf16_lo(pk[i])),
-                          fmaf(G.step, v[2 * i + 1], G.decay * bf16_hi(pk[i])));
+      pk[i] = pack_bf16x2(fmaf(step, v[2 * i], decay * bf16_lo(pk[i])),
+                          fmaf(step, v[2 * i + 1], decay * bf16_hi(pk[i])));
     warp_store_rows64(static_cast<__nv_bfloat16*>(G.w_ptrs[prob]) + (long long)r0 * G.N + c0, G.N, lane, buf, pk);
   } else if constexpr (EPI == EPI_STORE) {
     pack_row64(v, pk);

@@ -112,3 +112,49 @@ def test_captured_step_replays_like_direct_calls(hp):
     for a, b in zip(WC + MC, WE + ME):
         assert torch.equal(a, b)
     del graph
+
+
+def test_device_learning_rate_under_a_captured_graph(hp):
+    """With hparams.lr_wd pointing at a device (lr, wd) pair, the kernels read
+    the learning rate when they run: one captured step replayed under a
+    changing schedule matches direct calls made with those values on the host,
+    bit for bit (GEMM path, thin path and NorMuon's row pass)."""
+    g = torch.Generator(device=DEV)
+    g.manual_seed(12)
+    shapes = [(256, 768), (768, 256), (16, 300), (300, 24)]
+    W0 = [(torch.randn(sh, device=DEV, generator=g) * 0.02).to(torch.bfloat16) for sh in shapes]
+    Gs = [(torch.randn(sh, device=DEV, generator=g) * 1e-3).to(torch.bfloat16) for sh in shapes]
+    M0 = [torch.randn(sh, device=DEV, generator=g) * 1e-4 for sh in shapes]
+    base = {k: v for k, v in hp.items() if k not in ("lr", "wd")}
+    lr_wd = torch.tensor([0.02, 0.1], device=DEV, dtype=torch.float32)
+    dev_hp = mc.make_hparams(lr_wd=lr_wd, **base)
+    WE, ME = [w.clone() for w in W0], [m.clone() for m in M0]
+    WC, MC = [w.clone() for w in W0], [m.clone() for m in M0]
+    wsE, wsC = _workspace_for(WE, Gs, ME, hp), _workspace_for(WC, Gs, MC, hp)
+    mc.muon_step([W0[0].clone()], Gs[:1], [M0[0].clone()], **hp)   # set-up call, on copies
+    torch.cuda.synchronize()
+    side = torch.cuda.Stream()
+    side.wait_stream(torch.cuda.current_stream())
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph, stream=side):
+        mc.muon_step(WC, Gs, MC, workspace=wsC, hparams=dev_hp)
+    torch.cuda.synchronize()
+    for lr in (0.02, 0.01, 0.003):
+        lr_wd.copy_(torch.tensor([lr, 0.1], device=DEV))
+        graph.replay()
+        mc.muon_step(WE, Gs, ME, workspace=wsE, hparams=mc.make_hparams(lr=lr, wd=0.1, **base))
+        torch.cuda.synchronize()
+        for a, b in zip(WC + MC, WE + ME):
+            assert torch.equal(a, b), lr
+    del graph
+    # NorMuon: the device pair against the host values, directly
+    vs0 = [torch.rand(r, device=DEV, generator=g) * 1e-6 for r, _ in shapes]
+    W1, M1, V1 = [w.clone() for w in W0], [m.clone() for m in M0], [v.clone() for v in vs0]
+    W2, M2, V2 = [w.clone() for w in W0], [m.clone() for m in M0], [v.clone() for v in vs0]
+    lr_wd.copy_(torch.tensor([0.007, 0.05], device=DEV))
+    mc.normuon_step(W1, Gs, M1, V1, hparams=mc.make_hparams(lr_wd=lr_wd, **base))
+    mc.normuon_step(W2, Gs, M2, V2, hparams=mc.make_hparams(lr=0.007, wd=0.05, **base))
+    torch.cuda.synchronize()
+    assert mc.device_status() == mc.MC_OK, mc.last_error()
+    for a, b in zip(W1 + M1 + V1, W2 + M2 + V2):
+        assert torch.equal(a, b)
