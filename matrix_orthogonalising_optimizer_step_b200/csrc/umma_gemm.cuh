@@ -40,7 +40,8 @@
 // pair's B is split between the two SMs).  No TMA multicast is used.
 //
 // Warp roles (320 threads per CTA):
-//   warp 0      TMA producer: ring of {A 128x64, one or two B 128x64} bf16 tiles,
+//   warp 0      TMA producer: ring of stages, each one or two k-blocks of
+//               {A 128x64, one or two B 128x64} bf16 tiles (TileCfg::KPS),
 //               128-byte swizzled, K-major or MN-major per group.  Both CTAs'
 //               copies complete on the leader CTA's "full" barrier.
 //   warp 1      TMEM allocation (512 columns, both CTAs, 2-SM form); in the
@@ -51,7 +52,11 @@
 //               group (w-2)/4 of the tile; the leader's "accumulator empty"
 //               barrier counts both CTAs' epilogue warps.  Whole 32-row
 //               blocks move to and from global memory through a per-warp
-//               shared-memory buffer (coalesced rows; see epi_fast64).
+//               shared-memory buffer (TMA where the operand has a tensor map,
+//               else coalesced rows; see epi_tma_block and epi_fast64).
+// Every role starts after griddepcontrol.wait: the prologue (barriers, TMEM,
+// tensor-map prefetch) may overlap the previous kernel of the stream when the
+// launch allows programmatic serialisation.
 #pragma once
 
 #include <climits>
