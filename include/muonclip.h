@@ -461,6 +461,14 @@ typedef struct {
 int mc_profile_begin(void);
 int mc_profile_end(mc_kernel_stat* out, int max_rows, int* rows);
 
+/*
+ * mc_struct_size -- host-only: sizeof of this header's structures as the
+ * library was built, for bindings that lay the structures out themselves:
+ * 0 mc_param, 1 mc_hparams, 2 mc_normuon, 3 mc_clip_slice, 4 mc_kernel_stat;
+ * 0 for any other index.
+ */
+size_t mc_struct_size(int which);
+
 #ifdef __cplusplus
 }
 #endif

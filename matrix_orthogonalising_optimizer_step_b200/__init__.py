@@ -29,7 +29,8 @@ EXPORTS = ("mc_muon_workspace_size", "mc_muon_step", "mc_qk_workspace_size", "mc
            "mc_qk_clip", "mc_last_error", "mc_device_status", "mc_profile_begin", "mc_profile_end",
            "mc_qk_max_logit_static", "mc_qk_clip_slices", "mc_mla_workspace_size", "mc_mla_max_logit",
            "mc_shard_plan", "mc_normuon_workspace_size", "mc_normuon_step", "mc_polar_express_coeffs",
-           "mc_muon_host_grads_workspace_size", "mc_muon_step_host_grads", "mc_selftest_bounded_wait")
+           "mc_muon_host_grads_workspace_size", "mc_muon_step_host_grads", "mc_selftest_bounded_wait",
+           "mc_struct_size")
 MC_QK_STATIC_MAX_ELEMS = 1 << 24
 MC_QK_STATIC_MAX_HEADS = 4096
 
@@ -121,6 +122,8 @@ def load_library():
     lib.mc_shard_plan.restype = i32
     lib.mc_selftest_bounded_wait.argtypes = [ctypes.c_longlong, vp]
     lib.mc_selftest_bounded_wait.restype = i32
+    lib.mc_struct_size.argtypes = [i32]
+    lib.mc_struct_size.restype = sz
     lib.mc_profile_begin.argtypes = []
     lib.mc_profile_begin.restype = i32
     lib.mc_profile_end.argtypes = [P(McKernelStat), i32, P(ctypes.c_int)]

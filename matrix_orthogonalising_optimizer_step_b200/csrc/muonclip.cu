@@ -1675,6 +1675,17 @@ __global__ void bounded_wait_selftest_kernel(int* err, long long limit) {
 }
 }  // namespace mc
 
+MC_API size_t mc_struct_size(int which) {
+  switch (which) {
+    case 0: return sizeof(mc_param);
+    case 1: return sizeof(mc_hparams);
+    case 2: return sizeof(mc_normuon);
+    case 3: return sizeof(mc_clip_slice);
+    case 4: return sizeof(mc_kernel_stat);
+    default: return 0;
+  }
+}
+
 MC_API int mc_selftest_bounded_wait(long long limit_cycles, void* stream) {
   if (limit_cycles < 1000 || limit_cycles > kWaitLimitCycles)
     return fail(MC_ERR_INVAL, "limit_cycles must be in [1000, 2^32]");

@@ -33,6 +33,14 @@ def test_header_declares_the_three_operations():
         assert n in names
 
 
+def test_binding_structures_match_the_header(lib):
+    """The ctypes layouts of the binding have the sizes of the C structures
+    the library was built with (a field added on one side only fails here)."""
+    for which, cls in enumerate((mc.McParam, mc.McHparams, mc.McNormuon, mc.McClipSlice, mc.McKernelStat)):
+        assert lib.mc_struct_size(which) == ctypes.sizeof(cls), cls.__name__
+    assert lib.mc_struct_size(5) == 0
+
+
 def test_library_exports_every_declared_symbol(lib):
     names = declared_functions()
     assert set(names) == set(mc.EXPORTS)
