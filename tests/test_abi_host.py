@@ -83,6 +83,10 @@ def test_argument_errors_return_codes_without_a_gpu(lib):
     assert lib.mc_muon_step(a, 1, P(hp), None, 0, None, None) == mc.MC_ERR_INVAL
     a = _params(1); a[0].g = a[0].g + 2
     assert lib.mc_muon_step(a, 1, P(hp), None, 0, None, None) == mc.MC_ERR_ALIGN
+    # a device (lr, wd) pair must be 4-byte aligned (its values are the caller's)
+    h = mc.make_hparams(); h.lr_wd = 0x900002
+    assert lib.mc_muon_step(arr, 2, P(h), None, 0, None, None) == mc.MC_ERR_ALIGN
+    assert lib.mc_muon_workspace_size(arr, 2, P(h)) == 0
     # n == 0 is a no-op
     assert lib.mc_muon_step(arr, 0, P(hp), None, 0, None, None) == mc.MC_OK
     # QK
