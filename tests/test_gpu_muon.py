@@ -265,3 +265,16 @@ def test_matrix_past_2_31_elements(hp, r, c):
     del W, G, M, X0, O, P
     mc.release_workspaces()
     torch.cuda.empty_cache()
+
+
+def test_many_matrices_tables_in_several_launches(hp):
+    """Four hundred small matrices in one call: their parameter tables (about
+    38 KB) go up in two table launches (32704 bytes of parameters at most per
+    launch).  Every matrix is checked against the oracle."""
+    shapes = [(64, 96), (96, 64), (48, 80), (128, 128)]
+    mats = [wl.generic_matrix(*shapes[i % 4], seed=1000 + i) for i in range(400)]
+    mc.profile_begin()
+    outs = run_step(mats, hp)
+    k = mc.profile_end()
+    assert k["table_upload"]["launches"] == 2, k["table_upload"]
+    check_all(mats, hp, outs, "many")
