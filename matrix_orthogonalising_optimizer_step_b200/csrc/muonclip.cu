@@ -1208,7 +1208,9 @@ int run_muon(const mc_param* params, int n, const mc_hparams* hp, const mc_normu
         eo = &Mp.x_e32[par ^ 1];
         ei = &Mp.x_e32[par];
         ei2 = &Mp.xl_e32;
-      } else if (!final_apply && !mixed && Mp.ok_x64) {
+      } else if (!final_apply && !mixed && Mp.ok_x64 && !(last && nm)) {
+        // (NorMuon's last apply writes the fp32 NS output through the
+        // warp-coalesced path instead)
         eo = &Mp.x_e64[par ^ 1];
       }
       add_to_batch(applies[wide_apply], *st, g.tall ? Mp.x_k[par] : Mp.b_k, g.tall ? Mp.b_k : Mp.x_mn[par], G,

@@ -176,7 +176,7 @@ struct GemmGroup {
   long long xf_ld, xf_bs;
   int xf_read;             // EPI_APPLY*: take a*X from hi + lo
   int xl_write;            // EPI_APPLY: store the new iterate's lo half to xl
-  int xf_write;            // EPI_APPLY: store the new iterate in fp32 to xf
+  int xf_write;            // EPI_APPLY: store the new (last) iterate in fp32 to xf instead of d
   void* const* w_ptrs;     // per-problem weight (EPI_APPLY_FINAL), row-major M x N
   float* const* u_ptrs;    // per-problem update output, entries may be null
   const float* scale;      // per-problem s, or null for 1
@@ -521,14 +521,14 @@ __device__ __forceinline__ void epi_finish(const GemmGroup& G, int prob, int r, 
       if (full) {
         if (G.xf_write) store_f32x16(X + c0, o);
         if (G.xl_write) store_bf16x16(XL + c0, lo);
-        store_bf16x16(D + c0, o);
+        if (!G.xf_write) store_bf16x16(D + c0, o);
       } else {
 #pragma unroll
         for (int j = 0; j < 16; ++j)
           if (c0 + j < G.N) {
             if (G.xf_write) X[c0 + j] = o[j];
             if (G.xl_write) XL[c0 + j] = __float2bfloat16_rn(lo[j]);
-            D[c0 + j] = __float2bfloat16_rn(o[j]);
+            if (!G.xf_write) D[c0 + j] = __float2bfloat16_rn(o[j]);
           }
       }
     } else {
@@ -668,6 +668,28 @@ __device__ __forceinline__ void warp_store_rows64(__nv_bfloat16* base, long long
 __device__ __forceinline__ uint32_t epi_swz32(int row, int chunk) {
   return static_cast<uint32_t>(row * 64 + ((chunk ^ ((row >> 1) & 3)) << 4));
 }
+// One warp's 32 rows x 32 fp32 columns (each thread's `in` is its own row)
+// to global memory: own row into the buffer (128 bytes, swizzled chunks),
+// then four 128-byte row segments per warp store.
+__device__ __forceinline__ void warp_store_rows32f(float* base, long long ld, int lane, uint8_t* buf,
+                                                   const float* in) {
+#pragma unroll
+  for (int c = 0; c < 8; ++c)
+    *reinterpret_cast<float4*>(buf + epi_swz(lane, c)) = make_float4(in[4 * c], in[4 * c + 1], in[4 * c + 2], in[4 * c + 3]);
+  __syncwarp();
+#pragma unroll
+  for (int k0 = 0; k0 < 8; k0 += 4) {
+    float4 g[4];
+#pragma unroll
+    for (int k = 0; k < 4; ++k)
+      g[k] = *reinterpret_cast<const float4*>(buf + epi_swz(4 * (k0 + k) + (lane >> 3), lane & 7));
+#pragma unroll
+    for (int k = 0; k < 4; ++k)
+      *reinterpret_cast<float4*>(base + (long long)(4 * (k0 + k) + (lane >> 3)) * ld + (lane & 7) * 4) = g[k];
+  }
+  __syncwarp();
+}
+
 __device__ __forceinline__ void warp_issue_rows32(const __nv_bfloat16* base, long long ld, int lane, uint4 (&g)[4]) {
 #pragma unroll
   for (int k = 0; k < 4; ++k)
@@ -730,7 +752,8 @@ __device__ __forceinline__ bool epi_fast_ok(const GemmGroup& G, int prob, int r0
     }
     return true;
   } else if constexpr (EPI == EPI_APPLY || EPI == EPI_APPLY_MIXED) {
-    if (G.xf_write || (G.d_ld & 7) != 0 || (G.xl_write && (G.xl_ld & 7) != 0)) return false;
+    if ((G.d_ld & 7) != 0 || (G.xl_write && (G.xl_ld & 7) != 0)) return false;
+    if (G.xf_write && (EPI == EPI_APPLY_MIXED || G.tma_epi || (G.xf_ld & 3) != 0)) return false;
     if (EPI == EPI_APPLY_MIXED && ((G.xh_ld | G.xl_ld) & 7) != 0) return false;
     return true;
   } else if constexpr (EPI == EPI_APPLY_FINAL) {
@@ -805,9 +828,17 @@ __device__ __forceinline__ void epi_fast64(const GemmGroup& G, int prob, int r0,
       pm += 2 * ld;
     }
   } else if constexpr (EPI == EPI_APPLY) {
-    __nv_bfloat16* D = static_cast<__nv_bfloat16*>(G.d) + (long long)prob * G.d_bs + (long long)r0 * G.d_ld + c0;
-    pack_row64(v, pk);
-    warp_store_rows64(D, G.d_ld, lane, buf, pk);
+    if (G.xf_write) {
+      // the NS output in fp32 (NorMuon's row pass reads it), two 32-column
+      // halves; nothing reads a bf16 copy of the last iterate
+      float* X = G.xf + (long long)prob * G.xf_bs + (long long)r0 * G.xf_ld + c0;
+      warp_store_rows32f(X, G.xf_ld, lane, buf, v);
+      warp_store_rows32f(X + 32, G.xf_ld, lane, buf, v + 32);
+    } else {
+      __nv_bfloat16* D = static_cast<__nv_bfloat16*>(G.d) + (long long)prob * G.d_bs + (long long)r0 * G.d_ld + c0;
+      pack_row64(v, pk);
+      warp_store_rows64(D, G.d_ld, lane, buf, pk);
+    }
   } else if constexpr (EPI == EPI_APPLY_FINAL) {
     warp_rows_from_frags(ga, lane, buf, pk);
     float decay, step;
